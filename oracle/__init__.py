@@ -1,0 +1,144 @@
+"""fp64 CPU oracle for the selective-SSM (S6) forward scan.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
+baseline may import this package; the product path never does.  It shares no
+code with the CUDA library (the only common dependency is the seeded input
+generator in `ssm_inputs`, which holds none of the scan's arithmetic).
+
+The arithmetic lives in `ssm_oracle.c` (plain fp64 loop; see its header for the
+passages it follows).  This wrapper only converts the generated tensors exactly
+to float64 and marshals pointers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_oracle.so")
+_lib = None
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("dim", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("nheads", ctypes.c_int64), ("ngroups", ctypes.c_int64)]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with plain gcc: fp64, no FMA contraction, no fast-math."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+                               "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def load(path: Optional[str] = None):
+    """Load the oracle library (optionally another build of it, e.g. in a test)."""
+    lib = ctypes.CDLL(path or build())
+    p = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_selective_scan_f64.restype = ctypes.c_int
+    lib.oracle_selective_scan_f64.argtypes = [
+        ctypes.POINTER(_Dims), p, p, p, p, p, p, p, p, ctypes.c_int, p,
+        ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, p, p, p, ctypes.c_int]
+    return lib
+
+
+def _get_lib():
+    global _lib
+    if _lib is None:
+        _lib = load()
+    return _lib
+
+
+def _nthreads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _f64(a) -> Optional[np.ndarray]:
+    """Exact float64 copy of a tensor given as float64/float32 or bf16 bits (uint16)."""
+    if a is None:
+        return None
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        b = a.astype(np.uint32) << 16
+        return np.ascontiguousarray(b.view(np.float32).astype(np.float64))
+    return np.ascontiguousarray(a.astype(np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def selective_scan(batch: int, dim: int, seqlen: int, dstate: int, u, delta, A, B, C, D=None, z=None,
+                   delta_bias=None, softplus: bool = True, nheads: int = 0, ngroups: int = 1,
+                   h0=None, channels: Optional[Sequence[int]] = None, nthreads: Optional[int] = None,
+                   lib=None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Run the fp64 oracle.
+
+    Returns (out, last_state, mag) in float64.  Full mode: out/mag (batch, dim, L),
+    last_state (batch, dim, N).  Row mode (`channels` = flat ids b*dim + d; u, z,
+    delta and h0 given as the matching rows): out/mag (nch, L), last_state (nch, N).
+    """
+    H = nheads if nheads else dim
+    dims = _Dims(batch, dim, seqlen, dstate, H, ngroups)
+    uu, dd, AA, BB, CC = _f64(u), _f64(delta), _f64(A), _f64(B), _f64(C)
+    DD, zz, bb, hh = _f64(D), _f64(z), _f64(delta_bias), _f64(h0)
+    if channels is None:
+        rows = batch * dim
+        ch = None
+        nch = 0
+    else:
+        ch = np.ascontiguousarray(np.asarray(channels, dtype=np.int64))
+        rows = nch = int(ch.size)
+    # size checks (the C side trusts these)
+    exp_u = rows * seqlen
+    exp_delta = (batch * H if channels is None else rows) * seqlen
+    if uu.size != exp_u or dd.size != exp_delta:
+        raise ValueError("u / delta size does not match the problem")
+    if zz is not None and zz.size != exp_u:
+        raise ValueError("z size does not match the problem")
+    if BB.size != batch * ngroups * dstate * seqlen or CC.size != BB.size:
+        raise ValueError("B / C size does not match the problem")
+    if AA.size != (dim * dstate if H == dim else H):
+        raise ValueError("A size does not match the problem")
+    if DD is not None and DD.size != dim:
+        raise ValueError("D size does not match the problem")
+    if bb is not None and bb.size != H:
+        raise ValueError("delta_bias size does not match the problem")
+    if hh is not None and hh.size != rows * dstate:
+        raise ValueError("h0 size does not match the problem")
+    out = np.empty(rows * seqlen, dtype=np.float64)
+    mag = np.empty(rows * seqlen, dtype=np.float64)
+    last = np.empty(rows * dstate, dtype=np.float64)
+    lib = lib or _get_lib()
+    rc = lib.oracle_selective_scan_f64(
+        ctypes.byref(dims), _ptr(uu), _ptr(dd), _ptr(AA), _ptr(BB), _ptr(CC), _ptr(DD), _ptr(zz), _ptr(bb),
+        1 if softplus else 0, _ptr(hh),
+        ch.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)) if ch is not None else None, nch,
+        _ptr(out), _ptr(last), _ptr(mag), nthreads or _nthreads())
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    if channels is None:
+        return (out.reshape(batch, dim, seqlen), last.reshape(batch, dim, dstate),
+                mag.reshape(batch, dim, seqlen))
+    return out.reshape(rows, seqlen), last.reshape(rows, dstate), mag.reshape(rows, seqlen)
+
+
+def run_inputs(dims, inputs: dict, channels=None, h0=None, nthreads=None, lib=None):
+    """Convenience: run on a dict produced by `ssm_inputs.make_inputs`."""
+    return selective_scan(dims.batch, dims.dim, dims.seqlen, dims.dstate, inputs["u"], inputs["delta"],
+                          inputs["A"], inputs["B"], inputs["C"], inputs.get("D"), inputs.get("z"),
+                          inputs.get("delta_bias"), bool(inputs.get("softplus", True)), dims.nheads,
+                          dims.ngroups, h0=h0, channels=channels, nthreads=nthreads, lib=lib)

@@ -1,0 +1,409 @@
+"""Throughput of the selective-scan (S6) forward on B200: one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one forward scan (the whole hot path: softplus, discretisation,
+recurrence, readout, D skip, gate, final state) over one batch of synthetic
+input.  `value` is B*D*L elements per second over all ranks, with inputs
+resident in HBM; `e2e` is the same metric through the host-buffer C-ABI entry
+point with the host<->device copies inside the timed region.
+
+The scan does not shard across GPUs beyond independent replicas: with N > 1
+(torchrun) every rank runs the same workload on its own GPU with no collective
+on the data path (weak scaling); the only collectives are the barrier and the
+max-over-ranks of the timed interval.
+
+`--impl reference` times the fp64 CPU oracle instead (rank 0 only), on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "selective-scan Gelem/s (B*D*L/s) fwd and % of HBM/MUFU roofline on 1 B200"
+UNIT = "Gelem/s"
+DEFAULT_WORKLOAD = "mamba-130m"
+L2_BYTES = 126 * 1024 * 1024
+SMS = 148
+EX2_PER_CLK_PER_SM = 16          # MUFU ex2 issue rate per SM per clock (sm_80 .. sm_100 family)
+NOMINAL_SM_MHZ = 1965.0
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+def _rank_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", 6650.0)), float(d.get("sm_max_mhz", NOMINAL_SM_MHZ)), "measured"
+    return 6650.0, NOMINAL_SM_MHZ, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML on a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - no NVML
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def _alg_bytes(d, with_state=True):
+    """Algorithmic HBM bytes of one forward call: every input read once, every output written once."""
+    e = 2 if d.dtype == "bf16" else 4
+    bdl = d.batch * d.dim * d.seqlen
+    b = 3 * bdl * e if d.H == d.dim else 2 * bdl * e + d.batch * d.H * d.seqlen * e   # u, z (+delta)
+    b += bdl * e                                                                        # out
+    b += 2 * d.batch * d.ngroups * d.dstate * d.seqlen * e                               # B, C
+    b += (d.dim * d.dstate if d.H == d.dim else d.H) * 4 + d.dim * 4 + d.H * 4          # A, D, bias
+    if with_state:
+        b += d.batch * d.dim * d.dstate * 4                                             # last_state
+    return b
+
+
+def _exps(d):
+    """exp count of the metric: B*D*L*N (one exp per state per step)."""
+    return d.batch * d.dim * d.seqlen * d.dstate
+
+
+def _kernel_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_30_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_from_profiles(workload):
+    """dram bytes per launch from a committed ncu summary, if it was taken on this kernel source."""
+    p = os.path.join(PROFILE_DIR, "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(workload)
+    if not ent or ent.get("kernel_src_sha") != _kernel_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def _to_dev(arr, dev):
+    import torch
+    if arr is None:
+        return None
+    if arr.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(arr)).to(dev)
+
+
+def _to_pinned(arr):
+    import torch
+    if arr is None:
+        return None
+    t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16) if arr.dtype == np.uint16
+                         else np.ascontiguousarray(arr))
+    return t.pin_memory()
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_sample(d, recipe, seed, target_s=12.0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of channels of the workload."""
+    import oracle
+    import ssm_inputs as si
+    cores = _cores()
+    total = d.batch * d.dim
+    rng = np.random.default_rng(7)
+
+    def run(nch):
+        ch = sorted(int(c) for c in rng.choice(total, size=min(total, nch), replace=False))
+        rows = si.make_inputs(d, recipe, seed, channels=ch)
+        t0 = time.perf_counter()
+        oracle.run_inputs(d, rows, channels=ch, nthreads=cores)
+        return time.perf_counter() - t0, len(ch)
+
+    # calibrate on one channel per core, then size the sample to about target_s
+    dt, n = run(min(total, cores))
+    per_ch = dt / max(1, n) * cores
+    nch = int(max(cores, min(total, target_s * cores / max(per_ch, 1e-9))))
+    dt, n = run(nch)
+    elems = n * d.seqlen
+    return {"value": elems / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {total} channels x L={d.seqlen} (N={d.dstate}), fp64, {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args):
+    rank, _, world = _rank_env()
+    if rank != 0:
+        return
+    import ssm_inputs as si
+    w = si.WORKLOADS[args.workload]
+    d = w.dims
+    per_step = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        target = max(1.0, min(20.0, 150.0 / max(1, args.warmup + args.steps)))
+        r = cpu_oracle_sample(d, w.recipe, w.seed, target_s=target)
+        if i >= args.warmup:
+            per_step.append(r["value"])
+            base = r
+    v = statistics.median(per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded splitmix64)",
+            "config": {"workload": w.name, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen,
+                       "dstate": d.dstate, "nheads": d.H, "ngroups": d.ngroups, "io_dtype": d.dtype},
+            "cpu_baseline": dict(base, value=v),
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import ssm_inputs as si
+    import selective_state_space_30_b200 as ssm
+
+    rank, local, world = _rank_env()
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = si.WORKLOADS[args.workload]
+    d = w.dims
+    io = ssm.SSM_BF16 if d.dtype == "bf16" else ssm.SSM_F32
+    inp = si.make_inputs(d, w.recipe, w.seed)
+    names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+    alg_bytes = _alg_bytes(d)
+    # enough copies that consecutive steps never find their inputs in L2
+    copies = max(2, int(np.ceil(3 * L2_BYTES / alg_bytes)))
+    sets = []
+    for _ in range(copies):
+        t = {k: _to_dev(inp[k], dev) for k in names}
+        t["out"] = torch.empty_like(t["u"])
+        t["last"] = torch.empty(d.batch, d.dim, d.dstate, dtype=torch.float32, device=dev)
+        sets.append(t)
+    dims = ssm.make_dims(d.batch, d.dim, d.seqlen, d.dstate, d.H, d.ngroups, io)
+    plan = ssm.ssm_scan_plan(dims, local)
+    info = ssm.ssm_scan_plan_info(plan)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step(i):
+        t = sets[i % copies]
+        ssm.ssm_selective_scan_fwd(plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                   t["delta_bias"], w.recipe.softplus, dims, t["out"], t["last"], sh)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step(i)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    st = ssm.ssm_scan_device_status(plan, sh)
+    if st != ssm.SSM_OK:
+        raise RuntimeError(f"device status {ssm.ssm_status_string(st)}")
+
+    elems = d.batch * d.dim * d.seqlen
+    ms_per_step = total_ms / args.steps
+    value = world * elems * args.steps / (total_ms * 1e-3) / 1e9
+
+    # roofline of the scan kernel (one launch per step)
+    hbm_gbs, sm_max_mhz, peak_src = _peaks()
+    avg_launch_s = statistics.mean(launch_ms) * 1e-3
+    exps = _exps(d)
+    mufu_peak = SMS * EX2_PER_CLK_PER_SM * sm_max_mhz * 1e6        # ex2/s at the max SM clock
+    # MUFU rate measured in this process (probe kernel), at whatever clock the GPU runs
+    sink = torch.empty(SMS * 8 * 256, device=dev)
+    ssm.ssm_probe_ex2(sink, SMS * 8, 64, sh)
+    torch.cuda.synchronize(dev)
+    pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pe0.record(stream)
+    ssm.ssm_probe_ex2(sink, SMS * 8, 2048, sh)
+    pe1.record(stream)
+    torch.cuda.synchronize(dev)
+    probe_rate = SMS * 8 * 256 * 2048 * 16 / (pe0.elapsed_time(pe1) * 1e-3)
+    t_roof = max(alg_bytes / (hbm_gbs * 1e9), exps / mufu_peak)
+    traffic = _traffic_from_profiles(w.name)
+    roof = {"bound": "alu", "achieved": exps / avg_launch_s / 1e9, "peak": mufu_peak / 1e9, "unit": "Gexp/s",
+            "frac": (exps / avg_launch_s) / mufu_peak, "traffic": traffic,
+            "what": "MUFU ex2: B*D*L*N exps per launch / mean launch time; peak = 148 SM x 16 ex2/clk x "
+                    f"{sm_max_mhz:.0f} MHz (derived)",
+            "roofline_frac": t_roof / avg_launch_s,
+            "hbm": {"achieved": alg_bytes / avg_launch_s / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                    "frac": alg_bytes / avg_launch_s / 1e9 / hbm_gbs, "peak_source": peak_src,
+                    "alg_bytes_per_launch": alg_bytes},
+            "mufu_probe_gexps": probe_rate / 1e9,
+            "frac_of_probe": (exps / avg_launch_s) / probe_rate}
+
+    # end to end through the host-buffer entry point: pinned host inputs, copies in the timed region
+    e2e = None
+    if not args.no_e2e:
+        hp = {k: _to_pinned(inp[k]) for k in names}
+        hout = torch.empty(d.batch, d.dim, d.seqlen, dtype=torch.int16 if d.dtype == "bf16" else torch.float32,
+                           pin_memory=True)
+        hlast = torch.empty(d.batch, d.dim, d.dstate, dtype=torch.float32, pin_memory=True)
+        e2e_steps = max(3, min(args.steps, 50))
+
+        def hstep():
+            ssm.ssm_selective_scan_fwd_host(plan, hp["u"], hp["delta"], hp["A"], hp["B"], hp["C"], hp["D"],
+                                            hp["z"], hp["delta_bias"], w.recipe.softplus, dims, hout, hlast, sh)
+        for _ in range(2):
+            hstep()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            hstep()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([ems], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        h2d = sum(hp[k].numel() * hp[k].element_size() for k in names if hp[k] is not None)
+        d2h = hout.numel() * hout.element_size() + hlast.numel() * hlast.element_size()
+        e2e = {"value": world * elems * e2e_steps / (ems * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
+               "path": "ssm_selective_scan_fwd_host (pinned host buffers)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(d, w.recipe, w.seed)
+
+    ssm.ssm_scan_destroy(plan)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 (bf16 I/O)" if d.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded splitmix64; shapes/inits of the Mamba layer)",
+            "config": {"workload": w.name, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen, "dstate": d.dstate,
+                       "nheads": d.H, "ngroups": d.ngroups, "io_dtype": d.dtype, "parallelism": f"replicas x{world}",
+                       "l2": f"{copies} rotating input sets of {alg_bytes / 1e6:.0f} MB (> 3x 126 MB L2), no flush",
+                       "kernel": info["variant"], "grid": info["grid"], "block": info["block"]},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clk.summary(), "gpu_launches": args.steps * info["launches_per_call"]}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,162 @@
+/*
+ * ssm_scan.h -- C ABI of the B200 (sm_100a) selective-SSM (S6) forward scan.
+ *
+ * The operation (Mamba "architecture-details" page, section "How S6 Works";
+ * "Agent 229: SSM optimization patterns" page, section 7 "Selective Attention
+ * Mechanism" for A_bar = exp(delta*A)): for every batch row b, channel d and
+ * state n, walking t = 0 .. L-1 from h = 0,
+ *
+ *     dt      = softplus(delta[b,hd,t] + delta_bias[hd])     (or without softplus)
+ *     h[n]    = exp(dt * A[d,n]) * h[n] + dt * B[b,g,n,t] * u[b,d,t]
+ *     y       = sum_n C[b,g,n,t] * h[n] + D[d] * u[b,d,t]
+ *     out     = y * silu(z[b,d,t]),     silu(z) = z / (1 + exp(-z))
+ *
+ * and the state after the last step is returned as last_state[b,d,:].
+ * hd = d / (dim/nheads) is the channel's head (hd = d when nheads == dim) and
+ * g = d / (dim/ngroups) its B/C group.  With nheads < dim, A holds one scalar
+ * per head (A[hd] for every n), the layout of Mamba-2 ("SKILL" page, Mamba-2
+ * section: headdim, ngroups, d_state=128).
+ *
+ * Arithmetic: fp32 in registers (state, dt, products), inputs and outputs in
+ * the I/O dtype (fp32 or bf16, rounded to nearest even on output).
+ *
+ * Layouts -- every tensor is contiguous, row-major, in device memory owned by
+ * the caller:
+ *   u, z, out    (batch, dim, seqlen)          io dtype
+ *   delta        (batch, nheads, seqlen)       io dtype
+ *   B, C         (batch, ngroups, dstate, seqlen) io dtype
+ *   A            (dim, dstate) fp32, or (nheads) fp32 when nheads < dim
+ *   D            (dim) fp32                     nullable: no skip term
+ *   delta_bias   (nheads) fp32                  nullable: zero bias
+ *   z            nullable: no gate (out = y)
+ *   last_state   (batch, dim, dstate) fp32      nullable: not written
+ *
+ * Errors: every call returns an ssm_status_t.  Argument checks happen on the
+ * host before anything is launched; kernel-side conditions (a bounded wait
+ * that ran out, a debug bounds check) are recorded in the plan's device status
+ * word and read back with ssm_scan_device_status.  No call traps, asserts or
+ * aborts on the device.
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA stream type, declared without including the CUDA headers:
+ * a cudaStream_t converts to it as is; NULL is the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st* ssm_stream_t;
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1, /* NULL required pointer, bad size, dims != plan dims, destroyed plan */
+    SSM_ERR_UNSUPPORTED = 2, /* a shape or dtype no kernel here handles (e.g. dstate not in {8,16,32,64,128}) */
+    SSM_ERR_CUDA = 3,        /* a CUDA runtime call failed (allocation, launch, copy) */
+    SSM_ERR_TIMEOUT = 4,     /* device side: a bounded inter-CTA wait gave up */
+    SSM_ERR_BOUNDS = 5       /* device side: a debug-build bounds check fired */
+} ssm_status_t;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
+
+/* Problem shape.  nheads == dim is the S6 layout (per-channel delta, A, bias);
+ * nheads < dim gives one delta row, bias and scalar A per head.  dim must be a
+ * multiple of nheads and of ngroups. */
+typedef struct {
+    int64_t batch;    /* B */
+    int64_t dim;      /* D: channels (d_inner) */
+    int64_t seqlen;   /* L */
+    int64_t dstate;   /* N */
+    int64_t nheads;   /* H: == dim for S6 */
+    int64_t ngroups;  /* G: B/C groups */
+    int32_t io_dtype; /* ssm_dtype_t of u, delta, z, B, C, out */
+    int32_t reserved; /* must be 0 */
+} ssm_dims_t;
+
+typedef struct ssm_plan_s* ssm_plan_t;
+
+/*
+ * Create a plan for one problem shape on one device: validates the shape,
+ * picks the kernel and allocates the plan's own device workspace (the status
+ * word and the chunk-carry buffers).  The plan belongs to the caller until
+ * ssm_scan_destroy.  Returns SSM_ERR_INVALID_ARG for a NULL out_plan or a bad
+ * shape, SSM_ERR_UNSUPPORTED for a shape no kernel handles, SSM_ERR_CUDA when
+ * the device cannot be used or the workspace cannot be allocated.
+ */
+int ssm_scan_plan(ssm_plan_t* out_plan, const ssm_dims_t* dims, int device);
+
+/*
+ * The forward scan (the operation above), asynchronous on `stream`.
+ * `dims` must equal the plan's dims.  Pointers are device pointers owned by
+ * the caller and are not kept after the call returns; `out` must not alias an
+ * input.  softplus != 0 applies softplus to delta + delta_bias.
+ * Allocates nothing.  One plan must not run on two streams at once.
+ * Returns SSM_ERR_INVALID_ARG for a NULL required pointer (u, delta, A, B, C,
+ * out) or mismatched dims, SSM_ERR_CUDA if the launch fails.
+ */
+int ssm_selective_scan_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A,
+                           const void* B, const void* C, const float* D, const void* z,
+                           const float* delta_bias, int softplus, const ssm_dims_t* dims, void* out,
+                           float* last_state, ssm_stream_t stream);
+
+/*
+ * Same as ssm_selective_scan_fwd, starting from the state h0 (batch, dim, dstate)
+ * fp32 instead of zero (h0 == NULL means zero).  Running [0, L1) and then
+ * [L1, L) with h0 = the first call's last_state gives the same result as one
+ * run over [0, L) ("Agent 229" page, section 9 "Chunked Computation": the final
+ * state of a chunk is the initial state of the next).  h0 may alias last_state.
+ */
+int ssm_selective_scan_fwd_h0(ssm_plan_t plan, const void* u, const void* delta, const float* A,
+                              const void* B, const void* C, const float* D, const void* z,
+                              const float* delta_bias, int softplus, const ssm_dims_t* dims,
+                              const float* h0, void* out, float* last_state, ssm_stream_t stream);
+
+/*
+ * End-to-end variant: the same arguments as ssm_selective_scan_fwd but every
+ * tensor pointer is HOST memory (pinned memory makes the copies asynchronous).
+ * The plan allocates device copies on first use (kept until ssm_scan_destroy);
+ * each call copies the inputs host->device, runs the scan and copies out (and
+ * last_state, if given) device->host, all on `stream`.  The host outputs are
+ * complete once the stream is synchronised.
+ */
+int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delta, const float* A,
+                                const void* B, const void* C, const float* D, const void* z,
+                                const float* delta_bias, int softplus, const ssm_dims_t* dims,
+                                void* out, float* last_state, ssm_stream_t stream);
+
+/* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
+int ssm_scan_destroy(ssm_plan_t plan);
+
+/*
+ * Synchronise `stream`, return the kernel-side status recorded since the last
+ * call (SSM_OK, SSM_ERR_TIMEOUT, SSM_ERR_BOUNDS) and clear it.
+ */
+int ssm_scan_device_status(ssm_plan_t plan, ssm_stream_t stream);
+
+/* Static, human-readable text for a status code. */
+const char* ssm_status_string(int status);
+
+/*
+ * Launch facts of the plan's kernel, for measurement and tests: the grid size,
+ * threads per CTA, dynamic shared memory bytes, kernel launches per forward
+ * call, and the variant name (static string).  Any output pointer may be NULL.
+ */
+int ssm_scan_plan_info(ssm_plan_t plan, int* grid, int* block, int* smem_bytes, int* launches_per_call,
+                       const char** variant);
+
+/*
+ * Measurement helper (not part of the scan): runs `blocks` CTAs of 256 threads,
+ * each thread issuing `iters` x 16 independent ex2.approx operations, and
+ * writes a checksum per thread to `sink` (blocks*256 floats, device memory).
+ * The bench times it to measure the MUFU ex2 rate of the GPU it runs on.
+ */
+int ssm_probe_ex2(float* sink, int blocks, int iters, ssm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

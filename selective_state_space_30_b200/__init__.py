@@ -1,0 +1,132 @@
+"""B200-native selective-SSM (S6) forward scan.
+
+The product is the CUDA library `libssmscan.so` (C ABI: include/ssm_scan.h).
+This package binds it with ctypes (`_abi`, same names as the C entry points)
+and adds a small torch-tensor front end:
+
+    out, last_state = selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus=True)
+
+PyTorch is only used for device memory and streams; the scan runs in the
+library's kernels.  There is no CPU or PyTorch fallback.
+"""
+from __future__ import annotations
+
+import threading
+from typing import Dict, Optional, Tuple
+
+from . import _abi
+from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, SSM_ERR_TIMEOUT,  # noqa: F401
+                   SSM_ERR_UNSUPPORTED, SSM_F32, SSM_OK, SsmError, load_library, make_dims, ssm_dims_t,
+                   ssm_probe_ex2, ssm_scan_destroy, ssm_scan_device_status, ssm_scan_plan, ssm_scan_plan_info,
+                   ssm_selective_scan_fwd, ssm_selective_scan_fwd_h0, ssm_selective_scan_fwd_host,
+                   ssm_status_string)
+
+__all__ = ["selective_scan_fwd", "selective_scan_fwd_host", "Plan", "get_plan", "ssm_scan_plan",
+           "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0", "ssm_selective_scan_fwd_host",
+           "ssm_scan_destroy", "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info",
+           "ssm_probe_ex2", "make_dims", "SsmError", "load_library"]
+
+
+class Plan:
+    """Owns one ssm_plan_t (a problem shape on one device)."""
+
+    def __init__(self, batch, dim, seqlen, dstate, nheads=0, ngroups=1, io_dtype=SSM_BF16, device=0):
+        self.dims = make_dims(batch, dim, seqlen, dstate, nheads, ngroups, io_dtype)
+        self.device = int(device)
+        self.handle = ssm_scan_plan(self.dims, self.device)
+
+    def info(self) -> dict:
+        return ssm_scan_plan_info(self.handle)
+
+    def device_status(self, stream=None) -> int:
+        return ssm_scan_device_status(self.handle, stream)
+
+    def close(self) -> None:
+        if self.handle:
+            ssm_scan_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):  # pragma: no cover - interpreter shutdown order varies
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+_plans: Dict[tuple, Plan] = {}
+_plans_lock = threading.Lock()
+
+
+def get_plan(batch, dim, seqlen, dstate, nheads=0, ngroups=1, io_dtype=SSM_BF16, device=0) -> Plan:
+    key = (batch, dim, seqlen, dstate, nheads or dim, ngroups, io_dtype, device)
+    with _plans_lock:
+        p = _plans.get(key)
+        if p is None:
+            p = Plan(batch, dim, seqlen, dstate, nheads, ngroups, io_dtype, device)
+            _plans[key] = p
+        return p
+
+
+def _shapes(u, delta, A, B):
+    import torch
+    if u.dim() != 3 or delta.dim() != 3 or B.dim() != 4:
+        raise ValueError("u, delta: (batch, dim|nheads, seqlen); B, C: (batch, ngroups, dstate, seqlen)")
+    batch, dim, seqlen = u.shape
+    nheads = delta.shape[1]
+    ngroups, dstate = B.shape[1], B.shape[2]
+    if u.dtype == torch.bfloat16:
+        io = SSM_BF16
+    elif u.dtype == torch.float32:
+        io = SSM_F32
+    else:
+        raise ValueError("u must be bfloat16 or float32")
+    return batch, dim, seqlen, dstate, nheads, ngroups, io
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
+                       h0=None, return_last_state: bool = True, out=None, last_state=None,
+                       stream=None) -> Tuple[object, Optional[object]]:
+    """Forward scan on CUDA tensors (layouts as in include/ssm_scan.h).
+
+    Returns (out, last_state); last_state is None when return_last_state is False.
+    Output tensors are allocated with torch on u's device unless given.
+    """
+    import torch
+    batch, dim, seqlen, dstate, nheads, ngroups, io = _shapes(u, delta, A, B)
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("h0", h0)):
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError(f"{name} must be a CUDA tensor")
+            if not t.is_contiguous():
+                raise ValueError(f"{name} must be contiguous")
+    dev = u.device.index if u.device.index is not None else torch.cuda.current_device()
+    plan = get_plan(batch, dim, seqlen, dstate, nheads, ngroups, io, dev)
+    if out is None:
+        out = torch.empty_like(u)
+    if return_last_state and last_state is None:
+        last_state = torch.empty((batch, dim, dstate), dtype=torch.float32, device=u.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(u.device).cuda_stream
+    ssm_selective_scan_fwd_h0(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, h0, out,
+                              last_state if return_last_state else None, stream)
+    return out, (last_state if return_last_state else None)
+
+
+def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
+                            out=None, last_state=None, return_last_state: bool = True, device: int = 0,
+                            stream=None):
+    """End-to-end call on HOST tensors (pinned for asynchronous copies): the library
+    copies the inputs to the device, runs the scan and copies the results back."""
+    import torch
+    batch, dim, seqlen, dstate, nheads, ngroups, io = _shapes(u, delta, A, B)
+    plan = get_plan(batch, dim, seqlen, dstate, nheads, ngroups, io, device)
+    if out is None:
+        out = torch.empty_like(u, pin_memory=True)
+    if return_last_state and last_state is None:
+        last_state = torch.empty((batch, dim, dstate), dtype=torch.float32, pin_memory=True)
+    if stream is None:
+        stream = torch.cuda.current_stream(device).cuda_stream
+    ssm_selective_scan_fwd_host(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, out,
+                                last_state if return_last_state else None, stream)
+    return out, (last_state if return_last_state else None)

@@ -1,0 +1,6 @@
+// Instantiations of the forward-scan kernel for f32 I/O, N = 8 states.
+#include "scan_kernel.cuh"
+
+namespace ssm {
+SSM_DEFINE_PICK(float, f32, 8)
+}  // namespace ssm

@@ -1,0 +1,107 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every symbol
+include/*.h declares, and rejects bad arguments on the host.  No compute calls."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if not f.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", f)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(ssm_[A-Za-z0-9_]+)\s*\(", text, re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_30_b200 import build, _abi
+    build.build()
+    return _abi.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_scan_destroy"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    from selective_state_space_30_b200 import _abi
+    assert names == set(_abi.EXPORTS), "binding and header disagree"
+
+
+def test_status_strings(lib):
+    import selective_state_space_30_b200 as ssm
+    for code in range(6):
+        s = ssm.ssm_status_string(code)
+        assert s and s != "unknown status"
+    assert ssm.ssm_status_string(99) == "unknown status"
+
+
+def test_host_side_argument_checks(lib):
+    import selective_state_space_30_b200 as ssm
+    from selective_state_space_30_b200 import _abi
+    good = ssm.make_dims(2, 32, 64, 16, 32, 1, ssm.SSM_BF16)
+    # NULL out_plan
+    assert lib.ssm_scan_plan(None, ctypes.byref(good), 0) == ssm.SSM_ERR_INVALID_ARG
+    bad = [
+        ssm.make_dims(2, 30, 64, 16, 4, 1, ssm.SSM_BF16),   # dim not a multiple of nheads
+        ssm.make_dims(2, 32, 64, 16, 32, 3, ssm.SSM_BF16),  # dim not a multiple of ngroups
+        ssm.make_dims(-1, 32, 64, 16, 32, 1, ssm.SSM_BF16),
+        ssm.make_dims(2, 0, 64, 16, 32, 1, ssm.SSM_BF16),
+        ssm.make_dims(2, 32, 64, 0, 32, 1, ssm.SSM_BF16),
+        _abi.ssm_dims_t(2, 32, 64, 16, 32, 1, 7, 0),         # unknown dtype
+        _abi.ssm_dims_t(2, 32, 64, 16, 32, 1, 1, 5),         # reserved != 0
+    ]
+    for d in bad:
+        p = ctypes.c_void_p()
+        assert lib.ssm_scan_plan(ctypes.byref(p), ctypes.byref(d), 0) == ssm.SSM_ERR_INVALID_ARG
+        assert p.value is None
+    p = ctypes.c_void_p()
+    unsupported = ssm.make_dims(2, 32, 64, 24, 32, 1, ssm.SSM_BF16)   # N = 24: no kernel
+    assert lib.ssm_scan_plan(ctypes.byref(p), ctypes.byref(unsupported), 0) == ssm.SSM_ERR_UNSUPPORTED
+    # a NULL plan is rejected by every entry point that needs one
+    assert lib.ssm_selective_scan_fwd(None, None, None, None, None, None, None, None, None, 1,
+                                      ctypes.byref(good), None, None, None) == ssm.SSM_ERR_INVALID_ARG
+    assert lib.ssm_scan_device_status(None, None) == ssm.SSM_ERR_INVALID_ARG
+    assert lib.ssm_scan_plan_info(None, None, None, None, None, None) == ssm.SSM_ERR_INVALID_ARG
+    assert lib.ssm_scan_destroy(None) == ssm.SSM_OK
+    assert lib.ssm_probe_ex2(None, 1, 1, None) == ssm.SSM_ERR_INVALID_ARG
+
+
+def test_plan_without_a_gpu_reports_cuda_error(lib):
+    import torch
+    import selective_state_space_30_b200 as ssm
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    d = ssm.make_dims(2, 32, 64, 16, 32, 1, ssm.SSM_BF16)
+    p = ctypes.c_void_p()
+    assert lib.ssm_scan_plan(ctypes.byref(p), ctypes.byref(d), 0) == ssm.SSM_ERR_CUDA
+
+
+def test_product_path_never_touches_the_oracle():
+    """The package and its CUDA sources name neither the oracle nor the input generator."""
+    pkg = os.path.join(ROOT, "selective_state_space_30_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"\b(import\s+oracle|from\s+oracle|ssm_oracle|oracle_selective)", text), f
+                assert "ssm_inputs" not in text, f
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f.endswith((".py", ".c")):
+            text = open(os.path.join(ROOT, "oracle", f)).read()
+            assert "selective_state_space_30_b200" not in text and "libssmscan" not in text, f
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from selective_state_space_30_b200 import _abi
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _abi.load_library(str(tmp_path / "libssmscan.so"))

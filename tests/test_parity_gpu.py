@@ -1,0 +1,244 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI (needs a B200)."""
+import numpy as np
+import pytest
+
+import oracle
+import ssm_inputs as si
+from parity import check_out, check_state, oracle_rows, run_gpu, sample_channels, to_host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(dims, recipe, seed=0, h0=None, inp=None):
+    inp = inp if inp is not None else si.make_inputs(dims, recipe, seed)
+    out, last = run_gpu(dims, inp, h0=h0)
+    ro, rl, rm = oracle.run_inputs(dims, inp, h0=h0)
+    rep = check_out(to_host_f64(out), ro, rm, dims.dtype)
+    check_state(to_host_f64(last), rl)
+    return rep
+
+
+# --------------------------------------------------------------- the five workloads
+
+def test_tiny_f32_full():
+    w = si.WORKLOADS["tiny-f32"]
+    rep = _full_check(w.dims, w.recipe, w.seed)
+    assert rep["strict_pass"] == rep["n"]
+
+
+@pytest.mark.parametrize("name", ["mamba-130m", "mamba-1.4b", "mamba-2.8b-long", "mamba2-n128"])
+def test_workload_full_size_sampled(name):
+    """Full-size run in the bench's launch configuration; sampled channels checked
+    against the oracle, every output checked finite, state checked on the sample."""
+    w = si.WORKLOADS[name]
+    d = w.dims
+    inp = si.make_inputs(d, w.recipe, w.seed)
+    out, last = run_gpu(d, inp)
+    o = to_host_f64(out)
+    assert np.all(np.isfinite(o)), "non-finite output"
+    ls = last.cpu().numpy()
+    assert np.all(np.isfinite(ls)), "non-finite last_state"
+    ch = sample_channels(d, 64 if d.seqlen * d.dstate > 1 << 19 else 192)
+    ro, rl, rm = oracle_rows(d, inp, ch)
+    g = np.stack([o[c // d.dim, c % d.dim] for c in ch])
+    gl = np.stack([ls[c // d.dim, c % d.dim] for c in ch]).astype(np.float64)
+    rep = check_out(g, ro, rm, d.dtype, what=name)
+    check_state(gl, rl, what=name + " last_state")
+    print(name, rep)
+
+
+# --------------------------------------------------------------- small shapes, many tiles, ragged
+
+SMALL = [
+    # (batch, dim, L, N, nheads, ngroups, dtype)
+    (2, 80, 300, 16, 0, 1, "bf16"),     # partial channel tile, ragged L, unaligned rows (scalar loads)
+    (2, 80, 304, 16, 0, 1, "bf16"),     # 16-byte rows, ragged last block
+    (3, 40, 257, 16, 0, 1, "f32"),
+    (2, 64, 260, 16, 0, 1, "f32"),
+    (2, 96, 200, 16, 0, 2, "bf16"),     # two B/C groups
+    (2, 64, 200, 128, 4, 1, "bf16"),    # scalar A per head, N = 128
+    (1, 48, 96, 128, 3, 1, "f32"),
+    (2, 64, 136, 128, 0, 1, "bf16"),    # per-channel A with N = 128
+    (2, 24, 120, 8, 0, 1, "bf16"),
+    (2, 40, 88, 32, 0, 1, "bf16"),
+    (1, 40, 72, 64, 0, 1, "f32"),
+    (2, 64, 160, 64, 8, 2, "bf16"),
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+def test_small_full(shape):
+    b, dm, L, N, H, G, dt = shape
+    dims = si.Dims(b, dm, L, N, nheads=H, ngroups=G, dtype=dt)
+    head = dims.head_mode
+    recipe = si.Recipe(a_init="neg_uniform_1_16" if (head or N != 16) else "neg_n_plus_1",
+                       d_init="normal", delta_init="normal_half")
+    if not head and N != 16:
+        # per-channel A drawn per (d, n)
+        recipe = si.Recipe(a_init="neg_uniform_1_16", d_init="normal", delta_init="normal_half")
+    _full_check(dims, recipe, seed=3)
+
+
+@pytest.mark.parametrize("softplus,has_D,has_z,has_bias", [(False, True, True, True), (True, False, True, True),
+                                                         (True, True, False, True), (True, True, True, False),
+                                                         (False, False, False, False)])
+def test_optional_inputs(softplus, has_D, has_z, has_bias):
+    dims = si.Dims(2, 40, 100, 16, dtype="bf16")
+    r = si.Recipe(d_init="normal", delta_init="normal_half", softplus=softplus, has_D=has_D, has_z=has_z,
+                  has_bias=has_bias)
+    inp = si.make_inputs(dims, r, 5)
+    if not softplus:
+        # without softplus the step is delta + bias itself: keep it positive and small
+        delta = np.abs(si.to_f64(inp["delta"])) * 0.05
+        inp["delta"] = np.array([si.f64_to_bf16_bits(x) for x in delta.ravel()],
+                                dtype=np.uint16).reshape(delta.shape)
+        if has_bias:
+            inp["delta_bias"] = np.logaddexp(0.0, inp["delta_bias"].astype(np.float64)).astype(np.float32)
+    _full_check(dims, r, inp=inp)
+
+
+@pytest.mark.parametrize("L", [1, 2, 7, 31, 32, 33, 64])
+def test_short_sequences(L):
+    for dt in ("bf16", "f32"):
+        dims = si.Dims(2, 40, L, 16, dtype=dt)
+        _full_check(dims, si.Recipe(d_init="normal", delta_init="normal_half"), seed=L)
+
+
+def test_empty():
+    import torch
+    for dims in (si.Dims(0, 32, 64, 16), si.Dims(2, 32, 0, 16)):
+        inp = si.make_inputs(dims, si.Recipe(), 0)
+        out, last = run_gpu(dims, inp)
+        assert out.numel() == dims.batch * dims.dim * dims.seqlen
+        assert torch.all(last == 0)  # no steps: the state stays zero
+
+
+def test_initial_state_and_chunk_split():
+    """h0 input against the oracle, and [0,L1) + [L1,L) with the carried state equals one run."""
+    dims = si.Dims(2, 64, 384, 16, dtype="bf16")
+    r = si.Recipe(d_init="normal", delta_init="normal_half")
+    inp = si.make_inputs(dims, r, 9)
+    rng = np.random.default_rng(0)
+    h0 = rng.standard_normal((dims.batch, dims.dim, dims.dstate)).astype(np.float32)
+    _full_check(dims, r, inp=inp, h0=h0)
+    out, last = run_gpu(dims, inp)
+    for L1 in (128, 96, 100):
+        d1 = si.Dims(2, 64, L1, 16, dtype="bf16")
+        d2 = si.Dims(2, 64, dims.seqlen - L1, 16, dtype="bf16")
+        cut = lambda k, a, lo, hi: np.ascontiguousarray(a[..., lo:hi]) if k in ("u", "delta", "z", "B", "C") else a
+        i1 = {k: cut(k, v, 0, L1) for k, v in inp.items()}
+        i2 = {k: cut(k, v, L1, dims.seqlen) for k, v in inp.items()}
+        o1, s1 = run_gpu(d1, i1)
+        o2, s2 = run_gpu(d2, i2, h0=s1.cpu().numpy())
+        o12 = np.concatenate([to_host_f64(o1), to_host_f64(o2)], axis=2)
+        if L1 % 32 == 0:
+            # block boundaries line up: the same fp32 operations in the same order
+            assert np.array_equal(o12, to_host_f64(out)), f"split at {L1} not bit-exact"
+            assert np.array_equal(s2.cpu().numpy(), last.cpu().numpy())
+        else:
+            ro, rl, rm = oracle.run_inputs(dims, inp)
+            check_out(o12, ro, rm, "bf16")
+            check_state(s2.cpu().numpy().astype(np.float64), rl)
+
+
+def test_misaligned_pointers_take_scalar_path():
+    """Inputs at an odd 2-byte offset (not 16-byte aligned) give the same results as aligned ones."""
+    import torch
+    import selective_state_space_30_b200 as ssm
+    from parity import to_device
+    dims = si.Dims(2, 40, 96, 16, dtype="bf16")
+    inp = si.make_inputs(dims, si.Recipe(d_init="normal", delta_init="normal_half"), 4)
+    ref, ref_last = run_gpu(dims, inp)
+    d = ssm.make_dims(2, 40, 96, 16, 40, 1, ssm.SSM_BF16)
+
+    def shifted(a):
+        t = to_device(a)
+        buf = torch.empty(t.numel() + 1, dtype=t.dtype, device="cuda")
+        v = buf[1:].view(t.shape)
+        v.copy_(t)
+        return v
+    dev = {k: shifted(inp[k]) for k in ("u", "delta", "B", "C", "z")}
+    A, D, bias = to_device(inp["A"]), to_device(inp["D"]), to_device(inp["delta_bias"])
+    outbuf = torch.empty(2 * 40 * 96 + 1, dtype=torch.bfloat16, device="cuda")
+    out = outbuf[1:].view(2, 40, 96)
+    last = torch.empty(2, 40, 16, device="cuda")
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        ssm.ssm_selective_scan_fwd(plan, dev["u"], dev["delta"], A, dev["B"], dev["C"], D, dev["z"], bias, True,
+                                   d, out, last, None)
+        torch.cuda.synchronize()
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    assert torch.equal(out, ref) and torch.equal(last, ref_last)
+
+
+def test_host_entry_point_matches_device_path():
+    import torch
+    import selective_state_space_30_b200 as ssm
+    dims = si.Dims(2, 64, 256, 16, dtype="bf16")
+    inp = si.make_inputs(dims, si.Recipe(d_init="normal", delta_init="normal_half"), 6)
+    ref, ref_last = run_gpu(dims, inp)
+    d = ssm.make_dims(2, 64, 256, 16, 64, 1, ssm.SSM_BF16)
+    host = {k: np.ascontiguousarray(inp[k]) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    out = np.empty((2, 64, 256), dtype=np.uint16)
+    last = np.empty((2, 64, 16), dtype=np.float32)
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        ssm.ssm_selective_scan_fwd_host(plan, host["u"], host["delta"], host["A"], host["B"], host["C"],
+                                        host["D"], host["z"], host["delta_bias"], True, d, out, last, None)
+        torch.cuda.synchronize()
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    got = torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)
+    assert torch.equal(got, ref.cpu())
+    assert np.array_equal(last, ref_last.cpu().numpy())
+
+
+def test_deterministic():
+    w = si.WORKLOADS["mamba-130m"]
+    d = si.Dims(2, 256, 512, 16, dtype="bf16")
+    inp = si.make_inputs(d, w.recipe, 1)
+    o1, s1 = run_gpu(d, inp)
+    o2, s2 = run_gpu(d, inp)
+    import torch
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_argument_errors_on_gpu():
+    import selective_state_space_30_b200 as ssm
+    import torch
+    d = ssm.make_dims(1, 32, 64, 16, 32, 1, ssm.SSM_BF16)
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        x = torch.zeros(1, 32, 64, dtype=torch.bfloat16, device="cuda")
+        A = torch.zeros(32, 16, device="cuda")
+        BC = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
+        other = ssm.make_dims(1, 32, 65, 16, 32, 1, ssm.SSM_BF16)
+        rc = ssm.ssm_selective_scan_fwd(plan, x, x, A, BC, BC, None, None, None, True, other, x, None, None,
+                                        check=False)
+        assert rc == ssm.SSM_ERR_INVALID_ARG
+        rc = ssm.ssm_selective_scan_fwd(plan, None, x, A, BC, BC, None, None, None, True, d, x, None, None,
+                                        check=False)
+        assert rc == ssm.SSM_ERR_INVALID_ARG
+        rc = ssm.ssm_selective_scan_fwd(plan, x, x, A, BC, BC, None, None, None, True, d, x, None, None,
+                                        check=False)
+        assert rc == ssm.SSM_OK
+        assert ssm.ssm_scan_device_status(plan) == ssm.SSM_OK
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    with pytest.raises(ssm.SsmError):
+        ssm.ssm_scan_plan(ssm.make_dims(1, 32, 64, 24, 32, 1, ssm.SSM_BF16), 0)  # N = 24: no kernel
+
+
+def test_torch_front_end():
+    import torch
+    import selective_state_space_30_b200 as ssm
+    from parity import to_device
+    dims = si.Dims(2, 64, 128, 16, dtype="bf16")
+    inp = si.make_inputs(dims, si.Recipe(d_init="normal", delta_init="normal_half"), 2)
+    ref, ref_last = run_gpu(dims, inp)
+    t = {k: to_device(inp[k]) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    out, last = ssm.selective_scan_fwd(t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                       t["delta_bias"], softplus=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref) and torch.equal(last, ref_last)

@@ -264,6 +264,7 @@ def run_ours(args):
     dims = ssm.make_dims(d.batch, d.dim, d.seqlen, d.dstate, d.H, d.ngroups, io)
     plan = ssm.ssm_scan_plan(dims, local)
     info = ssm.ssm_scan_plan_info(plan)
+    sched = ssm.ssm_scan_plan_schedule(plan)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
 
@@ -381,7 +382,8 @@ def run_ours(args):
             "config": {"workload": w.name, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen, "dstate": d.dstate,
                        "nheads": d.H, "ngroups": d.ngroups, "io_dtype": d.dtype, "parallelism": f"replicas x{world}",
                        "l2": f"{copies} rotating input sets of {alg_bytes / 1e6:.0f} MB (> 3x 126 MB L2), no flush",
-                       "kernel": info["variant"], "grid": info["grid"], "block": info["block"]},
+                       "kernel": info["variant"], "grid": info["grid"], "block": info["block"],
+                       "schedule": sched},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk.summary(), "gpu_launches": args.steps * info["launches_per_call"]}
     print(json.dumps(line), flush=True)

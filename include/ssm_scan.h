@@ -127,6 +127,38 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
                                 const float* delta_bias, int softplus, const ssm_dims_t* dims,
                                 void* out, float* last_state, ssm_stream_t stream);
 
+/*
+ * Plan options (mostly for tests).  Changing SEG_LEN, CONSUMER_WARPS or
+ * WORKERS re-plans the schedule (synchronises the device).
+ *   SSM_OPT_SPIN_LIMIT         polls a chained wait makes before it gives up and
+ *                              records SSM_ERR_TIMEOUT (default about 2M, i.e. ~1 s)
+ *   SSM_OPT_INJECT_STALL       test hook, nonzero: every chained wait waits for a
+ *                              flag that no worker ever sets, so it runs out and the
+ *                              call reports SSM_ERR_TIMEOUT (outputs are then invalid);
+ *                              0 switches it off
+ *   SSM_OPT_SEG_LEN            force the segment length (rounded up to 32 steps);
+ *                              0 = automatic
+ *   SSM_OPT_CONSUMER_WARPS     force 4 or 8 consumer warps per CTA; 0 = automatic
+ *   SSM_OPT_WORKERS            cap the number of persistent CTAs; 0 = one per SM
+ * Returns SSM_ERR_INVALID_ARG for an unknown option or a bad value.
+ */
+typedef enum {
+    SSM_OPT_SPIN_LIMIT = 1,
+    SSM_OPT_INJECT_STALL = 2,
+    SSM_OPT_SEG_LEN = 3,
+    SSM_OPT_CONSUMER_WARPS = 4,
+    SSM_OPT_WORKERS = 5
+} ssm_option_t;
+int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value);
+
+/*
+ * The plan's schedule: consumer warps per CTA, segment length (time steps per
+ * work unit), channel tiles, segments per tile and persistent CTAs.  NULL
+ * outputs are skipped.
+ */
+int ssm_scan_plan_schedule(ssm_plan_t plan, int* consumer_warps, int* seg_len, int* n_tiles, int* n_seg,
+                           int* n_ctas);
+
 /* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
 int ssm_scan_destroy(ssm_plan_t plan);
 

@@ -25,8 +25,14 @@ SSM_BF16 = 1
 
 # every exported symbol declared in include/ssm_scan.h
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
-           "ssm_selective_scan_fwd_host", "ssm_scan_destroy", "ssm_scan_device_status",
-           "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
+           "ssm_selective_scan_fwd_host", "ssm_scan_set_option", "ssm_scan_plan_schedule", "ssm_scan_destroy",
+           "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
+
+SSM_OPT_SPIN_LIMIT = 1
+SSM_OPT_INJECT_STALL = 2
+SSM_OPT_SEG_LEN = 3
+SSM_OPT_CONSUMER_WARPS = 4
+SSM_OPT_WORKERS = 5
 
 
 class SsmError(RuntimeError):
@@ -68,6 +74,8 @@ def load_library(path: Optional[str] = None):
     lib.ssm_scan_plan_info.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32),
                                        ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_char_p)]
     lib.ssm_probe_ex2.argtypes = [vp, i32, i32, vp]
+    lib.ssm_scan_set_option.argtypes = [vp, i32, i64]
+    lib.ssm_scan_plan_schedule.argtypes = [vp] + [ctypes.POINTER(i32)] * 5
     for name in EXPORTS:
         if name != "ssm_status_string":
             getattr(lib, name).restype = i32
@@ -159,6 +167,16 @@ def ssm_scan_plan_info(plan: int) -> dict:
                                              ctypes.byref(n), ctypes.byref(name)), "ssm_scan_plan_info")
     return {"grid": g.value, "block": b.value, "smem_bytes": s.value, "launches_per_call": n.value,
             "variant": name.value.decode()}
+
+
+def ssm_scan_set_option(plan: int, option: int, value: int) -> int:
+    return _check(load_library().ssm_scan_set_option(plan, int(option), int(value)), "ssm_scan_set_option")
+
+
+def ssm_scan_plan_schedule(plan: int) -> dict:
+    v = [ctypes.c_int() for _ in range(5)]
+    _check(load_library().ssm_scan_plan_schedule(plan, *[ctypes.byref(x) for x in v]), "ssm_scan_plan_schedule")
+    return dict(zip(("consumer_warps", "seg_len", "n_tiles", "n_seg", "n_ctas"), (x.value for x in v)))
 
 
 def ssm_probe_ex2(sink, blocks: int, iters: int, stream=None) -> int:

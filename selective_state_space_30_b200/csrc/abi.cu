@@ -1,7 +1,9 @@
 // C ABI of the selective-scan library (declared in include/ssm_scan.h):
-// argument checks, plans, kernel choice and launch.
+// argument checks, plans (kernel choice, schedule, workspace) and launches.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -26,35 +28,51 @@ __global__ void __launch_bounds__(256) probe_ex2_kernel(float* sink, int iters) 
     sink[blockIdx.x * 256 + threadIdx.x] = s;
 }
 
-static bool pick_variant(int dtype, int64_t N, bool head, bool vec, Variant* v) {
+static bool pick_variant(int dtype, int64_t N, bool head, bool vec, int w, Variant* v) {
     const bool bf = dtype == SSM_BF16;
     switch (N) {
-        case 8: return bf ? pick_bf16_n8(head, vec, v) : pick_f32_n8(head, vec, v);
-        case 16: return bf ? pick_bf16_n16(head, vec, v) : pick_f32_n16(head, vec, v);
-        case 32: return bf ? pick_bf16_n32(head, vec, v) : pick_f32_n32(head, vec, v);
-        case 64: return bf ? pick_bf16_n64(head, vec, v) : pick_f32_n64(head, vec, v);
-        case 128: return bf ? pick_bf16_n128(head, vec, v) : pick_f32_n128(head, vec, v);
+        case 8: return bf ? pick_bf16_n8(head, vec, w, v) : pick_f32_n8(head, vec, w, v);
+        case 16: return bf ? pick_bf16_n16(head, vec, w, v) : pick_f32_n16(head, vec, w, v);
+        case 32: return bf ? pick_bf16_n32(head, vec, w, v) : pick_f32_n32(head, vec, w, v);
+        case 64: return bf ? pick_bf16_n64(head, vec, w, v) : pick_f32_n64(head, vec, w, v);
+        case 128: return bf ? pick_bf16_n128(head, vec, w, v) : pick_f32_n128(head, vec, w, v);
         default: return false;
     }
 }
 
 }  // namespace ssm
 
-// ------------------------------------------------------------------- C ABI
+// ------------------------------------------------------------------- plans
 
 struct ssm_plan_s {
     uint32_t magic;
     ssm_dims_t dims;
     int device;
-    int* d_status;
+    int sm_count;
+    // schedule
+    int w;                 // consumer warps per CTA
+    int threads;
+    int ch_per_tile;
+    int smem;
+    int tiles_per_group, n_tiles, n_seg, seg_len;
+    unsigned n_units, n_ctas;
+    int grid;
+    const char* name;
+    // options
+    unsigned spin_limit;
+    int64_t force_seg_len, force_k, force_workers;
+    // workspace: header | flags[n_tiles] | carry[n_tiles][CW][N]
+    unsigned char* ws;
+    size_t ws_bytes, flags_off, carry_off;
     // lazily allocated device mirrors for the host-buffer entry point
-    void* h_bufs[11];
-    size_t h_sizes[11];
+    void* h_bufs[10];
+    size_t h_sizes[10];
 };
 
 namespace {
 constexpr uint32_t kMagic = 0x53534d31u;  // "SSM1"
 constexpr uint32_t kDead = 0xdeadbeefu;
+constexpr unsigned kDefaultSpinLimit = 1u << 21;  // ~0.3-1 s of polling before a wait gives up
 
 bool dims_ok(const ssm_dims_t* d) {
     if (!d) return false;
@@ -63,10 +81,10 @@ bool dims_ok(const ssm_dims_t* d) {
     if (d->dim % d->nheads || d->dim % d->ngroups) return false;
     if (d->io_dtype != SSM_F32 && d->io_dtype != SSM_BF16) return false;
     if (d->reserved != 0) return false;
-    // element offsets must fit the kernel's 64-bit arithmetic comfortably
     const int64_t lim = (int64_t)1 << 46;
-    if (d->batch > lim / d->dim || d->batch * d->dim > lim / (d->seqlen > 0 ? d->seqlen : 1)) return false;
-    if (d->batch * d->ngroups > lim / (d->dstate * (d->seqlen > 0 ? d->seqlen : 1))) return false;
+    const int64_t L = d->seqlen > 0 ? d->seqlen : 1;
+    if (d->batch > lim / d->dim || d->batch * d->dim > lim / L) return false;
+    if (d->batch * d->ngroups > lim / (d->dstate * L)) return false;
     return true;
 }
 
@@ -76,15 +94,7 @@ bool same_dims(const ssm_dims_t* a, const ssm_dims_t* b) {
 }
 
 bool plan_ok(const ssm_plan_t p) { return p && p->magic == kMagic; }
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int tiles_per_group(const ssm_dims_t& d, int ch) {
-    const int64_t Dg = d.dim / d.ngroups;
-    return (int)((Dg + ch - 1) / ch);
-}
-
-int64_t grid_of(const ssm_dims_t& d, int ch) { return d.batch * d.ngroups * tiles_per_group(d, ch); }
 
 int set_device(int dev) {
     int cur = -1;
@@ -93,31 +103,168 @@ int set_device(int dev) {
     return SSM_OK;
 }
 
+bool head_mode(const ssm_dims_t& d) { return d.nheads != d.dim; }
+
+// Choose the consumer-warp count, segment length and grid; (re)allocate the workspace.
+int schedule(ssm_plan_s* p) {
+    const ssm_dims_t& d = p->dims;
+    const bool head = head_mode(d);
+    const int64_t Dg = d.dim / d.ngroups;
+    auto tiles_for = [&](int ct) { return d.batch * d.ngroups * ((Dg + ct - 1) / ct); };
+    ssm::Variant v8, v4;
+    if (!ssm::pick_variant(d.io_dtype, d.dstate, head, true, 8, &v8)) return SSM_ERR_UNSUPPORTED;
+    if (!ssm::pick_variant(d.io_dtype, d.dstate, head, true, 4, &v4)) return SSM_ERR_UNSUPPORTED;
+    // eight consumer warps (two per SM sub-partition) unless that leaves SMs without a tile
+    int w = 8;
+    if (p->force_k == 4 || p->force_k == 8) w = (int)p->force_k;
+    else if (tiles_for(v8.ch_per_tile) < p->sm_count) w = 4;
+    const ssm::Variant& v = w == 8 ? v8 : v4;
+    if (v.smem > 48 * 1024 &&
+        cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, v.fn, v.threads, v.smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (occ < 1) return SSM_ERR_UNSUPPORTED;
+    const int64_t n_tiles = tiles_for(v.ch_per_tile);
+    int64_t ctas = p->sm_count;  // one persistent CTA per SM
+    if (p->force_workers > 0 && p->force_workers < ctas) ctas = p->force_workers;
+    // segments: about 16 units per CTA, segments of at least 128 steps
+    const int64_t L = d.seqlen;
+    int64_t seg_len;
+    if (p->force_seg_len > 0) {
+        seg_len = (p->force_seg_len + ssm::kTB - 1) / ssm::kTB * ssm::kTB;
+    } else {
+        int64_t n_seg = (16 * ctas + n_tiles - 1) / (n_tiles > 0 ? n_tiles : 1);
+        const int64_t max_seg = (L + 127) / 128;
+        if (n_seg > max_seg) n_seg = max_seg;
+        if (n_seg < 1) n_seg = 1;
+        seg_len = ((L + n_seg - 1) / n_seg + ssm::kTB - 1) / ssm::kTB * ssm::kTB;
+    }
+    if (seg_len < ssm::kTB) seg_len = ssm::kTB;
+    const int64_t n_seg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
+    const int64_t n_units = n_tiles * n_seg;
+    if (n_units >= (int64_t)1 << 31 || seg_len > (int64_t)1 << 30) return SSM_ERR_UNSUPPORTED;
+    if (ctas > n_units) ctas = n_units;
+    if (ctas < 1) ctas = 1;
+    p->w = w;
+    p->threads = v.threads;
+    p->ch_per_tile = v.ch_per_tile;
+    p->smem = v.smem;
+    p->tiles_per_group = (int)((Dg + v.ch_per_tile - 1) / v.ch_per_tile);
+    p->n_tiles = (int)n_tiles;
+    p->n_seg = (int)n_seg;
+    p->seg_len = (int)seg_len;
+    p->n_units = (unsigned)n_units;
+    p->n_ctas = (unsigned)ctas;
+    p->grid = (int)ctas;
+    p->name = v.name;
+    // workspace: header | flags[n_tiles] | carry[n_tiles][CT][N]
+    const size_t flags_off = 64;
+    const size_t carry_off = (flags_off + (size_t)n_tiles * 4 + 255) / 256 * 256;
+    const size_t bytes = carry_off + (size_t)n_tiles * v.ch_per_tile * d.dstate * 4;
+    if (p->ws && p->ws_bytes < bytes) {
+        cudaFree(p->ws);
+        p->ws = nullptr;
+    }
+    if (!p->ws) {
+        if (cudaMalloc(&p->ws, bytes) != cudaSuccess) {
+            p->ws = nullptr;
+            return SSM_ERR_CUDA;
+        }
+        p->ws_bytes = bytes;
+    }
+    p->flags_off = flags_off;
+    p->carry_off = carry_off;
+    if (cudaMemset(p->ws, 0, p->ws_bytes) != cudaSuccess) return SSM_ERR_CUDA;
+    return SSM_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tensor_map_encoder() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+        tried = true;
+    }
+    return fn;
+}
+
+// A (rows x cols) row-major tensor seen as 2-D boxes of 32 steps x box_rows rows.
+bool encode_rows(CUtensorMap* m, const void* base, int esz, uint64_t cols, uint64_t rows, uint32_t box_rows,
+                 CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = tensor_map_encoder();
+    if (!enc || cols == 0 || rows == 0) return false;
+    const cuuint64_t gdim[2] = {cols, rows};
+    const cuuint64_t gstride[1] = {cols * (uint64_t)esz};
+    const cuuint32_t box[2] = {(cuuint32_t)ssm::kTB, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+               const_cast<void*>(base), gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A, const void* B, const void* C,
                const float* D, const void* z, const float* delta_bias, int softplus, const float* h0, void* out,
                float* last_state, cudaStream_t stream) {
     const ssm_dims_t& d = plan->dims;
-    const bool head = d.nheads != d.dim;
+    if (d.batch == 0) return SSM_OK;
     // Vector loads/stores need every per-lane chunk (up to 16 elements) wholly
     // inside or outside a row and 16-byte aligned: L % 16 == 0 plus aligned bases.
-    const bool vec = (d.seqlen % 16 == 0) && aligned16(u) && aligned16(delta) && aligned16(B) &&
-                     aligned16(C) && aligned16(out) && (!z || aligned16(z));
+    bool vec = d.seqlen > 0 && (d.seqlen % 16 == 0) && aligned16(u) && aligned16(delta) && aligned16(B) &&
+               aligned16(C) && aligned16(out) && (!z || aligned16(z));
+    const int esz = d.io_dtype == SSM_BF16 ? 2 : 4;
+    const int64_t P = d.dim / d.nheads;
+    const int ct = plan->ch_per_tile;
+    int delta_rows = ct;
+    if (head_mode(d)) {
+        delta_rows = (int)((ct - 1) / P + 2);
+        if (delta_rows > ct) delta_rows = ct;
+    }
+    ssm::TensorMaps tm;
+    std::memset(&tm, 0, sizeof(tm));
+    if (vec) {
+        const CUtensorMapSwizzle bc_swz = esz == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+        const uint64_t L = (uint64_t)d.seqlen;
+        vec = encode_rows(&tm.u, u, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              encode_rows(&tm.delta, delta, esz, L, (uint64_t)(d.batch * d.nheads), delta_rows,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              (!z || encode_rows(&tm.z, z, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE)) &&
+              encode_rows(&tm.B, B, esz, L, (uint64_t)(d.batch * d.ngroups * d.dstate), (uint32_t)d.dstate, bc_swz) &&
+              encode_rows(&tm.C, C, esz, L, (uint64_t)(d.batch * d.ngroups * d.dstate), (uint32_t)d.dstate, bc_swz);
+        // a shape the tensor maps cannot describe takes the element-copy path
+    }
     ssm::Variant v;
-    if (!ssm::pick_variant(d.io_dtype, d.dstate, head, vec, &v)) return SSM_ERR_UNSUPPORTED;
-    if (d.batch == 0) return SSM_OK;
+    if (!ssm::pick_variant(d.io_dtype, d.dstate, head_mode(d), vec, plan->w, &v)) return SSM_ERR_UNSUPPORTED;
     ssm::FwdParams prm;
     prm.u = u; prm.delta = delta; prm.A = A; prm.B = B; prm.C = C; prm.D = D; prm.z = z;
-    prm.bias = delta_bias; prm.h0 = h0; prm.out = out; prm.last_state = last_state; prm.status = plan->d_status;
-    prm.batch = d.batch; prm.dim = d.dim; prm.seqlen = d.seqlen; prm.nheads = d.nheads; prm.ngroups = d.ngroups;
+    prm.bias = delta_bias; prm.h0 = h0; prm.out = out; prm.last_state = last_state;
+    prm.ws = reinterpret_cast<ssm::WsHeader*>(plan->ws);
+    prm.flags = reinterpret_cast<unsigned*>(plan->ws + plan->flags_off);
+    prm.carry = reinterpret_cast<float*>(plan->ws + plan->carry_off);
+    prm.dim = d.dim; prm.seqlen = d.seqlen; prm.nheads = d.nheads; prm.ngroups = d.ngroups;
     prm.softplus = softplus ? 1 : 0;
-    prm.tiles_per_group = tiles_per_group(d, v.ch_per_cta);
-    const int64_t grid = grid_of(d, v.ch_per_cta);
-    if (grid > 0x7fffffff) return SSM_ERR_UNSUPPORTED;
-    if (v.smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
-            return SSM_ERR_CUDA;
-    }
-    v.fn<<<(unsigned)grid, ssm::kThreads, v.smem, stream>>>(prm);
+    prm.tiles_per_group = plan->tiles_per_group;
+    prm.n_tiles = plan->n_tiles;
+    prm.n_seg = plan->n_seg;
+    prm.seg_len = plan->seg_len;
+    prm.n_units = plan->n_units;
+    prm.n_ctas = plan->n_ctas;
+    prm.spin_limit = plan->spin_limit;
+    prm.delta_rows = delta_rows;
+    if (v.smem > 48 * 1024 &&
+        cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    v.fn<<<plan->grid, v.threads, v.smem, stream>>>(prm, tm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 }  // namespace
@@ -141,7 +288,7 @@ int ssm_scan_plan(ssm_plan_t* out_plan, const ssm_dims_t* dims, int device) {
     *out_plan = nullptr;
     if (!dims_ok(dims)) return SSM_ERR_INVALID_ARG;
     ssm::Variant v;
-    if (!ssm::pick_variant(dims->io_dtype, dims->dstate, dims->nheads != dims->dim, true, &v))
+    if (!ssm::pick_variant(dims->io_dtype, dims->dstate, dims->nheads != dims->dim, true, 8, &v))
         return SSM_ERR_UNSUPPORTED;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return SSM_ERR_CUDA;
@@ -151,17 +298,61 @@ int ssm_scan_plan(ssm_plan_t* out_plan, const ssm_dims_t* dims, int device) {
     p->magic = kMagic;
     p->dims = *dims;
     p->device = device;
-    if (cudaMalloc(&p->d_status, sizeof(int)) != cudaSuccess) {
+    p->spin_limit = kDefaultSpinLimit;
+    if (cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
         delete p;
         return SSM_ERR_CUDA;
     }
-    if (cudaMemset(p->d_status, 0, sizeof(int)) != cudaSuccess) {
-        cudaFree(p->d_status);
+    const int rc = schedule(p);
+    if (rc != SSM_OK) {
+        if (p->ws) cudaFree(p->ws);
         delete p;
-        return SSM_ERR_CUDA;
+        return rc;
     }
     *out_plan = p;
     return SSM_OK;
+}
+
+int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
+    if (!plan_ok(plan)) return SSM_ERR_INVALID_ARG;
+    if (set_device(plan->device) != SSM_OK) return SSM_ERR_CUDA;
+    switch (option) {
+        case SSM_OPT_SPIN_LIMIT:
+            if (value < 1 || value > 0x7fffffff) return SSM_ERR_INVALID_ARG;
+            plan->spin_limit = (unsigned)value;
+            return SSM_OK;
+        case SSM_OPT_INJECT_STALL: {
+            if (cudaDeviceSynchronize() != cudaSuccess) return SSM_ERR_CUDA;
+            const unsigned v = value ? 1u : 0u;
+            return cudaMemcpy(plan->ws + offsetof(ssm::WsHeader, inject), &v, sizeof(v), cudaMemcpyHostToDevice) ==
+                           cudaSuccess
+                       ? SSM_OK
+                       : SSM_ERR_CUDA;
+        }
+        case SSM_OPT_SEG_LEN:
+        case SSM_OPT_CONSUMER_WARPS:
+        case SSM_OPT_WORKERS: {
+            if (value < 0) return SSM_ERR_INVALID_ARG;
+            if (option == SSM_OPT_CONSUMER_WARPS && value != 0 && value != 4 && value != 8)
+                return SSM_ERR_INVALID_ARG;
+            if (cudaDeviceSynchronize() != cudaSuccess) return SSM_ERR_CUDA;
+            unsigned inject = 0;
+            if (cudaMemcpy(&inject, plan->ws + offsetof(ssm::WsHeader, inject), sizeof(inject),
+                           cudaMemcpyDeviceToHost) != cudaSuccess)
+                return SSM_ERR_CUDA;
+            if (option == SSM_OPT_SEG_LEN) plan->force_seg_len = value;
+            if (option == SSM_OPT_CONSUMER_WARPS) plan->force_k = value;
+            if (option == SSM_OPT_WORKERS) plan->force_workers = value;
+            const int rc = schedule(plan);
+            if (rc != SSM_OK) return rc;
+            return cudaMemcpy(plan->ws + offsetof(ssm::WsHeader, inject), &inject, sizeof(inject),
+                              cudaMemcpyHostToDevice) == cudaSuccess
+                       ? SSM_OK
+                       : SSM_ERR_CUDA;
+        }
+        default:
+            return SSM_ERR_INVALID_ARG;
+    }
 }
 
 int ssm_selective_scan_fwd_h0(ssm_plan_t plan, const void* u, const void* delta, const float* A, const void* B,
@@ -234,8 +425,8 @@ int ssm_scan_destroy(ssm_plan_t plan) {
     if (!plan_ok(plan)) return SSM_ERR_INVALID_ARG;
     set_device(plan->device);
     cudaDeviceSynchronize();
-    cudaFree(plan->d_status);
-    for (int i = 0; i < 11; ++i)
+    if (plan->ws) cudaFree(plan->ws);
+    for (int i = 0; i < 10; ++i)
         if (plan->h_bufs[i]) cudaFree(plan->h_bufs[i]);
     plan->magic = kDead;
     delete plan;
@@ -246,26 +437,40 @@ int ssm_scan_device_status(ssm_plan_t plan, ssm_stream_t stream) {
     if (!plan_ok(plan)) return SSM_ERR_INVALID_ARG;
     if (set_device(plan->device) != SSM_OK) return SSM_ERR_CUDA;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    int h = 0;
-    if (cudaMemcpyAsync(&h, plan->d_status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return SSM_ERR_CUDA;
+    ssm::WsHeader h;
+    if (cudaMemcpyAsync(&h, plan->ws, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return SSM_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return SSM_ERR_CUDA;
-    if (cudaMemsetAsync(plan->d_status, 0, sizeof(int), s) != cudaSuccess) return SSM_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return SSM_ERR_CUDA;
-    return h;
+    if (h.status != SSM_OK || h.ticket != 0 || h.done != 0) {
+        // clear the status and put the scheduler back into its initial state (the test hook stays)
+        const unsigned inject = h.inject;
+        if (cudaMemsetAsync(plan->ws, 0, plan->carry_off, s) != cudaSuccess) return SSM_ERR_CUDA;
+        if (cudaMemcpyAsync(plan->ws + offsetof(ssm::WsHeader, inject), &inject, sizeof(inject),
+                            cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return SSM_ERR_CUDA;
+    }
+    return h.status;
 }
 
 int ssm_scan_plan_info(ssm_plan_t plan, int* grid, int* block, int* smem_bytes, int* launches_per_call,
                        const char** variant) {
     if (!plan_ok(plan)) return SSM_ERR_INVALID_ARG;
-    const ssm_dims_t& d = plan->dims;
-    ssm::Variant v;
-    if (!ssm::pick_variant(d.io_dtype, d.dstate, d.nheads != d.dim, d.seqlen % 16 == 0, &v))
-        return SSM_ERR_UNSUPPORTED;
-    if (grid) *grid = (int)grid_of(d, v.ch_per_cta);
-    if (block) *block = ssm::kThreads;
-    if (smem_bytes) *smem_bytes = v.smem;
-    if (launches_per_call) *launches_per_call = d.batch > 0 ? 1 : 0;
-    if (variant) *variant = v.name;
+    if (grid) *grid = plan->grid;
+    if (block) *block = plan->threads;
+    if (smem_bytes) *smem_bytes = plan->smem;
+    if (launches_per_call) *launches_per_call = plan->dims.batch > 0 ? 1 : 0;
+    if (variant) *variant = plan->name;
+    return SSM_OK;
+}
+
+int ssm_scan_plan_schedule(ssm_plan_t plan, int* consumer_warps, int* seg_len, int* n_tiles, int* n_seg,
+                           int* n_ctas) {
+    if (!plan_ok(plan)) return SSM_ERR_INVALID_ARG;
+    if (consumer_warps) *consumer_warps = plan->w;
+    if (seg_len) *seg_len = plan->seg_len;
+    if (n_tiles) *n_tiles = plan->n_tiles;
+    if (n_seg) *n_seg = plan->n_seg;
+    if (n_ctas) *n_ctas = (int)plan->n_ctas;
     return SSM_OK;
 }
 

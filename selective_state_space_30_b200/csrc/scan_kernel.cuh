@@ -1,42 +1,68 @@
 #pragma once
-// Selective-SSM (S6) forward scan kernel for B200 (sm_100a): the template.
+// Selective-SSM (S6) forward scan kernel for B200 (sm_100a).
 //
-// What it computes is stated in include/ssm_scan.h (the recurrence of the
-// Mamba "architecture-details" page, section "How S6 Works", with
-// A_bar = exp(dt*A) from the "Agent 229: SSM optimization patterns" page,
-// section 7), plus softplus(delta + bias), the D skip, the silu(z) gate and the
-// final state.
+// What it computes is stated in include/ssm_scan.h: the recurrence of the
+// Mamba "architecture-details" page (section "How S6 Works") with
+// A_bar = exp(dt*A) (the "Agent 229: SSM optimization patterns" page, section 7),
+// plus dt = softplus(delta + bias), the D skip, the silu(z) gate and the final state.
 //
-// Kernel design (state-parallel, register-resident recurrence):
-//  * The N states of one channel are split over TPC lanes of a warp (S = N/TPC
-//    states per lane).  The states of a channel never interact except through
-//    y = sum_n C_n h_n, so each lane runs its S recurrences sequentially over t
-//    with no scan across time at all: one ex2 and four FP32 operations per
-//    (t, n) -- the minimum the recurrence needs.  The per-lane partial sums of y
-//    are reduced through shared memory once per block of TB time steps.
-//  * A warp holds 32/TPC channels of one batch row; a CTA holds kWarps warps.
-//    Channels never straddle a CTA's B/C group, so the B/C tile of a time block
-//    is staged once in shared memory (fp32, [t][n]) and read by every channel.
-//  * Per-(channel, t) work -- softplus, dt*u, the gate, the D skip, the
-//    conversions and the 16-byte loads/stores -- is spread over the TPC lanes
-//    of the channel (each lane owns TB/TPC consecutive steps), so it is done once.
-//  * Global loads for block k+1 are issued before the recurrence of block k
-//    (register double buffering), one __syncthreads per block.
-//  * exp runs as ex2.approx with A pre-scaled by log2(e) once per lane.
-//  * Time steps past L (the ragged last block) get dt = 0, i.e. dA = 1 and no
-//    input, so the state is carried unchanged to last_state.
+// Design (B200-first):
+//
+//  * State-parallel, register-resident recurrence.  The N states of a channel
+//    are split over TPC lanes of a warp (S = N/TPC states per lane); each lane
+//    runs its states sequentially over t.  States only meet in
+//    y = sum_n C_n h_n, so there is no scan across time inside a segment: one
+//    ex2 per (t, n) plus four FP32 operations (issued as packed f32x2).
+//  * Warp-specialised persistent CTAs, one per SM: a producer warp and W
+//    consumer warps (two per SM sub-partition when W = 8, since ex2 issues per
+//    sub-partition and a second warp hides the latency of the first).
+//    - The producer takes work units -- (channel tile of W*CW channels, L
+//      segment) -- from a global ticket counter in segment-major order, waits
+//      (bounded) for the previous segment of the tile to publish its state,
+//      loads the unit's parameters and incoming state into shared memory, and
+//      streams each 32-step block of u, delta, z rows and B, C rows into a
+//      STAGES-deep shared-memory ring with cp.async.bulk, completing on an
+//      mbarrier.  It also publishes each finished segment's state (carry
+//      buffer, then a release flag).  All global-memory latency sits in this
+//      warp.
+//    - Consumer warps only compute: wait for a full stage, run the block,
+//      arrive on the stage's empty barrier.  No CTA-wide barrier.
+//  * A unit's predecessor was ticketed earlier by a running producer, so the
+//    chain always progresses; every wait is bounded and records
+//    SSM_ERR_TIMEOUT in the workspace status instead of hanging.
+//  * B and C rows sit in shared memory in transposed row order (state s of
+//    lane group j at row s*TPC + j) with a 16-byte row pad, so the TPC lanes of
+//    a channel read different banks.
+//  * The per-(channel, t) work -- softplus, dt*u, the gate, the D skip -- is
+//    spread over the TPC lanes of the channel (lane j owns steps
+//    [j*TPT, (j+1)*TPT) of the block).  The per-lane partial sums of y are
+//    reduce-scattered with shuffles per window of steps.
+//  * softplus(x) = max(x,0) + log1p(2^(-|x| log2 e)) with one ex2 and a degree-9
+//    polynomial for log1p(e)/e on [0, 1] (fitted here; ~1.6e-7 relative error).
+//  * Steps past L in the ragged last block get dt = 0 (dA = 1, no input) and
+//    zeroed B, C, so the state reaches last_state unchanged.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+
 #include "ssm_scan.h"
 
 namespace ssm {
 
-constexpr int kTB = 32;     // time steps per block
-constexpr int kWarps = 4;   // warps per CTA
-constexpr int kThreads = kWarps * 32;
+constexpr int kTB = 32;      // time steps per block
+constexpr int kStages = 3;   // shared-memory ring depth (2 where 3 do not fit)
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Device workspace owned by the plan (zeroed at plan creation; the last CTA of
+// every launch puts the counters and flags back to zero).
+struct WsHeader {
+    unsigned ticket;  // next unit to hand out
+    unsigned done;    // CTAs that have finished
+    int status;       // kernel-side ssm_status_t (first error wins)
+    unsigned inject;  // test hook: nonzero makes chained waits wait for a flag nobody sets
+};
 
 struct FwdParams {
     const void* u;
@@ -50,10 +76,24 @@ struct FwdParams {
     const float* h0;
     void* out;
     float* last_state;
-    int* status;
-    int64_t batch, dim, seqlen, nheads, ngroups;
+    WsHeader* ws;
+    unsigned* flags;   // [n_tiles]: segments of the tile whose final state is published
+    float* carry;      // [n_tiles][CT][N]
+    int64_t dim, seqlen, nheads, ngroups;
     int softplus;
     int tiles_per_group;
+    int n_tiles;
+    int n_seg;
+    int seg_len;       // multiple of kTB
+    unsigned n_units;
+    unsigned n_ctas;
+    unsigned spin_limit;
+    int delta_rows;    // rows of the delta box: CT (S6 layout) or the heads a tile can touch
+};
+
+// The five 2-D tensor maps (time x rows) the producer loads boxes through.
+struct TensorMaps {
+    CUtensorMap u, delta, z, B, C;
 };
 
 // ----------------------------------------------------------------- helpers
@@ -64,13 +104,62 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// softplus(x) = log(1 + e^x); above 20 it equals x to fp32 precision.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// packed fp32 pairs (sm_100 f32x2 instructions)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// log(1 + e^x) = max(x, 0) + log1p(e), e = 2^(-|x| log2 e) in (0, 1];
+// log1p(e) = e * q(e) with q a degree-9 polynomial fitted to log1p(e)/e on [0, 1].
 __device__ __forceinline__ float softplus_f32(float x) {
-    return x > 20.f ? x : log1pf(expf(x));
+    const float e = ex2_approx(-fabsf(x) * kLog2e);
+    float q = -0.0032440342474728823f;
+    q = fmaf(q, e, 0.019851503893733025f);
+    q = fmaf(q, e, -0.0569596104323864f);
+    q = fmaf(q, e, 0.10603662580251694f);
+    q = fmaf(q, e, -0.15305596590042114f);
+    q = fmaf(q, e, 0.1967594027519226f);
+    q = fmaf(q, e, -0.24954134225845337f);
+    q = fmaf(q, e, 0.3332996368408203f);
+    q = fmaf(q, e, -0.4999990165233612f);
+    q = fmaf(q, e, 1.0f);
+    return fmaxf(x, 0.f) + e * q;
 }
 
 __device__ __forceinline__ float silu_f32(float z) {
-    return __fdividef(z, 1.f + ex2_approx(-z * kLog2e));
+    return z * rcp_approx(1.f + ex2_approx(-z * kLog2e));
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 template <typename T> struct IO;
@@ -81,66 +170,21 @@ template <> struct IO<float> {
 template <> struct IO<__nv_bfloat16> {
     static constexpr int kBytes = 2;
     __device__ static float get(const uint32_t* w, int e) {
-        uint32_t x = w[e >> 1];
+        const uint32_t x = w[e >> 1];
         return __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
     }
 };
 
-// CNT consecutive elements of a row, starting at t, kept as raw 32-bit words.
+// CNT consecutive elements of a row held as raw 32-bit words.
 template <typename T, int CNT>
 struct Chunk {
-    static constexpr int kWords = CNT * IO<T>::kBytes / 4;
+    static constexpr int kWords = (CNT * IO<T>::kBytes + 3) / 4;
     uint32_t w[kWords];
 };
 
-// VEC: the chunk is wholly in or out of range and its start is aligned to its
-// size (up to 16 bytes) -> vector loads of 16 or 8 bytes.
-template <typename T, int CNT, bool VEC>
-__device__ __forceinline__ void load_chunk(Chunk<T, CNT>& c, const T* row, int64_t t, int64_t L) {
-    constexpr int W = Chunk<T, CNT>::kWords;
-    if constexpr (VEC) {
-        static_assert(W % 2 == 0, "vector chunk must be a multiple of 8 bytes");
-        if (t < L) {
-            if constexpr (W % 4 == 0) {
-                const uint4* p = reinterpret_cast<const uint4*>(row + t);
-#pragma unroll
-                for (int q = 0; q < W / 4; ++q) {
-                    const uint4 v = __ldg(p + q);
-                    c.w[4 * q + 0] = v.x; c.w[4 * q + 1] = v.y; c.w[4 * q + 2] = v.z; c.w[4 * q + 3] = v.w;
-                }
-            } else {
-                const uint2* p = reinterpret_cast<const uint2*>(row + t);
-#pragma unroll
-                for (int q = 0; q < W / 2; ++q) {
-                    const uint2 v = __ldg(p + q);
-                    c.w[2 * q + 0] = v.x; c.w[2 * q + 1] = v.y;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int q = 0; q < W; ++q) c.w[q] = 0u;
-        }
-    } else {
-        if constexpr (IO<T>::kBytes == 4) {
-#pragma unroll
-            for (int e = 0; e < CNT; ++e)
-                c.w[e] = (t + e < L) ? __float_as_uint(__ldg(reinterpret_cast<const float*>(row) + t + e)) : 0u;
-        } else {
-            const unsigned short* r = reinterpret_cast<const unsigned short*>(row);
-#pragma unroll
-            for (int q = 0; q < CNT / 2; ++q) {
-                const uint32_t lo = (t + 2 * q < L) ? (uint32_t)__ldg(r + t + 2 * q) : 0u;
-                const uint32_t hi = (t + 2 * q + 1 < L) ? (uint32_t)__ldg(r + t + 2 * q + 1) : 0u;
-                c.w[q] = lo | (hi << 16);
-            }
-        }
-    }
-}
-
-// Store CNT consecutive outputs (rounded to nearest even for bf16).
 template <typename T, int CNT, bool VEC>
 __device__ __forceinline__ void store_chunk(T* row, int64_t t, int64_t L, const float (&v)[CNT]) {
-    constexpr int W = CNT * IO<T>::kBytes / 4;
+    constexpr int W = (CNT * IO<T>::kBytes + 3) / 4;
     uint32_t w[W];
     if constexpr (IO<T>::kBytes == 4) {
 #pragma unroll
@@ -158,9 +202,11 @@ __device__ __forceinline__ void store_chunk(T* row, int64_t t, int64_t L, const 
 #pragma unroll
                 for (int q = 0; q < W / 4; ++q)
                     reinterpret_cast<uint4*>(row + t)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-            } else {
+            } else if constexpr (W % 2 == 0) {
 #pragma unroll
                 for (int q = 0; q < W / 2; ++q) reinterpret_cast<uint2*>(row + t)[q] = make_uint2(w[2 * q], w[2 * q + 1]);
+            } else {
+                reinterpret_cast<uint32_t*>(row + t)[0] = w[0];
             }
         }
     } else {
@@ -172,251 +218,720 @@ __device__ __forceinline__ void store_chunk(T* row, int64_t t, int64_t L, const 
         } else {
             unsigned short* r = reinterpret_cast<unsigned short*>(row);
 #pragma unroll
-            for (int q = 0; q < CNT / 2; ++q) {
-                if (t + 2 * q < L) r[t + 2 * q] = (unsigned short)(w[q] & 0xFFFFu);
-                if (t + 2 * q + 1 < L) r[t + 2 * q + 1] = (unsigned short)(w[q] >> 16);
-            }
+            for (int e = 0; e < CNT; ++e)
+                if (t + e < L) r[t + e] = (unsigned short)(w[e >> 1] >> (16 * (e & 1)));
         }
     }
 }
 
+// Reduce-scatter of a window of WT partial sums over the TPC lanes of a channel
+// group (lane bits below TPC): each step halves the values a lane holds, then
+// any remaining lane bits are summed by butterfly.  On return the lane holds the
+// totals for window positions [off, off + max(1, WT/TPC)).
+template <int WT, int TPC>
+__device__ __forceinline__ void window_reduce(float (&a)[WT], int j, int& off) {
+    off = 0;
+#pragma unroll
+    for (int s = 0; (TPC >> (s + 1)) >= 1; ++s) {
+        const int m = TPC >> (s + 1);
+        if ((WT >> s) >= 2) {
+            const int half = WT >> (s + 1);
+            const bool up = (j & m) != 0;
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float lo = a[i], hi = a[half + i];
+                a[i] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, m);
+            }
+            off += up ? half : 0;
+        } else {
+            a[0] += __shfl_xor_sync(0xffffffffu, a[0], m);
+        }
+    }
+}
+
+// ------------------------------------------------------ barriers and copies
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+// non-blocking probe of a phase
+__device__ __forceinline__ bool mbar_test(uint64_t* b, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// probe that may suspend the thread for a short, hardware-bounded time
+__device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for a phase: false (and SSM_ERR_TIMEOUT recorded) after budget_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, unsigned parity, uint64_t budget_ns, int* status) {
+    if (mbar_try(b, parity)) return true;
+    const uint64_t t0 = now_ns();
+    while (true) {
+        if (mbar_try(b, parity)) return true;
+        if (now_ns() - t0 > budget_ns) {
+            atomicCAS(status, SSM_OK, SSM_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+// A float range src[i0, i0 + cnt) of an array of `total` elements, planned as one
+// bulk copy of its 16-byte aligned superset when that superset stays inside the
+// array (else: element copies).  off = position of i0 in the destination.
+struct RangeCopy {
+    int64_t start;   // first element copied
+    int n;           // elements copied
+    int off;         // i0 - start
+    bool bulk;
+};
+__device__ __forceinline__ RangeCopy plan_range(const float* src, int64_t i0, int cnt, int64_t total) {
+    RangeCopy r;
+    const int64_t s4 = i0 & ~(int64_t)3;
+    const int64_t e4 = (i0 + cnt + 3) & ~(int64_t)3;
+    const bool aligned_base = (reinterpret_cast<uintptr_t>(src) & 15u) == 0;
+    r.bulk = aligned_base && cnt > 0 && e4 <= total;
+    r.start = r.bulk ? s4 : i0;
+    r.n = r.bulk ? (int)(e4 - s4) : cnt;
+    r.off = (int)(i0 - r.start);
+    return r;
+}
+
+// warp-uniform decision taken by lane 0
+__device__ __forceinline__ bool lane0_says(bool v) { return __shfl_sync(0xffffffffu, v ? 1 : 0, 0) != 0; }
+
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // ------------------------------------------------------------ kernel config
 
-template <typename T, int N>
+template <typename T, int N, int W, bool HEAD_A>
 struct Cfg {
-    static constexpr int TPC = (N <= 8) ? 2 : (N == 16 ? 4 : 8);  // lanes per channel
-    static constexpr int S = N / TPC;                               // states per lane
-    static constexpr int CPW = 32 / TPC;                            // channels per warp
-    static constexpr int CH = kWarps * CPW;                         // channels per CTA
-    static constexpr int TPT = kTB / TPC;                           // steps per lane in pro/epilogue
-    static constexpr int VE = 16 / IO<T>::kBytes;                   // elements per 16-byte B/C chunk
-    static constexpr int BC_CHUNKS = 2 * N * (kTB / VE);            // B/C chunks per time block
-    static constexpr int BC_PER_THREAD = (BC_CHUNKS + kThreads - 1) / kThreads;
-    static constexpr int ROW = kTB + 4;                             // padded smem row (floats)
-    // shared memory layout (floats)
-    static constexpr int OFF_BC = 0;                                // [2 buf][2 B/C][kTB][N]
-    static constexpr int SZ_BC = 2 * 2 * kTB * N;
-    static constexpr int OFF_DT = OFF_BC + SZ_BC;                   // [kWarps][CPW][ROW] dt
-    static constexpr int OFF_DTU = OFF_DT + kWarps * CPW * ROW;     // dt*u
-    static constexpr int OFF_DA = OFF_DTU + kWarps * CPW * ROW;     // dA (scalar-A-per-head only)
-    static constexpr int OFF_Y = OFF_DA + kWarps * CPW * ROW;       // [kWarps][CPW*TPC][ROW] partial y
-    static constexpr int SMEM_FLOATS = OFF_Y + kWarps * CPW * TPC * ROW;
-    static constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
-    static_assert(S % 4 == 0, "states per lane must be a multiple of 4");
-    static_assert(TPT % 4 == 0, "steps per lane must be a multiple of 4");
-    // the host takes the vector path only when L % 16 == 0, which keeps every
-    // per-lane chunk wholly inside or outside a row only if chunks are <= 16
-    static_assert(TPT <= 16 && VE <= 16, "chunks longer than 16 elements break the L % 16 rule");
+    static constexpr int ESZ = IO<T>::kBytes;
+    static constexpr int S = (N >= 64) ? N / 8 : 4;       // states per lane
+    static constexpr int TPC = N / S;                      // lanes per channel (2, 4 or 8)
+    static constexpr int GW = 32 / TPC;                    // channels per consumer warp
+    static constexpr int CT = W * GW;                      // channels per tile
+    static constexpr int TPT = kTB / TPC;                  // steps per lane in prologue / epilogue
+    static constexpr int WT = (ESZ == 4 || S >= 16) ? 4 : 8;  // steps per B/C register window
+    static constexpr int RB = kTB * ESZ;                   // bytes of one block row
+    static constexpr int ROW = kTB + 4;                    // per-warp float rows (padded)
+    static constexpr int NA = HEAD_A ? 1 : S;
+    // one ring stage (1024-byte aligned): B box | C box (N rows each, hardware
+    // swizzled) | u box | delta box | z box (CT rows each) | header
+    static constexpr int OFF_BC = 0;
+    static constexpr int OFF_IN = OFF_BC + 2 * N * RB;
+    static constexpr int OFF_HDR = OFF_IN + 3 * CT * RB;
+    static constexpr int STAGE = (OFF_HDR + 64 + 1023) / 1024 * 1024;
+    // unit parameter slot (floats): A, D, bias (each with room for a 16-byte
+    // aligned superset of the needed range) and the incoming state
+    static constexpr int P_A = 0;
+    static constexpr int P_D = P_A + (HEAD_A ? CT : CT * N) + 8;
+    static constexpr int P_BIAS = P_D + CT + 8;
+    static constexpr int P_H = P_BIAS + CT + 8;
+    static constexpr int PSLOT = P_H + CT * N;
+    static constexpr int CSLOT = CT * N;                   // outgoing state slot (floats)
+    // per consumer warp (floats): dt, dt*u, (dA), reduced y
+    static constexpr int W_DT = 0;
+    static constexpr int W_DU = GW * ROW;
+    static constexpr int W_DA = 2 * GW * ROW;
+    static constexpr int W_Y = (HEAD_A ? 3 : 2) * GW * ROW;
+    static constexpr int WARP_F = W_Y + GW * ROW;
+    // shared memory map (bytes)
+    static constexpr int OFF_STAGES = 1024;                // barriers live below
+    static constexpr int REST = 2 * PSLOT * 4 + 2 * CSLOT * 4 + W * WARP_F * 4;
+    static constexpr int STG = OFF_STAGES + kStages * STAGE + REST <= 227 * 1024 ? kStages : 2;
+    static constexpr int OFF_PSLOT = OFF_STAGES + STG * STAGE;
+    static constexpr int OFF_CSLOT = OFF_PSLOT + 2 * PSLOT * 4;
+    static constexpr int OFF_WARP = OFF_CSLOT + 2 * CSLOT * 4;
+    static constexpr int SMEM = OFF_WARP + W * WARP_F * 4;
+    static constexpr int THREADS = 32 * (W + 1);
+    static_assert(S % 2 == 0 && TPC >= 2 && TPC <= 8, "lane split");
+    static_assert(TPT % 4 == 0 && TPT <= 16, "steps per lane must be 4..16");
+    static_assert(STAGE % 16 == 0 && (PSLOT * 4) % 16 == 0 && (WARP_F * 4) % 16 == 0, "16-byte aligned smem");
+    static_assert(2 * kStages + 6 <= 128, "barriers fit below OFF_STAGES");
+    static_assert((N * RB) % 512 == 0, "C box keeps the swizzle phase");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
+
+// Byte offset of element t of row r inside a B or C box, as the tensor-map
+// swizzle lays it out: 16-byte chunks XORed with row bits (64-byte rows: bits 1-2
+// of the row; 128-byte rows: bits 0-2).
+template <int ESZ>
+__device__ __forceinline__ int bc_off(int r, int t) {
+    constexpr int RB = kTB * ESZ;
+    const int byte = t * ESZ;
+    const int swz = RB == 64 ? ((r >> 1) & 3) : (r & 7);
+    return r * RB + ((((byte >> 4) ^ swz) & (RB / 16 - 1)) << 4) + (byte & 15);
+}
+
+// barrier slots
+enum { BAR_FULL = 0, BAR_EMPTY = kStages, BAR_PEMPTY = 2 * kStages, BAR_CFULL = 2 * kStages + 2,
+       BAR_CEMPTY = 2 * kStages + 4 };
+
+// per-block header written by the producer into its ring stage
+struct BlockHdr {
+    int64_t t0, t1;     // first step of the block; end of the unit's range
+    int b, g, ci0;      // batch row, group, first channel-in-group of the tile
+    int tile, seg;
+    int flags;          // kFirst | kLast | kFinalSeg | kEnd
+    int pslot;          // parameter slot of the unit
+    int cseq;           // outgoing-state sequence number (last block of a non-final segment)
+    int oa, od, ob;     // where element 0 of the tile's A, D, bias ranges sit in their slot regions
+    int pad;
+};
+constexpr int kFirst = 1, kLast = 2, kFinalSeg = 4, kEnd = 8;
+static_assert(sizeof(BlockHdr) <= 64, "header fits its slot");
 
 // ------------------------------------------------------------------- kernel
 
-template <typename T, int N, bool HEAD_A, bool VEC>
-__global__ void __launch_bounds__(kThreads)
-scan_fwd_kernel(const FwdParams p) {
-    using C = Cfg<T, N>;
-    constexpr int TPC = C::TPC, S = C::S, CPW = C::CPW, CH = C::CH, TPT = C::TPT, VE = C::VE, ROW = C::ROW;
-    extern __shared__ __align__(16) float smem[];
+template <typename T, int N, int W, bool HEAD_A, bool VEC>
+__global__ void __launch_bounds__(Cfg<T, N, W, HEAD_A>::THREADS, 1)
+scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
+    using Cf = Cfg<T, N, W, HEAD_A>;
+    constexpr int S = Cf::S, TPC = Cf::TPC, GW = Cf::GW, CT = Cf::CT, TPT = Cf::TPT, WT = Cf::WT;
+    constexpr int ROW = Cf::ROW, NA = Cf::NA, ESZ = Cf::ESZ, RB = Cf::RB;
+    constexpr int NST = Cf::STG;  // ring stages
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
 
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int cw = lane / TPC, j = lane % TPC;
-
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t Dm = p.dim, L = p.seqlen, H = p.nheads, G = p.ngroups;
-    const int64_t Dg = Dm / G;
-    const int64_t bg = blockIdx.x / p.tiles_per_group;
-    const int64_t ti = blockIdx.x % p.tiles_per_group;
-    const int64_t b = bg / G, g = bg % G;
-    const int64_t ci = ti * CH + warp * CPW + cw;
-    const bool valid = ci < Dg;
-    const int64_t d = g * Dg + (valid ? ci : 0);
-    const int64_t hd = d / (Dm / H);
+    const int64_t Dg = Dm / G, P = Dm / H;
+    int* status = &p.ws->status;
+    const uint64_t budget = (uint64_t)p.spin_limit * 256ull;  // ns
 
-    const T* u_row = reinterpret_cast<const T*>(p.u) + (b * Dm + d) * L;
-    const T* z_row = p.z ? reinterpret_cast<const T*>(p.z) + (b * Dm + d) * L : nullptr;
-    const T* dl_row = reinterpret_cast<const T*>(p.delta) + (b * H + hd) * L;
-    T* out_row = reinterpret_cast<T*>(p.out) + (b * Dm + d) * L;
-    const T* Bbase = reinterpret_cast<const T*>(p.B) + (b * G + g) * (int64_t)N * L;
-    const T* Cbase = reinterpret_cast<const T*>(p.C) + (b * G + g) * (int64_t)N * L;
-
-    // per-lane constants
-    float a2[HEAD_A ? 1 : S];
-    if constexpr (HEAD_A) {
-        a2[0] = __ldg(p.A + hd) * kLog2e;
-    } else {
-#pragma unroll
-        for (int s = 0; s < S; ++s) a2[s] = __ldg(p.A + d * N + j * S + s) * kLog2e;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(bars + BAR_FULL + s, 1);
+            mbar_init(bars + BAR_EMPTY + s, W);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bars + BAR_PEMPTY + s, W);
+            mbar_init(bars + BAR_CFULL + s, W);
+            mbar_init(bars + BAR_CEMPTY + s, 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    const float Dd = p.D ? __ldg(p.D + d) : 0.f;
-    const float bias = p.bias ? __ldg(p.bias + hd) : 0.f;
-    float h[S];
-#pragma unroll
-    for (int s = 0; s < S; ++s) h[s] = p.h0 ? p.h0[(b * Dm + d) * N + j * S + s] : 0.f;
+    __syncthreads();
 
-    float* sBC = smem + C::OFF_BC;
-    float* sdt = smem + C::OFF_DT + (warp * CPW + cw) * ROW;
-    float* sdtu = smem + C::OFF_DTU + (warp * CPW + cw) * ROW;
-    float* sdA = smem + C::OFF_DA + (warp * CPW + cw) * ROW;
-    float* sy_w = smem + C::OFF_Y + warp * CPW * TPC * ROW;
+    if (warp == W) {
+        // ============================================================ producer
+        unsigned fill = 0;          // blocks produced
+        unsigned ucount = 0;        // units started
+        unsigned pub_head = 0, pub_tail = 0;
+        int pub_tile[2] = {0, 0}, pub_seg[2] = {0, 0};
+        bool alive = true;
 
-    // register prefetch buffers
-    Chunk<T, TPT> pu, pdl, pz;
-    Chunk<T, VE> pbc[C::BC_PER_THREAD];
-
-    auto issue_loads = [&](int64_t t0) {
-        const int64_t tl = t0 + j * TPT;
-        if (valid) {
-            load_chunk<T, TPT, VEC>(pu, u_row, tl, L);
-            load_chunk<T, TPT, VEC>(pdl, dl_row, tl, L);
-            if (z_row) load_chunk<T, TPT, VEC>(pz, z_row, tl, L);
-        }
-#pragma unroll
-        for (int k = 0; k < C::BC_PER_THREAD; ++k) {
-            const int c = tid + k * kThreads;
-            if (c < C::BC_CHUNKS) {
-                const int tc = c % (kTB / VE);
-                const int n = (c / (kTB / VE)) % N;
-                const int which = c / (N * (kTB / VE));
-                const T* row = (which ? Cbase : Bbase) + (int64_t)n * L;
-                load_chunk<T, VE, VEC>(pbc[k], row, t0 + tc * VE, L);
-            }
-        }
-    };
-
-    const int64_t nblk = (L + kTB - 1) / kTB;
-    if (nblk > 0) issue_loads(0);
-
-    for (int64_t k = 0; k < nblk; ++k) {
-        const int64_t t0 = k * kTB;
-        const int buf = (int)(k & 1);
-        // -- prologue: dt, dt*u (and dA) for this lane's TPT steps
-        float ucur[TPT], zcur[TPT];
-#pragma unroll
-        for (int i = 0; i < TPT; ++i) {
-            const bool in = valid && (t0 + j * TPT + i < L);
-            const float uv = in ? IO<T>::get(pu.w, i) : 0.f;
-            const float x = (in ? IO<T>::get(pdl.w, i) : 0.f) + bias;
-            float dt = p.softplus ? softplus_f32(x) : x;
-            dt = in ? dt : 0.f;
-            ucur[i] = uv;
-            zcur[i] = (in && z_row) ? IO<T>::get(pz.w, i) : 0.f;
-            sdt[j * TPT + i] = dt;
-            sdtu[j * TPT + i] = dt * uv;
-            if constexpr (HEAD_A) sdA[j * TPT + i] = ex2_approx(dt * a2[0]);
-        }
-        // -- stage the B/C tile (fp32, [t][n]) into buffer `buf`
-        float* sB = sBC + buf * 2 * kTB * N;
-#pragma unroll
-        for (int q = 0; q < C::BC_PER_THREAD; ++q) {
-            const int c = tid + q * kThreads;
-            if (c < C::BC_CHUNKS) {
-                const int tc = c % (kTB / VE);
-                const int n = (c / (kTB / VE)) % N;
-                const int which = c / (N * (kTB / VE));
-                float* dst = sB + which * kTB * N;
-#pragma unroll
-                for (int e = 0; e < VE; ++e) dst[(tc * VE + e) * N + n] = IO<T>::get(pbc[q].w, e);
-            }
-        }
-        __syncthreads();
-        if (k + 1 < nblk) issue_loads(t0 + kTB);
-
-        // -- the recurrence over this block
-        const float* sBt = sB;
-        const float* sCt = sB + kTB * N;
-        float yp[kTB];
-#pragma unroll
-        for (int tq = 0; tq < kTB; tq += 4) {
-            const float4 dt4 = *reinterpret_cast<const float4*>(sdt + tq);
-            const float4 du4 = *reinterpret_cast<const float4*>(sdtu + tq);
-            float4 da4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if constexpr (HEAD_A) da4 = *reinterpret_cast<const float4*>(sdA + tq);
-            const float dtv[4] = {dt4.x, dt4.y, dt4.z, dt4.w};
-            const float duv[4] = {du4.x, du4.y, du4.z, du4.w};
-            const float dav[4] = {da4.x, da4.y, da4.z, da4.w};
-#pragma unroll
-            for (int tt = 0; tt < 4; ++tt) {
-                const int t = tq + tt;
-                float Bv[S], Cv[S];
-#pragma unroll
-                for (int s4 = 0; s4 < S; s4 += 4) {
-                    const float4 bb = *reinterpret_cast<const float4*>(sBt + t * N + j * S + s4);
-                    const float4 cc = *reinterpret_cast<const float4*>(sCt + t * N + j * S + s4);
-                    Bv[s4] = bb.x; Bv[s4 + 1] = bb.y; Bv[s4 + 2] = bb.z; Bv[s4 + 3] = bb.w;
-                    Cv[s4] = cc.x; Cv[s4 + 1] = cc.y; Cv[s4 + 2] = cc.z; Cv[s4 + 3] = cc.w;
+        // publish the outgoing state of finished segments (oldest first); every
+        // loop decision below is taken by lane 0 and broadcast, so the warp never diverges
+        auto service = [&](bool block) {
+            while (pub_head < pub_tail) {
+                const int slot = pub_head & 1;
+                const unsigned par = (pub_head >> 1) & 1;
+                bool ready;
+                if (block) ready = lane0_says(lane == 0 ? mbar_wait(bars + BAR_CFULL + slot, par, budget, status) : false);
+                else ready = lane0_says(lane == 0 ? mbar_test(bars + BAR_CFULL + slot, par) : false);
+                if (!ready) {
+                    if (block) alive = false;
+                    return;
                 }
-                float y = 0.f;
-#pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    const float dA = HEAD_A ? dav[tt] : ex2_approx(dtv[tt] * a2[HEAD_A ? 0 : s]);
-                    h[s] = fmaf(dA, h[s], duv[tt] * Bv[s]);
-                    y = fmaf(Cv[s], h[s], y);
+                __syncwarp();  // order the other lanes' reads after lane 0's acquire
+                const float* cs = reinterpret_cast<const float*>(smem + Cf::OFF_CSLOT) + slot * Cf::CSLOT;
+                const int tile = slot ? pub_tile[1] : pub_tile[0];
+                const int seg = slot ? pub_seg[1] : pub_seg[0];
+                float* dst = p.carry + (int64_t)tile * CT * N;
+                for (int i = lane; i < CT * N; i += 32) __stcg(dst + i, cs[i]);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) {
+                    st_release(p.flags + tile, (unsigned)seg + 1u);
+                    mbar_arrive(bars + BAR_CEMPTY + slot);
                 }
-                yp[t] = y;
+                ++pub_head;
             }
-        }
-        // -- reduce the partial sums of y over the channel's TPC lanes
-        float* myrow = sy_w + (cw * TPC + j) * ROW;
-#pragma unroll
-        for (int tq = 0; tq < kTB; tq += 4)
-            *reinterpret_cast<float4*>(myrow + tq) = make_float4(yp[tq], yp[tq + 1], yp[tq + 2], yp[tq + 3]);
-        __syncwarp();
-        float o[TPT];
-#pragma unroll
-        for (int i = 0; i < TPT; ++i) o[i] = Dd * ucur[i];
-#pragma unroll
-        for (int jj = 0; jj < TPC; ++jj) {
-            const float* r = sy_w + (cw * TPC + jj) * ROW + j * TPT;
-#pragma unroll
-            for (int i4 = 0; i4 < TPT; i4 += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(r + i4);
-                o[i4] += v.x; o[i4 + 1] += v.y; o[i4 + 2] += v.z; o[i4 + 3] += v.w;
+        };
+
+        // wait for a free ring stage, publishing finished segments meanwhile
+        auto acquire_stage = [&](unsigned f) -> bool {
+            if (f < NST) return true;
+            uint64_t* e = bars + BAR_EMPTY + f % NST;
+            const unsigned par = ((f / NST) - 1) & 1;
+            const uint64_t t0 = now_ns();
+            while (!lane0_says(lane == 0 ? mbar_test(e, par) : false)) {
+                service(false);
+                if (lane0_says(lane == 0 ? now_ns() - t0 > budget : false)) {
+                    if (lane == 0) atomicCAS(status, SSM_OK, SSM_ERR_TIMEOUT);
+                    return false;
+                }
             }
+            __syncwarp();
+            return true;
+        };
+
+        while (alive) {
+            unsigned tk = 0;
+            if (lane == 0) tk = atomicAdd(&p.ws->ticket, 1u);
+            tk = __shfl_sync(0xffffffffu, tk, 0);
+            if (tk >= p.n_units) break;
+            const int seg = (int)(tk / (unsigned)p.n_tiles);
+            const int tile = (int)(tk % (unsigned)p.n_tiles);
+            const int bg = tile / p.tiles_per_group, ti = tile % p.tiles_per_group;
+            const int64_t b = bg / G, g = bg % G, ci0 = (int64_t)ti * CT;
+            const int64_t t0u = (int64_t)seg * p.seg_len;
+            const int64_t t1u = t0u + p.seg_len < L ? t0u + p.seg_len : L;
+            const int nblk = L > 0 ? (int)((t1u - t0u + kTB - 1) / kTB) : 1;
+            const bool final_seg = seg + 1 >= p.n_seg;
+            const int pslot = ucount & 1;
+
+            // the parameter slot must have been read by the consumers (unit ucount-2)
+            if (ucount >= 2) {
+                const unsigned par = ((ucount >> 1) - 1) & 1;
+                const uint64_t tw = now_ns();
+                while (!lane0_says(lane == 0 ? mbar_test(bars + BAR_PEMPTY + pslot, par) : false)) {
+                    service(false);
+                    if (lane0_says(lane == 0 ? now_ns() - tw > budget : false)) {
+                        if (lane == 0) atomicCAS(status, SSM_OK, SSM_ERR_TIMEOUT);
+                        alive = false;
+                        break;
+                    }
+                }
+                if (!alive) break;
+                __syncwarp();
+            }
+            // the previous segment of the tile must have published its state
+            bool carry_ok = true;
+            if (seg > 0) {
+                const unsigned need = (unsigned)seg + (p.ws->inject ? 0x40000000u : 0u);
+                const uint64_t tw = now_ns();
+                while (true) {
+                    // 0 = ready, 1 = keep waiting, 2 = give up
+                    int verdict = 1;
+                    if (lane == 0) {
+                        if (ld_acquire(p.flags + tile) >= need) verdict = 0;
+                        else if (*reinterpret_cast<volatile int*>(status) != SSM_OK) verdict = 2;
+                        else if (now_ns() - tw > budget) {
+                            atomicCAS(status, SSM_OK, SSM_ERR_TIMEOUT);
+                            verdict = 2;
+                        }
+                    }
+                    verdict = __shfl_sync(0xffffffffu, verdict, 0);
+                    if (verdict == 0) break;
+                    if (verdict == 2) { carry_ok = false; break; }
+                    service(false);
+                    __nanosleep(200);
+                }
+                __syncwarp();
+            }
+            // parameters and incoming state of the unit -> parameter slot, by bulk
+            // copies that complete on the unit's first-block barrier (element copies
+            // only where a range is not 16-byte aligned inside its array)
+            float* ps = reinterpret_cast<float*>(smem + Cf::OFF_PSLOT) + pslot * Cf::PSLOT;
+            const int nvalid_u = (int)(Dg - ci0 < CT ? Dg - ci0 : CT);
+            const int64_t d0 = g * Dg + ci0;
+            const int64_t h_lo = d0 / P, h_hi = (d0 + nvalid_u - 1) / P;
+            const RangeCopy rA = HEAD_A ? plan_range(p.A, h_lo, (int)(h_hi - h_lo + 1), H)
+                                        : plan_range(p.A, d0 * N, nvalid_u * N, Dm * N);
+            const RangeCopy rD = plan_range(p.D, d0, nvalid_u, Dm);
+            const RangeCopy rB = plan_range(p.bias, h_lo, (int)(h_hi - h_lo + 1), H);
+            const float* hsrc = seg == 0 ? (p.h0 ? p.h0 + (b * Dm + d0) * N : nullptr)
+                                         : (carry_ok ? p.carry + (int64_t)tile * CT * N : nullptr);
+            const int hcnt = seg == 0 ? nvalid_u * N : CT * N;
+            const bool hbulk = hsrc && (reinterpret_cast<uintptr_t>(hsrc) & 15u) == 0 && (hcnt % 4) == 0;
+            unsigned ptx = (rA.bulk ? rA.n * 4u : 0u) + (p.D && rD.bulk ? rD.n * 4u : 0u) +
+                           (p.bias && rB.bulk ? rB.n * 4u : 0u) + (hbulk ? hcnt * 4u : 0u);
+            // element copies and zero fills (generic stores, published by the first block's arrive)
+            if (!rA.bulk)
+                for (int i = lane; i < rA.n; i += 32) ps[Cf::P_A + i] = __ldg(p.A + rA.start + i);
+            if (!p.D) for (int i = lane; i < CT; i += 32) ps[Cf::P_D + i] = 0.f;
+            else if (!rD.bulk) for (int i = lane; i < rD.n; i += 32) ps[Cf::P_D + i] = __ldg(p.D + rD.start + i);
+            if (!p.bias) for (int i = lane; i < CT + 8; i += 32) ps[Cf::P_BIAS + i] = 0.f;
+            else if (!rB.bulk) for (int i = lane; i < rB.n; i += 32) ps[Cf::P_BIAS + i] = __ldg(p.bias + rB.start + i);
+            if (!hsrc) for (int i = lane; i < CT * N; i += 32) ps[Cf::P_H + i] = 0.f;
+            else if (!hbulk) for (int i = lane; i < hcnt; i += 32) ps[Cf::P_H + i] = __ldcg(hsrc + i);
+            if (hbulk && seg > 0) asm volatile("fence.proxy.async.global;" ::: "memory");
+            int cseq = 0;
+            if (!final_seg) {
+                // at most two outgoing states in flight: publish the oldest first
+                while (pub_tail - pub_head >= 2 && alive) service(true);
+                cseq = (int)pub_tail;
+                if (pub_tail & 1) { pub_tile[1] = tile; pub_seg[1] = seg; }
+                else { pub_tile[0] = tile; pub_seg[0] = seg; }
+                ++pub_tail;
+            }
+            __syncwarp();
+            // stream the unit's blocks
+            for (int kb = 0; kb < nblk && alive; ++kb, ++fill) {
+                if (!acquire_stage(fill)) { alive = false; break; }
+                const int st = fill % NST;
+                unsigned char* sb = smem + Cf::OFF_STAGES + st * Cf::STAGE;
+                uint64_t* full = bars + BAR_FULL + st;
+                const int64_t t0 = t0u + (int64_t)kb * kTB;
+                const int64_t nv = L - t0 < kTB ? (L - t0 > 0 ? L - t0 : 0) : kTB;  // valid steps in the block
+                int nvalid = (int)(Dg - ci0 < CT ? Dg - ci0 : CT);
+                if (lane == 0) {
+                    BlockHdr* hd = reinterpret_cast<BlockHdr*>(sb + Cf::OFF_HDR);
+                    hd->b = (int)b; hd->g = (int)g; hd->ci0 = (int)ci0; hd->t0 = t0; hd->t1 = t1u;
+                    hd->tile = tile; hd->seg = seg;
+                    hd->flags = (kb == 0 ? kFirst : 0) | (kb == nblk - 1 ? kLast : 0) | (final_seg ? kFinalSeg : 0);
+                    hd->pslot = pslot; hd->cseq = cseq;
+                    hd->oa = rA.off; hd->od = rD.off; hd->ob = rB.off;
+                }
+                const unsigned extra_tx = kb == 0 ? ptx : 0u;
+                // the unit's parameter bulk copies ride on its first block's barrier
+                auto issue_params = [&]() {
+                    if (kb != 0 || lane != 0) return;
+                    if (rA.bulk) bulk_g2s(ps + Cf::P_A, p.A + rA.start, rA.n * 4u, full);
+                    if (p.D && rD.bulk) bulk_g2s(ps + Cf::P_D, p.D + rD.start, rD.n * 4u, full);
+                    if (p.bias && rB.bulk) bulk_g2s(ps + Cf::P_BIAS, p.bias + rB.start, rB.n * 4u, full);
+                    if (hbulk) bulk_g2s(ps + Cf::P_H, hsrc, hcnt * 4u, full);
+                };
+                const int ntens = p.z ? 3 : 2;
+                const int64_t d0b = g * Dg + ci0;          // first channel of the tile
+                const int64_t hrow0 = HEAD_A ? d0b / P : d0b;  // first delta row of the tile
+                if (VEC) {
+                    // five 2-D boxes; the tensor maps zero-fill whatever lies past L or past the last row
+                    const unsigned bytes = (unsigned)RB * (unsigned)(2 * N + CT + p.delta_rows + (ntens == 3 ? CT : 0));
+                    if (lane == 0) {
+                        mbar_arrive_tx(full, bytes + extra_tx);
+                        const int x = (int)t0;
+                        tma_2d(sb + Cf::OFF_BC, &tm.B, x, (int)((b * G + g) * N), full);
+                        tma_2d(sb + Cf::OFF_BC + N * RB, &tm.C, x, (int)((b * G + g) * N), full);
+                        tma_2d(sb + Cf::OFF_IN, &tm.u, x, (int)(b * Dm + d0b), full);
+                        tma_2d(sb + Cf::OFF_IN + CT * RB, &tm.delta, x, (int)(b * H + hrow0), full);
+                        if (ntens == 3) tma_2d(sb + Cf::OFF_IN + 2 * CT * RB, &tm.z, x, (int)(b * Dm + d0b), full);
+                    }
+                    __syncwarp();
+                    issue_params();
+                } else {
+                    // guarded element copies into the same layout (unaligned rows, ragged tails)
+                    const T* Bb = reinterpret_cast<const T*>(p.B) + (b * G + g) * (int64_t)N * L;
+                    const T* Cb = reinterpret_cast<const T*>(p.C) + (b * G + g) * (int64_t)N * L;
+                    for (int e = lane; e < 2 * N * kTB; e += 32) {
+                        const int r = e / kTB, tt = e % kTB;
+                        const int w = r / N, n = r % N;
+                        const T* src = (w ? Cb : Bb) + (int64_t)n * L;
+                        *reinterpret_cast<T*>(sb + Cf::OFF_BC + w * N * RB + bc_off<ESZ>(n, tt)) =
+                            tt < nv ? src[t0 + tt] : T(0.f);
+                    }
+                    for (int e = lane; e < ntens * CT * kTB; e += 32) {
+                        const int r = e / kTB, tt = e % kTB;
+                        const int w = r / CT, lcr = r % CT;
+                        const T* src = nullptr;
+                        if (w == 1) {
+                            const int64_t hr = hrow0 + lcr;
+                            if (lcr < p.delta_rows && hr < H) src = reinterpret_cast<const T*>(p.delta) + (b * H + hr) * L;
+                        } else if (lcr < nvalid) {
+                            src = reinterpret_cast<const T*>(w == 0 ? p.u : p.z) + (b * Dm + d0b + lcr) * L;
+                        }
+                        *reinterpret_cast<T*>(sb + Cf::OFF_IN + (w * CT + lcr) * RB + tt * ESZ) =
+                            (src && tt < nv) ? src[t0 + tt] : T(0.f);
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (extra_tx) mbar_arrive_tx(full, extra_tx);
+                        else mbar_arrive(full);
+                    }
+                    __syncwarp();
+                    issue_params();
+                }
+                service(false);
+            }
+            ++ucount;
         }
-        if (z_row) {
-#pragma unroll
-            for (int i = 0; i < TPT; ++i) o[i] *= silu_f32(zcur[i]);
+        // end-of-work marker for the consumers
+        if (acquire_stage(fill)) {
+            const int st = fill % NST;
+            if (lane == 0) {
+                reinterpret_cast<BlockHdr*>(smem + Cf::OFF_STAGES + st * Cf::STAGE + Cf::OFF_HDR)->flags = kEnd;
+                mbar_arrive(bars + BAR_FULL + st);
+            }
+            ++fill;
         }
-        if (valid) store_chunk<T, TPT, VEC>(out_row, t0 + j * TPT, L, o);
-        __syncwarp();
+        while (pub_head < pub_tail && alive) service(true);
+        // the last CTA to finish resets the counters and flags for the next launch
+        unsigned last = 0;
+        if (lane == 0) {
+            __threadfence();
+            last = atomicAdd(&p.ws->done, 1u) == p.n_ctas - 1u;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+            __threadfence();
+            for (int i = lane; i < p.n_tiles; i += 32) p.flags[i] = 0u;
+            if (lane == 0) {
+                p.ws->ticket = 0u;
+                p.ws->done = 0u;
+            }
+            __threadfence();
+        }
+        return;
     }
 
-    if (valid && p.last_state) {
-        float* ls = p.last_state + (b * Dm + d) * N + j * S;
+    // ================================================================ consumers
+    const int cg = lane / TPC, j = lane % TPC;
+    const int lc = warp * GW + cg;   // channel of the lane within the tile
+    float* wf = reinterpret_cast<float*>(smem + Cf::OFF_WARP) + warp * Cf::WARP_F;
+    float* rdt = wf + Cf::W_DT + cg * ROW;
+    float* rdu = wf + Cf::W_DU + cg * ROW;
+    float* rda = wf + Cf::W_DA + cg * ROW;
+    float* ry = wf + Cf::W_Y + cg * ROW;
+
+    float a2[NA], h[S];
+    float Dd = 0.f, bias = 0.f;
 #pragma unroll
-        for (int s = 0; s < S; ++s) ls[s] = h[s];
+    for (int s = 0; s < NA; ++s) a2[s] = 0.f;
+#pragma unroll
+    for (int s = 0; s < S; ++s) h[s] = 0.f;
+
+    for (unsigned c = 0;; ++c) {
+        const int st = c % NST;
+        unsigned char* sb = smem + Cf::OFF_STAGES + st * Cf::STAGE;
+        if (!__all_sync(0xffffffffu, mbar_wait(bars + BAR_FULL + st, (c / NST) & 1, budget, status))) break;
+        const BlockHdr hd = *reinterpret_cast<const BlockHdr*>(sb + Cf::OFF_HDR);
+        if (hd.flags & kEnd) break;
+        const int64_t ci = hd.ci0 + lc;
+        const bool ok = ci < Dg;
+        const int64_t d = hd.g * Dg + (ok ? ci : 0);
+        const int64_t t0 = hd.t0;
+        if (hd.flags & kFirst) {
+            const float* ps = reinterpret_cast<const float*>(smem + Cf::OFF_PSLOT) + hd.pslot * Cf::PSLOT;
+            const int64_t h_lo = (hd.g * Dg + hd.ci0) / P;
+            const int hrel = ok ? (int)(d / P - h_lo) : 0;
+            if constexpr (HEAD_A) {
+                a2[0] = ps[Cf::P_A + hd.oa + hrel] * kLog2e;
+            } else {
+#pragma unroll
+                for (int s = 0; s < S; ++s) a2[s] = ps[Cf::P_A + hd.oa + lc * N + s * TPC + j] * kLog2e;
+            }
+            Dd = ps[Cf::P_D + hd.od + lc];
+            bias = ps[Cf::P_BIAS + hd.ob + hrel];
+#pragma unroll
+            for (int s = 0; s < S; ++s) h[s] = ps[Cf::P_H + lc * N + s * TPC + j];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars + BAR_PEMPTY + hd.pslot);
+        }
+        const unsigned char* urow = sb + Cf::OFF_IN + lc * RB + j * TPT * ESZ;
+        const int64_t drow_i = HEAD_A ? (d / P - (hd.g * Dg + hd.ci0) / P) : lc;
+        const unsigned char* drow = sb + Cf::OFF_IN + (CT + drow_i) * RB + j * TPT * ESZ;
+        const unsigned char* zrow = sb + Cf::OFF_IN + (2 * CT + lc) * RB + j * TPT * ESZ;
+        // -------- prologue: dt, dt*u (dA) of this lane's steps
+        {
+            Chunk<T, TPT> cu, cd;
+#pragma unroll
+            for (int q = 0; q < Chunk<T, TPT>::kWords; ++q) {
+                cu.w[q] = reinterpret_cast<const uint32_t*>(urow)[q];
+                cd.w[q] = reinterpret_cast<const uint32_t*>(drow)[q];
+            }
+            float vdt[TPT], vdu[TPT];
+#pragma unroll
+            for (int i = 0; i < TPT; ++i) {
+                const bool in = t0 + j * TPT + i < hd.t1;
+                const float x = IO<T>::get(cd.w, i) + bias;
+                float dt = p.softplus ? softplus_f32(x) : x;
+                dt = in ? dt : 0.f;
+                vdt[i] = dt;
+                vdu[i] = in ? dt * IO<T>::get(cu.w, i) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < TPT; i += 4) {
+                *reinterpret_cast<float4*>(rdt + j * TPT + i) = make_float4(vdt[i], vdt[i + 1], vdt[i + 2], vdt[i + 3]);
+                *reinterpret_cast<float4*>(rdu + j * TPT + i) = make_float4(vdu[i], vdu[i + 1], vdu[i + 2], vdu[i + 3]);
+            }
+            if constexpr (HEAD_A) {
+#pragma unroll
+                for (int i = 0; i < TPT; i += 4)
+                    *reinterpret_cast<float4*>(rda + j * TPT + i) =
+                        make_float4(ex2_approx(vdt[i] * a2[0]), ex2_approx(vdt[i + 1] * a2[0]),
+                                    ex2_approx(vdt[i + 2] * a2[0]), ex2_approx(vdt[i + 3] * a2[0]));
+            }
+        }
+        __syncwarp();
+        // -------- the recurrence, one window of WT steps at a time
+        const unsigned char* bcb = sb + Cf::OFF_BC;
+#pragma unroll 1
+        for (int tw = 0; tw < kTB; tw += WT) {
+            uint32_t bw[S][WT * ESZ / 4], cw_[S][WT * ESZ / 4];
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                const unsigned char* rb = bcb + bc_off<ESZ>(s * TPC + j, tw);
+                const unsigned char* rc = bcb + N * RB + bc_off<ESZ>(s * TPC + j, tw);
+                if constexpr (WT * ESZ == 16) {
+                    const uint4 vb = *reinterpret_cast<const uint4*>(rb);
+                    const uint4 vc = *reinterpret_cast<const uint4*>(rc);
+                    bw[s][0] = vb.x; bw[s][1] = vb.y; bw[s][2] = vb.z; bw[s][3] = vb.w;
+                    cw_[s][0] = vc.x; cw_[s][1] = vc.y; cw_[s][2] = vc.z; cw_[s][3] = vc.w;
+                } else {
+                    const uint2 vb = *reinterpret_cast<const uint2*>(rb);
+                    const uint2 vc = *reinterpret_cast<const uint2*>(rc);
+                    bw[s][0] = vb.x; bw[s][1] = vb.y;
+                    cw_[s][0] = vc.x; cw_[s][1] = vc.y;
+                }
+            }
+            float dtv[WT], duv[WT], dav[HEAD_A ? WT : 1];
+#pragma unroll
+            for (int q = 0; q < WT; q += 4) {
+                const float4 a = *reinterpret_cast<const float4*>(rdt + tw + q);
+                const float4 bq = *reinterpret_cast<const float4*>(rdu + tw + q);
+                dtv[q] = a.x; dtv[q + 1] = a.y; dtv[q + 2] = a.z; dtv[q + 3] = a.w;
+                duv[q] = bq.x; duv[q + 1] = bq.y; duv[q + 2] = bq.z; duv[q + 3] = bq.w;
+                if constexpr (HEAD_A) {
+                    const float4 cq = *reinterpret_cast<const float4*>(rda + tw + q);
+                    dav[q] = cq.x; dav[q + 1] = cq.y; dav[q + 2] = cq.z; dav[q + 3] = cq.w;
+                }
+            }
+            float yw[WT];
+#pragma unroll
+            for (int tt = 0; tt < WT; ++tt) {
+                const float2 dt2 = make_float2(dtv[tt], dtv[tt]);
+                const float2 du2 = make_float2(duv[tt], duv[tt]);
+                float2 y2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int s = 0; s < S; s += 2) {
+                    float2 dA;
+                    if constexpr (HEAD_A) {
+                        dA = make_float2(dav[tt], dav[tt]);
+                    } else {
+                        const float2 arg = mul2(dt2, make_float2(a2[s], a2[s + 1]));
+                        dA = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+                    }
+                    const float2 bb = make_float2(IO<T>::get(bw[s], tt), IO<T>::get(bw[s + 1], tt));
+                    const float2 cc = make_float2(IO<T>::get(cw_[s], tt), IO<T>::get(cw_[s + 1], tt));
+                    const float2 hh = fma2(dA, make_float2(h[s], h[s + 1]), mul2(du2, bb));
+                    h[s] = hh.x;
+                    h[s + 1] = hh.y;
+                    y2 = fma2(cc, hh, y2);
+                }
+                yw[tt] = y2.x + y2.y;
+            }
+            int off;
+            window_reduce<WT, TPC>(yw, j, off);
+            if (j % (TPC > WT ? TPC / WT : 1) == 0) {
+#pragma unroll
+                for (int i = 0; i < (WT >= TPC ? WT / TPC : 1); ++i) ry[tw + off + i] = yw[i];
+            }
+        }
+        // -------- end of a unit: the state goes to the outgoing slot (or last_state)
+        if (hd.flags & kLast) {
+            if (!(hd.flags & kFinalSeg)) {
+                const int slot = hd.cseq & 1;
+                if (hd.cseq >= 2)
+                    __all_sync(0xffffffffu, mbar_wait(bars + BAR_CEMPTY + slot, ((hd.cseq >> 1) - 1) & 1, budget, status));
+                float* cs = reinterpret_cast<float*>(smem + Cf::OFF_CSLOT) + slot * Cf::CSLOT;
+#pragma unroll
+                for (int s = 0; s < S; ++s) cs[lc * N + s * TPC + j] = h[s];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + BAR_CFULL + slot);
+            } else if (ok && p.last_state) {
+#pragma unroll
+                for (int s = 0; s < S; ++s) p.last_state[((int64_t)hd.b * Dm + d) * N + s * TPC + j] = h[s];
+            }
+        }
+        __syncwarp();
+        // -------- epilogue: (y + D u) * silu(z) for the lane's own steps
+        {
+            Chunk<T, TPT> cu, cz;
+#pragma unroll
+            for (int q = 0; q < Chunk<T, TPT>::kWords; ++q) {
+                cu.w[q] = reinterpret_cast<const uint32_t*>(urow)[q];
+                cz.w[q] = reinterpret_cast<const uint32_t*>(zrow)[q];
+            }
+            float o[TPT];
+#pragma unroll
+            for (int i = 0; i < TPT; i += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(ry + j * TPT + i);
+                o[i] = v.x; o[i + 1] = v.y; o[i + 2] = v.z; o[i + 3] = v.w;
+            }
+#pragma unroll
+            for (int i = 0; i < TPT; ++i) {
+                float v = fmaf(Dd, IO<T>::get(cu.w, i), o[i]);
+                if (p.z) v *= silu_f32(IO<T>::get(cz.w, i));
+                o[i] = v;
+            }
+            const int64_t tl = t0 + j * TPT;
+            if (ok && tl < hd.t1) {
+                T* orow = reinterpret_cast<T*>(p.out) + (hd.b * Dm + d) * L;
+                store_chunk<T, TPT, VEC>(orow, tl, hd.t1, o);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + BAR_EMPTY + st);
     }
 }
 
 // --------------------------------------------------------------- dispatch
 
-using KernelFn = void (*)(const FwdParams);
+using KernelFn = void (*)(const FwdParams, const TensorMaps);
 
 struct Variant {
     KernelFn fn;
     int smem;
-    int ch_per_cta;
+    int threads;
+    int ch_per_tile;   // CT
+    int dstate;
     const char* name;
 };
 
-template <typename T, int N, bool HEAD_A, bool VEC>
+template <typename T, int N, int W, bool HEAD_A, bool VEC>
 Variant make_variant(const char* name) {
-    return Variant{scan_fwd_kernel<T, N, HEAD_A, VEC>, Cfg<T, N>::SMEM_BYTES, Cfg<T, N>::CH, name};
+    using C = Cfg<T, N, W, HEAD_A>;
+    return Variant{scan_fwd_kernel<T, N, W, HEAD_A, VEC>, C::SMEM, C::THREADS, C::CT, N, name};
 }
 
-// One function per (io dtype, N) translation unit; see fwd_*.cu.
-#define SSM_DEFINE_PICK(T, TN, N)                                                                    \
-    bool pick_##TN##_n##N(bool head, bool vec, Variant* v) {                                        \
-        if (head)                                                                                   \
-            *v = vec ? make_variant<T, N, true, true>("sp_" #TN "_n" #N "_head_vec")                \
-                     : make_variant<T, N, true, false>("sp_" #TN "_n" #N "_head");                  \
-        else                                                                                        \
-            *v = vec ? make_variant<T, N, false, true>("sp_" #TN "_n" #N "_vec")                    \
-                     : make_variant<T, N, false, false>("sp_" #TN "_n" #N);                         \
-        return true;                                                                                \
+// One function per (io dtype, N) translation unit; see fwd_*.cu.  w = consumer warps (8 or 4).
+#define SSM_DEFINE_PICK(T, TN, N)                                                                         \
+    bool pick_##TN##_n##N(bool head, bool vec, int w, Variant* v) {                                      \
+        if (w == 8) {                                                                                    \
+            if (head)                                                                                    \
+                *v = vec ? make_variant<T, N, 8, true, true>("ws_" #TN "_n" #N "_w8_head_vec")           \
+                         : make_variant<T, N, 8, true, false>("ws_" #TN "_n" #N "_w8_head");             \
+            else                                                                                         \
+                *v = vec ? make_variant<T, N, 8, false, true>("ws_" #TN "_n" #N "_w8_vec")               \
+                         : make_variant<T, N, 8, false, false>("ws_" #TN "_n" #N "_w8");                 \
+        } else {                                                                                         \
+            if (head)                                                                                    \
+                *v = vec ? make_variant<T, N, 4, true, true>("ws_" #TN "_n" #N "_w4_head_vec")           \
+                         : make_variant<T, N, 4, true, false>("ws_" #TN "_n" #N "_w4_head");             \
+            else                                                                                         \
+                *v = vec ? make_variant<T, N, 4, false, true>("ws_" #TN "_n" #N "_w4_vec")               \
+                         : make_variant<T, N, 4, false, false>("ws_" #TN "_n" #N "_w4");                 \
+        }                                                                                                \
+        return true;                                                                                     \
     }
 
-#define SSM_DECLARE_PICK(TN, N) bool pick_##TN##_n##N(bool head, bool vec, Variant* v);
+#define SSM_DECLARE_PICK(TN, N) bool pick_##TN##_n##N(bool head, bool vec, int w, Variant* v);
 SSM_DECLARE_PICK(bf16, 8)
 SSM_DECLARE_PICK(bf16, 16)
 SSM_DECLARE_PICK(bf16, 32)

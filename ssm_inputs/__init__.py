@@ -248,7 +248,7 @@ def make_inputs(dims: Dims, recipe: Recipe, seed: int = 0,
 
     def normal_rows(name, row_len, rows_total, rows, scale=1.0):
         if rows is None:
-            return _gen_normal(seed, name, 0, rows_total * row_len, dt, scale).reshape(-1, row_len)
+            return _gen_normal(seed, name, 0, rows_total * row_len, dt, scale).reshape(rows_total, row_len)
         return np.stack([_gen_normal(seed, name, r * row_len, row_len, dt, scale) for r in rows]) \
             if len(rows) else np.empty((0, row_len), dtype=np.uint16 if dt == "bf16" else np.float32)
 

@@ -86,8 +86,12 @@ def to_host_f64(t) -> np.ndarray:
     return t.cpu().numpy().astype(np.float64)
 
 
-def run_gpu(dims: si.Dims, inp: dict, h0=None, with_state=True, device="cuda", stream=None):
-    """Run the CUDA path through the C ABI (plan, forward, device status, destroy)."""
+OPTION_CODES = {"spin_limit": 1, "inject_stall": 2, "seg_len": 3, "warps": 4, "ctas": 5}
+
+
+def run_gpu(dims: si.Dims, inp: dict, h0=None, with_state=True, device="cuda", stream=None, opts=None,
+            expect_status=0):
+    """Run the CUDA path through the C ABI (plan, options, forward, device status, destroy)."""
     import torch
     import selective_state_space_30_b200 as ssm
     io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
@@ -99,11 +103,13 @@ def run_gpu(dims: si.Dims, inp: dict, h0=None, with_state=True, device="cuda", s
     h0d = to_device(np.ascontiguousarray(h0, dtype=np.float32), device) if h0 is not None else None
     plan = ssm.ssm_scan_plan(d, torch.device(device).index or 0)
     try:
+        for k, v in (opts or {}).items():
+            ssm.ssm_scan_set_option(plan, OPTION_CODES[k], v)
         ssm.ssm_selective_scan_fwd_h0(plan, dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"],
                                       dev["z"], dev["delta_bias"], bool(inp.get("softplus", True)), d, h0d, out,
                                       last, stream)
         st = ssm.ssm_scan_device_status(plan, stream)
-        assert st == ssm.SSM_OK, f"device status {st}"
+        assert st == expect_status, f"device status {st}, expected {expect_status}"
         torch.cuda.synchronize()
     finally:
         ssm.ssm_scan_destroy(plan)

@@ -133,3 +133,10 @@ def test_workload_params_and_row_mode(name):
             assert np.array_equal(rows["u"][k], full["u"][b, dd])
             assert np.array_equal(rows["z"][k], full["z"][b, dd])
             assert np.array_equal(rows["delta"][k], full["delta"][b, dd // (d.dim // d.H)])
+
+
+def test_empty_shapes():
+    for d in (si.Dims(0, 32, 64, 16), si.Dims(2, 32, 0, 16)):
+        x = si.make_inputs(d, si.Recipe(), 0)
+        assert x["u"].shape == (d.batch, d.dim, d.seqlen)
+        assert x["B"].shape == (d.batch, 1, d.dstate, d.seqlen)

@@ -1,0 +1,102 @@
+"""The chained-carry scheduler on the GPU: results do not depend on the schedule
+(segment length, channels per lane, worker count) and a wait that runs out is
+reported as SSM_ERR_TIMEOUT without hanging the GPU (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssm_inputs as si
+from parity import check_out, check_state, run_gpu, to_host_f64
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    si.Dims(2, 80, 300, 16, dtype="bf16"),            # ragged L, partial channel tile, scalar loads
+    si.Dims(2, 64, 512, 16, dtype="bf16"),            # vector path
+    si.Dims(1, 48, 257, 16, dtype="f32"),
+    si.Dims(2, 64, 384, 128, nheads=4, dtype="bf16"),  # scalar A per head, N = 128
+    si.Dims(2, 32, 224, 64, ngroups=2, dtype="bf16"),
+]
+SCHEDULES = [dict(seg_len=32), dict(seg_len=64, warps=4), dict(seg_len=96, warps=8), dict(seg_len=32, ctas=1),
+             dict(seg_len=64, ctas=3, warps=8), dict(ctas=5), dict(seg_len=160, ctas=7, warps=4)]
+
+
+def _recipe(d):
+    if d.head_mode or d.dstate != 16:
+        return si.Recipe(a_init="neg_uniform_1_16", d_init="normal", delta_init="normal_half")
+    return si.Recipe(d_init="normal", delta_init="normal_half")
+
+
+@pytest.mark.parametrize("dims", SHAPES, ids=lambda d: f"{d.batch}x{d.dim}x{d.seqlen}x{d.dstate}h{d.H}g{d.ngroups}{d.dtype}")
+def test_schedule_invariance(dims):
+    inp = si.make_inputs(dims, _recipe(dims), 11)
+    ref_out, ref_last = run_gpu(dims, inp)
+    ro, rl, rm = oracle.run_inputs(dims, inp)
+    check_out(to_host_f64(ref_out), ro, rm, dims.dtype)
+    check_state(to_host_f64(ref_last), rl)
+    for opts in SCHEDULES:
+        out, last = run_gpu(dims, inp, opts=opts)
+        # segments and blocks are 32-step aligned: the same fp32 operations in the same order
+        assert torch.equal(out, ref_out), f"output differs under schedule {opts}"
+        assert torch.equal(last, ref_last), f"last_state differs under schedule {opts}"
+
+
+def test_schedule_with_initial_state():
+    dims = si.Dims(2, 64, 320, 16, dtype="bf16")
+    inp = si.make_inputs(dims, _recipe(dims), 12)
+    h0 = np.random.default_rng(3).standard_normal((2, 64, 16)).astype(np.float32)
+    ro, rl, rm = oracle.run_inputs(dims, inp, h0=h0)
+    for opts in (None, dict(seg_len=32), dict(seg_len=64, ctas=2)):
+        out, last = run_gpu(dims, inp, h0=h0, opts=opts)
+        check_out(to_host_f64(out), ro, rm, "bf16")
+        check_state(to_host_f64(last), rl)
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    """A chained wait on a flag that nothing sets gives up after the spin limit,
+    records SSM_ERR_TIMEOUT, and the next call on the same context is correct."""
+    import selective_state_space_30_b200 as ssm
+    from parity import to_device
+    dims = si.Dims(2, 64, 256, 16, dtype="bf16")
+    inp = si.make_inputs(dims, _recipe(dims), 13)
+    d = ssm.make_dims(2, 64, 256, 16, 64, 1, ssm.SSM_BF16)
+    t = {k: to_device(inp[k]) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    out = torch.empty_like(t["u"])
+    last = torch.empty(2, 64, 16, device="cuda")
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        ssm.ssm_scan_set_option(plan, ssm.SSM_OPT_SEG_LEN, 64)       # 4 chained segments per tile
+        ssm.ssm_scan_set_option(plan, ssm.SSM_OPT_SPIN_LIMIT, 2000)  # a few ms of polling
+        ssm.ssm_scan_set_option(plan, ssm.SSM_OPT_INJECT_STALL, 1)
+        ssm.ssm_selective_scan_fwd(plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                   t["delta_bias"], True, d, out, last, None)
+        assert ssm.ssm_scan_device_status(plan) == ssm.SSM_ERR_TIMEOUT
+        assert ssm.ssm_scan_device_status(plan) == ssm.SSM_OK          # reading clears it
+        ssm.ssm_scan_set_option(plan, ssm.SSM_OPT_INJECT_STALL, 0)
+        ssm.ssm_selective_scan_fwd(plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                   t["delta_bias"], True, d, out, last, None)
+        assert ssm.ssm_scan_device_status(plan) == ssm.SSM_OK
+        torch.cuda.synchronize()
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    ro, rl, rm = oracle.run_inputs(dims, inp)
+    check_out(to_host_f64(out), ro, rm, "bf16")
+    check_state(to_host_f64(last), rl)
+
+
+def test_option_errors():
+    import selective_state_space_30_b200 as ssm
+    d = ssm.make_dims(1, 32, 64, 16, 32, 1, ssm.SSM_BF16)
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        with pytest.raises(ssm.SsmError):
+            ssm.ssm_scan_set_option(plan, 99, 1)
+        with pytest.raises(ssm.SsmError):
+            ssm.ssm_scan_set_option(plan, ssm.SSM_OPT_CONSUMER_WARPS, 3)
+        with pytest.raises(ssm.SsmError):
+            ssm.ssm_scan_set_option(plan, ssm.SSM_OPT_SPIN_LIMIT, 0)
+        sch = ssm.ssm_scan_plan_schedule(plan)
+        assert sch["n_seg"] >= 1 and sch["seg_len"] % 32 == 0 and sch["consumer_warps"] in (4, 8)
+    finally:
+        ssm.ssm_scan_destroy(plan)

@@ -159,6 +159,28 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value);
 int ssm_scan_plan_schedule(ssm_plan_t plan, int* consumer_warps, int* seg_len, int* n_tiles, int* n_seg,
                            int* n_ctas);
 
+/*
+ * The forward scan without a plan and without any device allocation (no
+ * counterpart in the pages: this is a deployment convenience).  For callers that
+ * cannot call cudaMalloc -- code inside a framework that owns all device memory
+ * through its own pre-reserved pool, or a hot path that must not take an
+ * allocation's latency and failure mode.  Same arguments and layouts as
+ * ssm_selective_scan_fwd, minus the plan; device pointers, current device.
+ *   - Scratch comes from a fixed 8 MiB __device__ array held by every GPU that
+ *     loads the library until exit; a problem whose workspace does not fit
+ *     (about batch * dim * dstate * 4 bytes of carry states) returns
+ *     SSM_ERR_UNSUPPORTED without launching anything.
+ *   - The first call on a device looks up the array's address (once per device);
+ *     make that first call before any stream capture.
+ *   - All calls share the array: each clears its counters on its stream, and
+ *     calls whose kernels overlap on the GPU race and must not be made.
+ *   - Kernel-side conditions (a bounded wait that gave up) are not reported.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                                   const float* D, const void* z, const float* delta_bias, int softplus,
+                                   const ssm_dims_t* dims, void* out, float* last_state, ssm_stream_t stream);
+
 /* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
 int ssm_scan_destroy(ssm_plan_t plan);
 

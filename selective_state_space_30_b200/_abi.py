@@ -25,7 +25,8 @@ SSM_BF16 = 1
 
 # every exported symbol declared in include/ssm_scan.h
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
-           "ssm_selective_scan_fwd_host", "ssm_scan_set_option", "ssm_scan_plan_schedule", "ssm_scan_destroy",
+           "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_scan_set_option",
+           "ssm_scan_plan_schedule", "ssm_scan_destroy",
            "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
 
 SSM_OPT_SPIN_LIMIT = 1
@@ -67,6 +68,7 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_fwd.argtypes = fwd_args + [vp, vp, vp]
     lib.ssm_selective_scan_fwd_h0.argtypes = fwd_args + [vp, vp, vp, vp]
     lib.ssm_selective_scan_fwd_host.argtypes = fwd_args + [vp, vp, vp]
+    lib.ssm_selective_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, dims_p, vp, vp, vp]
     lib.ssm_scan_destroy.argtypes = [vp]
     lib.ssm_scan_device_status.argtypes = [vp, vp]
     lib.ssm_status_string.argtypes = [i32]
@@ -150,6 +152,15 @@ def ssm_selective_scan_fwd_host(plan: int, u, delta, A, B, C, D, z, delta_bias, 
         plan, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
         1 if softplus else 0, ctypes.byref(dims), _ptr(out), _ptr(last_state), _stream(stream))
     return _check(rc, "ssm_selective_scan_fwd_host") if check else rc
+
+
+def ssm_selective_scan_fwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dims: ssm_dims_t,
+                                   out, last_state, stream=None, check: bool = True) -> int:
+    """The forward scan without a plan or any device allocation (see include/ssm_scan.h)."""
+    rc = load_library().ssm_selective_scan_fwd_noalloc(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if softplus else 0, ctypes.byref(dims), _ptr(out), _ptr(last_state), _stream(stream))
+    return _check(rc, "ssm_selective_scan_fwd_noalloc") if check else rc
 
 
 def ssm_scan_destroy(plan: Optional[int]) -> int:

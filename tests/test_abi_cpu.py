@@ -34,7 +34,10 @@ def test_every_declared_symbol_is_exported(lib):
     for n in sorted(names):
         assert hasattr(lib, n), f"{n} declared in include/ but not exported"
     from selective_state_space_30_b200 import _abi
+    import selective_state_space_30_b200 as pkg
     assert names == set(_abi.EXPORTS), "binding and header disagree"
+    for n in names:
+        assert callable(getattr(pkg, n, None)), f"package does not expose {n}"
 
 
 def test_status_strings(lib):

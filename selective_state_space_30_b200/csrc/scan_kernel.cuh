@@ -37,8 +37,8 @@
 //    spread over the TPC lanes of the channel (lane j owns steps
 //    [j*TPT, (j+1)*TPT) of the block).  The per-lane partial sums of y are
 //    reduce-scattered with shuffles per window of steps.
-//  * softplus(x) = max(x,0) + log1p(2^(-|x| log2 e)) with one ex2 and a degree-9
-//    polynomial for log1p(e)/e on [0, 1] (fitted here; ~1.6e-7 relative error).
+//  * softplus(x) = max(x,0) + log1p(2^(-|x| log2 e)) with one ex2 and a degree-7
+//    polynomial for log1p(e)/e on [0, 1] (fitted here; ~3.3e-7 relative error).
 //  * Steps past L in the ragged last block get dt = 0 (dA = 1, no input) and
 //    zeroed B, C, so the state reaches last_state unchanged.
 #include <cuda.h>
@@ -131,25 +131,39 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     return d;
 }
 
-// log(1 + e^x) = max(x, 0) + log1p(e), e = 2^(-|x| log2 e) in (0, 1];
-// log1p(e) = e * q(e) with q a degree-9 polynomial fitted to log1p(e)/e on [0, 1].
-__device__ __forceinline__ float softplus_f32(float x) {
-    const float e = ex2_approx(-fabsf(x) * kLog2e);
-    float q = -0.0032440342474728823f;
-    q = fmaf(q, e, 0.019851503893733025f);
-    q = fmaf(q, e, -0.0569596104323864f);
-    q = fmaf(q, e, 0.10603662580251694f);
-    q = fmaf(q, e, -0.15305596590042114f);
-    q = fmaf(q, e, 0.1967594027519226f);
-    q = fmaf(q, e, -0.24954134225845337f);
-    q = fmaf(q, e, 0.3332996368408203f);
-    q = fmaf(q, e, -0.4999990165233612f);
-    q = fmaf(q, e, 1.0f);
-    return fmaxf(x, 0.f) + e * q;
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
 }
 
-__device__ __forceinline__ float silu_f32(float z) {
-    return z * rcp_approx(1.f + ex2_approx(-z * kLog2e));
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
+
+// softplus on a pair: max(x,0) + e*q(e), e = 2^(-|x| log2 e) in (0, 1], q a degree-7
+// polynomial fitted to log1p(e)/e on [0, 1] (max relative error about 3.3e-7).
+__device__ __forceinline__ float2 softplus2(float2 x) {
+    const float2 a = mul2(make_float2(fabsf(x.x), fabsf(x.y)), dup2(-kLog2e));
+    const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+    float2 q = dup2(-0.008539234288036823f);
+    q = fma2(q, e, dup2(0.044089723378419876f));
+    q = fma2(q, e, dup2(-0.10768184065818787f));
+    q = fma2(q, e, dup2(0.17745250463485718f));
+    q = fma2(q, e, dup2(-0.2449546605348587f));
+    q = fma2(q, e, dup2(0.33275479078292847f));
+    q = fma2(q, e, dup2(-0.4999740421772003f));
+    q = fma2(q, e, dup2(0.9999998211860657f));
+    return fma2(e, q, make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)));
+}
+
+// silu(z) = z / (1 + e^-z) on a pair
+__device__ __forceinline__ float2 silu2(float2 z) {
+    const float2 a = mul2(z, dup2(-kLog2e));
+    const float2 d = add2(make_float2(ex2_approx(a.x), ex2_approx(a.y)), dup2(1.f));
+    return mul2(z, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
 }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -166,12 +180,20 @@ template <typename T> struct IO;
 template <> struct IO<float> {
     static constexpr int kBytes = 4;
     __device__ static float get(const uint32_t* w, int e) { return __uint_as_float(w[e]); }
+    // elements e, e+1 (e even)
+    __device__ static float2 get2(const uint32_t* w, int e) {
+        return make_float2(__uint_as_float(w[e]), __uint_as_float(w[e + 1]));
+    }
 };
 template <> struct IO<__nv_bfloat16> {
     static constexpr int kBytes = 2;
     __device__ static float get(const uint32_t* w, int e) {
         const uint32_t x = w[e >> 1];
         return __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
+    }
+    __device__ static float2 get2(const uint32_t* w, int e) {
+        const uint32_t x = w[e >> 1];
+        return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
     }
 };
 
@@ -237,10 +259,20 @@ __device__ __forceinline__ void window_reduce(float (&a)[WT], int j, int& off) {
         if ((WT >> s) >= 2) {
             const int half = WT >> (s + 1);
             const bool up = (j & m) != 0;
+            float recv[WT / 2 > 0 ? WT / 2 : 1];
 #pragma unroll
-            for (int i = 0; i < half; ++i) {
-                const float lo = a[i], hi = a[half + i];
-                a[i] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, m);
+            for (int i = 0; i < half; ++i) recv[i] = __shfl_xor_sync(0xffffffffu, up ? a[i] : a[half + i], m);
+            if (half % 2 == 0) {
+#pragma unroll
+                for (int i = 0; i < half; i += 2) {
+                    const float2 k2 = up ? make_float2(a[half + i], a[half + i + 1]) : make_float2(a[i], a[i + 1]);
+                    const float2 r2 = add2(k2, make_float2(recv[i], recv[i + 1]));
+                    a[i] = r2.x;
+                    a[i + 1] = r2.y;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < half; ++i) a[i] = (up ? a[half + i] : a[i]) + recv[i];
             }
             off += up ? half : 0;
         } else {
@@ -489,13 +521,17 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             if (f < NST) return true;
             uint64_t* e = bars + BAR_EMPTY + f % NST;
             const unsigned par = ((f / NST) - 1) & 1;
+            // the suspending try_wait keeps the producer off the issue slots it shares
+            // with the consumer warps of its SM sub-partition
+            if (lane0_says(lane == 0 ? mbar_try(e, par) : false)) { __syncwarp(); return true; }
             const uint64_t t0 = now_ns();
-            while (!lane0_says(lane == 0 ? mbar_test(e, par) : false)) {
+            while (!lane0_says(lane == 0 ? mbar_try(e, par) : false)) {
                 service(false);
                 if (lane0_says(lane == 0 ? now_ns() - t0 > budget : false)) {
                     if (lane == 0) atomicCAS(status, SSM_OK, SSM_ERR_TIMEOUT);
                     return false;
                 }
+                __nanosleep(256);
             }
             __syncwarp();
             return true;
@@ -520,8 +556,9 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             if (ucount >= 2) {
                 const unsigned par = ((ucount >> 1) - 1) & 1;
                 const uint64_t tw = now_ns();
-                while (!lane0_says(lane == 0 ? mbar_test(bars + BAR_PEMPTY + pslot, par) : false)) {
+                while (!lane0_says(lane == 0 ? mbar_try(bars + BAR_PEMPTY + pslot, par) : false)) {
                     service(false);
+                    __nanosleep(256);
                     if (lane0_says(lane == 0 ? now_ns() - tw > budget : false)) {
                         if (lane == 0) atomicCAS(status, SSM_OK, SSM_ERR_TIMEOUT);
                         alive = false;
@@ -708,6 +745,19 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
     float* rdu = wf + Cf::W_DU + cg * ROW;
     float* rda = wf + Cf::W_DA + cg * ROW;
     float* ry = wf + Cf::W_Y + cg * ROW;
+    // this lane's states are n = s*TPC + j; byte offsets of their rows' windows in a B/C box
+    constexpr int NWIN = kTB / WT;
+    constexpr bool OFF_TABLE = S * NWIN <= 16;
+    int boff[OFF_TABLE ? S * NWIN : S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        if constexpr (OFF_TABLE) {
+#pragma unroll
+            for (int w = 0; w < NWIN; ++w) boff[s * NWIN + w] = bc_off<ESZ>(s * TPC + j, w * WT);
+        } else {
+            boff[s] = s * TPC + j;
+        }
+    }
 
     float a2[NA], h[S];
     float Dd = 0.f, bias = 0.f;
@@ -747,7 +797,8 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
         const int64_t drow_i = HEAD_A ? (d / P - (hd.g * Dg + hd.ci0) / P) : lc;
         const unsigned char* drow = sb + Cf::OFF_IN + (CT + drow_i) * RB + j * TPT * ESZ;
         const unsigned char* zrow = sb + Cf::OFF_IN + (2 * CT + lc) * RB + j * TPT * ESZ;
-        // -------- prologue: dt, dt*u (dA) of this lane's steps
+        const bool full_blk = t0 + kTB <= hd.t1;
+        // -------- prologue: dt, dt*u (dA) of this lane's steps, two at a time
         {
             Chunk<T, TPT> cu, cd;
 #pragma unroll
@@ -757,13 +808,17 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             }
             float vdt[TPT], vdu[TPT];
 #pragma unroll
-            for (int i = 0; i < TPT; ++i) {
-                const bool in = t0 + j * TPT + i < hd.t1;
-                const float x = IO<T>::get(cd.w, i) + bias;
-                float dt = p.softplus ? softplus_f32(x) : x;
-                dt = in ? dt : 0.f;
-                vdt[i] = dt;
-                vdu[i] = in ? dt * IO<T>::get(cu.w, i) : 0.f;
+            for (int i = 0; i < TPT; i += 2) {
+                const float2 x = add2(IO<T>::get2(cd.w, i), dup2(bias));
+                float2 dt = p.softplus ? softplus2(x) : x;
+                if (!full_blk) {
+                    // steps past the end of the unit: no step (dA = 1, no input); their u is zero-filled
+                    if (t0 + j * TPT + i >= hd.t1) dt.x = 0.f;
+                    if (t0 + j * TPT + i + 1 >= hd.t1) dt.y = 0.f;
+                }
+                const float2 du = mul2(dt, IO<T>::get2(cu.w, i));
+                vdt[i] = dt.x; vdt[i + 1] = dt.y;
+                vdu[i] = du.x; vdu[i + 1] = du.y;
             }
 #pragma unroll
             for (int i = 0; i < TPT; i += 4) {
@@ -779,15 +834,19 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             }
         }
         __syncwarp();
-        // -------- the recurrence, one window of WT steps at a time
+        // -------- the recurrence, one window of WT steps at a time (unrolled)
         const unsigned char* bcb = sb + Cf::OFF_BC;
-#pragma unroll 1
-        for (int tw = 0; tw < kTB; tw += WT) {
+#pragma unroll
+        for (int w = 0; w < NWIN; ++w) {
+            const int tw = w * WT;
             uint32_t bw[S][WT * ESZ / 4], cw_[S][WT * ESZ / 4];
 #pragma unroll
             for (int s = 0; s < S; ++s) {
-                const unsigned char* rb = bcb + bc_off<ESZ>(s * TPC + j, tw);
-                const unsigned char* rc = bcb + N * RB + bc_off<ESZ>(s * TPC + j, tw);
+                int off;
+                if constexpr (OFF_TABLE) off = boff[s * NWIN + w];
+                else off = bc_off<ESZ>(boff[s], tw);
+                const unsigned char* rb = bcb + off;
+                const unsigned char* rc = bcb + N * RB + off;
                 if constexpr (WT * ESZ == 16) {
                     const uint4 vb = *reinterpret_cast<const uint4*>(rb);
                     const uint4 vc = *reinterpret_cast<const uint4*>(rc);
@@ -815,14 +874,14 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             float yw[WT];
 #pragma unroll
             for (int tt = 0; tt < WT; ++tt) {
-                const float2 dt2 = make_float2(dtv[tt], dtv[tt]);
-                const float2 du2 = make_float2(duv[tt], duv[tt]);
+                const float2 dt2 = dup2(dtv[tt]);
+                const float2 du2 = dup2(duv[tt]);
                 float2 y2 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int s = 0; s < S; s += 2) {
                     float2 dA;
                     if constexpr (HEAD_A) {
-                        dA = make_float2(dav[tt], dav[tt]);
+                        dA = dup2(dav[tt]);
                     } else {
                         const float2 arg = mul2(dt2, make_float2(a2[s], a2[s + 1]));
                         dA = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
@@ -860,7 +919,7 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             }
         }
         __syncwarp();
-        // -------- epilogue: (y + D u) * silu(z) for the lane's own steps
+        // -------- epilogue: (y + D u) * silu(z) for the lane's own steps, two at a time
         {
             Chunk<T, TPT> cu, cz;
 #pragma unroll
@@ -875,10 +934,11 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
                 o[i] = v.x; o[i + 1] = v.y; o[i + 2] = v.z; o[i + 3] = v.w;
             }
 #pragma unroll
-            for (int i = 0; i < TPT; ++i) {
-                float v = fmaf(Dd, IO<T>::get(cu.w, i), o[i]);
-                if (p.z) v *= silu_f32(IO<T>::get(cz.w, i));
-                o[i] = v;
+            for (int i = 0; i < TPT; i += 2) {
+                float2 v = fma2(dup2(Dd), IO<T>::get2(cu.w, i), make_float2(o[i], o[i + 1]));
+                if (p.z) v = mul2(v, silu2(IO<T>::get2(cz.w, i)));
+                o[i] = v.x;
+                o[i + 1] = v.y;
             }
             const int64_t tl = t0 + j * TPT;
             if (ok && tl < hd.t1) {

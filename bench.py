@@ -48,6 +48,55 @@ def _rank_env():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+# ------------------------------------------------------------------ ranks
+# One process per GPU (torchrun).  The scan shards only as independent
+# replicas, so the only collectives are the barriers around the timed region
+# and the max over ranks of its length; every rank takes them in the same order.
+
+def init_ranks(backend: str, local: int, timeout_s: float = 120.0) -> int:
+    """Join the process group named by the torchrun environment; returns the world size."""
+    import datetime
+    import torch.distributed as dist
+    _, _, world = _rank_env()
+    if world > 1 and not dist.is_initialized():
+        kw = {}
+        if backend == "nccl":
+            import torch
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+    return world
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (the identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, elems_per_rank_step: int, steps: int, ms: float) -> float:
+    """Whole-job Gelem/s: every rank's elements over the slowest rank's time."""
+    return world * elems_per_rank_step * steps / (ms * 1e-3) / 1e9
+
+
+def finish_ranks():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if dist.get_world_size() > 1:
+            dist.barrier()
+        dist.destroy_process_group()
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -188,21 +237,32 @@ def cpu_oracle_sample(d, recipe, seed, target_s=12.0):
     total = d.batch * d.dim
     rng = np.random.default_rng(7)
 
-    def run(nch):
+    def run(nch, reps=1):
         ch = sorted(int(c) for c in rng.choice(total, size=min(total, nch), replace=False))
         rows = si.make_inputs(d, recipe, seed, channels=ch)
         t0 = time.perf_counter()
-        oracle.run_inputs(d, rows, channels=ch, nthreads=cores)
+        for _ in range(reps):
+            oracle.run_inputs(d, rows, channels=ch, nthreads=cores)
         return time.perf_counter() - t0, len(ch)
 
-    # calibrate on one channel per core, then size the sample to about target_s
-    dt, n = run(min(total, cores))
-    per_ch = dt / max(1, n) * cores
-    nch = int(max(cores, min(total, target_s * cores / max(per_ch, 1e-9))))
-    dt, n = run(nch)
-    elems = n * d.seqlen
+    # grow the sample until it takes about target_s (the whole workload, repeated,
+    # when one pass over it takes less than that)
+    nch, reps = min(total, cores), 1
+    while True:
+        dt, n = run(nch, reps)
+        if dt >= target_s / 3:
+            break
+        grow = target_s / max(dt, 1e-3)
+        if nch < total:
+            nch = int(min(total, nch * min(grow, 64.0)))
+        elif reps < 1000:
+            reps = int(min(1000, reps * min(grow, 64.0)))
+        else:
+            break
+    elems = n * d.seqlen * reps
+    what = f"{n} of {total} channels" if n < total else f"all {total} channels" + (f", {reps} passes" if reps > 1 else "")
     return {"value": elems / dt / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n} of {total} channels x L={d.seqlen} (N={d.dstate}), fp64, {dt:.1f} s"}
+            "sample": f"{what} x L={d.seqlen} (N={d.dstate}), fp64, {dt:.1f} s"}
 
 
 # ------------------------------------------------------------------ arms
@@ -235,16 +295,13 @@ def run_reference(args):
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
     import ssm_inputs as si
     import selective_state_space_30_b200 as ssm
 
     rank, local, world = _rank_env()
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    init_ranks("nccl", local)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = si.WORKLOADS[args.workload]
@@ -276,8 +333,7 @@ def run_ours(args):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    barrier()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(local) as clk:
@@ -287,21 +343,16 @@ def run_ours(args):
             step(i)
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    total_ms = starts[0].elapsed_time(ends[-1])
+    barrier()
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]), dev)
     st = ssm.ssm_scan_device_status(plan, sh)
     if st != ssm.SSM_OK:
         raise RuntimeError(f"device status {ssm.ssm_status_string(st)}")
 
     elems = d.batch * d.dim * d.seqlen
     ms_per_step = total_ms / args.steps
-    value = world * elems * args.steps / (total_ms * 1e-3) / 1e9
+    value = job_throughput(world, elems, args.steps, total_ms)
 
     # roofline of the scan kernel (one launch per step)
     hbm_gbs, sm_max_mhz, peak_src = _peaks()
@@ -346,22 +397,17 @@ def run_ours(args):
         for _ in range(2):
             hstep()
         torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
+        barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(e2e_steps):
             hstep()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
         h2d = sum(hp[k].numel() * hp[k].element_size() for k in names if hp[k] is not None)
         d2h = hout.numel() * hout.element_size() + hlast.numel() * hlast.element_size()
-        e2e = {"value": world * elems * e2e_steps / (ems * 1e-3) / 1e9, "unit": UNIT,
+        e2e = {"value": job_throughput(world, elems, e2e_steps, ems), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
                "path": "ssm_selective_scan_fwd_host (pinned host buffers)"}
 
@@ -370,9 +416,7 @@ def run_ours(args):
         cpu = cpu_oracle_sample(d, w.recipe, w.seed)
 
     ssm.ssm_scan_destroy(plan)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    finish_ranks()
     if rank != 0:
         return
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

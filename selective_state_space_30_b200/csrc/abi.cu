@@ -129,19 +129,9 @@ int schedule(ssm_plan_s* p) {
     const int64_t n_tiles = tiles_for(v.ch_per_tile);
     int64_t ctas = p->sm_count;  // one persistent CTA per SM
     if (p->force_workers > 0 && p->force_workers < ctas) ctas = p->force_workers;
-    // segments: about 16 units per CTA, segments of at least 128 steps
     const int64_t L = d.seqlen;
-    int64_t seg_len;
-    if (p->force_seg_len > 0) {
-        seg_len = (p->force_seg_len + ssm::kTB - 1) / ssm::kTB * ssm::kTB;
-    } else {
-        int64_t n_seg = (16 * ctas + n_tiles - 1) / (n_tiles > 0 ? n_tiles : 1);
-        const int64_t max_seg = (L + 127) / 128;
-        if (n_seg > max_seg) n_seg = max_seg;
-        if (n_seg < 1) n_seg = 1;
-        seg_len = ((L + n_seg - 1) / n_seg + ssm::kTB - 1) / ssm::kTB * ssm::kTB;
-    }
-    if (seg_len < ssm::kTB) seg_len = ssm::kTB;
+    const int64_t seg_len = p->force_seg_len > 0 ? (p->force_seg_len + ssm::kTB - 1) / ssm::kTB * ssm::kTB
+                                                 : ssm::default_seg_len(L, n_tiles, ctas);
     const int64_t n_seg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
     const int64_t n_units = n_tiles * n_seg;
     if (n_units >= (int64_t)1 << 31 || seg_len > (int64_t)1 << 30) return SSM_ERR_UNSUPPORTED;

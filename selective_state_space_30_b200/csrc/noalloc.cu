@@ -158,7 +158,7 @@ extern "C" int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, 
     if (d.batch == 0) return SSM_OK;
 
     // the schedule: the same policy as a plan (eight consumer warps unless that leaves SMs idle,
-    // one persistent CTA per SM, about 16 units per CTA, segments of at least 128 steps)
+    // one persistent CTA per SM, the default segment length)
     const int64_t Dg = d.dim / d.ngroups;
     auto tiles_for = [&](int ct) { return d.batch * d.ngroups * ((Dg + ct - 1) / ct); };
     const int w = tiles_for(v8.ch_per_tile) < sms ? 4 : 8;
@@ -166,13 +166,8 @@ extern "C" int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, 
     const int64_t n_tiles = tiles_for(ct);
     int64_t ctas = sms;
     const int64_t L = d.seqlen;
-    int64_t n_seg = (16 * ctas + n_tiles - 1) / n_tiles;
-    const int64_t max_seg = (L + 127) / 128;
-    if (n_seg > max_seg) n_seg = max_seg;
-    if (n_seg < 1) n_seg = 1;
-    int64_t seg_len = ((L + n_seg - 1) / n_seg + ssm::kTB - 1) / ssm::kTB * ssm::kTB;
-    if (seg_len < ssm::kTB) seg_len = ssm::kTB;
-    n_seg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
+    const int64_t seg_len = ssm::default_seg_len(L, n_tiles, ctas);
+    const int64_t n_seg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
     const int64_t n_units = n_tiles * n_seg;
     if (n_units >= (int64_t)1 << 31) return SSM_ERR_UNSUPPORTED;
     if (ctas > n_units) ctas = n_units;

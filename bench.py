@@ -433,6 +433,93 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ decode step
+
+DECODE_SHAPES = {
+    # one generation step of a Mamba-1.4B layer (d_inner 4096, N 16) for 256 sequences
+    "decode-mamba-1.4b-b256": dict(batch=256, dim=4096, dstate=16, nheads=4096, ngroups=1, dtype="bf16"),
+    # one step of the Mamba-2-style layer (32 heads x 64, N 128) for 64 sequences
+    "decode-mamba2-n128-b64": dict(batch=64, dim=2048, dstate=128, nheads=32, ngroups=1, dtype="bf16"),
+}
+
+
+def _decode_bytes(sh):
+    """Algorithmic HBM bytes of one step: the state read and written, u, delta, z read, out written,
+    B and C read, A, D, bias read."""
+    e = 2 if sh["dtype"] == "bf16" else 4
+    b, d, n, h, g = sh["batch"], sh["dim"], sh["dstate"], sh["nheads"], sh["ngroups"]
+    return (2 * b * d * n * 4 + 3 * b * d * e + b * h * e + 2 * b * g * n * e +
+            (d * n if h == d else h) * 4 + d * 4 + h * 4)
+
+
+def run_decode(args):
+    """ssm_selective_state_update on a decode shape: one JSON line (GB/s against the HBM roofline)."""
+    import torch
+    import ssm_inputs as si
+    import selective_state_space_30_b200 as ssm
+    rank, local, world = _rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+    init_ranks("nccl", local)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sh = DECODE_SHAPES[args.workload]
+    dims = si.Dims(sh["batch"], sh["dim"], 1, sh["dstate"], nheads=sh["nheads"] if sh["nheads"] != sh["dim"] else 0,
+                   ngroups=sh["ngroups"], dtype=sh["dtype"])
+    rec = si.Recipe(a_init="neg_uniform_1_16" if dims.head_mode else "neg_n_plus_1", d_init="normal",
+                    delta_init="normal_half")
+    inp = si.make_inputs(dims, rec, 0)
+    names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+    alg = _decode_bytes(sh)
+    copies = max(2, int(np.ceil(3 * L2_BYTES / alg)))
+    sets = []
+    for i in range(copies):
+        t = {k: _to_dev(inp[k], dev) for k in names}
+        t["state"] = torch.randn(dims.batch, dims.dim, dims.dstate, device=dev, generator=None)
+        t["out"] = torch.empty_like(t["u"])
+        sets.append(t)
+    io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
+    d = ssm.make_dims(dims.batch, dims.dim, 1, dims.dstate, dims.H, dims.ngroups, io)
+    stream = torch.cuda.current_stream(dev)
+    sh_ = stream.cuda_stream
+
+    def step(i):
+        t = sets[i % copies]
+        ssm.ssm_selective_state_update(d, t["state"], t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                       t["delta_bias"], True, t["out"], sh_)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    total = max_over_ranks(e0.elapsed_time(e1), dev)
+    hbm_gbs, _, src = _peaks()
+    finish_ranks()
+    if rank != 0:
+        return
+    gbs = alg / (ms * 1e-3) / 1e9
+    line = {"metric": "selective-state-update (decode step) GB/s on 1 B200", "op": "decode",
+            "value": world * dims.batch * dims.dim * args.steps / (total * 1e-3) / 1e9, "unit": "Gelem/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 (bf16 I/O)" if dims.dtype == "bf16" else "f32", "data": "synthetic (seeded splitmix64)",
+            "config": dict(sh, workload=args.workload,
+                           l2=f"{copies} rotating state/input sets of {alg / 1e6:.0f} MB, no flush"),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                         "traffic": None, "peak_source": src, "alg_bytes_per_launch": alg},
+            "clocks": clk.summary(), "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -442,9 +529,16 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--op", default="scan", choices=["scan", "decode"],
+                    help="scan: the forward scan (the headline metric); decode: the single-step state update")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.op == "decode":
+        if args.workload == DEFAULT_WORKLOAD:
+            args.workload = "decode-mamba-1.4b-b256"
+        run_decode(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

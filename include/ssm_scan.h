@@ -57,7 +57,7 @@ typedef enum {
     SSM_ERR_UNSUPPORTED = 2, /* a shape or dtype no kernel here handles (e.g. dstate not in {8,16,32,64,128}) */
     SSM_ERR_CUDA = 3,        /* a CUDA runtime call failed (allocation, launch, copy) */
     SSM_ERR_TIMEOUT = 4,     /* device side: a bounded inter-CTA wait gave up */
-    SSM_ERR_BOUNDS = 5       /* device side: a debug-build bounds check fired */
+    SSM_ERR_BOUNDS = 5       /* device side: a bounds or alignment check fired */
 } ssm_status_t;
 
 typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
@@ -92,7 +92,9 @@ int ssm_scan_plan(ssm_plan_t* out_plan, const ssm_dims_t* dims, int device);
  * The forward scan (the operation above), asynchronous on `stream`.
  * `dims` must equal the plan's dims.  Pointers are device pointers owned by
  * the caller and are not kept after the call returns; `out` must not alias an
- * input.  softplus != 0 applies softplus to delta + delta_bias.
+ * input.  softplus != 0 applies softplus to delta + delta_bias; with softplus
+ * == 0, delta + delta_bias is dt itself and must be >= 0 (with A <= 0 every
+ * exp(dt*A) is then <= 1; a dt*A above about 88 overflows fp32).
  * Allocates nothing.  One plan must not run on two streams at once.
  * Returns SSM_ERR_INVALID_ARG for a NULL required pointer (u, delta, A, B, C,
  * out) or mismatched dims, SSM_ERR_CUDA if the launch fails.
@@ -128,8 +130,8 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
                                 void* out, float* last_state, ssm_stream_t stream);
 
 /*
- * Plan options (mostly for tests).  Changing SEG_LEN, CONSUMER_WARPS or
- * WORKERS re-plans the schedule (synchronises the device).
+ * Plan options (mostly for tests).  Changing SEG_LEN, CONSUMER_WARPS, WORKERS or
+ * STATES_PER_LANE re-plans the schedule (synchronises the device).
  *   SSM_OPT_SPIN_LIMIT         polls a chained wait makes before it gives up and
  *                              records SSM_ERR_TIMEOUT (default about 2M, i.e. ~1 s)
  *   SSM_OPT_INJECT_STALL       test hook, nonzero: every chained wait waits for a
@@ -138,8 +140,14 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
  *                              0 switches it off
  *   SSM_OPT_SEG_LEN            force the segment length (rounded up to 32 steps);
  *                              0 = automatic
- *   SSM_OPT_CONSUMER_WARPS     force 4 or 8 consumer warps per CTA; 0 = automatic
+ *   SSM_OPT_CONSUMER_WARPS     force 4, 8 or 16 consumer warps per CTA (16 exists for
+ *                              dstate <= 16 with 2 states per lane); 0 = automatic
  *   SSM_OPT_WORKERS            cap the number of persistent CTAs; 0 = one per SM
+ *   SSM_OPT_STATES_PER_LANE    force the states each lane holds (2 or 4 for dstate <= 16,
+ *                              4 for dstate 32, dstate/8 above); 0 = automatic.  A
+ *                              combination with CONSUMER_WARPS that no kernel has makes
+ *                              the call return SSM_ERR_UNSUPPORTED and keeps the
+ *                              previous setting.
  * Returns SSM_ERR_INVALID_ARG for an unknown option or a bad value.
  */
 typedef enum {
@@ -147,7 +155,8 @@ typedef enum {
     SSM_OPT_INJECT_STALL = 2,
     SSM_OPT_SEG_LEN = 3,
     SSM_OPT_CONSUMER_WARPS = 4,
-    SSM_OPT_WORKERS = 5
+    SSM_OPT_WORKERS = 5,
+    SSM_OPT_STATES_PER_LANE = 6
 } ssm_option_t;
 int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value);
 
@@ -180,6 +189,31 @@ int ssm_scan_plan_schedule(ssm_plan_t plan, int* consumer_warps, int* seg_len, i
 int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,
                                    const float* D, const void* z, const float* delta_bias, int softplus,
                                    const ssm_dims_t* dims, void* out, float* last_state, ssm_stream_t stream);
+
+/*
+ * One step of the recurrence with the state kept in device memory: the
+ * inference mode of the Mamba "architecture-details" page ("Parallel
+ * Algorithm": the sequential, RNN-style mode; "Memory Efficiency": a
+ * constant-size state and no cache of past inputs).  For every (b, d):
+ *
+ *     dt = softplus(delta[b,hd] + delta_bias[hd]),   h = state[b,d,:]
+ *     h[n] = exp(dt * A[d,n]) * h[n] + dt * B[b,g,n] * u[b,d]
+ *     out[b,d] = (sum_n C[b,g,n] * h[n] + D[d] * u[b,d]) * silu(z[b,d])
+ *     state[b,d,:] = h                       (overwritten in place)
+ *
+ * This is exactly ssm_selective_scan_fwd_h0 with seqlen 1 and h0 = last_state
+ * = state.  dims->seqlen must be 1: u, z, out are (batch, dim), delta is
+ * (batch, nheads), B and C are (batch, ngroups, dstate), in the io dtype; A, D,
+ * delta_bias and the fp32 state (batch, dim, dstate) are as for the scan.  No
+ * plan and no workspace: the call allocates nothing and launches one kernel on
+ * `stream`.  state must be 16-byte aligned, B and C 8-byte (bf16) or 16-byte
+ * (fp32) aligned, and A 16-byte aligned in the per-channel layout; otherwise
+ * SSM_ERR_UNSUPPORTED.  SSM_ERR_INVALID_ARG for a NULL required pointer (state,
+ * u, delta, A, B, C, out), seqlen != 1 or a bad shape.
+ */
+int ssm_selective_state_update(const ssm_dims_t* dims, float* state, const void* u, const void* delta,
+                               const float* A, const void* B, const void* C, const float* D, const void* z,
+                               const float* delta_bias, int softplus, void* out, ssm_stream_t stream);
 
 /* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
 int ssm_scan_destroy(ssm_plan_t plan);

@@ -25,7 +25,8 @@ SSM_BF16 = 1
 
 # every exported symbol declared in include/ssm_scan.h
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
-           "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_scan_set_option",
+           "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update",
+           "ssm_scan_set_option",
            "ssm_scan_plan_schedule", "ssm_scan_destroy",
            "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
 
@@ -34,6 +35,7 @@ SSM_OPT_INJECT_STALL = 2
 SSM_OPT_SEG_LEN = 3
 SSM_OPT_CONSUMER_WARPS = 4
 SSM_OPT_WORKERS = 5
+SSM_OPT_STATES_PER_LANE = 6
 
 
 class SsmError(RuntimeError):
@@ -69,6 +71,7 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_fwd_h0.argtypes = fwd_args + [vp, vp, vp, vp]
     lib.ssm_selective_scan_fwd_host.argtypes = fwd_args + [vp, vp, vp]
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, dims_p, vp, vp, vp]
+    lib.ssm_selective_state_update.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
     lib.ssm_scan_destroy.argtypes = [vp]
     lib.ssm_scan_device_status.argtypes = [vp, vp]
     lib.ssm_status_string.argtypes = [i32]
@@ -161,6 +164,15 @@ def ssm_selective_scan_fwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
         1 if softplus else 0, ctypes.byref(dims), _ptr(out), _ptr(last_state), _stream(stream))
     return _check(rc, "ssm_selective_scan_fwd_noalloc") if check else rc
+
+
+def ssm_selective_state_update(dims: ssm_dims_t, state, u, delta, A, B, C, D, z, delta_bias, softplus: bool,
+                               out, stream=None, check: bool = True) -> int:
+    """One recurrence step with the state updated in place (see include/ssm_scan.h)."""
+    rc = load_library().ssm_selective_state_update(
+        ctypes.byref(dims), _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), 1 if softplus else 0, _ptr(out), _stream(stream))
+    return _check(rc, "ssm_selective_state_update") if check else rc
 
 
 def ssm_scan_destroy(plan: Optional[int]) -> int:

@@ -8,6 +8,7 @@
 #include <cstring>
 #include <new>
 
+#include "layout.h"
 #include "scan_kernel.cuh"
 #include "ssm_scan.h"
 
@@ -28,18 +29,6 @@ __global__ void __launch_bounds__(256) probe_ex2_kernel(float* sink, int iters) 
     sink[blockIdx.x * 256 + threadIdx.x] = s;
 }
 
-static bool pick_variant(int dtype, int64_t N, bool head, bool vec, int w, Variant* v) {
-    const bool bf = dtype == SSM_BF16;
-    switch (N) {
-        case 8: return bf ? pick_bf16_n8(head, vec, w, v) : pick_f32_n8(head, vec, w, v);
-        case 16: return bf ? pick_bf16_n16(head, vec, w, v) : pick_f32_n16(head, vec, w, v);
-        case 32: return bf ? pick_bf16_n32(head, vec, w, v) : pick_f32_n32(head, vec, w, v);
-        case 64: return bf ? pick_bf16_n64(head, vec, w, v) : pick_f32_n64(head, vec, w, v);
-        case 128: return bf ? pick_bf16_n128(head, vec, w, v) : pick_f32_n128(head, vec, w, v);
-        default: return false;
-    }
-}
-
 }  // namespace ssm
 
 // ------------------------------------------------------------------- plans
@@ -51,6 +40,7 @@ struct ssm_plan_s {
     int sm_count;
     // schedule
     int w;                 // consumer warps per CTA
+    int spl;               // states per lane
     int threads;
     int ch_per_tile;
     int smem;
@@ -60,7 +50,7 @@ struct ssm_plan_s {
     const char* name;
     // options
     unsigned spin_limit;
-    int64_t force_seg_len, force_k, force_workers;
+    int64_t force_seg_len, force_w, force_spl, force_workers;
     // workspace: header | flags[n_tiles] | carry[n_tiles][CW][N]
     unsigned char* ws;
     size_t ws_bytes, flags_off, carry_off;
@@ -108,17 +98,11 @@ bool head_mode(const ssm_dims_t& d) { return d.nheads != d.dim; }
 // Choose the consumer-warp count, segment length and grid; (re)allocate the workspace.
 int schedule(ssm_plan_s* p) {
     const ssm_dims_t& d = p->dims;
-    const bool head = head_mode(d);
     const int64_t Dg = d.dim / d.ngroups;
-    auto tiles_for = [&](int ct) { return d.batch * d.ngroups * ((Dg + ct - 1) / ct); };
-    ssm::Variant v8, v4;
-    if (!ssm::pick_variant(d.io_dtype, d.dstate, head, true, 8, &v8)) return SSM_ERR_UNSUPPORTED;
-    if (!ssm::pick_variant(d.io_dtype, d.dstate, head, true, 4, &v4)) return SSM_ERR_UNSUPPORTED;
-    // eight consumer warps (two per SM sub-partition) unless that leaves SMs without a tile
-    int w = 8;
-    if (p->force_k == 4 || p->force_k == 8) w = (int)p->force_k;
-    else if (tiles_for(v8.ch_per_tile) < p->sm_count) w = 4;
-    const ssm::Variant& v = w == 8 ? v8 : v4;
+    ssm::Layout lay;
+    if (!ssm::choose_layout(d, p->sm_count, (int)p->force_w, (int)p->force_spl, &lay)) return SSM_ERR_UNSUPPORTED;
+    const int w = lay.w;
+    const ssm::Variant& v = lay.v;
     if (v.smem > 48 * 1024 &&
         cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
         return SSM_ERR_CUDA;
@@ -126,7 +110,7 @@ int schedule(ssm_plan_s* p) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, v.fn, v.threads, v.smem) != cudaSuccess)
         return SSM_ERR_CUDA;
     if (occ < 1) return SSM_ERR_UNSUPPORTED;
-    const int64_t n_tiles = tiles_for(v.ch_per_tile);
+    const int64_t n_tiles = ssm::layout_tiles(d, v.ch_per_tile);
     int64_t ctas = p->sm_count;  // one persistent CTA per SM
     if (p->force_workers > 0 && p->force_workers < ctas) ctas = p->force_workers;
     const int64_t L = d.seqlen;
@@ -138,6 +122,7 @@ int schedule(ssm_plan_s* p) {
     if (ctas > n_units) ctas = n_units;
     if (ctas < 1) ctas = 1;
     p->w = w;
+    p->spl = lay.spl;
     p->threads = v.threads;
     p->ch_per_tile = v.ch_per_tile;
     p->smem = v.smem;
@@ -234,7 +219,8 @@ int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A
         // a shape the tensor maps cannot describe takes the element-copy path
     }
     ssm::Variant v;
-    if (!ssm::pick_variant(d.io_dtype, d.dstate, head_mode(d), vec, plan->w, &v)) return SSM_ERR_UNSUPPORTED;
+    if (!ssm::pick_variant(d.io_dtype, d.dstate, head_mode(d), vec, plan->w, plan->spl, &v))
+        return SSM_ERR_UNSUPPORTED;
     ssm::FwdParams prm;
     prm.u = u; prm.delta = delta; prm.A = A; prm.B = B; prm.C = C; prm.D = D; prm.z = z;
     prm.bias = delta_bias; prm.h0 = h0; prm.out = out; prm.last_state = last_state;
@@ -278,8 +264,8 @@ int ssm_scan_plan(ssm_plan_t* out_plan, const ssm_dims_t* dims, int device) {
     *out_plan = nullptr;
     if (!dims_ok(dims)) return SSM_ERR_INVALID_ARG;
     ssm::Variant v;
-    if (!ssm::pick_variant(dims->io_dtype, dims->dstate, dims->nheads != dims->dim, true, 8, &v))
-        return SSM_ERR_UNSUPPORTED;
+    ssm::Layout probe;
+    if (!ssm::choose_layout(*dims, 1, 0, 0, &probe)) return SSM_ERR_UNSUPPORTED;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return SSM_ERR_CUDA;
     if (set_device(device) != SSM_OK) return SSM_ERR_CUDA;
@@ -321,20 +307,31 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
         }
         case SSM_OPT_SEG_LEN:
         case SSM_OPT_CONSUMER_WARPS:
-        case SSM_OPT_WORKERS: {
+        case SSM_OPT_WORKERS:
+        case SSM_OPT_STATES_PER_LANE: {
             if (value < 0) return SSM_ERR_INVALID_ARG;
-            if (option == SSM_OPT_CONSUMER_WARPS && value != 0 && value != 4 && value != 8)
+            if (option == SSM_OPT_CONSUMER_WARPS && value != 0 && value != 4 && value != 8 && value != 16)
+                return SSM_ERR_INVALID_ARG;
+            if (option == SSM_OPT_STATES_PER_LANE && value != 0 && value != 2 && value != 4 && value != 8 &&
+                value != 16)
                 return SSM_ERR_INVALID_ARG;
             if (cudaDeviceSynchronize() != cudaSuccess) return SSM_ERR_CUDA;
             unsigned inject = 0;
             if (cudaMemcpy(&inject, plan->ws + offsetof(ssm::WsHeader, inject), sizeof(inject),
                            cudaMemcpyDeviceToHost) != cudaSuccess)
                 return SSM_ERR_CUDA;
-            if (option == SSM_OPT_SEG_LEN) plan->force_seg_len = value;
-            if (option == SSM_OPT_CONSUMER_WARPS) plan->force_k = value;
-            if (option == SSM_OPT_WORKERS) plan->force_workers = value;
+            int64_t* field = option == SSM_OPT_SEG_LEN         ? &plan->force_seg_len
+                             : option == SSM_OPT_CONSUMER_WARPS ? &plan->force_w
+                             : option == SSM_OPT_STATES_PER_LANE ? &plan->force_spl
+                                                                 : &plan->force_workers;
+            const int64_t old = *field;
+            *field = value;
             const int rc = schedule(plan);
-            if (rc != SSM_OK) return rc;
+            if (rc != SSM_OK) {
+                // no kernel for that combination: keep the previous option and schedule
+                *field = old;
+                return rc;
+            }
             return cudaMemcpy(plan->ws + offsetof(ssm::WsHeader, inject), &inject, sizeof(inject),
                               cudaMemcpyHostToDevice) == cudaSuccess
                        ? SSM_OK

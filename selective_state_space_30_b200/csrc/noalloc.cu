@@ -32,6 +32,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include "layout.h"
 #include "scan_kernel.cuh"
 #include "ssm_scan.h"
 
@@ -89,18 +90,6 @@ bool dims_valid(const ssm_dims_t* d) {
     return true;
 }
 
-bool pick(int dtype, int64_t N, bool head, bool vec, int w, ssm::Variant* v) {
-    const bool bf = dtype == SSM_BF16;
-    switch (N) {
-        case 8: return bf ? ssm::pick_bf16_n8(head, vec, w, v) : ssm::pick_f32_n8(head, vec, w, v);
-        case 16: return bf ? ssm::pick_bf16_n16(head, vec, w, v) : ssm::pick_f32_n16(head, vec, w, v);
-        case 32: return bf ? ssm::pick_bf16_n32(head, vec, w, v) : ssm::pick_f32_n32(head, vec, w, v);
-        case 64: return bf ? ssm::pick_bf16_n64(head, vec, w, v) : ssm::pick_f32_n64(head, vec, w, v);
-        case 128: return bf ? ssm::pick_bf16_n128(head, vec, w, v) : ssm::pick_f32_n128(head, vec, w, v);
-        default: return false;
-    }
-}
-
 typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -146,9 +135,6 @@ extern "C" int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, 
     if (d.batch > 0 && d.seqlen > 0 && (!u || !delta || !B || !C || !out)) return SSM_ERR_INVALID_ARG;
     if (!A) return SSM_ERR_INVALID_ARG;
     const bool head = d.nheads != d.dim;
-    ssm::Variant v8, v4;
-    if (!pick(d.io_dtype, d.dstate, head, true, 8, &v8) || !pick(d.io_dtype, d.dstate, head, true, 4, &v4))
-        return SSM_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
     void* scratch = nullptr;
@@ -157,13 +143,14 @@ extern "C" int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, 
     if (rc != SSM_OK) return rc;
     if (d.batch == 0) return SSM_OK;
 
-    // the schedule: the same policy as a plan (eight consumer warps unless that leaves SMs idle,
-    // one persistent CTA per SM, the default segment length)
+    // the schedule: the same policy as a plan (the default lane layout, one persistent CTA
+    // per SM, the default segment length)
     const int64_t Dg = d.dim / d.ngroups;
-    auto tiles_for = [&](int ct) { return d.batch * d.ngroups * ((Dg + ct - 1) / ct); };
-    const int w = tiles_for(v8.ch_per_tile) < sms ? 4 : 8;
-    const int ct = w == 8 ? v8.ch_per_tile : v4.ch_per_tile;
-    const int64_t n_tiles = tiles_for(ct);
+    ssm::Layout lay;
+    if (!ssm::choose_layout(d, sms, 0, 0, &lay)) return SSM_ERR_UNSUPPORTED;
+    const int w = lay.w;
+    const int ct = lay.v.ch_per_tile;
+    const int64_t n_tiles = ssm::layout_tiles(d, ct);
     int64_t ctas = sms;
     const int64_t L = d.seqlen;
     const int64_t seg_len = ssm::default_seg_len(L, n_tiles, ctas);
@@ -198,7 +185,7 @@ extern "C" int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, 
               encode(&tm.C, C, esz, L, d.batch * d.ngroups * d.dstate, (uint32_t)d.dstate, bc);
     }
     ssm::Variant v;
-    if (!pick(d.io_dtype, d.dstate, head, vec, w, &v)) return SSM_ERR_UNSUPPORTED;
+    if (!ssm::pick_variant(d.io_dtype, d.dstate, head, vec, w, lay.spl, &v)) return SSM_ERR_UNSUPPORTED;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     unsigned char* ws = static_cast<unsigned char*>(scratch);

@@ -9,13 +9,15 @@
 // Design (B200-first):
 //
 //  * State-parallel, register-resident recurrence.  The N states of a channel
-//    are split over TPC lanes of a warp (S = N/TPC states per lane); each lane
-//    runs its states sequentially over t.  States only meet in
+//    are split over TPC lanes of a warp (S = N/TPC states per lane, S = 2 or 4
+//    for N <= 16, 4 for N = 32, N/8 above); each lane runs its states
+//    sequentially over t.  States only meet in
 //    y = sum_n C_n h_n, so there is no scan across time inside a segment: one
 //    ex2 per (t, n) plus four FP32 operations (issued as packed f32x2).
 //  * Warp-specialised persistent CTAs, one per SM: a producer warp and W
-//    consumer warps (two per SM sub-partition when W = 8, since ex2 issues per
-//    sub-partition and a second warp hides the latency of the first).
+//    consumer warps (W = 16, 8 or 4: four, two or one per SM sub-partition; ex2
+//    issues per sub-partition and the kernel is latency-bound, so the most warps
+//    that still give every SM a channel tile win).
 //    - The producer takes work units -- (channel tile of W*CW channels, L
 //      segment) -- from a global ticket counter in segment-major order, waits
 //      (bounded) for the previous segment of the tile to publish its state,
@@ -369,10 +371,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
 
 // ------------------------------------------------------------ kernel config
 
-template <typename T, int N, int W, bool HEAD_A>
+template <typename T, int N, int W, bool HEAD_A, int SPL>
 struct Cfg {
     static constexpr int ESZ = IO<T>::kBytes;
-    static constexpr int S = (N >= 64) ? N / 8 : 4;       // states per lane
+    static constexpr int S = SPL;                          // states per lane
     static constexpr int TPC = N / S;                      // lanes per channel (2, 4 or 8)
     static constexpr int GW = 32 / TPC;                    // channels per consumer warp
     static constexpr int CT = W * GW;                      // channels per tile
@@ -410,7 +412,7 @@ struct Cfg {
     static constexpr int OFF_WARP = OFF_CSLOT + 2 * CSLOT * 4;
     static constexpr int SMEM = OFF_WARP + W * WARP_F * 4;
     static constexpr int THREADS = 32 * (W + 1);
-    static_assert(S % 2 == 0 && TPC >= 2 && TPC <= 8, "lane split");
+    static_assert(S % 2 == 0 && N % S == 0 && TPC >= 2 && TPC <= 8, "lane split");
     static_assert(TPT % 4 == 0 && TPT <= 16, "steps per lane must be 4..16");
     static_assert(STAGE % 16 == 0 && (PSLOT * 4) % 16 == 0 && (WARP_F * 4) % 16 == 0, "16-byte aligned smem");
     static_assert(2 * kStages + 6 <= 128, "barriers fit below OFF_STAGES");
@@ -449,10 +451,10 @@ static_assert(sizeof(BlockHdr) <= 64, "header fits its slot");
 
 // ------------------------------------------------------------------- kernel
 
-template <typename T, int N, int W, bool HEAD_A, bool VEC>
-__global__ void __launch_bounds__(Cfg<T, N, W, HEAD_A>::THREADS, 1)
+template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC>
+__global__ void __launch_bounds__(Cfg<T, N, W, HEAD_A, SPL>::THREADS, 1)
 scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
-    using Cf = Cfg<T, N, W, HEAD_A>;
+    using Cf = Cfg<T, N, W, HEAD_A, SPL>;
     constexpr int S = Cf::S, TPC = Cf::TPC, GW = Cf::GW, CT = Cf::CT, TPT = Cf::TPT, WT = Cf::WT;
     constexpr int ROW = Cf::ROW, NA = Cf::NA, ESZ = Cf::ESZ, RB = Cf::RB;
     constexpr int NST = Cf::STG;  // ring stages
@@ -465,6 +467,11 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
     int* status = &p.ws->status;
     const uint64_t budget = (uint64_t)p.spin_limit * 256ull;  // ns
 
+    // the swizzle of the B and C boxes assumes a 1024-byte aligned base
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(status, SSM_OK, SSM_ERR_BOUNDS);
+        return;
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(bars + BAR_FULL + s, 1);
@@ -986,34 +993,50 @@ struct Variant {
     const char* name;
 };
 
-template <typename T, int N, int W, bool HEAD_A, bool VEC>
+template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC>
 Variant make_variant(const char* name) {
-    using C = Cfg<T, N, W, HEAD_A>;
-    return Variant{scan_fwd_kernel<T, N, W, HEAD_A, VEC>, C::SMEM, C::THREADS, C::CT, N, name};
+    using C = Cfg<T, N, W, HEAD_A, SPL>;
+    return Variant{scan_fwd_kernel<T, N, W, HEAD_A, SPL, VEC>, C::SMEM, C::THREADS, C::CT, N, name};
 }
 
-// One function per (io dtype, N) translation unit; see fwd_*.cu.  w = consumer warps (8 or 4).
-#define SSM_DEFINE_PICK(T, TN, N)                                                                         \
-    bool pick_##TN##_n##N(bool head, bool vec, int w, Variant* v) {                                      \
-        if (w == 8) {                                                                                    \
+// The lane layouts compiled for a state size N: (consumer warps W, states per lane S).
+//   N <= 16: (16, 2), (8, 4), (8, 2), (4, 4), (4, 2);  N = 32: (8, 4), (4, 4);
+//   N >= 64: (8, N/8), (4, N/8).
+constexpr bool layout_exists(int N, int w, int spl) {
+    if (N <= 16) return (w == 16 && spl == 2) || ((w == 8 || w == 4) && (spl == 2 || spl == 4));
+    if (N == 32) return (w == 8 || w == 4) && spl == 4;
+    return (w == 8 || w == 4) && spl == N / 8;
+}
+
+// One function per (io dtype, N) translation unit; see fwd_*.cu.
+#define SSM_PICK_ONE(T, TN, N, W, SPL)                                                                   \
+    if (w == W && spl == SPL) {                                                                          \
+        if constexpr (layout_exists(N, W, SPL)) {                                                        \
             if (head)                                                                                    \
-                *v = vec ? make_variant<T, N, 8, true, true>("ws_" #TN "_n" #N "_w8_head_vec")           \
-                         : make_variant<T, N, 8, true, false>("ws_" #TN "_n" #N "_w8_head");             \
+                *v = vec ? make_variant<T, N, W, true, SPL, true>("ws_" #TN "_n" #N "_w" #W "s" #SPL "_head_vec") \
+                         : make_variant<T, N, W, true, SPL, false>("ws_" #TN "_n" #N "_w" #W "s" #SPL "_head");   \
             else                                                                                         \
-                *v = vec ? make_variant<T, N, 8, false, true>("ws_" #TN "_n" #N "_w8_vec")               \
-                         : make_variant<T, N, 8, false, false>("ws_" #TN "_n" #N "_w8");                 \
-        } else {                                                                                         \
-            if (head)                                                                                    \
-                *v = vec ? make_variant<T, N, 4, true, true>("ws_" #TN "_n" #N "_w4_head_vec")           \
-                         : make_variant<T, N, 4, true, false>("ws_" #TN "_n" #N "_w4_head");             \
-            else                                                                                         \
-                *v = vec ? make_variant<T, N, 4, false, true>("ws_" #TN "_n" #N "_w4_vec")               \
-                         : make_variant<T, N, 4, false, false>("ws_" #TN "_n" #N "_w4");                 \
+                *v = vec ? make_variant<T, N, W, false, SPL, true>("ws_" #TN "_n" #N "_w" #W "s" #SPL "_vec")     \
+                         : make_variant<T, N, W, false, SPL, false>("ws_" #TN "_n" #N "_w" #W "s" #SPL);          \
+            return true;                                                                                 \
         }                                                                                                \
-        return true;                                                                                     \
+        return false;                                                                                    \
+    }
+#define SSM_DEFINE_PICK(T, TN, N)                                                                         \
+    bool pick_##TN##_n##N(bool head, bool vec, int w, int spl, Variant* v) {                             \
+        SSM_PICK_ONE(T, TN, N, 16, 2)                                                                    \
+        SSM_PICK_ONE(T, TN, N, 8, 2)                                                                     \
+        SSM_PICK_ONE(T, TN, N, 8, 4)                                                                     \
+        SSM_PICK_ONE(T, TN, N, 4, 2)                                                                     \
+        SSM_PICK_ONE(T, TN, N, 4, 4)                                                                     \
+        SSM_PICK_ONE(T, TN, N, 8, 8)                                                                     \
+        SSM_PICK_ONE(T, TN, N, 4, 8)                                                                     \
+        SSM_PICK_ONE(T, TN, N, 8, 16)                                                                    \
+        SSM_PICK_ONE(T, TN, N, 4, 16)                                                                    \
+        return false;                                                                                    \
     }
 
-#define SSM_DECLARE_PICK(TN, N) bool pick_##TN##_n##N(bool head, bool vec, int w, Variant* v);
+#define SSM_DECLARE_PICK(TN, N) bool pick_##TN##_n##N(bool head, bool vec, int w, int spl, Variant* v);
 SSM_DECLARE_PICK(bf16, 8)
 SSM_DECLARE_PICK(bf16, 16)
 SSM_DECLARE_PICK(bf16, 32)

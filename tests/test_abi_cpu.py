@@ -79,6 +79,21 @@ def test_host_side_argument_checks(lib):
     assert lib.ssm_probe_ex2(None, 1, 1, None) == ssm.SSM_ERR_INVALID_ARG
 
 
+def test_state_update_host_checks(lib):
+    """ssm_selective_state_update rejects bad arguments before touching the GPU."""
+    import selective_state_space_30_b200 as ssm
+    a, mis = 0x10000, 0x10004   # stand-in device addresses: 16-byte aligned, and not
+    args = lambda st: (st, a, a, a, a, a, None, None, None, 1, a, None)  # noqa: E731
+    f = lib.ssm_selective_state_update
+    assert f(None, *args(a)) == ssm.SSM_ERR_INVALID_ARG
+    assert f(ctypes.byref(ssm.make_dims(2, 64, 2, 16, 64, 1, ssm.SSM_BF16)), *args(a)) == ssm.SSM_ERR_INVALID_ARG
+    assert f(ctypes.byref(ssm.make_dims(2, 64, 1, 24, 64, 1, ssm.SSM_BF16)), *args(a)) == ssm.SSM_ERR_UNSUPPORTED
+    d = ssm.make_dims(2, 64, 1, 16, 64, 1, ssm.SSM_BF16)
+    assert f(ctypes.byref(d), *args(None)) == ssm.SSM_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), *args(mis)) == ssm.SSM_ERR_UNSUPPORTED
+    assert f(ctypes.byref(ssm.make_dims(0, 64, 1, 16, 64, 1, ssm.SSM_BF16)), *args(None)) == ssm.SSM_OK
+
+
 def test_plan_without_a_gpu_reports_cuda_error(lib):
     import torch
     import selective_state_space_30_b200 as ssm

@@ -20,6 +20,10 @@ SHAPES = [
 ]
 SCHEDULES = [dict(seg_len=32), dict(seg_len=64, warps=4), dict(seg_len=96, warps=8), dict(seg_len=32, ctas=1),
              dict(seg_len=64, ctas=3, warps=8), dict(ctas=5), dict(seg_len=160, ctas=7, warps=4)]
+# N <= 16: the other lane layouts (consumer warps x states per lane); the same
+# per-state arithmetic, so the results stay bit-identical
+SCHEDULES_SMALL_N = [dict(warps=16, states_per_lane=2), dict(warps=8, states_per_lane=2, seg_len=64, ctas=3),
+                     dict(warps=4, states_per_lane=2), dict(warps=16, states_per_lane=2, seg_len=32, ctas=1)]
 
 
 def _recipe(d):
@@ -35,7 +39,8 @@ def test_schedule_invariance(dims):
     ro, rl, rm = oracle.run_inputs(dims, inp)
     check_out(to_host_f64(ref_out), ro, rm, dims.dtype)
     check_state(to_host_f64(ref_last), rl)
-    for opts in SCHEDULES:
+    scheds = SCHEDULES + (SCHEDULES_SMALL_N if dims.dstate <= 16 else [])
+    for opts in scheds:
         out, last = run_gpu(dims, inp, opts=opts)
         # segments and blocks are 32-step aligned: the same fp32 operations in the same order
         assert torch.equal(out, ref_out), f"output differs under schedule {opts}"
@@ -98,5 +103,39 @@ def test_option_errors():
             ssm.ssm_scan_set_option(plan, ssm.SSM_OPT_SPIN_LIMIT, 0)
         sch = ssm.ssm_scan_plan_schedule(plan)
         assert sch["n_seg"] >= 1 and sch["seg_len"] % 32 == 0 and sch["consumer_warps"] in (4, 8)
+    finally:
+        ssm.ssm_scan_destroy(plan)
+
+
+def test_layout_option_checks():
+    import selective_state_space_30_b200 as ssm
+    from selective_state_space_30_b200 import _abi
+    lib = _abi.load_library()
+    # 8 x 1536 channels, N = 16: sixteen consumer warps with two states per lane fill the SMs
+    d = ssm.make_dims(8, 1536, 256, 16, 1536, 1, ssm.SSM_BF16)
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w16s2_vec"
+        assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_STATES_PER_LANE, 3) == ssm.SSM_ERR_INVALID_ARG
+        assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_CONSUMER_WARPS, 12) == ssm.SSM_ERR_INVALID_ARG
+        assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_STATES_PER_LANE, 4) == ssm.SSM_OK
+        assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w8s4_vec"
+        # sixteen warps exist only with two states per lane: refused, previous schedule kept
+        assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_CONSUMER_WARPS, 16) == ssm.SSM_ERR_UNSUPPORTED
+        assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w8s4_vec"
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    # 1 x 5120 channels: eight warps with two states per lane keep a tile per SM
+    d = ssm.make_dims(1, 5120, 256, 16, 5120, 1, ssm.SSM_BF16)
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w8s2_vec"
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    dh = ssm.make_dims(2, 64, 256, 128, 4, 1, ssm.SSM_BF16)
+    plan = ssm.ssm_scan_plan(dh, 0)
+    try:
+        assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_STATES_PER_LANE, 2) == ssm.SSM_ERR_UNSUPPORTED
+        assert ssm.ssm_scan_plan_info(plan)["variant"].endswith("s16_head_vec")
     finally:
         ssm.ssm_scan_destroy(plan)

@@ -47,6 +47,9 @@ def load(path: Optional[str] = None):
     lib.oracle_selective_scan_f64.argtypes = [
         ctypes.POINTER(_Dims), p, p, p, p, p, p, p, p, ctypes.c_int, p,
         ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, p, p, p, ctypes.c_int]
+    i64 = ctypes.c_int64
+    lib.oracle_causal_conv1d_f64.restype = ctypes.c_int
+    lib.oracle_causal_conv1d_f64.argtypes = [i64, i64, i64, i64, p, p, p, ctypes.c_int, p]
     return lib
 
 
@@ -142,3 +145,28 @@ def run_inputs(dims, inputs: dict, channels=None, h0=None, nthreads=None, lib=No
                           inputs["A"], inputs["B"], inputs["C"], inputs.get("D"), inputs.get("z"),
                           inputs.get("delta_bias"), bool(inputs.get("softplus", True)), dims.nheads,
                           dims.ngroups, h0=h0, channels=channels, nthreads=nthreads, lib=lib)
+
+
+def causal_conv1d(x, w, bias=None, silu: bool = True, lib=None) -> np.ndarray:
+    """The causal depthwise convolution (see `oracle_causal_conv1d_f64`) in fp64.
+
+    x: (batch, dim, seqlen) as float64/float32 or bf16 bits; w: (dim, width);
+    bias: (dim) or None.  Returns out (batch, dim, seqlen) float64.
+    """
+    xx, ww, bb = _f64(x), _f64(w), _f64(bias)
+    xs = np.asarray(x).shape
+    if len(xs) != 3:
+        raise ValueError("x must be (batch, dim, seqlen)")
+    batch, dim, seqlen = xs
+    if ww.ndim != 2 or ww.shape[0] != dim:
+        raise ValueError("w must be (dim, width)")
+    width = ww.shape[1]
+    if bb is not None and bb.size != dim:
+        raise ValueError("bias must be (dim)")
+    out = np.empty(batch * dim * seqlen, dtype=np.float64)
+    lib = lib or _get_lib()
+    rc = lib.oracle_causal_conv1d_f64(batch, dim, seqlen, width, _ptr(xx), _ptr(ww), _ptr(bb),
+                                      1 if silu else 0, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out.reshape(batch, dim, seqlen)

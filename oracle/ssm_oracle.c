@@ -159,3 +159,41 @@ int oracle_selective_scan_f64(const oracle_dims_t* dm, const double* u, const do
         if (live[t]) pthread_join(th[t], NULL);
     return 0;
 }
+
+/*
+ * Causal depthwise convolution over time: the local convolution in front of
+ * the SSM ("architecture-details" page, "Model Configuration": d_conv, the
+ * convolution width, and conv_bias; "Parameter Impact": d_conv is the local
+ * context window before the SSM).  Each channel has its own `width` taps; the
+ * input is zero before t = 0, so output t sees steps t-width+1 .. t only.
+ * Per batch b, channel d, step t, in fp64:
+ *
+ *   v = bias[d] + sum_{k=0}^{width-1} w[d][k] * x[b][d][t - (width-1) + k]
+ *   out[b][d][t] = silu ? v / (1 + exp(-v)) : v
+ *
+ * (the activation after the convolution is a flag: the pages name the
+ * convolution, not what follows it).  bias may be NULL (zero).
+ * Layouts: x, out (batch, dim, seqlen); w (dim, width); bias (dim).
+ * Returns 0, or -1 on a bad size or a missing required pointer.
+ */
+int oracle_causal_conv1d_f64(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, const double* x,
+                             const double* w, const double* bias, int silu, double* out) {
+    if (batch < 0 || dim <= 0 || seqlen < 0 || width <= 0) return -1;
+    if (!x || !w || !out) return -1;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const double* xr = x + (b * dim + d) * seqlen;
+            double* orow = out + (b * dim + d) * seqlen;
+            const double* wr = w + d * width;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                double v = bias ? bias[d] : 0.0;
+                for (int64_t k = 0; k < width; ++k) {
+                    const int64_t s = t - (width - 1) + k;
+                    if (s >= 0) v += wr[k] * xr[s];
+                }
+                orow[t] = silu ? v / (1.0 + exp(-v)) : v;
+            }
+        }
+    }
+    return 0;
+}

@@ -9,6 +9,7 @@ import subprocess
 import pytest
 
 import oracle
+from conv1d_pins import CONV_PINS
 from oracle_pins import ALL_PINS
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
@@ -32,6 +33,12 @@ MUTANTS = [
     ("initial state ignored", "h[n] = j->h0 ? j->h0[row * N + n] : 0.0;", "h[n] = 0.0;"),
     ("state not decayed", "h[n] = dA * h[n] +", "h[n] = h[n] +"),
     ("u squared", "* u[t];\n            y +=", "* u[t] * u[t];\n            y +="),
+    # the causal convolution
+    ("conv taps reversed", "v += wr[k] * xr[s];", "v += wr[width - 1 - k] * xr[s];"),
+    ("conv shifted by one step", "const int64_t s = t - (width - 1) + k;", "const int64_t s = t - width + k;"),
+    ("conv not causal (centred)", "const int64_t s = t - (width - 1) + k;", "const int64_t s = t - (width - 1) / 2 + k;"),
+    ("conv bias dropped", "double v = bias ? bias[d] : 0.0;", "double v = 0.0;"),
+    ("conv activation sigmoid", "orow[t] = silu ? v / (1.0 + exp(-v)) : v;", "orow[t] = silu ? 1.0 / (1.0 + exp(-v)) : v;"),
 ]
 
 
@@ -52,7 +59,7 @@ def _build_mutant(tmp_path, name, old, new):
 def test_mutant_is_caught(tmp_path, name, old, new):
     lib = _build_mutant(tmp_path, name, old, new)
     caught = []
-    for pin in ALL_PINS:
+    for pin in ALL_PINS + CONV_PINS:
         try:
             pin(lib)
         except AssertionError:

@@ -2,6 +2,7 @@
 import pytest
 
 import oracle
+from conv1d_pins import CONV_PINS
 from oracle_pins import ALL_PINS
 
 
@@ -12,4 +13,9 @@ def lib():
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
 def test_pin(pin, lib):
+    pin(lib)
+
+
+@pytest.mark.parametrize("pin", CONV_PINS, ids=lambda f: f.__name__)
+def test_conv_pin(pin, lib):
     pin(lib)

@@ -520,6 +520,81 @@ def run_decode(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ causal conv1d
+
+CONV_SHAPES = {
+    # the x of the mamba-130m layer: batch 8, d_inner 1536, L 2048, d_conv 4, bf16
+    "conv1d-mamba-130m": dict(batch=8, dim=1536, seqlen=2048, width=4, dtype="bf16"),
+    # the x of the mamba-1.4b layer: batch 4, d_inner 4096, L 4096
+    "conv1d-mamba-1.4b": dict(batch=4, dim=4096, seqlen=4096, width=4, dtype="bf16"),
+}
+
+
+def run_conv1d(args):
+    """ssm_causal_conv1d_fwd on a layer's x: one JSON line (GB/s against the HBM roofline)."""
+    import torch
+    import ssm_inputs as si
+    import selective_state_space_30_b200 as ssm
+    rank, local, world = _rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+    init_ranks("nccl", local)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sh = CONV_SHAPES[args.workload]
+    dims = si.Dims(sh["batch"], sh["dim"], sh["seqlen"], 16, dtype=sh["dtype"])
+    x = si.make_inputs(dims, si.Recipe(), 0)["u"]
+    e = 2 if sh["dtype"] == "bf16" else 4
+    elems = sh["batch"] * sh["dim"] * sh["seqlen"]
+    alg = 2 * elems * e + sh["dim"] * (sh["width"] + 1) * 4          # x read, out written, taps and bias
+    copies = max(2, int(np.ceil(3 * L2_BYTES / alg)))
+    rng = np.random.default_rng(0)
+    w = torch.from_numpy((rng.standard_normal((sh["dim"], sh["width"])) / 2).astype(np.float32)).to(dev)
+    b = torch.from_numpy((rng.standard_normal(sh["dim"]) * 0.1).astype(np.float32)).to(dev)
+    sets = []
+    for _ in range(copies):
+        xd = _to_dev(x, dev)
+        sets.append((xd, torch.empty_like(xd)))
+    io = ssm.SSM_BF16 if sh["dtype"] == "bf16" else ssm.SSM_F32
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        xd, od = sets[i % copies]
+        ssm.ssm_causal_conv1d_fwd(sh["batch"], sh["dim"], sh["seqlen"], sh["width"], io, xd, w, b, True, od,
+                                  stream.cuda_stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    total = max_over_ranks(e0.elapsed_time(e1), dev)
+    hbm_gbs, _, src = _peaks()
+    finish_ranks()
+    if rank != 0:
+        return
+    gbs = alg / (ms * 1e-3) / 1e9
+    line = {"metric": "causal conv1d (d_conv taps + SiLU) Gelem/s on 1 B200", "op": "conv1d",
+            "value": job_throughput(world, elems, args.steps, total), "unit": "Gelem/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 (bf16 I/O)" if sh["dtype"] == "bf16" else "f32", "data": "synthetic (seeded splitmix64)",
+            "config": dict(sh, workload=args.workload,
+                           l2=f"{copies} rotating input sets of {alg / 1e6:.0f} MB, no flush"),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                         "traffic": None, "peak_source": src, "alg_bytes_per_launch": alg},
+            "clocks": clk.summary(), "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,8 +604,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", default="scan", choices=["scan", "decode"],
-                    help="scan: the forward scan (the headline metric); decode: the single-step state update")
+    ap.add_argument("--op", default="scan", choices=["scan", "decode", "conv1d"],
+                    help="scan: the forward scan (the headline metric); decode: the single-step state update; "
+                         "conv1d: the causal convolution in front of the scan")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -538,6 +614,11 @@ def main():
         if args.workload == DEFAULT_WORKLOAD:
             args.workload = "decode-mamba-1.4b-b256"
         run_decode(args)
+        return
+    if args.op == "conv1d":
+        if args.workload == DEFAULT_WORKLOAD:
+            args.workload = "conv1d-mamba-130m"
+        run_conv1d(args)
         return
     if args.impl == "reference":
         run_reference(args)

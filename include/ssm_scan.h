@@ -140,8 +140,9 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
  *                              0 switches it off
  *   SSM_OPT_SEG_LEN            force the segment length (rounded up to 32 steps);
  *                              0 = automatic
- *   SSM_OPT_CONSUMER_WARPS     force 4, 8 or 16 consumer warps per CTA (16 exists for
- *                              dstate <= 16 with 2 states per lane); 0 = automatic
+ *   SSM_OPT_CONSUMER_WARPS     force 4, 8, 12 or 16 consumer warps per CTA (16 exists
+ *                              for dstate <= 16 with 2 states per lane, 12 for dstate
+ *                              16 with 4); 0 = automatic
  *   SSM_OPT_WORKERS            cap the number of persistent CTAs; 0 = one per SM
  *   SSM_OPT_STATES_PER_LANE    force the states each lane holds (2 or 4 for dstate <= 16,
  *                              4 for dstate 32, dstate/8 above); 0 = automatic.  A
@@ -214,6 +215,26 @@ int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, const float
 int ssm_selective_state_update(const ssm_dims_t* dims, float* state, const void* u, const void* delta,
                                const float* A, const void* B, const void* C, const float* D, const void* z,
                                const float* delta_bias, int softplus, void* out, ssm_stream_t stream);
+
+/*
+ * The causal depthwise convolution in front of the scan (Mamba
+ * "architecture-details" page, "Model Configuration": d_conv, the convolution
+ * width, and conv_bias; "Parameter Impact": the local context window before the
+ * SSM).  For every (b, d, t), with x taken as zero before t = 0:
+ *
+ *     v = bias[d] + sum_{k < width} w[d,k] * x[b,d,t - width + 1 + k]
+ *     out[b,d,t] = silu ? v / (1 + exp(-v)) : v
+ *
+ * x and out are (batch, dim, seqlen) in io_dtype (ssm_dtype_t), w is (dim,
+ * width) fp32, bias is (dim) fp32 or NULL (zero).  The pages name the
+ * convolution but not what follows it, so the SiLU is a flag.  width is 1 to 4
+ * (4 is the pages' standard), else SSM_ERR_UNSUPPORTED.  No plan, no workspace:
+ * one kernel on `stream`.  out must not alias x.  SSM_ERR_INVALID_ARG for a bad
+ * shape or dtype or a NULL x, w or out.
+ */
+int ssm_causal_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t width, int32_t io_dtype,
+                          const void* x, const float* w, const float* bias, int silu, void* out,
+                          ssm_stream_t stream);
 
 /* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
 int ssm_scan_destroy(ssm_plan_t plan);

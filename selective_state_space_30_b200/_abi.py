@@ -26,6 +26,7 @@ SSM_BF16 = 1
 # every exported symbol declared in include/ssm_scan.h
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
            "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update",
+           "ssm_causal_conv1d_fwd",
            "ssm_scan_set_option",
            "ssm_scan_plan_schedule", "ssm_scan_destroy",
            "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
@@ -72,6 +73,7 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_fwd_host.argtypes = fwd_args + [vp, vp, vp]
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, dims_p, vp, vp, vp]
     lib.ssm_selective_state_update.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+    lib.ssm_causal_conv1d_fwd.argtypes = [i64, i64, i64, i32, i32, vp, vp, vp, i32, vp, vp]
     lib.ssm_scan_destroy.argtypes = [vp]
     lib.ssm_scan_device_status.argtypes = [vp, vp]
     lib.ssm_status_string.argtypes = [i32]
@@ -173,6 +175,14 @@ def ssm_selective_state_update(dims: ssm_dims_t, state, u, delta, A, B, C, D, z,
         ctypes.byref(dims), _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), 1 if softplus else 0, _ptr(out), _stream(stream))
     return _check(rc, "ssm_selective_state_update") if check else rc
+
+
+def ssm_causal_conv1d_fwd(batch: int, dim: int, seqlen: int, width: int, io_dtype: int, x, w, bias,
+                          silu: bool, out, stream=None, check: bool = True) -> int:
+    """The causal depthwise convolution (see include/ssm_scan.h)."""
+    rc = load_library().ssm_causal_conv1d_fwd(int(batch), int(dim), int(seqlen), int(width), int(io_dtype), _ptr(x),
+                                              _ptr(w), _ptr(bias), 1 if silu else 0, _ptr(out), _stream(stream))
+    return _check(rc, "ssm_causal_conv1d_fwd") if check else rc
 
 
 def ssm_scan_destroy(plan: Optional[int]) -> int:

@@ -310,7 +310,8 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
         case SSM_OPT_WORKERS:
         case SSM_OPT_STATES_PER_LANE: {
             if (value < 0) return SSM_ERR_INVALID_ARG;
-            if (option == SSM_OPT_CONSUMER_WARPS && value != 0 && value != 4 && value != 8 && value != 16)
+            if (option == SSM_OPT_CONSUMER_WARPS && value != 0 && value != 4 && value != 8 && value != 12 &&
+                value != 16)
                 return SSM_ERR_INVALID_ARG;
             if (option == SSM_OPT_STATES_PER_LANE && value != 0 && value != 2 && value != 4 && value != 8 &&
                 value != 16)

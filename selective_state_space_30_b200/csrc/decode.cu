@@ -5,26 +5,22 @@
 // ssm_selective_state_update.
 //
 // The step is bound by HBM: every state row is read and written once, and the
-// exps per element are a handful.  Layout: TPC = N/4 lanes per channel, four
-// consecutive states per lane, so a warp reads and writes its state rows as
-// contiguous 16-byte pieces; the lanes of a channel sum y with shuffles.
+// exps per element are a handful.  The state rows reach shared memory by bulk
+// copies, so enough bytes are in flight to cover the HBM latency.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
+#include "scan_kernel.cuh"   // ex2_approx, softplus1, silu1, mbarrier and bulk-copy helpers
 #include "ssm_scan.h"
 
 namespace {
 
+using ssm::ex2_approx;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kThreads = 256;
-
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
+constexpr int kMaxGridY = 65535;
 
 template <typename T> __device__ __forceinline__ float ld_io(const T* p);
 template <> __device__ __forceinline__ float ld_io<float>(const float* p) { return __ldg(p); }
@@ -53,70 +49,140 @@ struct StepParams {
     const void *u, *delta, *B, *C, *z;
     const float *A, *D, *bias;
     void* out;
-    int64_t batch, dim, nheads, ngroups;
+    int64_t batch;
+    uint32_t dim, nheads, ngroups;
+    uint32_t head_dim, group_dim;   // dim / nheads, dim / ngroups
     int softplus;
 };
 
+// grid.y walks the batch rows, grid.x the chunks of R = 4096/N channels of a
+// row.  One thread bulk-copies the chunk's state rows (and, per channel, its A
+// rows) into shared memory with cp.async.bulk: 16 KB of state in flight per CTA
+// without holding registers, several CTAs per SM.  Then thread slots (channel,
+// lane j) -- N/4 lanes per channel, four states per lane -- update the states in
+// four passes and store them back with evict-first 16-byte stores; a warp covers
+// contiguous 512-byte stretches.
+template <int N>
+struct StepCfg {
+    static constexpr int TPC = N / 4;                 // lanes per channel
+    static constexpr int R = 4096 / N;                // channels per CTA
+    static constexpr int PASSES = R * TPC / kThreads; // slots per thread
+    static constexpr int STATE_BYTES = R * N * 4;     // 16 KB
+    static_assert(PASSES * kThreads == R * TPC, "whole passes");
+};
+
 template <typename T, int N>
-__global__ void __launch_bounds__(kThreads) state_update_kernel(const StepParams p) {
-    constexpr int TPC = N / 4;   // lanes per channel
-    const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    const int64_t ch = gid / TPC;           // flat (b, d)
-    const int j = (int)(gid % TPC);
-    const bool live = ch < p.batch * p.dim;
-    const int64_t c = live ? ch : 0;
-    const int64_t b = c / p.dim, d = c % p.dim;
-    const int64_t hd = d / (p.dim / p.nheads), g = d / (p.dim / p.ngroups);
+__global__ void __launch_bounds__(kThreads, 6) state_update_kernel(const StepParams p) {
+    using SC = StepCfg<N>;
+    constexpr uint32_t TPC = SC::TPC;
+    __shared__ __align__(128) float sh[SC::R * N];     // the chunk's states
+    __shared__ __align__(128) float sa[SC::R * N];     // the chunk's A rows (per-channel layout)
+    __shared__ __align__(8) uint64_t bar;
     const bool head = p.nheads != p.dim;
+    const uint32_t d0 = blockIdx.x * (uint32_t)SC::R;
+    const uint32_t nch = p.dim - d0 < (uint32_t)SC::R ? p.dim - d0 : (uint32_t)SC::R;
     const T* u = static_cast<const T*>(p.u);
     const T* dl = static_cast<const T*>(p.delta);
-    const float uu = ld_io<T>(u + c);
-    float x = ld_io<T>(dl + b * p.nheads + hd) + (p.bias ? __ldg(p.bias + hd) : 0.f);
-    // softplus(x) = max(x, 0) + log1p(exp(-|x|))
-    const float dt = p.softplus ? fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x))) : x;
-    const float du = dt * uu;
-    const int n0 = 4 * j;
-    const float4 bb = ld4<T>(static_cast<const T*>(p.B) + (b * p.ngroups + g) * N + n0);
-    const float4 cc = ld4<T>(static_cast<const T*>(p.C) + (b * p.ngroups + g) * N + n0);
-    float4 a;
-    if (head) {
-        const float ah = __ldg(p.A + hd);
-        a = make_float4(ah, ah, ah, ah);
-    } else {
-        a = __ldg(reinterpret_cast<const float4*>(p.A + d * N + n0));
+    if (threadIdx.x == 0) {
+        ssm::mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    float4* hp = reinterpret_cast<float4*>(p.state + c * N + n0);
-    float4 h = live ? *hp : make_float4(0.f, 0.f, 0.f, 0.f);
-    h.x = fmaf(ex2_approx(dt * a.x * kLog2e), h.x, du * bb.x);
-    h.y = fmaf(ex2_approx(dt * a.y * kLog2e), h.y, du * bb.y);
-    h.z = fmaf(ex2_approx(dt * a.z * kLog2e), h.z, du * bb.z);
-    h.w = fmaf(ex2_approx(dt * a.w * kLog2e), h.w, du * bb.w);
-    if (live) *hp = h;
-    float y = fmaf(cc.x, h.x, fmaf(cc.y, h.y, fmaf(cc.z, h.z, cc.w * h.w)));
-#pragma unroll
-    for (int m = TPC / 2; m >= 1; m >>= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
-    if (live && j == 0) {
-        y = fmaf(p.D ? __ldg(p.D + d) : 0.f, uu, y);
-        if (p.z) {
-            const float zz = ld_io<T>(static_cast<const T*>(p.z) + c);
-            y *= zz / (1.f + __expf(-zz));
+    __syncthreads();
+    unsigned phase = 0;
+    for (int64_t b = blockIdx.y; b < p.batch; b += gridDim.y, phase ^= 1u) {
+        const int64_t c0 = b * p.dim + d0;
+        if (threadIdx.x == 0) {
+            const unsigned bytes = nch * N * 4u;
+            ssm::mbar_arrive_tx(&bar, bytes * (head ? 1u : 2u));
+            ssm::bulk_g2s(sh, p.state + c0 * N, bytes, &bar);
+            if (!head) ssm::bulk_g2s(sa, p.A + (int64_t)d0 * N, bytes, &bar);
         }
-        st_io<T>(static_cast<T*>(p.out) + c, y);
+        // per-slot inputs from global memory while the bulk copies are in flight (B and C
+        // rows are shared by all channels of a group: they come from L1 in the passes below)
+        float uu[SC::PASSES], x[SC::PASSES];
+#pragma unroll
+        for (int k = 0; k < SC::PASSES; ++k) {
+            const uint32_t slot = threadIdx.x + (uint32_t)(k * kThreads);
+            const uint32_t lc = slot / TPC;
+            const uint32_t d = d0 + (lc < nch ? lc : 0u);
+            const uint32_t hd = head ? d / p.head_dim : d;
+            uu[k] = ld_io<T>(u + b * p.dim + d);
+            x[k] = ld_io<T>(dl + b * p.nheads + hd) + (p.bias ? __ldg(p.bias + hd) : 0.f);
+        }
+        // the copies complete (they depend on nothing else; the wait is bounded all the same,
+        // and a chunk that never arrived leaves its outputs NaN rather than hanging)
+        bool ready = true;
+        {
+            const uint64_t t0 = ssm::now_ns();
+            while (!ssm::mbar_try(&bar, phase)) {
+                if (ssm::now_ns() - t0 > 1000000000ull) { ready = false; break; }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < SC::PASSES; ++k) {
+            const uint32_t slot = threadIdx.x + (uint32_t)(k * kThreads);
+            const uint32_t lc = slot / TPC;
+            const bool live = lc < nch;
+            const uint32_t d = d0 + (live ? lc : 0u);
+            const uint32_t n0 = 4u * (slot % TPC);
+            const int64_t c = b * p.dim + d;
+            const uint32_t g = p.ngroups == 1 ? 0u : d / p.group_dim;
+            const int64_t bc = (b * p.ngroups + g) * N + n0;
+            const float4 bbk = ld4<T>(static_cast<const T*>(p.B) + bc);
+            const float4 cck = ld4<T>(static_cast<const T*>(p.C) + bc);
+            float4 a;
+            if (head) {
+                const float ah = __ldg(p.A + d / p.head_dim);
+                a = make_float4(ah, ah, ah, ah);
+            } else {
+                a = *reinterpret_cast<const float4*>(sa + (live ? lc : 0u) * N + n0);
+            }
+            float4 hk = *reinterpret_cast<const float4*>(sh + (live ? lc : 0u) * N + n0);
+            const float dt = p.softplus ? ssm::softplus1(x[k]) : x[k];
+            const float du = dt * uu[k];
+            const float s = dt * kLog2e;
+            hk.x = fmaf(ex2_approx(s * a.x), hk.x, du * bbk.x);
+            hk.y = fmaf(ex2_approx(s * a.y), hk.y, du * bbk.y);
+            hk.z = fmaf(ex2_approx(s * a.z), hk.z, du * bbk.z);
+            hk.w = fmaf(ex2_approx(s * a.w), hk.w, du * bbk.w);
+            if (live && ready) __stcs(reinterpret_cast<float4*>(p.state + c * N + n0), hk);
+            float y = fmaf(cck.x, hk.x, fmaf(cck.y, hk.y, fmaf(cck.z, hk.z, cck.w * hk.w)));
+#pragma unroll
+            for (uint32_t m = TPC / 2; m >= 1; m >>= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
+            if (live && n0 == 0) {
+                y = fmaf(p.D ? __ldg(p.D + d) : 0.f, uu[k], y);
+                if (p.z) y *= ssm::silu1(ld_io<T>(static_cast<const T*>(p.z) + c));
+                st_io<T>(static_cast<T*>(p.out) + c, ready ? y : __int_as_float(0x7FC00000));
+            }
+        }
+        // every thread is done with the chunk's shared copies before the next row's copies land
+        __syncthreads();
     }
 }
 
 template <typename T>
 int launch(const StepParams& prm, int64_t N, cudaStream_t s) {
-    const int64_t threads = prm.batch * prm.dim * (N / 4);
-    const int64_t blocks = (threads + kThreads - 1) / kThreads;
-    if (blocks > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;
-    if (blocks == 0) return SSM_OK;
+    const int64_t R = 4096 / N;
+    const int64_t bx = (prm.dim + R - 1) / R;
+    const int64_t by = prm.batch < kMaxGridY ? prm.batch : kMaxGridY;
+    if (bx == 0 || by == 0) return SSM_OK;
+    const dim3 g((unsigned)bx, (unsigned)by);
+    // shared memory holds the in-flight state: ask for the largest carveout
+    static const bool carve = [] {
+        cudaFuncSetAttribute(state_update_kernel<T, 8>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        cudaFuncSetAttribute(state_update_kernel<T, 16>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        cudaFuncSetAttribute(state_update_kernel<T, 32>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        cudaFuncSetAttribute(state_update_kernel<T, 64>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        cudaFuncSetAttribute(state_update_kernel<T, 128>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        return true;
+    }();
+    (void)carve;
     switch (N) {
-        case 8: state_update_kernel<T, 8><<<(unsigned)blocks, kThreads, 0, s>>>(prm); break;
-        case 16: state_update_kernel<T, 16><<<(unsigned)blocks, kThreads, 0, s>>>(prm); break;
-        case 32: state_update_kernel<T, 32><<<(unsigned)blocks, kThreads, 0, s>>>(prm); break;
-        case 64: state_update_kernel<T, 64><<<(unsigned)blocks, kThreads, 0, s>>>(prm); break;
-        case 128: state_update_kernel<T, 128><<<(unsigned)blocks, kThreads, 0, s>>>(prm); break;
+        case 8: state_update_kernel<T, 8><<<g, kThreads, 0, s>>>(prm); break;
+        case 16: state_update_kernel<T, 16><<<g, kThreads, 0, s>>>(prm); break;
+        case 32: state_update_kernel<T, 32><<<g, kThreads, 0, s>>>(prm); break;
+        case 64: state_update_kernel<T, 64><<<g, kThreads, 0, s>>>(prm); break;
+        case 128: state_update_kernel<T, 128><<<g, kThreads, 0, s>>>(prm); break;
         default: return SSM_ERR_UNSUPPORTED;
     }
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
@@ -146,10 +212,14 @@ extern "C" int ssm_selective_state_update(const ssm_dims_t* dims, float* state, 
     if (!aligned(state, 16) || !aligned(B, bc_align) || !aligned(C, bc_align) ||
         (d.nheads == d.dim && !aligned(A, 16)))
         return SSM_ERR_UNSUPPORTED;
+    // 32-bit index math within a batch row
+    if (d.dim * (N / 4) >= ((int64_t)1 << 31)) return SSM_ERR_UNSUPPORTED;
     StepParams prm;
     prm.state = state; prm.u = u; prm.delta = delta; prm.B = B; prm.C = C; prm.z = z;
     prm.A = A; prm.D = D; prm.bias = delta_bias; prm.out = out;
-    prm.batch = d.batch; prm.dim = d.dim; prm.nheads = d.nheads; prm.ngroups = d.ngroups;
+    prm.batch = d.batch;
+    prm.dim = (uint32_t)d.dim; prm.nheads = (uint32_t)d.nheads; prm.ngroups = (uint32_t)d.ngroups;
+    prm.head_dim = (uint32_t)(d.dim / d.nheads); prm.group_dim = (uint32_t)(d.dim / d.ngroups);
     prm.softplus = softplus ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return d.io_dtype == SSM_BF16 ? launch<__nv_bfloat16>(prm, N, s) : launch<float>(prm, N, s);

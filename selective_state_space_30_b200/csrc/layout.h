@@ -35,14 +35,15 @@ inline int64_t layout_tiles(const ssm_dims_t& d, int ct) {
 // The first layout in order of preference that gives every SM a channel tile,
 // else the one with the most tiles.  A segment of a tile runs after the
 // previous one, so tiles are the parallelism.  The kernel is latency-bound, so
-// the order prefers more consumer warps per SM sub-partition (16, then 8, then
-// 4) and, at equal warps, more states per lane (fewer instructions per state
-// update).  Measured on B200 with N = 16: 16 warps x 2 states beat 8 x 4 by
-// about 5 %, and 8 x 4 beat 4 x 4 by about 30 %.  force_w / force_spl (0 =
+// the order prefers many consumer warps per SM sub-partition and, among those,
+// more states per lane (fewer instructions per state update).  Measured on B200
+// with N = 16: 12 warps x 4 states beat 16 x 2 by about 7 % where they fill the
+// SMs (4 x 4096 channels), 16 x 2 beat 8 x 4 by about 5 %, and 8 x 4 beat 4 x 4
+// by about 30 %.  force_w / force_spl (0 =
 // free) restrict the candidates; false: no variant fits them.
 inline bool choose_layout(const ssm_dims_t& d, int sm_count, int force_w, int force_spl, Layout* out) {
     const bool head = d.nheads != d.dim;
-    static const int order[][2] = {{16, 2}, {8, 16}, {8, 8}, {8, 4}, {8, 2}, {4, 16}, {4, 8}, {4, 4}, {4, 2}};
+    static const int order[][2] = {{12, 4}, {16, 2}, {8, 16}, {8, 8}, {8, 4}, {8, 2}, {4, 16}, {4, 8}, {4, 4}, {4, 2}};
     bool found = false;
     Layout best{};
     int64_t best_tiles = -1;

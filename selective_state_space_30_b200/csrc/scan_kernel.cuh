@@ -145,28 +145,39 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
 
 __device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
 
-// softplus on a pair: max(x,0) + e*q(e), e = 2^(-|x| log2 e) in (0, 1], q a degree-7
-// polynomial fitted to log1p(e)/e on [0, 1] (max relative error about 3.3e-7).
+// softplus(x) = max(x,0) + e*q(e), e = 2^(-|x| log2 e) in (0, 1], q a degree-7
+// polynomial fitted to log1p(e)/e on [0, 1] (max relative error about 3.3e-7);
+// coefficients from the highest degree down.
+__device__ constexpr float kSoftplusQ[8] = {-0.008539234288036823f, 0.044089723378419876f, -0.10768184065818787f,
+                                            0.17745250463485718f,   -0.2449546605348587f,  0.33275479078292847f,
+                                            -0.4999740421772003f,   0.9999998211860657f};
+
+// softplus on a pair
 __device__ __forceinline__ float2 softplus2(float2 x) {
     const float2 a = mul2(make_float2(fabsf(x.x), fabsf(x.y)), dup2(-kLog2e));
     const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-    float2 q = dup2(-0.008539234288036823f);
-    q = fma2(q, e, dup2(0.044089723378419876f));
-    q = fma2(q, e, dup2(-0.10768184065818787f));
-    q = fma2(q, e, dup2(0.17745250463485718f));
-    q = fma2(q, e, dup2(-0.2449546605348587f));
-    q = fma2(q, e, dup2(0.33275479078292847f));
-    q = fma2(q, e, dup2(-0.4999740421772003f));
-    q = fma2(q, e, dup2(0.9999998211860657f));
+    float2 q = dup2(kSoftplusQ[0]);
+#pragma unroll
+    for (int i = 1; i < 8; ++i) q = fma2(q, e, dup2(kSoftplusQ[i]));
     return fma2(e, q, make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)));
 }
 
-// silu(z) = z / (1 + e^-z) on a pair
+__device__ __forceinline__ float softplus1(float x) {
+    const float e = ex2_approx(fabsf(x) * -kLog2e);
+    float q = kSoftplusQ[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) q = fmaf(q, e, kSoftplusQ[i]);
+    return fmaf(e, q, fmaxf(x, 0.f));
+}
+
+// silu(z) = z / (1 + e^-z) on a pair, and on one value
 __device__ __forceinline__ float2 silu2(float2 z) {
     const float2 a = mul2(z, dup2(-kLog2e));
     const float2 d = add2(make_float2(ex2_approx(a.x), ex2_approx(a.y)), dup2(1.f));
     return mul2(z, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
 }
+
+__device__ __forceinline__ float silu1(float z) { return z * rcp_approx(ex2_approx(z * -kLog2e) + 1.f); }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     unsigned v;
@@ -1000,10 +1011,13 @@ Variant make_variant(const char* name) {
 }
 
 // The lane layouts compiled for a state size N: (consumer warps W, states per lane S).
-//   N <= 16: (16, 2), (8, 4), (8, 2), (4, 4), (4, 2);  N = 32: (8, 4), (4, 4);
+//   N <= 16: (16, 2), (8, 4), (8, 2), (4, 4), (4, 2), and (12, 4) for N = 16;
+//   N = 32: (8, 4), (4, 4);
 //   N >= 64: (8, N/8), (4, N/8).
 constexpr bool layout_exists(int N, int w, int spl) {
-    if (N <= 16) return (w == 16 && spl == 2) || ((w == 8 || w == 4) && (spl == 2 || spl == 4));
+    if (N <= 16)
+        return (w == 16 && spl == 2) || (N == 16 && w == 12 && spl == 4) ||
+               ((w == 8 || w == 4) && (spl == 2 || spl == 4));
     if (N == 32) return (w == 8 || w == 4) && spl == 4;
     return (w == 8 || w == 4) && spl == N / 8;
 }
@@ -1025,6 +1039,7 @@ constexpr bool layout_exists(int N, int w, int spl) {
 #define SSM_DEFINE_PICK(T, TN, N)                                                                         \
     bool pick_##TN##_n##N(bool head, bool vec, int w, int spl, Variant* v) {                             \
         SSM_PICK_ONE(T, TN, N, 16, 2)                                                                    \
+        SSM_PICK_ONE(T, TN, N, 12, 4)                                                                    \
         SSM_PICK_ONE(T, TN, N, 8, 2)                                                                     \
         SSM_PICK_ONE(T, TN, N, 8, 4)                                                                     \
         SSM_PICK_ONE(T, TN, N, 4, 2)                                                                     \

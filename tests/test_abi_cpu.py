@@ -94,6 +94,18 @@ def test_state_update_host_checks(lib):
     assert f(ctypes.byref(ssm.make_dims(0, 64, 1, 16, 64, 1, ssm.SSM_BF16)), *args(None)) == ssm.SSM_OK
 
 
+def test_conv1d_host_checks(lib):
+    """ssm_causal_conv1d_fwd rejects bad arguments before touching the GPU."""
+    import selective_state_space_30_b200 as ssm
+    a = 0x10000
+    f = lib.ssm_causal_conv1d_fwd
+    assert f(1, 4, 16, 5, ssm.SSM_F32, a, a, None, 1, a, None) == ssm.SSM_ERR_UNSUPPORTED
+    assert f(1, 4, 16, 4, 9, a, a, None, 1, a, None) == ssm.SSM_ERR_INVALID_ARG
+    assert f(1, 0, 16, 4, ssm.SSM_F32, a, a, None, 1, a, None) == ssm.SSM_ERR_INVALID_ARG
+    assert f(1, 4, 16, 4, ssm.SSM_F32, None, a, None, 1, a, None) == ssm.SSM_ERR_INVALID_ARG
+    assert f(0, 4, 16, 4, ssm.SSM_F32, None, None, None, 1, None, None) == ssm.SSM_OK
+
+
 def test_plan_without_a_gpu_reports_cuda_error(lib):
     import torch
     import selective_state_space_30_b200 as ssm

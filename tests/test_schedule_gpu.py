@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import ssm_inputs as si
-from parity import check_out, check_state, run_gpu, to_host_f64
+from parity import OPTION_CODES, check_out, check_state, run_gpu, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -24,6 +24,7 @@ SCHEDULES = [dict(seg_len=32), dict(seg_len=64, warps=4), dict(seg_len=96, warps
 # per-state arithmetic, so the results stay bit-identical
 SCHEDULES_SMALL_N = [dict(warps=16, states_per_lane=2), dict(warps=8, states_per_lane=2, seg_len=64, ctas=3),
                      dict(warps=4, states_per_lane=2), dict(warps=16, states_per_lane=2, seg_len=32, ctas=1)]
+SCHEDULES_N16 = [dict(warps=12, states_per_lane=4), dict(warps=12, states_per_lane=4, seg_len=32, ctas=2)]
 
 
 def _recipe(d):
@@ -32,17 +33,39 @@ def _recipe(d):
     return si.Recipe(d_init="normal", delta_init="normal_half")
 
 
+def _states_per_lane(plan_variant: str) -> int:
+    """S of a variant name ws_<dtype>_n<N>_w<W>s<S>..."""
+    return int(plan_variant.split("_")[3].split("s")[1])
+
+
 @pytest.mark.parametrize("dims", SHAPES, ids=lambda d: f"{d.batch}x{d.dim}x{d.seqlen}x{d.dstate}h{d.H}g{d.ngroups}{d.dtype}")
 def test_schedule_invariance(dims):
+    """Every schedule agrees with the oracle; schedules with the same states per lane run
+    the same fp32 operations in the same order (segments and blocks are 32-step aligned),
+    so their results are bit-identical."""
+    import selective_state_space_30_b200 as ssm
     inp = si.make_inputs(dims, _recipe(dims), 11)
-    ref_out, ref_last = run_gpu(dims, inp)
     ro, rl, rm = oracle.run_inputs(dims, inp)
-    check_out(to_host_f64(ref_out), ro, rm, dims.dtype)
-    check_state(to_host_f64(ref_last), rl)
-    scheds = SCHEDULES + (SCHEDULES_SMALL_N if dims.dstate <= 16 else [])
+    scheds = [None] + SCHEDULES + (SCHEDULES_SMALL_N if dims.dstate <= 16 else []) + \
+        (SCHEDULES_N16 if dims.dstate == 16 else [])
+    io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
+    refs = {}
     for opts in scheds:
+        d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, io)
+        plan = ssm.ssm_scan_plan(d, 0)
+        try:
+            for k, v in (opts or {}).items():
+                ssm.ssm_scan_set_option(plan, OPTION_CODES[k], v)
+            spl = _states_per_lane(ssm.ssm_scan_plan_info(plan)["variant"])
+        finally:
+            ssm.ssm_scan_destroy(plan)
         out, last = run_gpu(dims, inp, opts=opts)
-        # segments and blocks are 32-step aligned: the same fp32 operations in the same order
+        if spl not in refs:
+            check_out(to_host_f64(out), ro, rm, dims.dtype)
+            check_state(to_host_f64(last), rl)
+            refs[spl] = (out, last)
+            continue
+        ref_out, ref_last = refs[spl]
         assert torch.equal(out, ref_out), f"output differs under schedule {opts}"
         assert torch.equal(last, ref_last), f"last_state differs under schedule {opts}"
 
@@ -117,12 +140,19 @@ def test_layout_option_checks():
     try:
         assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w16s2_vec"
         assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_STATES_PER_LANE, 3) == ssm.SSM_ERR_INVALID_ARG
-        assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_CONSUMER_WARPS, 12) == ssm.SSM_ERR_INVALID_ARG
+        assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_CONSUMER_WARPS, 6) == ssm.SSM_ERR_INVALID_ARG
         assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_STATES_PER_LANE, 4) == ssm.SSM_OK
         assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w8s4_vec"
         # sixteen warps exist only with two states per lane: refused, previous schedule kept
         assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_CONSUMER_WARPS, 16) == ssm.SSM_ERR_UNSUPPORTED
         assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w8s4_vec"
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    # 4 x 4096 channels: twelve warps with four states per lane still fill the SMs
+    d = ssm.make_dims(4, 4096, 256, 16, 4096, 1, ssm.SSM_BF16)
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        assert ssm.ssm_scan_plan_info(plan)["variant"] == "ws_bf16_n16_w12s4_vec"
     finally:
         ssm.ssm_scan_destroy(plan)
     # 1 x 5120 channels: eight warps with two states per lane keep a tile per SM

@@ -130,8 +130,8 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
                                 void* out, float* last_state, ssm_stream_t stream);
 
 /*
- * Plan options (mostly for tests).  Changing SEG_LEN, CONSUMER_WARPS, WORKERS or
- * STATES_PER_LANE re-plans the schedule (synchronises the device).
+ * Plan options (mostly for tests).  Changing SEG_LEN, CONSUMER_WARPS, WORKERS,
+ * STATES_PER_LANE or SSD re-plans the schedule (synchronises the device).
  *   SSM_OPT_SPIN_LIMIT         polls a chained wait makes before it gives up and
  *                              records SSM_ERR_TIMEOUT (default about 2M, i.e. ~1 s)
  *   SSM_OPT_INJECT_STALL       test hook, nonzero: every chained wait waits for a
@@ -149,6 +149,11 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
  *                              combination with CONSUMER_WARPS that no kernel has makes
  *                              the call return SSM_ERR_UNSUPPORTED and keeps the
  *                              previous setting.
+ *   SSM_OPT_SSD                the chunked tensor-core (state-space-dual) path for bf16
+ *                              I/O, nheads < dim with dim/nheads == 64, dstate 128 and
+ *                              seqlen a multiple of 128: 0 = use it where it applies
+ *                              (automatic), 1 = never (the scan kernel), 2 = required
+ *                              (SSM_ERR_UNSUPPORTED for a shape it does not cover)
  * Returns SSM_ERR_INVALID_ARG for an unknown option or a bad value.
  */
 typedef enum {
@@ -157,7 +162,8 @@ typedef enum {
     SSM_OPT_SEG_LEN = 3,
     SSM_OPT_CONSUMER_WARPS = 4,
     SSM_OPT_WORKERS = 5,
-    SSM_OPT_STATES_PER_LANE = 6
+    SSM_OPT_STATES_PER_LANE = 6,
+    SSM_OPT_SSD = 7
 } ssm_option_t;
 int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value);
 

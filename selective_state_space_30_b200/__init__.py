@@ -17,7 +17,7 @@ from typing import Dict, Optional, Tuple
 from . import _abi
 from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, SSM_ERR_TIMEOUT,  # noqa: F401
                    SSM_ERR_UNSUPPORTED, SSM_F32, SSM_OK, SSM_OPT_CONSUMER_WARPS, SSM_OPT_INJECT_STALL,
-                   SSM_OPT_SEG_LEN, SSM_OPT_SPIN_LIMIT, SSM_OPT_STATES_PER_LANE, SSM_OPT_WORKERS,
+                   SSM_OPT_SEG_LEN, SSM_OPT_SPIN_LIMIT, SSM_OPT_SSD, SSM_OPT_STATES_PER_LANE, SSM_OPT_WORKERS,
                    SsmError, load_library, make_dims,
                    ssm_dims_t, ssm_probe_ex2, ssm_scan_destroy, ssm_scan_device_status, ssm_scan_plan,
                    ssm_scan_plan_info, ssm_scan_plan_schedule, ssm_scan_set_option, ssm_selective_scan_fwd,

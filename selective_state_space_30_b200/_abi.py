@@ -37,6 +37,7 @@ SSM_OPT_SEG_LEN = 3
 SSM_OPT_CONSUMER_WARPS = 4
 SSM_OPT_WORKERS = 5
 SSM_OPT_STATES_PER_LANE = 6
+SSM_OPT_SSD = 7
 
 
 class SsmError(RuntimeError):

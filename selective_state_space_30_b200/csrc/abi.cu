@@ -9,6 +9,7 @@
 #include <new>
 
 #include "layout.h"
+#include "ssd.h"
 #include "scan_kernel.cuh"
 #include "ssm_scan.h"
 
@@ -41,6 +42,7 @@ struct ssm_plan_s {
     // schedule
     int w;                 // consumer warps per CTA
     int spl;               // states per lane
+    bool ssd;              // the chunked tensor-core path (per-head layout, dstate 128, head dim 64)
     int threads;
     int ch_per_tile;
     int smem;
@@ -50,7 +52,7 @@ struct ssm_plan_s {
     const char* name;
     // options
     unsigned spin_limit;
-    int64_t force_seg_len, force_w, force_spl, force_workers;
+    int64_t force_seg_len, force_w, force_spl, force_ssd, force_workers;
     // workspace: header | flags[n_tiles] | carry[n_tiles][CW][N]
     unsigned char* ws;
     size_t ws_bytes, flags_off, carry_off;
@@ -121,6 +123,9 @@ int schedule(ssm_plan_s* p) {
     if (n_units >= (int64_t)1 << 31 || seg_len > (int64_t)1 << 30) return SSM_ERR_UNSUPPORTED;
     if (ctas > n_units) ctas = n_units;
     if (ctas < 1) ctas = 1;
+    const bool ssd_ok = ssm::ssd_eligible(d);
+    if (p->force_ssd == 2 && !ssd_ok) return SSM_ERR_UNSUPPORTED;
+    p->ssd = ssd_ok && p->force_ssd != 1;
     p->w = w;
     p->spl = lay.spl;
     p->threads = v.threads;
@@ -176,12 +181,12 @@ EncodeTiledFn tensor_map_encoder() {
 
 // A (rows x cols) row-major tensor seen as 2-D boxes of 32 steps x box_rows rows.
 bool encode_rows(CUtensorMap* m, const void* base, int esz, uint64_t cols, uint64_t rows, uint32_t box_rows,
-                 CUtensorMapSwizzle swz) {
+                 CUtensorMapSwizzle swz, uint32_t box_cols = ssm::kTB) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc || cols == 0 || rows == 0) return false;
     const cuuint64_t gdim[2] = {cols, rows};
     const cuuint64_t gstride[1] = {cols * (uint64_t)esz};
-    const cuuint32_t box[2] = {(cuuint32_t)ssm::kTB, box_rows};
+    const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t es[2] = {1, 1};
     return enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                const_cast<void*>(base), gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
@@ -193,6 +198,30 @@ int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A
                float* last_state, cudaStream_t stream) {
     const ssm_dims_t& d = plan->dims;
     if (d.batch == 0) return SSM_OK;
+    if (plan->ssd) {
+        // the chunked tensor-core path: 16-byte aligned TMA sources, 8-byte aligned delta rows
+        ssm::SsdMaps maps;
+        std::memset(&maps, 0, sizeof(maps));
+        const uint64_t L = (uint64_t)d.seqlen;
+        const bool ok = aligned16(u) && aligned16(B) && aligned16(C) && (reinterpret_cast<uintptr_t>(delta) & 7u) == 0 &&
+                        encode_rows(&maps.u, u, 2, L, (uint64_t)(d.batch * d.dim), 64, CU_TENSOR_MAP_SWIZZLE_128B, 64) &&
+                        encode_rows(&maps.B, B, 2, L, (uint64_t)(d.batch * d.ngroups * d.dstate), 128,
+                                    CU_TENSOR_MAP_SWIZZLE_128B, 64) &&
+                        encode_rows(&maps.C, C, 2, L, (uint64_t)(d.batch * d.ngroups * d.dstate), 128,
+                                    CU_TENSOR_MAP_SWIZZLE_128B, 64);
+        if (ok) {
+            ssm::SsdParams sp;
+            sp.delta = static_cast<const __nv_bfloat16*>(delta); sp.A = A; sp.D = D; sp.bias = delta_bias;
+            sp.z = static_cast<const __nv_bfloat16*>(z); sp.h0 = h0;
+            sp.out = static_cast<__nv_bfloat16*>(out); sp.last_state = last_state;
+            sp.status = &reinterpret_cast<ssm::WsHeader*>(plan->ws)->status;
+            sp.batch = d.batch; sp.dim = d.dim; sp.seqlen = d.seqlen; sp.nheads = d.nheads; sp.ngroups = d.ngroups;
+            sp.softplus = softplus ? 1 : 0;
+            sp.spin_limit = plan->spin_limit;
+            return ssm::ssd_launch(sp, maps, d.batch * d.nheads, stream);
+        }
+        // an unaligned call takes the scan kernel below
+    }
     // Vector loads/stores need every per-lane chunk (up to 16 elements) wholly
     // inside or outside a row and 16-byte aligned: L % 16 == 0 plus aligned bases.
     bool vec = d.seqlen > 0 && (d.seqlen % 16 == 0) && aligned16(u) && aligned16(delta) && aligned16(B) &&
@@ -308,7 +337,8 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
         case SSM_OPT_SEG_LEN:
         case SSM_OPT_CONSUMER_WARPS:
         case SSM_OPT_WORKERS:
-        case SSM_OPT_STATES_PER_LANE: {
+        case SSM_OPT_STATES_PER_LANE:
+        case SSM_OPT_SSD: {
             if (value < 0) return SSM_ERR_INVALID_ARG;
             if (option == SSM_OPT_CONSUMER_WARPS && value != 0 && value != 4 && value != 8 && value != 12 &&
                 value != 16)
@@ -316,6 +346,7 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
             if (option == SSM_OPT_STATES_PER_LANE && value != 0 && value != 2 && value != 4 && value != 8 &&
                 value != 16)
                 return SSM_ERR_INVALID_ARG;
+            if (option == SSM_OPT_SSD && value > 2) return SSM_ERR_INVALID_ARG;
             if (cudaDeviceSynchronize() != cudaSuccess) return SSM_ERR_CUDA;
             unsigned inject = 0;
             if (cudaMemcpy(&inject, plan->ws + offsetof(ssm::WsHeader, inject), sizeof(inject),
@@ -324,6 +355,7 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
             int64_t* field = option == SSM_OPT_SEG_LEN         ? &plan->force_seg_len
                              : option == SSM_OPT_CONSUMER_WARPS ? &plan->force_w
                              : option == SSM_OPT_STATES_PER_LANE ? &plan->force_spl
+                             : option == SSM_OPT_SSD            ? &plan->force_ssd
                                                                  : &plan->force_workers;
             const int64_t old = *field;
             *field = value;
@@ -443,11 +475,12 @@ int ssm_scan_device_status(ssm_plan_t plan, ssm_stream_t stream) {
 int ssm_scan_plan_info(ssm_plan_t plan, int* grid, int* block, int* smem_bytes, int* launches_per_call,
                        const char** variant) {
     if (!plan_ok(plan)) return SSM_ERR_INVALID_ARG;
-    if (grid) *grid = plan->grid;
-    if (block) *block = plan->threads;
-    if (smem_bytes) *smem_bytes = plan->smem;
+    const bool ssd = plan->ssd;
+    if (grid) *grid = ssd ? (int)(plan->dims.batch * plan->dims.nheads) : plan->grid;
+    if (block) *block = ssd ? 256 : plan->threads;
+    if (smem_bytes) *smem_bytes = ssd ? ssm::ssd_smem_bytes() : plan->smem;
     if (launches_per_call) *launches_per_call = plan->dims.batch > 0 ? 1 : 0;
-    if (variant) *variant = plan->name;
+    if (variant) *variant = ssd ? "ssd_bf16_n128_p64_q128" : plan->name;
     return SSM_OK;
 }
 

@@ -5,10 +5,10 @@
 //
 //   out[b,d,t] = act(bias[d] + sum_{k<width} w[d,k] * x[b,d,t-width+1+k]),  x = 0 before t = 0
 //
-// HBM-bound: each element is read and written once.  A thread owns one
-// 16-byte chunk of a row (8 bf16 or 4 fp32 steps) and also reads the chunk
-// before it for the width-1 earlier steps; consecutive threads take
-// consecutive chunks of a row, so a warp reads and writes 512 contiguous bytes.
+// HBM-bound: each element is read and written once.  The row is cut into
+// 16-byte chunks (8 bf16 or 4 fp32 steps); a lane computes four chunks, 32
+// chunks apart, reading for each also the chunk before it for the width-1
+// earlier steps.
 // Rows whose length or base is not 16-byte aligned take a one-step-per-thread
 // path with the same arithmetic.
 #include <cuda_bf16.h>
@@ -81,47 +81,62 @@ __device__ __forceinline__ void taps(const ConvParams& p, int64_t d, float (&w)[
     b = p.bias ? __ldg(p.bias + d) : 0.f;
 }
 
-// 16-byte chunks: chunk c of row r covers steps [c*V, c*V + V); W (the width) is a
-// template parameter so every tap index is known at compile time
+// 16-byte chunks: chunk c of row r covers steps [c*V, c*V + V).  A warp owns a
+// tile of 32*CPC consecutive chunks of a row; lane l takes chunks l, l+32, ...,
+// so every load and store instruction of the warp covers 512 contiguous bytes.
+// Each chunk also needs the chunk before it for the earlier taps (mostly an L1
+// hit: it is the neighbour lane's chunk).  All loads are issued first.  W (the
+// width) is a template parameter so every tap index is known at compile time.
+constexpr int kCPC = 4;   // chunks per lane
+
 template <typename T, int W>
 __global__ void __launch_bounds__(kThreads) conv1d_vec_kernel(const ConvParams p) {
     using E = Elem<T>;
     constexpr int V = E::V;
     static_assert(W - 1 <= V, "the earlier steps fit in the previous chunk");
     const int64_t chunks = p.seqlen / V;
-    const int64_t g = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (g >= p.rows * chunks) return;
-    const int64_t r = g / chunks, c = g % chunks;
+    const int64_t tiles = (chunks + 32 * kCPC - 1) / (32 * kCPC);   // warp tiles per row
+    const int64_t wid = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= p.rows * tiles) return;
+    const int64_t r = wid / tiles, c0 = (wid % tiles) * (32 * kCPC) + lane;
     float w[W], b;
     taps<W>(p, r % p.dim, w, b);
     const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const char*>(p.x) + r * p.seqlen * sizeof(T));
-    // steps c*V - V .. c*V + V - 1 of the row (zero before t = 0)
-    float xv[2 * V];
-    {
-        float cur[V], prev[V];
-        E::unpack(__ldg(xr + c), cur);
-        if (c > 0) {
-            E::unpack(__ldg(xr + c - 1), prev);
-        } else {
+    uint4* orow = reinterpret_cast<uint4*>(static_cast<char*>(p.out) + r * p.seqlen * sizeof(T));
+    uint4 cur_raw[kCPC], prev_raw[kCPC];
 #pragma unroll
-            for (int i = 0; i < V; ++i) prev[i] = 0.f;
+    for (int q = 0; q < kCPC; ++q) {
+        const int64_t c = c0 + 32 * q;
+        const bool in = c < chunks;
+        cur_raw[q] = in ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+        prev_raw[q] = in && c > 0 ? __ldg(xr + c - 1) : make_uint4(0u, 0u, 0u, 0u);   // zero bits are 0.0
+    }
+#pragma unroll
+    for (int q = 0; q < kCPC; ++q) {
+        const int64_t c = c0 + 32 * q;
+        // steps of the previous chunk, then this one
+        float xv[2 * V];
+        {
+            float prev[V], cur[V];
+            E::unpack(prev_raw[q], prev);
+            E::unpack(cur_raw[q], cur);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                xv[i] = prev[i];
+                xv[V + i] = cur[i];
+            }
         }
+        float o[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            xv[i] = prev[i];
-            xv[V + i] = cur[i];
+            float v = b;
+#pragma unroll
+            for (int k = 0; k < W; ++k) v = fmaf(w[k], xv[V + i - (W - 1) + k], v);
+            o[i] = p.silu ? ssm::silu1(v) : v;
         }
+        if (c < chunks) orow[c] = E::pack(o);
     }
-    float o[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) {
-        float v = b;
-#pragma unroll
-        for (int k = 0; k < W; ++k) v = fmaf(w[k], xv[V + i - (W - 1) + k], v);
-        o[i] = p.silu ? ssm::silu1(v) : v;
-    }
-    uint4* orow = reinterpret_cast<uint4*>(static_cast<char*>(p.out) + r * p.seqlen * sizeof(T));
-    orow[c] = E::pack(o);
 }
 
 // one step per thread
@@ -144,7 +159,9 @@ __global__ void __launch_bounds__(kThreads) conv1d_scalar_kernel(const ConvParam
 
 template <typename T, int W>
 int launch_w(const ConvParams& p, bool vec, cudaStream_t s) {
-    const int64_t work = vec ? p.rows * (p.seqlen / Elem<T>::V) : p.rows * p.seqlen;
+    // vector path: one warp per tile of 32*kCPC chunks
+    const int64_t work = vec ? p.rows * ((p.seqlen / Elem<T>::V + 32 * kCPC - 1) / (32 * kCPC)) * 32
+                             : p.rows * p.seqlen;
     const int64_t blocks = (work + kThreads - 1) / kThreads;
     if (blocks == 0) return SSM_OK;
     if (blocks > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;

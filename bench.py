@@ -106,6 +106,28 @@ def _peaks():
     return 6650.0, NOMINAL_SM_MHZ, "fallback"
 
 
+def _bf16_tflops():
+    """Measured dense bf16 rate (burst: the kernel is timed in isolation), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f).get("bf16_tflops", 1590.0)), "measured"
+    return 1590.0, "fallback"
+
+
+SSD_Q = 128   # steps per chunk of the tensor-core (SSD) path
+
+
+def _ssd_flops(d):
+    """Algorithmic tensor-core flops of the chunked SSD path per call: per (batch row, head,
+    chunk) G = C B^T (2 Q Q N), M X (2 Q Q P), C H (2 Q N P), B'^T X (2 N Q P).  The bf16
+    hi/lo splits of M, B' and H double the executed MMAs of the last three; not counted."""
+    P = d.dim // d.H
+    N = d.dstate
+    per = 2 * SSD_Q * (SSD_Q * N + SSD_Q * P + N * P + N * P)
+    return d.batch * d.H * (d.seqlen // SSD_Q) * per
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -371,16 +393,31 @@ def run_ours(args):
     probe_rate = SMS * 8 * 256 * 2048 * 16 / (pe0.elapsed_time(pe1) * 1e-3)
     t_roof = max(alg_bytes / (hbm_gbs * 1e9), exps / mufu_peak)
     traffic = _traffic_from_profiles(w.name)
-    roof = {"bound": "alu", "achieved": exps / avg_launch_s / 1e9, "peak": mufu_peak / 1e9, "unit": "Gexp/s",
-            "frac": (exps / avg_launch_s) / mufu_peak, "traffic": traffic,
-            "what": "MUFU ex2: B*D*L*N exps per launch / mean launch time; peak = 148 SM x 16 ex2/clk x "
-                    f"{sm_max_mhz:.0f} MHz (derived)",
-            "roofline_frac": t_roof / avg_launch_s,
-            "hbm": {"achieved": alg_bytes / avg_launch_s / 1e9, "peak": hbm_gbs, "unit": "GB/s",
-                    "frac": alg_bytes / avg_launch_s / 1e9 / hbm_gbs, "peak_source": peak_src,
-                    "alg_bytes_per_launch": alg_bytes},
-            "mufu_probe_gexps": probe_rate / 1e9,
-            "frac_of_probe": (exps / avg_launch_s) / probe_rate}
+    hbm_obj = {"achieved": alg_bytes / avg_launch_s / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+               "frac": alg_bytes / avg_launch_s / 1e9 / hbm_gbs, "peak_source": peak_src,
+               "alg_bytes_per_launch": alg_bytes}
+    mufu_obj = {"achieved": exps / avg_launch_s / 1e9, "peak": mufu_peak / 1e9, "unit": "Gexp/s",
+                "frac": (exps / avg_launch_s) / mufu_peak,
+                "what": "MUFU ex2: B*D*L*N exps per launch / mean launch time; peak = 148 SM x 16 ex2/clk x "
+                        f"{sm_max_mhz:.0f} MHz (derived)",
+                "mufu_probe_gexps": probe_rate / 1e9, "frac_of_probe": (exps / avg_launch_s) / probe_rate}
+    if info["variant"].startswith("ssd_"):
+        # the chunked tensor-core path: the bound is the slower of HBM bytes and tensor flops
+        tf, tf_src = _bf16_tflops()
+        flops = _ssd_flops(d)
+        t_hbm, t_tc = alg_bytes / (hbm_gbs * 1e9), flops / (tf * 1e12)
+        tensor_obj = {"achieved": flops / avg_launch_s / 1e12, "peak": tf, "unit": "TFLOP/s",
+                      "frac": flops / avg_launch_s / 1e12 / tf, "peak_source": tf_src,
+                      "flops_per_launch": flops, "what": "algorithmic SSD flops (G, M X, C H, B'^T X per chunk)"}
+        main = dict(hbm_obj, bound="hbm") if t_hbm >= t_tc else dict(tensor_obj, bound="tensor")
+        roof = dict(main, traffic=traffic, roofline_frac=max(t_hbm, t_tc) / avg_launch_s,
+                    hbm=hbm_obj, tensor=tensor_obj,
+                    mufu_literal=dict(mufu_obj, note="B*D*L*N exps: the SSD path takes one exp per (t, head)"))
+    else:
+        roof = {"bound": "alu", "achieved": mufu_obj["achieved"], "peak": mufu_obj["peak"], "unit": "Gexp/s",
+                "frac": mufu_obj["frac"], "traffic": traffic, "what": mufu_obj["what"],
+                "roofline_frac": t_roof / avg_launch_s, "hbm": hbm_obj,
+                "mufu_probe_gexps": mufu_obj["mufu_probe_gexps"], "frac_of_probe": mufu_obj["frac_of_probe"]}
 
     # end to end through the host-buffer entry point: pinned host inputs, copies in the timed region
     e2e = None

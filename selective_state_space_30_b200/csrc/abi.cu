@@ -203,8 +203,11 @@ int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A
         ssm::SsdMaps maps;
         std::memset(&maps, 0, sizeof(maps));
         const uint64_t L = (uint64_t)d.seqlen;
-        const bool ok = aligned16(u) && aligned16(B) && aligned16(C) && (reinterpret_cast<uintptr_t>(delta) & 7u) == 0 &&
+        const bool ok = aligned16(u) && aligned16(B) && aligned16(C) && (!z || aligned16(z)) &&
+                        (reinterpret_cast<uintptr_t>(delta) & 7u) == 0 &&
                         encode_rows(&maps.u, u, 2, L, (uint64_t)(d.batch * d.dim), 64, CU_TENSOR_MAP_SWIZZLE_128B, 64) &&
+                        (!z || encode_rows(&maps.z, z, 2, L, (uint64_t)(d.batch * d.dim), 64,
+                                           CU_TENSOR_MAP_SWIZZLE_128B, 64)) &&
                         encode_rows(&maps.B, B, 2, L, (uint64_t)(d.batch * d.ngroups * d.dstate), 128,
                                     CU_TENSOR_MAP_SWIZZLE_128B, 64) &&
                         encode_rows(&maps.C, C, 2, L, (uint64_t)(d.batch * d.ngroups * d.dstate), 128,
@@ -477,7 +480,7 @@ int ssm_scan_plan_info(ssm_plan_t plan, int* grid, int* block, int* smem_bytes, 
     if (!plan_ok(plan)) return SSM_ERR_INVALID_ARG;
     const bool ssd = plan->ssd;
     if (grid) *grid = ssd ? (int)(plan->dims.batch * plan->dims.nheads) : plan->grid;
-    if (block) *block = ssd ? 256 : plan->threads;
+    if (block) *block = ssd ? 512 : plan->threads;
     if (smem_bytes) *smem_bytes = ssd ? ssm::ssd_smem_bytes() : plan->smem;
     if (launches_per_call) *launches_per_call = plan->dims.batch > 0 ? 1 : 0;
     if (variant) *variant = ssd ? "ssd_bf16_n128_p64_q128" : plan->name;

@@ -27,15 +27,16 @@ struct SsdParams {
 };
 
 // 2-D tensor maps (time x rows), 64-step boxes with the 128-byte swizzle:
-// u rows (batch*dim) in boxes of 64 rows, B and C rows (batch*ngroups*dstate) in boxes of 128 rows.
+// u and z rows (batch*dim) in boxes of 64 rows, B and C rows (batch*ngroups*dstate) in
+// boxes of 128 rows; z is unused (and may be left zero) when there is no gate.
 struct SsdMaps {
-    CUtensorMap u, B, C;
+    CUtensorMap u, z, B, C;
 };
 
 // bf16 I/O, nheads < dim with dim/nheads == 64, dstate == 128, seqlen a positive multiple of 128.
 bool ssd_eligible(const ssm_dims_t& d);
 int ssd_smem_bytes();
-// one CTA of 256 threads per (batch row, head): grid = batch * nheads
+// one CTA of 512 threads per (batch row, head): grid = batch * nheads
 int ssd_launch(const SsdParams& prm, const SsdMaps& maps, int64_t grid, cudaStream_t s);
 
 }  // namespace ssm

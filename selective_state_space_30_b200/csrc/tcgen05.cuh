@@ -52,11 +52,22 @@ __device__ __forceinline__ void ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+// 16 consecutive 32-bit TMEM columns of this thread's lane
+__device__ __forceinline__ void ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// ties the registers of an ld32 to a preceding wait_ld (volatile asm statements keep their order)
-__device__ __forceinline__ void after_wait(uint32_t (&r)[32]) {
+// ties the registers of an ld32 / ld16 to a preceding wait_ld (volatile asm statements keep their order)
+template <int R>
+__device__ __forceinline__ void after_wait(uint32_t (&r)[R]) {
+    static_assert(R % 8 == 0, "groups of eight");
 #pragma unroll
-    for (int i = 0; i < 32; i += 8)
+    for (int i = 0; i < R; i += 8)
         asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
                      "+r"(r[i + 6]), "+r"(r[i + 7]));
 }

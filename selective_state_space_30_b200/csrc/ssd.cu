@@ -13,7 +13,7 @@
 //   M  = G o [2^(cum_i - cum_j) dt_j]_{j <= i}   (causal decay mask)  threads
 //   Y  = M X + diag(2^cum) (C H)                 (Q x P)              tensor cores
 //   out = (Y + D x) silu(z)                                           threads
-//   B' = B diag(2^(cum_end - cum_j) dt_j)                             threads
+//   B' = B diag(w),  w_j = 2^(cum_end - cum_j) dt_j                   threads
 //   H  = 2^cum_end H + B'^T X                    (N x P)              tensor cores + threads
 //
 // Operands the tensor cores read: B, C and X straight from TMA boxes (128-byte
@@ -53,8 +53,9 @@ constexpr int OFF_X = 64 * 1024;         // X (u rows of the head): 2 boxes x 64
 constexpr int OFF_MB = 80 * 1024;        // M, later B': hi (2 atom columns x 128 rows x 128 B), then lo
 constexpr int OFF_H = 144 * 1024;        // H: hi (128 rows x 128 B), then lo
 constexpr int OFF_Z = 176 * 1024;        // z (gate rows of the head): 2 boxes x 64 rows x 128 B
-constexpr int OFF_DT = 192 * 1024;       // two chunks' dt[128] and cum[128] floats
-constexpr int OFF_BAR = OFF_DT + 2048;   // barriers: full (C, B), full (X), g, y, s; TMEM base slot
+constexpr int OFF_DT = 192 * 1024;       // two chunks' dt[128], cum[128], w[128] floats
+constexpr int kDec = 3 * kQ;             // floats of one chunk's decay vectors
+constexpr int OFF_BAR = OFF_DT + 2 * kDec * 4;   // barriers: full (C, B), full (X), g, y, s; TMEM base slot
 constexpr int kSmemSsd = OFF_BAR + 128 + 1024;   // + slack to align the base up to 1024 bytes
 constexpr uint32_t kTxCB = 2 * 16384 + 2 * 16384;
 constexpr uint32_t kTxX = 2 * 8192;   // X, and as much again for z when there is a gate
@@ -81,10 +82,11 @@ __device__ __forceinline__ float bf16_at(const unsigned char* tile, uint32_t r, 
     return __bfloat162float(__ushort_as_bfloat16(*reinterpret_cast<const unsigned short*>(tile + tc::sw128_off(r, c))));
 }
 
-// dt and the decay prefix cum (log2 units) of the chunk starting at t0, four steps
-// per lane of one warp, into sdt / scum
+// The decay vectors of the chunk starting at t0, four steps per lane of one warp:
+// dt, the prefix cum (log2 units), and w = 2^(cum_end - cum) dt, the weight of each
+// step's input in the chunk's final state (at most dt, since cum only falls).
 __device__ __forceinline__ void chunk_decay(const SsdParams& p, int64_t b, int64_t h, int64_t t0, float Ah, float bias,
-                                            int lane, float* sdt, float* scum) {
+                                            int lane, float* sdt, float* scum, float* sw) {
     const unsigned short* drow =
         reinterpret_cast<const unsigned short*>(p.delta) + (b * p.nheads + h) * p.seqlen + t0 + 4 * lane;
     const uint2 raw = *reinterpret_cast<const uint2*>(drow);
@@ -105,9 +107,16 @@ __device__ __forceinline__ void chunk_decay(const SsdParams& p, int64_t b, int64
         if (lane >= o) incl += v;
     }
     const float base = incl - run;
+    const float cend = __shfl_sync(0xffffffffu, incl, 31);
+    float cm[4], wv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        cm[e] = base + pre[e];
+        wv[e] = ex2_approx(cend - cm[e]) * dt[e];
+    }
     *reinterpret_cast<float4*>(sdt + 4 * lane) = make_float4(dt[0], dt[1], dt[2], dt[3]);
-    *reinterpret_cast<float4*>(scum + 4 * lane) =
-        make_float4(base + pre[0], base + pre[1], base + pre[2], base + pre[3]);
+    *reinterpret_cast<float4*>(scum + 4 * lane) = make_float4(cm[0], cm[1], cm[2], cm[3]);
+    *reinterpret_cast<float4*>(sw + 4 * lane) = make_float4(wv[0], wv[1], wv[2], wv[3]);
 }
 
 // 8 consecutive floats from shared memory (16-byte aligned)
@@ -131,7 +140,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
     uint64_t* mb_y = bars + 3;
     uint64_t* mb_s = bars + 4;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 64);
-    float* sdec = reinterpret_cast<float*>(smem + OFF_DT);   // [2][dt[128], cum[128]]
+    float* sdec = reinterpret_cast<float*>(smem + OFF_DT);   // [2][dt[128], cum[128], w[128]]
     unsigned char* sC = smem + OFF_C;
     unsigned char* sB = smem + OFF_B;
     unsigned char* sX = smem + OFF_X;
@@ -182,7 +191,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             if (gate) tma_2d(sZ + hb * 8192, &m.z, 64 * hb, x_row, full_x);
         }
     }
-    if (warp == 0) chunk_decay(p, b, h, 0, Ah, bias, lane, sdec, sdec + kQ);
+    if (warp == 0) chunk_decay(p, b, h, 0, Ah, bias, lane, sdec, sdec + kQ, sdec + 2 * kQ);
 
     // the state: row n = row, channels p0 .. p0+15; skip weights of those channels
     float H[16], Dv[16];
@@ -211,8 +220,9 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
     for (int c = 0; c < nchunks; ++c) {
         const int64_t t0 = (int64_t)c * kQ;
         const unsigned ph = (unsigned)c & 1u;
-        const float* sdt = sdec + (c & 1) * 2 * kQ;
+        const float* sdt = sdec + (c & 1) * kDec;
         const float* scum = sdt + kQ;
+        const float* sw = sdt + 2 * kQ;
         const bool with_state = c > 0 || have_h0;
 
         // ---- G = C B^T once the chunk's C and B tiles are in
@@ -230,16 +240,23 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             last_ph = ph;
         }
         // meanwhile: the next chunk's decay, and this step's gate inputs
-        if (warp == 0 && c + 1 < nchunks)
-            chunk_decay(p, b, h, t0 + kQ, Ah, bias, lane, sdec + ((c + 1) & 1) * 2 * kQ,
-                        sdec + ((c + 1) & 1) * 2 * kQ + kQ);
+        if (warp == 0 && c + 1 < nchunks) {
+            float* nd = sdec + ((c + 1) & 1) * kDec;
+            chunk_decay(p, b, h, t0 + kQ, Ah, bias, lane, nd, nd + kQ, nd + 2 * kQ);
+        }
 
         const bool ok_g = mbar_wait(mb_g, ph, budget, p.status);
         if (__syncthreads_or(!ok_g)) { failed = true; break; }
         tc::fence_after();
 
-        // ---- M = G o decay mask: row i = row, steps j0 .. j0+31
-        {
+        // ---- M = G o decay mask: row i = row, steps j0 .. j0+31 (a warp whose steps all lie
+        // after its rows writes zeros: the causal mask)
+        if (j0 > (uint32_t)(32 * quarter + 31)) {
+            const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 32; k += 8)
+                store_pair8(sMhi + (j0 >> 6) * 16384, sMlo + (j0 >> 6) * 16384, row, (j0 & 63u) + k, zero8);
+        } else {
             uint32_t gv[32];
             tc::ld32(trow + kColG + j0, gv);
             const float ci = scum[row];
@@ -314,22 +331,20 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
                 p.out[(b * Dm + d0 + p0 + k) * L + t0 + row] = __float2bfloat16_rn(v);
             }
         }
-        // ---- B' = B diag(2^(cum_end - cum_j) dt_j): row n = row, steps j0 .. j0+31
+        // ---- B' = B diag(w): row n = row, steps j0 .. j0+31
         {
-            const float cend = scum[kQ - 1];
             const unsigned char* bt = sB + (j0 >> 6) * 16384;
 #pragma unroll
             for (int k = 0; k < 32; k += 8) {
-                float cj[8], dj[8];
-                lds8f(scum + j0 + k, cj);
-                lds8f(sdt + j0 + k, dj);
+                float wj[8];
+                lds8f(sw + j0 + k, wj);
                 const uint4 raw = *reinterpret_cast<const uint4*>(bt + tc::sw128_off(row, (j0 & 63u) + k));
                 const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
                 float v[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const uint32_t bits = (e & 1) ? (w4[e >> 1] & 0xFFFF0000u) : (w4[e >> 1] << 16);
-                    v[e] = __uint_as_float(bits) * ex2_approx(cend - cj[e]) * dj[e];
+                    v[e] = __uint_as_float(bits) * wj[e];
                 }
                 store_pair8(sMhi + (j0 >> 6) * 16384, sMlo + (j0 >> 6) * 16384, row, (j0 & 63u) + k, v);
             }

@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for the selective-SSM (S6) forward scan.
+"""fp64 CPU oracle for the selective-SSM (S6) forward scan, its gradient (the
+backward scan) and the causal convolution in front of it.
 
 TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
 baseline may import this package; the product path never does.  It shares no
@@ -29,6 +30,13 @@ class _Dims(ctypes.Structure):
                 ("dstate", ctypes.c_int64), ("nheads", ctypes.c_int64), ("ngroups", ctypes.c_int64)]
 
 
+GRAD_NAMES = ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias", "dh0")
+
+
+class _Grads(ctypes.Structure):
+    _fields_ = [(k, ctypes.POINTER(ctypes.c_double)) for k in GRAD_NAMES]
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle with plain gcc: fp64, no FMA contraction, no fast-math."""
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
@@ -47,6 +55,10 @@ def load(path: Optional[str] = None):
     lib.oracle_selective_scan_f64.argtypes = [
         ctypes.POINTER(_Dims), p, p, p, p, p, p, p, p, ctypes.c_int, p,
         ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, p, p, p, ctypes.c_int]
+    lib.oracle_selective_scan_bwd_f64.restype = ctypes.c_int
+    lib.oracle_selective_scan_bwd_f64.argtypes = [
+        ctypes.POINTER(_Dims), p, p, p, p, p, p, p, p, ctypes.c_int, p, p, p,
+        ctypes.POINTER(_Grads), ctypes.POINTER(_Grads), ctypes.c_int]
     i64 = ctypes.c_int64
     lib.oracle_causal_conv1d_f64.restype = ctypes.c_int
     lib.oracle_causal_conv1d_f64.argtypes = [i64, i64, i64, i64, p, p, p, ctypes.c_int, p]
@@ -170,3 +182,67 @@ def causal_conv1d(x, w, bias=None, silu: bool = True, lib=None) -> np.ndarray:
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out.reshape(batch, dim, seqlen)
+
+
+def selective_scan_bwd(batch: int, dim: int, seqlen: int, dstate: int, u, delta, A, B, C, dout, D=None, z=None,
+                       delta_bias=None, softplus: bool = True, nheads: int = 0, ngroups: int = 1, h0=None,
+                       dlast=None, want_dh0: bool = False, nthreads: Optional[int] = None, lib=None):
+    """Gradients of the forward scan (see `oracle_selective_scan_bwd_f64`) in fp64.
+
+    dout has out's shape (batch, dim, L); dlast (optional) last_state's (batch, dim, N).
+    Returns (grads, mags): dicts name -> float64 array over GRAD_NAMES, shaped
+    du, dz (batch, dim, L); ddelta (batch, nheads, L); dA like A; dB, dC
+    (batch, ngroups, N, L); dD (dim); ddelta_bias (nheads); dh0 (batch, dim, N).
+    dz is None without z, dh0 unless want_dh0.  mags hold the magnitude sums
+    used by the tolerance checks.
+    """
+    H = nheads if nheads else dim
+    dims = _Dims(batch, dim, seqlen, dstate, H, ngroups)
+    arrs = {k: _f64(v) for k, v in dict(u=u, delta=delta, A=A, B=B, C=C, D=D, z=z, bias=delta_bias, h0=h0,
+                                          dout=dout, dlast=dlast).items()}
+    rows = batch * dim
+    if arrs["u"].size != rows * seqlen or arrs["dout"].size != rows * seqlen:
+        raise ValueError("u / dout size does not match the problem")
+    if arrs["delta"].size != batch * H * seqlen:
+        raise ValueError("delta size does not match the problem")
+    if arrs["z"] is not None and arrs["z"].size != rows * seqlen:
+        raise ValueError("z size does not match the problem")
+    nbc = batch * ngroups * dstate * seqlen
+    if arrs["B"].size != nbc or arrs["C"].size != nbc:
+        raise ValueError("B / C size does not match the problem")
+    nA = dim * dstate if H == dim else H
+    if arrs["A"].size != nA:
+        raise ValueError("A size does not match the problem")
+    if arrs["D"] is not None and arrs["D"].size != dim:
+        raise ValueError("D size does not match the problem")
+    if arrs["bias"] is not None and arrs["bias"].size != H:
+        raise ValueError("delta_bias size does not match the problem")
+    for k in ("h0", "dlast"):
+        if arrs[k] is not None and arrs[k].size != rows * dstate:
+            raise ValueError(f"{k} size does not match the problem")
+    shapes = dict(du=(batch, dim, seqlen), ddelta=(batch, H, seqlen), dA=(dim, dstate) if H == dim else (H,),
+                  dB=(batch, ngroups, dstate, seqlen), dC=(batch, ngroups, dstate, seqlen), dD=(dim,),
+                  dz=(batch, dim, seqlen), ddelta_bias=(H,), dh0=(batch, dim, dstate))
+    grads, mags = {}, {}
+    for k in GRAD_NAMES:
+        want = (k != "dz" or arrs["z"] is not None) and (k != "dh0" or want_dh0)
+        grads[k] = np.zeros(shapes[k], dtype=np.float64) if want else None
+        mags[k] = np.zeros(shapes[k], dtype=np.float64) if want else None
+    gs = _Grads(*[_ptr(grads[k]) for k in GRAD_NAMES])
+    ms = _Grads(*[_ptr(mags[k]) for k in GRAD_NAMES])
+    lib = lib or _get_lib()
+    rc = lib.oracle_selective_scan_bwd_f64(
+        ctypes.byref(dims), _ptr(arrs["u"]), _ptr(arrs["delta"]), _ptr(arrs["A"]), _ptr(arrs["B"]), _ptr(arrs["C"]),
+        _ptr(arrs["D"]), _ptr(arrs["z"]), _ptr(arrs["bias"]), 1 if softplus else 0, _ptr(arrs["h0"]),
+        _ptr(arrs["dout"]), _ptr(arrs["dlast"]), ctypes.byref(gs), ctypes.byref(ms), nthreads or _nthreads())
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return grads, mags
+
+
+def run_inputs_bwd(dims, inputs: dict, dout, dlast=None, h0=None, want_dh0=False, nthreads=None, lib=None):
+    """Convenience: the backward on a dict produced by `ssm_inputs.make_inputs`."""
+    return selective_scan_bwd(dims.batch, dims.dim, dims.seqlen, dims.dstate, inputs["u"], inputs["delta"],
+                              inputs["A"], inputs["B"], inputs["C"], dout, inputs.get("D"), inputs.get("z"),
+                              inputs.get("delta_bias"), bool(inputs.get("softplus", True)), dims.nheads,
+                              dims.ngroups, h0=h0, dlast=dlast, want_dh0=want_dh0, nthreads=nthreads, lib=lib)

@@ -9,6 +9,7 @@ import subprocess
 import pytest
 
 import oracle
+from bwd_pins import BWD_PINS
 from conv1d_pins import CONV_PINS
 from oracle_pins import ALL_PINS
 
@@ -39,6 +40,22 @@ MUTANTS = [
     ("conv not causal (centred)", "const int64_t s = t - (width - 1) + k;", "const int64_t s = t - (width - 1) / 2 + k;"),
     ("conv bias dropped", "double v = bias ? bias[d] : 0.0;", "double v = 0.0;"),
     ("conv activation sigmoid", "orow[t] = silu ? v / (1.0 + exp(-v)) : v;", "orow[t] = silu ? 1.0 / (1.0 + exp(-v)) : v;"),
+    # the backward scan
+    ("bwd dt drops the decay term", "ddt += gs[n] * Bg[n * L + t] * u[t] + gdA * a * dA;",
+     "ddt += gs[n] * Bg[n * L + t] * u[t];"),
+    ("bwd state gradient not decayed", "gs[n] = dA * gs[n];", ""),
+    ("bwd decay gradient uses h_t", "const double gdA = gs[n] * hp[n];", "const double gdA = gs[n] * hc[n];"),
+    ("bwd softplus derivative dropped", "const double sp = j->softplus ? sigmoid_f64(x) : 1.0;",
+     "const double sp = 1.0;"),
+    ("bwd dB without dt", "j->g.dB[bc] += gs[n] * dt * u[t];", "j->g.dB[bc] += gs[n] * u[t];"),
+    ("bwd dC from the previous state", "j->g.dC[bc] += dy * hc[n];", "j->g.dC[bc] += dy * hp[n];"),
+    ("bwd dz through silu itself", "j->g.dz[row * L + t] = go[t] * y * dsilu;",
+     "j->g.dz[row * L + t] = go[t] * y * silu_f64(z[t]);"),
+    ("bwd readout gradient not added", "gs[n] += dy * Cg[n * L + t];", ""),
+    ("bwd dlast ignored", "gs[n] = j->dlast ? j->dlast[row * N + n] : 0.0;", "gs[n] = 0.0;"),
+    ("bwd du misses the skip", "double du = dy * Dd,", "double du = 0.0 * Dd,"),
+    ("bwd dA without dt", "j->g.dA[ai] += gdA * dt * dA;", "j->g.dA[ai] += gdA * dA;"),
+    ("bwd gate gradient ungated", "const double dy = go[t] * gate;", "const double dy = go[t];"),
 ]
 
 
@@ -59,7 +76,7 @@ def _build_mutant(tmp_path, name, old, new):
 def test_mutant_is_caught(tmp_path, name, old, new):
     lib = _build_mutant(tmp_path, name, old, new)
     caught = []
-    for pin in ALL_PINS + CONV_PINS:
+    for pin in ALL_PINS + CONV_PINS + BWD_PINS:
         try:
             pin(lib)
         except AssertionError:

@@ -40,6 +40,7 @@
 #ifndef SSM_SCAN_H
 #define SSM_SCAN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -241,6 +242,66 @@ int ssm_selective_state_update(const ssm_dims_t* dims, float* state, const void*
 int ssm_causal_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t width, int32_t io_dtype,
                           const void* x, const float* w, const float* bias, int silu, void* out,
                           ssm_stream_t stream);
+
+/*
+ * Gradients of the forward scan (ssm_selective_scan_fwd_h0), for training: the
+ * backward pass.  The states are not kept by the forward; this call recomputes
+ * them ("Agent 229: SSM optimization patterns" page, section 4 "Activation
+ * Recomputation": recompute in the backward pass, checkpoint at chunk
+ * boundaries; Mamba "architecture-details" page, "Memory Efficiency").  Given
+ * dout = dLoss/dout and dlast = dLoss/dlast_state (nullable: zero), with
+ * dt, dA = exp(dt*A), h, y as in the forward and g the gradient of the state
+ * carried back from step t+1 (dlast at the last step):
+ *
+ *     dy    = dout * silu(z)                g[n] += dy * C[n]    (= dLoss/dh_t)
+ *     dB[n] += g[n] * dt * u                dC[n] += dy * h_t[n]  (summed over channels)
+ *     du    = dt * sum_n g[n] B[n] + dy * D
+ *     ddt   = u * sum_n g[n] B[n] + sum_n g[n] h_(t-1)[n] A[n] dA[n]
+ *     dA[n] += g[n] h_(t-1)[n] dt dA[n]        g[n] *= dA[n]   (carried to t-1)
+ *     ddelta = ddt * sigmoid(delta + delta_bias)  (ddt without softplus)
+ *     ddelta_bias += ddelta,  dD += dy * u,  dz = dout * y * silu'(z)
+ *     dh0 = g after step 0
+ *
+ * Covered: the S6 layout (nheads == dim), dstate 16, dim/ngroups a multiple of
+ * 32; other shapes return SSM_ERR_UNSUPPORTED.  Inputs and layouts are the
+ * forward's (h0 nullable: zero); dout is (batch, dim, seqlen) in the io dtype,
+ * dlast (batch, dim, dstate) fp32.  Outputs (ssm_grads_t, device memory owned
+ * by the caller, every one overwritten):
+ *     du, dz        (batch, dim, seqlen) io dtype; dz required iff z != NULL
+ *     ddelta        (batch, nheads, seqlen) io dtype
+ *     dA            like A, fp32
+ *     dB, dC        (batch, ngroups, dstate, seqlen) fp32
+ *     dD            (dim) fp32, nullable: not computed
+ *     ddelta_bias   (nheads) fp32, nullable: not computed
+ *     dh0           (batch, dim, dstate) fp32, nullable: not computed
+ * The call allocates nothing: `workspace` (device, 256-byte aligned, at least
+ * ssm_selective_scan_bwd_workspace_size bytes; about batch*dim*seqlen*4 bytes of
+ * state checkpoints plus per-tile dB/dC rows) is the caller's and is scratch
+ * after the call.  Two kernels on `stream`; the sums run in a fixed order, so
+ * repeated calls give identical bits.  A, h0, dlast and dh0 must be 8-byte
+ * aligned (else SSM_ERR_UNSUPPORTED).  SSM_ERR_INVALID_ARG for a NULL required
+ * pointer (u, delta, A, B, C, dout, grads, du, ddelta, dA, dB, dC, workspace),
+ * a bad shape or a workspace that is too small.
+ */
+typedef struct {
+    void* du;
+    void* ddelta;
+    float* dA;
+    float* dB;
+    float* dC;
+    float* dD;
+    void* dz;
+    float* ddelta_bias;
+    float* dh0;
+} ssm_grads_t;
+
+int ssm_selective_scan_bwd_workspace_size(const ssm_dims_t* dims, size_t* bytes);
+
+int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, const void* delta, const float* A,
+                           const void* B, const void* C, const float* D, const void* z,
+                           const float* delta_bias, int softplus, const float* h0, const void* dout,
+                           const float* dlast, const ssm_grads_t* grads, void* workspace,
+                           size_t workspace_bytes, ssm_stream_t stream);
 
 /* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
 int ssm_scan_destroy(ssm_plan_t plan);

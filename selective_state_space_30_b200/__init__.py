@@ -22,12 +22,14 @@ from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, 
                    ssm_dims_t, ssm_probe_ex2, ssm_scan_destroy, ssm_scan_device_status, ssm_scan_plan,
                    ssm_scan_plan_info, ssm_scan_plan_schedule, ssm_scan_set_option, ssm_selective_scan_fwd,
                    ssm_selective_scan_fwd_h0, ssm_selective_scan_fwd_host, ssm_selective_scan_fwd_noalloc,
-                   ssm_selective_state_update, ssm_causal_conv1d_fwd,
+                   ssm_selective_state_update, ssm_causal_conv1d_fwd, ssm_selective_scan_bwd,
+                   ssm_selective_scan_bwd_workspace_size, ssm_grads_t, GRAD_NAMES,
                    ssm_status_string)
 
 __all__ = ["selective_scan_fwd", "selective_scan_fwd_host", "Plan", "get_plan", "ssm_scan_plan",
            "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0", "ssm_selective_scan_fwd_host",
            "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update", "ssm_causal_conv1d_fwd",
+           "selective_scan_bwd", "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_workspace_size",
            "ssm_scan_destroy", "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info",
            "ssm_scan_set_option", "ssm_scan_plan_schedule",
            "ssm_probe_ex2", "make_dims", "SsmError", "load_library"]
@@ -136,3 +138,37 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     ssm_selective_scan_fwd_host(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, out,
                                 last_state if return_last_state else None, stream)
     return out, (last_state if return_last_state else None)
+
+
+def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None, softplus: bool = True,
+                       h0=None, dlast=None, want_dh0: bool = False, workspace=None, stream=None) -> dict:
+    """Gradients of the forward scan on CUDA tensors (see include/ssm_scan.h,
+    ssm_selective_scan_bwd).  Returns a dict over GRAD_NAMES: du, ddelta, dz in
+    u's dtype; dA, dB, dC, dD, ddelta_bias, dh0 fp32 (dz None without z, dh0
+    only with want_dh0; dD and ddelta_bias are the gradients at D = 0 / bias = 0
+    when those are not given).  The workspace is allocated with torch unless
+    given (uint8, at least ssm_selective_scan_bwd_workspace_size bytes)."""
+    import torch
+    batch, dim, seqlen, dstate, nheads, ngroups, io = _shapes(u, delta, A, B)
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("dout", dout), ("D", D),
+                    ("z", z), ("delta_bias", delta_bias), ("h0", h0), ("dlast", dlast)):
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError(f"{name} must be a CUDA tensor")
+            if not t.is_contiguous():
+                raise ValueError(f"{name} must be contiguous")
+    dims = make_dims(batch, dim, seqlen, dstate, nheads, ngroups, io)
+    nbytes = ssm_selective_scan_bwd_workspace_size(dims)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=u.device)
+    f32 = dict(dtype=torch.float32, device=u.device)
+    g = {"du": torch.empty_like(u), "ddelta": torch.empty_like(delta), "dA": torch.empty(A.shape, **f32),
+         "dB": torch.empty(B.shape, **f32), "dC": torch.empty(C.shape, **f32),
+         "dD": torch.empty((dim,), **f32), "dz": torch.empty_like(z) if z is not None else None,
+         "ddelta_bias": torch.empty((nheads,), **f32),
+         "dh0": torch.empty((batch, dim, dstate), **f32) if want_dh0 else None}
+    if stream is None:
+        stream = torch.cuda.current_stream(u.device).cuda_stream
+    ssm_selective_scan_bwd(dims, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dout, dlast, g, workspace,
+                           workspace.numel() * workspace.element_size(), stream)
+    return g

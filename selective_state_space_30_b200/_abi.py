@@ -26,7 +26,7 @@ SSM_BF16 = 1
 # every exported symbol declared in include/ssm_scan.h
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
            "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update",
-           "ssm_causal_conv1d_fwd",
+           "ssm_causal_conv1d_fwd", "ssm_selective_scan_bwd_workspace_size", "ssm_selective_scan_bwd",
            "ssm_scan_set_option",
            "ssm_scan_plan_schedule", "ssm_scan_destroy",
            "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
@@ -52,6 +52,14 @@ class ssm_dims_t(ctypes.Structure):
                 ("io_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+class ssm_grads_t(ctypes.Structure):
+    _fields_ = [("du", ctypes.c_void_p), ("ddelta", ctypes.c_void_p), ("dA", ctypes.c_void_p),
+                ("dB", ctypes.c_void_p), ("dC", ctypes.c_void_p), ("dD", ctypes.c_void_p),
+                ("dz", ctypes.c_void_p), ("ddelta_bias", ctypes.c_void_p), ("dh0", ctypes.c_void_p)]
+
+
+GRAD_NAMES = tuple(f[0] for f in ssm_grads_t._fields_)
+
 _lib = None
 
 
@@ -75,6 +83,9 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, dims_p, vp, vp, vp]
     lib.ssm_selective_state_update.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
     lib.ssm_causal_conv1d_fwd.argtypes = [i64, i64, i64, i32, i32, vp, vp, vp, i32, vp, vp]
+    lib.ssm_selective_scan_bwd_workspace_size.argtypes = [dims_p, ctypes.POINTER(ctypes.c_size_t)]
+    lib.ssm_selective_scan_bwd.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
+                                           ctypes.POINTER(ssm_grads_t), vp, ctypes.c_size_t, vp]
     lib.ssm_scan_destroy.argtypes = [vp]
     lib.ssm_scan_device_status.argtypes = [vp, vp]
     lib.ssm_status_string.argtypes = [i32]
@@ -184,6 +195,27 @@ def ssm_causal_conv1d_fwd(batch: int, dim: int, seqlen: int, width: int, io_dtyp
     rc = load_library().ssm_causal_conv1d_fwd(int(batch), int(dim), int(seqlen), int(width), int(io_dtype), _ptr(x),
                                               _ptr(w), _ptr(bias), 1 if silu else 0, _ptr(out), _stream(stream))
     return _check(rc, "ssm_causal_conv1d_fwd") if check else rc
+
+
+def ssm_selective_scan_bwd_workspace_size(dims: ssm_dims_t, check: bool = True) -> int:
+    """Bytes of device scratch ssm_selective_scan_bwd needs for `dims` (see include/ssm_scan.h)."""
+    n = ctypes.c_size_t()
+    rc = load_library().ssm_selective_scan_bwd_workspace_size(ctypes.byref(dims), ctypes.byref(n))
+    if check:
+        _check(rc, "ssm_selective_scan_bwd_workspace_size")
+    return int(n.value) if rc == SSM_OK else -rc
+
+
+def ssm_selective_scan_bwd(dims: ssm_dims_t, u, delta, A, B, C, D, z, delta_bias, softplus: bool, h0, dout,
+                           dlast, grads: dict, workspace, workspace_bytes: int, stream=None,
+                           check: bool = True) -> int:
+    """Gradients of the forward scan (see include/ssm_scan.h); `grads` maps GRAD_NAMES to outputs or None."""
+    g = ssm_grads_t(*[_ptr(grads.get(k)) for k in GRAD_NAMES])
+    rc = load_library().ssm_selective_scan_bwd(
+        ctypes.byref(dims), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if softplus else 0, _ptr(h0), _ptr(dout), _ptr(dlast), ctypes.byref(g), _ptr(workspace),
+        int(workspace_bytes), _stream(stream))
+    return _check(rc, "ssm_selective_scan_bwd") if check else rc
 
 
 def ssm_scan_destroy(plan: Optional[int]) -> int:

@@ -1,0 +1,519 @@
+// Backward of the selective scan: the gradients of every input of the forward
+// scan, given dout (and optionally the gradient of the final state).  The
+// states are not stored by the forward; this pass recomputes them ("Agent
+// 229: SSM optimization patterns" page, section 4 "Activation Recomputation",
+// checkpoints at chunk boundaries; Mamba "architecture-details" page, "Memory
+// Efficiency": training recomputes activations in the backward pass).
+// Declared in include/ssm_scan.h as ssm_selective_scan_bwd.
+//
+// With x_t = delta_t + bias, dt_t = softplus(x_t), dA_tn = exp(dt_t a_n),
+// h_t = dA_t h_(t-1) + dt_t B_t u_t, y_t = C_t.h_t + D u_t, out_t = y_t silu(z_t)
+// and g the gradient of the state carried from t+1 (g = dlast after the last
+// step), walking t down:
+//
+//   dy = dout silu(z)             g_n += dy C_tn   (dLoss/dh_tn)
+//   dB_tn += g_n dt u_t           dC_tn += dy h_tn           (summed over channels)
+//   du_t = dt sum_n g_n B_tn + dy D
+//   ddt_t = u_t sum_n g_n B_tn + sum_n g_n h_(t-1)n a_n dA_tn
+//   da_n += g_n h_(t-1)n dt dA_tn g_n <- dA_tn g_n
+//   ddelta_t = ddt_t sigmoid(x_t),  dbias += ddelta_t,  dz_t = dout y_t silu'(z_t)
+//
+// One CTA takes 32 channels of one batch row (S6 layout, dstate 16): eight
+// warps, each four channels x 8 lanes x 2 states.  Pass 1 runs the recurrence
+// forward and stores the state at the start of every 8-step window (the
+// checkpoints).  Pass 2 walks the 32-step blocks backwards; per window it
+// recomputes the 8 states and decays from the checkpoint into registers, then
+// runs the window in reverse.  Sums over the states (y, sum g B, the decay term)
+// are transposed shuffle reductions inside the 8 lanes of a channel; dB and dC,
+// sums over channels, go through shared memory to per-CTA partial rows, which a
+// second kernel adds in a fixed order with the per-row dA, dD and dbias
+// partials: the result does not depend on scheduling.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "scan_kernel.cuh"   // ex2_approx, rcp_approx, softplus1, kLog2e
+#include "ssm_scan.h"
+
+namespace ssm {
+namespace {
+
+constexpr int kN = 16;         // states per channel
+constexpr int kBT = 32;        // steps per staged block
+constexpr int kWin = 8;        // steps per recomputed window (= one 8-lane reduction)
+constexpr int kCT = 32;        // channels per CTA
+constexpr int kThreads = 256;  // 8 warps x 4 channels x 8 lanes
+constexpr int kStageRows = 4 * kCT + 2 * kN;   // u, delta, z, dout rows; B, C rows
+
+struct BwdParams {
+    const void *u, *delta, *z, *dout, *B, *C;
+    const float *A, *D, *bias, *h0, *dlast;
+    void *du, *ddelta, *dz;
+    float* dh0;
+    float *ckpt, *dBp, *dCp, *dAp, *dDp, *dbp;   // workspace
+    int64_t batch, dim, seqlen, ngroups;
+    int tiles_per_row;   // dim / kCT
+    int softplus;
+};
+
+template <typename T> struct Io;
+template <> struct Io<float> {
+    using raw = float;
+    __device__ static float f(raw v) { return v; }
+    __device__ static raw from(float v) { return v; }
+};
+template <> struct Io<__nv_bfloat16> {
+    using raw = unsigned short;
+    __device__ static float f(raw v) { return __uint_as_float((uint32_t)v << 16); }
+    __device__ static raw from(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
+};
+
+// shared memory (bytes)
+template <typename T>
+struct Smem {
+    static constexpr int kRow = kBT * (int)sizeof(T) + 16;        // staged row stride (16-byte padded)
+    static constexpr int STAGE = 0;
+    static constexpr int P = STAGE + kStageRows * kRow;           // float4 [kCT][kBT]: dt, dt*u, dy, dout*silu'(z)
+    static constexpr int U = P + kCT * kBT * 16;                  // float2 [kCT][kBT]: u, sigmoid(x)
+    static constexpr int BC = U + kCT * kBT * 8;                  // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
+    static constexpr int RED = BC + kBT * 8 * 16;                 // float4 [kCT][kWin][8]: dB, dC terms
+    static constexpr int TOTAL = RED + kCT * kWin * 8 * 16;
+};
+
+// rows x kBT steps [t0, t0 + kBT) of `rows` rows (row r at src + r * stride) into
+// shared memory, zero past L.  vec: 16-byte chunks (rows 16-byte aligned, L a
+// multiple of the chunk), else element by element.
+template <typename T>
+__device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int64_t stride, int rows, int64_t t0,
+                                           int64_t L, bool vec, int tid) {
+    using R = typename Io<T>::raw;
+    constexpr int E = 16 / (int)sizeof(T);
+    constexpr int CPR = kBT / E;
+    if (vec) {
+        for (int i = tid; i < rows * CPR; i += kThreads) {
+            const int r = i / CPR, k = i % CPR;
+            const int64_t t = t0 + (int64_t)k * E;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (t < L) v = __ldg(reinterpret_cast<const uint4*>(src + r * stride + t));
+            *reinterpret_cast<uint4*>(dst + r * Smem<T>::kRow + k * 16) = v;
+        }
+    } else {
+        const R* s = reinterpret_cast<const R*>(src);
+        for (int i = tid; i < rows * kBT; i += kThreads) {
+            const int r = i / kBT, k = i % kBT;
+            const int64_t t = t0 + k;
+            reinterpret_cast<R*>(dst + r * Smem<T>::kRow)[k] = t < L ? s[r * stride + t] : (R)0;
+        }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float staged(const unsigned char* base, int row, int k) {
+    return Io<T>::f(reinterpret_cast<const typename Io<T>::raw*>(base + row * Smem<T>::kRow)[k]);
+}
+
+__device__ __forceinline__ float sigmoid1(float x) { return rcp_approx(1.f + ex2_approx(x * -kLog2e)); }
+
+// One step of the recurrence on the lane's two states (the same expression in
+// both passes, so the recomputed states equal the checkpointed ones bit for bit).
+__device__ __forceinline__ void fwd_step(float2& h, float2& dA, float dt, float dtu, float b0, float b1, float2 al) {
+    dA = make_float2(ex2_approx(dt * al.x), ex2_approx(dt * al.y));
+    h.x = fmaf(dA.x, h.x, dtu * b0);
+    h.y = fmaf(dA.y, h.y, dtu * b1);
+}
+
+// Sum of v over the 8 lanes of a channel (lane bits 0-2 = j), transposed: lane j
+// gets the total of element j.  Three halvings, 4 + 2 + 1 shuffles.
+__device__ __forceinline__ float reduce8(const float (&v)[8], int j) {
+    float a[4], b[2];
+    const bool h2 = j & 4, h1 = j & 2, h0 = j & 1;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = h2 ? v[i] : v[i + 4];
+        const float keep = h2 ? v[i + 4] : v[i];
+        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = h1 ? a[i] : a[i + 2];
+        const float keep = h1 ? a[i + 2] : a[i];
+        b[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    const float send = h0 ? b[0] : b[1];
+    const float keep = h0 ? b[1] : b[0];
+    return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p) {
+    using S = Smem<T>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    unsigned char* stage = smem + S::STAGE;
+    float4* sP = reinterpret_cast<float4*>(smem + S::P);
+    float2* sU = reinterpret_cast<float2*>(smem + S::U);
+    float4* sBC = reinterpret_cast<float4*>(smem + S::BC);
+    float4* sR = reinterpret_cast<float4*>(smem + S::RED);
+    float* sRf = reinterpret_cast<float*>(smem + S::RED);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = lane >> 3, j = lane & 7;
+    const int c = warp * 4 + q;                    // channel within the tile
+    const int64_t cta = blockIdx.x;                // = b * tiles_per_row + tile
+    const int64_t b = cta / p.tiles_per_row;
+    const int64_t L = p.seqlen, Dm = p.dim, G = p.ngroups;
+    const int64_t row0 = cta * kCT;                // first (b, d) row of the tile
+    const int64_t d0 = row0 - b * Dm;
+    const int64_t g = d0 / (Dm / G);
+    const int64_t d = d0 + c;
+    const T* u = static_cast<const T*>(p.u) + row0 * L;
+    const T* dl = static_cast<const T*>(p.delta) + row0 * L;
+    const T* zz = p.z ? static_cast<const T*>(p.z) + row0 * L : nullptr;
+    const T* go = static_cast<const T*>(p.dout) + row0 * L;
+    const T* Bg = static_cast<const T*>(p.B) + (b * G + g) * kN * L;
+    const T* Cg = static_cast<const T*>(p.C) + (b * G + g) * kN * L;
+    const bool vec = (L % (16 / (int64_t)sizeof(T))) == 0 &&
+                     ((reinterpret_cast<uintptr_t>(p.u) | reinterpret_cast<uintptr_t>(p.delta) |
+                       reinterpret_cast<uintptr_t>(p.z) | reinterpret_cast<uintptr_t>(p.dout) |
+                       reinterpret_cast<uintptr_t>(p.B) | reinterpret_cast<uintptr_t>(p.C)) & 15u) == 0;
+    const int nblk = (int)((L + kBT - 1) / kBT);
+    const int nwin = nblk * (kBT / kWin);
+    float* ckpt = p.ckpt + cta * (int64_t)nwin * kCT * kN;
+
+    const float2 Aln = make_float2(__ldg(p.A + d * kN + 2 * j), __ldg(p.A + d * kN + 2 * j + 1));
+    const float2 al = make_float2(Aln.x * kLog2e, Aln.y * kLog2e);
+    const float bias_c = p.bias ? __ldg(p.bias + d) : 0.f;
+    const float Dc = p.D ? __ldg(p.D + d) : 0.f;
+
+    // ---------------- pass 1: the recurrence forward, checkpoints at every window start
+    float2 h = p.h0 ? *reinterpret_cast<const float2*>(p.h0 + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
+    for (int blk = 0; blk < nblk; ++blk) {
+        const int64_t t0 = (int64_t)blk * kBT;
+        __syncthreads();   // the previous block is done with the staged rows and the B tile
+        stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
+        stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
+        stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
+        __syncthreads();
+        // dt and dt*u of this warp's 4 channels, lane = step
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int cc = warp * 4 + i;
+            const float uv = staged<T>(stage, cc, lane);
+            const float xv = staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
+            float dt = p.softplus ? softplus1(xv) : xv;
+            if (t0 + lane >= L) dt = 0.f;
+            sP[cc * kBT + lane] = make_float4(dt, dt * uv, 0.f, 0.f);
+        }
+        {
+            const int t = tid >> 3, jj = tid & 7;
+            const unsigned char* sb = stage + 4 * kCT * S::kRow;
+            sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t), 0.f, 0.f);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < kBT / kWin; ++w) {
+            *reinterpret_cast<float2*>(ckpt + ((int64_t)(blk * (kBT / kWin) + w) * kCT + c) * kN + 2 * j) = h;
+#pragma unroll 4
+            for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
+                const float4 pv = sP[c * kBT + t];
+                const float4 bc = sBC[t * 8 + j];
+                float2 dA;
+                fwd_step(h, dA, pv.x, pv.y, bc.x, bc.y, al);
+            }
+        }
+    }
+
+    // ---------------- pass 2: blocks backwards, windows recomputed from their checkpoints
+    float2 gs = p.dlast ? *reinterpret_cast<const float2*>(p.dlast + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
+    float2 dAacc = make_float2(0.f, 0.f);
+    float dbias = 0.f, dDacc = 0.f;
+    float* dBrow = p.dBp + cta * kN * L;
+    float* dCrow = p.dCp + cta * kN * L;
+    for (int blk = nblk - 1; blk >= 0; --blk) {
+        const int64_t t0 = (int64_t)blk * kBT;
+        __syncthreads();
+        stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
+        stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
+        if (zz) stage_rows<T>(stage + 2 * kCT * S::kRow, zz, L, kCT, t0, L, vec, tid);
+        stage_rows<T>(stage + 3 * kCT * S::kRow, go, L, kCT, t0, L, vec, tid);
+        stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
+        stage_rows<T>(stage + (4 * kCT + kN) * S::kRow, Cg, L, kN, t0, L, vec, tid);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int cc = warp * 4 + i;
+            const bool valid = t0 + lane < L;
+            const float uv = staged<T>(stage, cc, lane);
+            const float xv = staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
+            const float gov = staged<T>(stage + 3 * kCT * S::kRow, cc, lane);
+            float dt = p.softplus ? softplus1(xv) : xv;
+            float sp = p.softplus ? sigmoid1(xv) : 1.f;
+            if (!valid) dt = sp = 0.f;
+            float dy = gov, dzf = 0.f;
+            if (zz) {
+                const float zv = staged<T>(stage + 2 * kCT * S::kRow, cc, lane);
+                const float s = sigmoid1(zv);
+                dy = gov * zv * s;
+                dzf = gov * (s * fmaf(zv, 1.f - s, 1.f));
+            }
+            sP[cc * kBT + lane] = make_float4(dt, dt * uv, dy, dzf);
+            sU[cc * kBT + lane] = make_float2(uv, sp);
+        }
+        {
+            const int t = tid >> 3, jj = tid & 7;
+            const unsigned char* sb = stage + 4 * kCT * S::kRow;
+            const unsigned char* sc = stage + (4 * kCT + kN) * S::kRow;
+            sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t),
+                                          staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
+        }
+        __syncthreads();
+
+        for (int w = kBT / kWin - 1; w >= 0; --w) {
+            const int tw = w * kWin;   // first step of the window within the block
+            const float2 he = *reinterpret_cast<const float2*>(ckpt + ((int64_t)(blk * (kBT / kWin) + w) * kCT + c) * kN + 2 * j);
+            float2 hr[kWin], dAr[kWin];
+            float yw;   // y of step j of the window, summed over the states
+            {
+                float2 hh = he;
+                float yp[kWin];
+#pragma unroll
+                for (int t = 0; t < kWin; ++t) {
+                    const float4 pv = sP[c * kBT + tw + t];
+                    const float4 bc = sBC[(tw + t) * 8 + j];
+                    fwd_step(hh, dAr[t], pv.x, pv.y, bc.x, bc.y, al);
+                    hr[t] = hh;
+                    yp[t] = fmaf(bc.z, hh.x, bc.w * hh.y);
+                }
+                yw = reduce8(yp, j);
+            }
+            float gb[kWin], qq[kWin];
+#pragma unroll
+            for (int t = kWin - 1; t >= 0; --t) {
+                const float4 pv = sP[c * kBT + tw + t];
+                const float4 bc = sBC[(tw + t) * 8 + j];
+                gs.x = fmaf(pv.z, bc.z, gs.x);   // + dy C: now dLoss/dh_t
+                gs.y = fmaf(pv.z, bc.w, gs.y);
+                const float2 hp = t > 0 ? hr[t - 1] : he;
+                const float2 e = make_float2(gs.x * hp.x * dAr[t].x, gs.y * hp.y * dAr[t].y);
+                dAacc.x = fmaf(e.x, pv.x, dAacc.x);
+                dAacc.y = fmaf(e.y, pv.x, dAacc.y);
+                gb[t] = fmaf(gs.x, bc.x, gs.y * bc.y);
+                qq[t] = fmaf(e.x, Aln.x, e.y * Aln.y);
+                sR[(c * kWin + t) * 8 + j] = make_float4(gs.x * pv.y, gs.y * pv.y, pv.z * hr[t].x, pv.z * hr[t].y);
+                gs.x *= dAr[t].x;                // carry to t-1
+                gs.y *= dAr[t].y;
+                asm volatile("" ::: "memory");   // keep the next step's loads here (register pressure)
+            }
+            const float GB = reduce8(gb, j), Q = reduce8(qq, j);
+            __syncwarp();
+            {
+                // lane j: step tw + j of channel c
+                const int t = tw + j;
+                const float4 pv = sP[c * kBT + t];
+                const float2 uv = sU[c * kBT + t];
+                const float dd = fmaf(uv.x, GB, Q) * uv.y;
+                dbias += dd;
+                dDacc = fmaf(pv.z, uv.x, dDacc);
+                sP[c * kBT + t] = make_float4(fmaf(pv.x, GB, pv.z * Dc), dd, fmaf(Dc, uv.x, yw) * pv.w, 0.f);
+            }
+            __syncthreads();
+            // dB, dC of these 8 steps summed over the tile's channels, in channel order
+            {
+                float sum = 0.f;
+#pragma unroll 8
+                for (int cc = 0; cc < kCT; ++cc) sum += sRf[cc * (kWin * 8 * 4) + tid];
+                const int i = tid >> 5, jj = (tid >> 2) & 7, comp = tid & 3;
+                const int64_t t = t0 + tw + i;
+                if (t < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + t] = sum;
+            }
+            __syncthreads();
+        }
+        // the block's du, ddelta, dz rows of this warp's channels (lane = step)
+        __syncwarp();
+        if (t0 + lane < L) {
+            using R = typename Io<T>::raw;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int cc = warp * 4 + i;
+                const float4 o = sP[cc * kBT + lane];
+                const int64_t at = (row0 + cc) * L + t0 + lane;
+                static_cast<R*>(p.du)[at] = Io<T>::from(o.x);
+                static_cast<R*>(p.ddelta)[at] = Io<T>::from(o.y);
+                if (zz) static_cast<R*>(p.dz)[at] = Io<T>::from(o.z);
+            }
+        }
+    }
+
+    // ---------------- per-row partials of the parameter gradients; dh0
+    if (p.dh0) *reinterpret_cast<float2*>(p.dh0 + (row0 + c) * kN + 2 * j) = gs;
+    *reinterpret_cast<float2*>(p.dAp + (row0 + c) * kN + 2 * j) = dAacc;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+        dbias += __shfl_xor_sync(0xffffffffu, dbias, o);
+        dDacc += __shfl_xor_sync(0xffffffffu, dDacc, o);
+    }
+    if (j == 0) {
+        p.dbp[row0 + c] = dbias;
+        p.dDp[row0 + c] = dDacc;
+    }
+}
+
+// dB, dC: sum of the per-tile rows of the group; dA, dD, dbias: sum over batch rows.
+__global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, float* dA, float* dB, float* dC,
+                                                         float* dD, float* dbias) {
+    const int64_t Dm = p.dim, L = p.seqlen, G = p.ngroups;
+    const int64_t nbc = p.batch * G * kN * L;
+    const int64_t tpg = (Dm / G) / kCT;   // tiles per group
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < 2 * nbc) {
+        const bool isC = i >= nbc;
+        const int64_t k = isC ? i - nbc : i;
+        const int64_t t = k % L, n = (k / L) % kN, bg = k / (L * kN);
+        const int64_t b = bg / G, g = bg % G;
+        const float* src = (isC ? p.dCp : p.dBp) + ((b * p.tiles_per_row + g * tpg) * kN + n) * L + t;
+        float s = 0.f;
+        for (int64_t m = 0; m < tpg; ++m) s += src[m * kN * L];
+        (isC ? dC : dB)[k] = s;
+        return;
+    }
+    const int64_t k = i - 2 * nbc;
+    if (k < Dm * kN) {
+        float s = 0.f;
+        for (int64_t b = 0; b < p.batch; ++b) s += p.dAp[b * Dm * kN + k];
+        dA[k] = s;
+        return;
+    }
+    const int64_t e = k - Dm * kN;
+    if (e < 2 * Dm) {
+        const bool isb = e >= Dm;
+        const int64_t dd = isb ? e - Dm : e;
+        float* dst = isb ? dbias : dD;
+        if (!dst) return;
+        const float* src = isb ? p.dbp : p.dDp;
+        float s = 0.f;
+        for (int64_t b = 0; b < p.batch; ++b) s += src[b * Dm + dd];
+        dst[dd] = s;
+    }
+}
+
+struct WsLayout {
+    int64_t ckpt, dBp, dCp, dAp, dDp, dbp, total;   // byte offsets
+};
+
+__host__ int64_t align256(int64_t v) { return (v + 255) & ~(int64_t)255; }
+
+WsLayout ws_layout(const ssm_dims_t& d) {
+    const int64_t rows = d.batch * d.dim;
+    const int64_t ctas = rows / kCT;
+    const int64_t nwin = ((d.seqlen + kBT - 1) / kBT) * (kBT / kWin);
+    WsLayout w;
+    w.ckpt = 0;
+    w.dBp = align256(w.ckpt + ctas * nwin * kCT * kN * 4);
+    w.dCp = align256(w.dBp + ctas * kN * d.seqlen * 4);
+    w.dAp = align256(w.dCp + ctas * kN * d.seqlen * 4);
+    w.dDp = align256(w.dAp + rows * kN * 4);
+    w.dbp = align256(w.dDp + rows * 4);
+    w.total = align256(w.dbp + rows * 4);
+    return w;
+}
+
+int check_dims(const ssm_dims_t* d) {
+    if (!d || d->batch < 0 || d->dim <= 0 || d->seqlen < 0 || d->dstate <= 0 || d->nheads <= 0 || d->ngroups <= 0)
+        return SSM_ERR_INVALID_ARG;
+    if (d->dim % d->nheads || d->dim % d->ngroups || d->reserved != 0) return SSM_ERR_INVALID_ARG;
+    if (d->io_dtype != SSM_F32 && d->io_dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+    if (d->batch > ((int64_t)1 << 40) / d->dim || (d->seqlen > 0 && d->batch * d->dim > ((int64_t)1 << 40) / d->seqlen))
+        return SSM_ERR_INVALID_ARG;
+    // what the kernel covers: the S6 layout, dstate 16, whole 32-channel tiles inside a group
+    if (d->nheads != d->dim || d->dstate != kN || (d->dim / d->ngroups) % kCT != 0) return SSM_ERR_UNSUPPORTED;
+    if (d->batch * d->dim / kCT > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;
+    return SSM_OK;
+}
+
+template <typename T>
+int launch(const BwdParams& prm, float* dA, float* dB, float* dC, float* dD, float* dbias, int64_t ctas,
+           cudaStream_t s) {
+    constexpr int smem = Smem<T>::TOTAL;
+    static const bool attr =
+        cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+    if (!attr) return SSM_ERR_CUDA;
+    scan_bwd_kernel<T><<<(unsigned)ctas, kThreads, smem, s>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
+    const int64_t work = 2 * prm.batch * prm.ngroups * kN * prm.seqlen + prm.dim * kN + 2 * prm.dim;
+    const int64_t blocks = (work + 255) / 256;
+    if (blocks > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;
+    scan_bwd_finalize<<<(unsigned)blocks, 256, 0, s>>>(prm, dA, dB, dC, dD, dbias);
+    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace ssm
+
+extern "C" int ssm_selective_scan_bwd_workspace_size(const ssm_dims_t* dims, size_t* bytes) {
+    using namespace ssm;
+    if (!bytes) return SSM_ERR_INVALID_ARG;
+    const int rc = check_dims(dims);
+    if (rc != SSM_OK) return rc;
+    *bytes = (size_t)ws_layout(*dims).total;
+    return SSM_OK;
+}
+
+extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, const void* delta, const float* A,
+                                      const void* B, const void* C, const float* D, const void* z,
+                                      const float* delta_bias, int softplus, const float* h0, const void* dout,
+                                      const float* dlast, const ssm_grads_t* grads, void* workspace,
+                                      size_t workspace_bytes, ssm_stream_t stream) {
+    using namespace ssm;
+    const int rc = check_dims(dims);
+    if (rc != SSM_OK) return rc;
+    if (!grads || !grads->dA) return SSM_ERR_INVALID_ARG;
+    if (dims->batch == 0 || dims->seqlen == 0) {
+        // no steps (the per-step tensors are empty and may be NULL): every gradient is zero, dh0 = dlast
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        const int64_t rows = dims->batch * dims->dim, esz = dims->io_dtype == SSM_BF16 ? 2 : 4;
+        const int64_t nbc = dims->batch * dims->ngroups * kN * dims->seqlen * 4;
+        bool ok = cudaMemsetAsync(grads->dA, 0, dims->dim * kN * 4, s) == cudaSuccess;
+        if (grads->dD) ok = ok && cudaMemsetAsync(grads->dD, 0, dims->dim * 4, s) == cudaSuccess;
+        if (grads->ddelta_bias) ok = ok && cudaMemsetAsync(grads->ddelta_bias, 0, dims->dim * 4, s) == cudaSuccess;
+        if (nbc) ok = ok && cudaMemsetAsync(grads->dB, 0, nbc, s) == cudaSuccess &&
+                      cudaMemsetAsync(grads->dC, 0, nbc, s) == cudaSuccess;
+        if (rows * dims->seqlen) {
+            ok = ok && cudaMemsetAsync(grads->du, 0, rows * dims->seqlen * esz, s) == cudaSuccess &&
+                 cudaMemsetAsync(grads->ddelta, 0, rows * dims->seqlen * esz, s) == cudaSuccess;
+            if (grads->dz) ok = ok && cudaMemsetAsync(grads->dz, 0, rows * dims->seqlen * esz, s) == cudaSuccess;
+        }
+        if (grads->dh0 && rows) {
+            ok = ok && (dlast ? cudaMemcpyAsync(grads->dh0, dlast, rows * kN * 4, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(grads->dh0, 0, rows * kN * 4, s)) == cudaSuccess;
+        }
+        return ok ? SSM_OK : SSM_ERR_CUDA;
+    }
+    if (!u || !delta || !A || !B || !C || !dout) return SSM_ERR_INVALID_ARG;
+    if (!grads->du || !grads->ddelta || !grads->dB || !grads->dC) return SSM_ERR_INVALID_ARG;
+    if (z && !grads->dz) return SSM_ERR_INVALID_ARG;
+    const WsLayout w = ws_layout(*dims);
+    if (!workspace || workspace_bytes < (size_t)w.total) return SSM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) || (reinterpret_cast<uintptr_t>(A) & 7u) ||
+        (h0 && (reinterpret_cast<uintptr_t>(h0) & 7u)) || (dlast && (reinterpret_cast<uintptr_t>(dlast) & 7u)) ||
+        (grads->dh0 && (reinterpret_cast<uintptr_t>(grads->dh0) & 7u)))
+        return SSM_ERR_UNSUPPORTED;
+    BwdParams prm;
+    prm.u = u; prm.delta = delta; prm.z = z; prm.dout = dout; prm.B = B; prm.C = C;
+    prm.A = A; prm.D = D; prm.bias = delta_bias; prm.h0 = h0; prm.dlast = dlast;
+    prm.du = grads->du; prm.ddelta = grads->ddelta; prm.dz = grads->dz; prm.dh0 = grads->dh0;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    prm.ckpt = reinterpret_cast<float*>(ws + w.ckpt);
+    prm.dBp = reinterpret_cast<float*>(ws + w.dBp);
+    prm.dCp = reinterpret_cast<float*>(ws + w.dCp);
+    prm.dAp = reinterpret_cast<float*>(ws + w.dAp);
+    prm.dDp = reinterpret_cast<float*>(ws + w.dDp);
+    prm.dbp = reinterpret_cast<float*>(ws + w.dbp);
+    prm.batch = dims->batch; prm.dim = dims->dim; prm.seqlen = dims->seqlen; prm.ngroups = dims->ngroups;
+    prm.tiles_per_row = (int)(dims->dim / kCT);
+    prm.softplus = softplus ? 1 : 0;
+    const int64_t ctas = dims->batch * dims->dim / kCT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return dims->io_dtype == SSM_BF16
+               ? launch<__nv_bfloat16>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, ctas, s)
+               : launch<float>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, ctas, s);
+}

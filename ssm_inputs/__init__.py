@@ -45,7 +45,8 @@ _NORMAL, _UNIFORM, _LOGUNIFORM, _CONST, _SPINV_LOGUNIFORM = 0, 1, 2, 3, 4
 _F64, _F32, _BF16 = 0, 1, 2
 
 # fixed stream ids: one independent stream per tensor, in this order
-STREAMS = {"A": 0, "D": 1, "dt": 2, "u": 3, "delta": 4, "z": 5, "B": 6, "C": 7}
+STREAMS = {"A": 0, "D": 1, "dt": 2, "u": 3, "delta": 4, "z": 5, "B": 6, "C": 7,
+           "dout": 8, "dlast": 9, "h0": 10}
 
 
 def build(force: bool = False) -> str:
@@ -274,6 +275,22 @@ def make_inputs(dims: Dims, recipe: Recipe, seed: int = 0,
         z = z.reshape(Bt, Dm, L) if z is not None else None
         delta = delta.reshape(Bt, H, L)
     out.update({"u": u, "delta": delta, "z": z, "B": Bm, "C": Cm, "softplus": recipe.softplus})
+    return out
+
+
+def make_grad_inputs(dims: Dims, seed: int = 0, dlast: bool = False, h0: bool = False
+                     ) -> Dict[str, Optional[np.ndarray]]:
+    """The incoming gradients of a backward pass: dout (batch, dim, L) in the I/O
+    dtype, N(0, 1); optionally dlast, the gradient of last_state, and an initial
+    state h0, both (batch, dim, N) fp32 N(0, 1)."""
+    dims.validate()
+    Bt, Dm, L, N = dims.batch, dims.dim, dims.seqlen, dims.dstate
+    out = {"dout": _gen_normal(seed, "dout", 0, Bt * Dm * L, dims.dtype).reshape(Bt, Dm, L),
+           "dlast": None, "h0": None}
+    if dlast:
+        out["dlast"] = _gen_normal(seed, "dlast", 0, Bt * Dm * N, "f32").reshape(Bt, Dm, N)
+    if h0:
+        out["h0"] = _gen_normal(seed, "h0", 0, Bt * Dm * N, "f32").reshape(Bt, Dm, N)
     return out
 
 

@@ -1,0 +1,143 @@
+"""The backward scan (ssm_selective_scan_bwd) against the fp64 oracle's gradients.
+
+Tolerance, per gradient element, from the oracle's magnitude sums (mag: the same
+sum with every term and the carried state / state gradient replaced by their
+absolute values; see oracle_selective_scan_bwd_f64):
+
+    |gpu - ref| <= 1e-4 * mag  (+ ulp_bf16(ref) for the bf16 outputs du, ddelta, dz)
+
+The kernel forms every gradient in fp32 with the forward's approximations
+(ex2.approx for exp, a polynomial softplus, rcp.approx in the sigmoids), so its
+error is a small multiple of 2^-22 of the terms it sums, grown along the state
+and gradient recurrences; 1e-4 * mag is the forward's gating bound.  A wrong
+term moves a gradient by O(mag).  Needs a B200.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssm_inputs as si
+from parity import bf16_ulp, to_device, to_host_f64
+
+pytestmark = pytest.mark.gpu
+
+BF16_OUT = ("du", "ddelta", "dz")
+
+
+def _recipe(kind):
+    if kind == "c2":   # the mamba-130m recipe: delta ~ N(0, 0.5), D ~ N(0, 1)
+        return si.Recipe(d_init="normal", delta_init="normal_half")
+    if kind == "plain":
+        return si.Recipe(has_D=False, has_z=False, has_bias=False, delta_init="normal_half")
+    return si.Recipe()
+
+
+def run_bwd(dims, inp, gin, want_dh0=False, softplus=True):
+    import selective_state_space_30_b200 as ssm
+    dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    g = ssm.selective_scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], to_device(gin["dout"]),
+                               dev["D"], dev["z"], dev["delta_bias"], softplus, h0=to_device(gin.get("h0")),
+                               dlast=to_device(gin.get("dlast")), want_dh0=want_dh0)
+    torch.cuda.synchronize()
+    return g
+
+
+def check_grads(g, ref, mag, dtype, what=""):
+    for k, r in ref.items():
+        if r is None:
+            assert g.get(k) is None, f"{what}{k}: expected no output"
+            continue
+        got = to_host_f64(g[k]).reshape(r.shape)
+        assert np.all(np.isfinite(got)), f"{what}{k}: non-finite values"
+        err = np.abs(got - r)
+        tol = 1e-4 * mag[k]
+        if dtype == "bf16" and k in BF16_OUT:
+            tol = tol + bf16_ulp(r)
+        bad = err > tol
+        if bad.any():
+            i = int(np.argmax(bad.ravel()))
+            raise AssertionError(f"{what}{k}: {int(bad.sum())} of {bad.size} outside tolerance; first at flat {i}: "
+                                 f"gpu={got.ravel()[i]!r} ref={r.ravel()[i]!r} mag={mag[k].ravel()[i]!r}")
+
+
+CASES = [
+    # (dims, recipe, dlast, h0, softplus)
+    (si.Dims(2, 64, 100, 16, dtype="bf16"), "c2", True, True, True),       # ragged tail, h0 and dlast
+    (si.Dims(1, 32, 64, 16, dtype="f32"), "default", False, False, True),  # two whole blocks
+    (si.Dims(2, 64, 77, 16, dtype="f32"), "c2", True, False, True),        # L not a multiple of 4: element loads
+    (si.Dims(2, 128, 96, 16, ngroups=2, dtype="bf16"), "c2", False, True, True),   # two groups
+    (si.Dims(1, 96, 33, 16, dtype="bf16"), "plain", True, False, True),    # no z, D, bias; 33 = a block + 1
+    (si.Dims(3, 32, 8, 16, dtype="bf16"), "default", False, False, True),  # shorter than a block
+    (si.Dims(2, 32, 200, 16, dtype="f32"), "default", False, False, False),  # softplus off
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[0].batch}x{c[0].dim}x{c[0].seqlen}g{c[0].ngroups}"
+                                                      f"{c[0].dtype}-{c[1]}{'-sp' if c[4] else '-nosp'}")
+def test_bwd_matches_oracle(case):
+    dims, kind, dlast, h0, softplus = case
+    inp = si.make_inputs(dims, _recipe(kind), 41)
+    if not softplus:   # dt = delta + bias is dt itself and must be >= 0 (the caller's contract)
+        inp["delta"] = (np.abs(si.make_inputs(dims, _recipe("c2"), 41)["delta"]) * np.float32(0.05)).astype(np.float32)
+        inp["delta_bias"] = np.zeros_like(inp["delta_bias"])
+    inp["softplus"] = softplus
+    gin = si.make_grad_inputs(dims, 42, dlast=dlast, h0=h0)
+    ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin["dlast"], h0=gin["h0"], want_dh0=True)
+    g = run_bwd(dims, inp, gin, want_dh0=True, softplus=softplus)
+    check_grads(g, ref, mag, dims.dtype)
+
+
+def test_bwd_is_deterministic():
+    dims = si.Dims(2, 64, 130, 16, dtype="bf16")
+    inp = si.make_inputs(dims, _recipe("c2"), 43)
+    gin = si.make_grad_inputs(dims, 44, dlast=True)
+    a = run_bwd(dims, inp, gin)
+    b = run_bwd(dims, inp, gin)
+    for k in a:
+        if a[k] is not None:
+            assert torch.equal(a[k], b[k]), f"{k} differs between two identical calls"
+
+
+def test_bwd_no_steps():
+    """seqlen 0: every gradient is zero and dh0 = dlast."""
+    dims = si.Dims(2, 32, 0, 16, dtype="bf16")
+    inp = si.make_inputs(dims, _recipe("c2"), 45)
+    gin = si.make_grad_inputs(dims, 46, dlast=True)
+    g = run_bwd(dims, inp, gin, want_dh0=True)
+    assert torch.equal(g["dh0"].cpu(), torch.from_numpy(gin["dlast"]))
+    for k in ("dA", "dD", "ddelta_bias"):
+        assert torch.count_nonzero(g[k]) == 0
+
+
+def test_bwd_argument_checks():
+    import selective_state_space_30_b200 as ssm
+    x = torch.zeros(1 << 16, device="cuda")
+    y = torch.zeros(1 << 16, device="cuda")
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    grads = {k: y for k in ("du", "ddelta", "dA", "dB", "dC")}
+
+    def call(dims, z=None, g=grads, nbytes=ws.numel()):
+        return ssm.ssm_selective_scan_bwd(dims, x, x, x, x, x, None, z, None, True, None, x, None, g, ws, nbytes,
+                                          check=False)
+    ok = ssm.make_dims(1, 32, 16, 16, 0, 1, ssm.SSM_BF16)
+    assert ssm.ssm_selective_scan_bwd_workspace_size(ok) <= ws.numel()
+    assert call(ssm.make_dims(1, 32, 16, 128, 0, 1, ssm.SSM_BF16)) == ssm.SSM_ERR_UNSUPPORTED    # dstate 128
+    assert call(ssm.make_dims(1, 64, 16, 16, 2, 1, ssm.SSM_BF16)) == ssm.SSM_ERR_UNSUPPORTED     # per-head layout
+    assert call(ssm.make_dims(1, 48, 16, 16, 0, 1, ssm.SSM_BF16)) == ssm.SSM_ERR_UNSUPPORTED     # dim not x32
+    assert call(ok, z=x) == ssm.SSM_ERR_INVALID_ARG                                              # z without dz
+    assert call(ok, nbytes=16) == ssm.SSM_ERR_INVALID_ARG                                        # workspace too small
+    assert call(ok, g=dict(grads, dB=None)) == ssm.SSM_ERR_INVALID_ARG                           # missing output
+    assert call(ok) == ssm.SSM_OK
+
+
+def test_bwd_full_size_mamba_130m():
+    """The bench workload (mamba-130m: 8 x 1536 x 2048, N = 16, bf16), every gradient against
+    the full fp64 oracle backward."""
+    w = si.workload("mamba-130m")
+    dims = w.dims
+    inp = si.make_inputs(dims, w.recipe, w.seed)
+    gin = si.make_grad_inputs(dims, 1)
+    ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"])
+    g = run_bwd(dims, inp, gin)
+    check_grads(g, ref, mag, dims.dtype, what="mamba-130m ")

@@ -214,15 +214,26 @@ def _kernel_hash():
     return h.hexdigest()[:16]
 
 
-def _traffic_from_profiles(workload):
-    """dram bytes per launch from a committed ncu summary, if it was taken on this kernel source."""
+def _src_hash(files):
+    """Hash of kernel source files under csrc/ (what a committed traffic figure was measured on)."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_30_b200", "csrc")
+    for f in files:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_from_profiles(workload, key=None, sha=None):
+    """dram bytes per launch from a committed ncu summary, if it was taken on this kernel source.
+    key: the entry name (default: the workload); sha: the source hash to match (default: the scan kernel's)."""
     p = os.path.join(PROFILE_DIR, "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    ent = d.get(workload)
-    if not ent or ent.get("kernel_src_sha") != _kernel_hash():
+    ent = d.get(key or workload)
+    if not ent or ent.get("kernel_src_sha") != (sha or _kernel_hash()):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -633,6 +644,99 @@ def run_conv1d(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ backward scan
+
+BWD_WORKLOADS = ("mamba-130m", "mamba-1.4b", "mamba-2.8b-long")
+
+
+def _bwd_bytes(d):
+    """Algorithmic HBM bytes of one backward call: u, delta, z, dout, B, C, A, D, bias read;
+    du, ddelta, dz written in the I/O dtype, dB, dC fp32, dA, dD, dbias fp32."""
+    e = 2 if d.dtype == "bf16" else 4
+    elems = d.batch * d.dim * d.seqlen
+    bc = d.batch * d.ngroups * d.dstate * d.seqlen
+    return 7 * elems * e + 2 * bc * e + 2 * bc * 4 + 2 * (d.dim * d.dstate + 2 * d.dim) * 4
+
+
+def run_bwd(args):
+    """ssm_selective_scan_bwd on a layer shape: one JSON line (Gelem/s; roofline against the MUFU ex2 rate,
+    B*D*L*N exps: each dA of the forward must be formed again at least once)."""
+    import torch
+    import ssm_inputs as si
+    import selective_state_space_30_b200 as ssm
+    rank, local, world = _rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+    init_ranks("nccl", local)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = si.workload(args.workload)
+    d = w.dims
+    inp = si.make_inputs(d, w.recipe, w.seed)
+    gin = si.make_grad_inputs(d, 1)
+    t = {k: _to_dev(inp[k], dev) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    dout = _to_dev(gin["dout"], dev)
+    io = ssm.SSM_BF16 if d.dtype == "bf16" else ssm.SSM_F32
+    dims = ssm.make_dims(d.batch, d.dim, d.seqlen, d.dstate, d.H, d.ngroups, io)
+    nws = ssm.ssm_selective_scan_bwd_workspace_size(dims)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"du": torch.empty_like(t["u"]), "ddelta": torch.empty_like(t["delta"]), "dA": torch.empty_like(t["A"]),
+         "dB": torch.empty(t["B"].shape, **f32), "dC": torch.empty(t["C"].shape, **f32),
+         "dD": torch.empty((d.dim,), **f32), "dz": torch.empty_like(t["z"]),
+         "ddelta_bias": torch.empty((d.H,), **f32), "dh0": None}
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = sum(int(x.numel() * x.element_size()) for x in list(t.values()) + [dout] if x is not None)
+
+    def step():
+        ssm.ssm_selective_scan_bwd(dims, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                   t["delta_bias"], True, None, dout, None, g, ws, nws, stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    total = max_over_ranks(e0.elapsed_time(e1), dev)
+    hbm_gbs, sm_max_mhz, src = _peaks()
+    finish_ranks()
+    if rank != 0:
+        return
+    elems = d.batch * d.dim * d.seqlen
+    exps = _exps(d)
+    mufu_peak = SMS * EX2_PER_CLK_PER_SM * sm_max_mhz * 1e6 / 1e9
+    gexps = exps / (ms * 1e-3) / 1e9
+    alg = _bwd_bytes(d)
+    gbs = alg / (ms * 1e-3) / 1e9
+    line = {"metric": "selective-scan backward Gelem/s (B*D*L/s) on 1 B200", "op": "bwd",
+            "value": job_throughput(world, elems, args.steps, total), "unit": "Gelem/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 (bf16 I/O)" if d.dtype == "bf16" else "f32", "data": "synthetic (seeded splitmix64)",
+            "config": {"workload": args.workload, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen,
+                       "dstate": d.dstate, "io_dtype": d.dtype, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs {in_bytes / 1e6:.0f} MB and workspace {nws / 1e6:.0f} MB (> 126 MB L2), "
+                             "no flush"},
+            "roofline": {"bound": "alu", "achieved": gexps, "peak": mufu_peak, "unit": "Gexp/s",
+                         "frac": gexps / mufu_peak,
+                         "traffic": _traffic_from_profiles(args.workload, key="bwd:" + args.workload,
+                                                           sha=_src_hash(("bwd.cu",))),
+                         "peak_source": f"148 SMs x 16 ex2/clk x {sm_max_mhz:.0f} MHz ({src} sm_max_mhz)",
+                         "exps_per_launch": exps,
+                         "hbm": {"achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                                 "alg_bytes_per_launch": alg, "peak_source": src}},
+            "clocks": clk.summary(), "gpu_launches": 2 * args.steps}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -642,9 +746,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", default="scan", choices=["scan", "decode", "conv1d"],
+    ap.add_argument("--op", default="scan", choices=["scan", "decode", "conv1d", "bwd"],
                     help="scan: the forward scan (the headline metric); decode: the single-step state update; "
-                         "conv1d: the causal convolution in front of the scan")
+                         "conv1d: the causal convolution in front of the scan; bwd: the backward scan")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -657,6 +761,13 @@ def main():
         if args.workload == DEFAULT_WORKLOAD:
             args.workload = "conv1d-mamba-130m"
         run_conv1d(args)
+        return
+    if args.op == "bwd":
+        if args.workload == DEFAULT_WORKLOAD:
+            args.workload = "mamba-130m"
+        if args.workload not in BWD_WORKLOADS:
+            raise SystemExit(f"--op bwd runs on {BWD_WORKLOADS}")
+        run_bwd(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -69,16 +69,21 @@ template <> struct Io<__nv_bfloat16> {
     __device__ static raw from(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 };
 
-// shared memory (bytes)
+// shared memory (bytes).  The per-step rows P and U have kPS = kBT + 1 entries per
+// channel, so the four channels a warp reads at one step sit in different banks.
+constexpr int kPS = kBT + 1;
 template <typename T>
 struct Smem {
     static constexpr int kRow = kBT * (int)sizeof(T) + 16;        // staged row stride (16-byte padded)
     static constexpr int STAGE = 0;
-    static constexpr int P = STAGE + kStageRows * kRow;           // float4 [kCT][kBT]: dt, dt*u, dy, dout*silu'(z)
-    static constexpr int U = P + kCT * kBT * 16;                  // float2 [kCT][kBT]: u, sigmoid(x)
-    static constexpr int BC = U + kCT * kBT * 8;                  // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
-    static constexpr int RED = BC + kBT * 8 * 16;                 // float4 [kCT][kWin][8]: dB, dC terms
-    static constexpr int TOTAL = RED + kCT * kWin * 8 * 16;
+    static constexpr int P = STAGE + kStageRows * kRow;           // float4 [kCT][kPS]: dt, dt*u, dy, dout*silu'(z)
+    static constexpr int U = P + kCT * kPS * 16;                  // float2 [kCT][kPS]: u, sigmoid(x)
+    static constexpr int BC = U + kCT * kPS * 8;                  // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
+    static constexpr int RED = BC + kBT * 8 * 16;                 // float4 [bufs][kCT][kWin][8]: dB, dC terms
+    static constexpr int kRedBytes = kCT * kWin * 8 * 16;
+    // two reduction buffers (one barrier per window) where two CTAs per SM still fit
+    static constexpr int kRedBufs = RED + 2 * kRedBytes <= 112 * 1024 ? 2 : 1;
+    static constexpr int TOTAL = RED + kRedBufs * kRedBytes;
 };
 
 // rows x kBT steps [t0, t0 + kBT) of `rows` rows (row r at src + r * stride) into
@@ -115,12 +120,13 @@ __device__ __forceinline__ float staged(const unsigned char* base, int row, int 
 
 __device__ __forceinline__ float sigmoid1(float x) { return rcp_approx(1.f + ex2_approx(x * -kLog2e)); }
 
-// One step of the recurrence on the lane's two states (the same expression in
-// both passes, so the recomputed states equal the checkpointed ones bit for bit).
+// One step of the recurrence on the lane's two states, as f32x2 pairs (the same
+// expression in both passes, so the recomputed states equal the checkpointed ones
+// bit for bit).
 __device__ __forceinline__ void fwd_step(float2& h, float2& dA, float dt, float dtu, float b0, float b1, float2 al) {
-    dA = make_float2(ex2_approx(dt * al.x), ex2_approx(dt * al.y));
-    h.x = fmaf(dA.x, h.x, dtu * b0);
-    h.y = fmaf(dA.y, h.y, dtu * b1);
+    const float2 arg = mul2(dup2(dt), al);
+    dA = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+    h = fma2(dA, h, mul2(dup2(dtu), make_float2(b0, b1)));
 }
 
 // Sum of v over the 8 lanes of a channel (lane bits 0-2 = j), transposed: lane j
@@ -154,7 +160,6 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
     float2* sU = reinterpret_cast<float2*>(smem + S::U);
     float4* sBC = reinterpret_cast<float4*>(smem + S::BC);
     float4* sR = reinterpret_cast<float4*>(smem + S::RED);
-    float* sRf = reinterpret_cast<float*>(smem + S::RED);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = lane >> 3, j = lane & 7;
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             const float xv = staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
             float dt = p.softplus ? softplus1(xv) : xv;
             if (t0 + lane >= L) dt = 0.f;
-            sP[cc * kBT + lane] = make_float4(dt, dt * uv, 0.f, 0.f);
+            sP[cc * kPS + lane] = make_float4(dt, dt * uv, 0.f, 0.f);
         }
         {
             const int t = tid >> 3, jj = tid & 7;
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             *reinterpret_cast<float2*>(ckpt + ((int64_t)(blk * (kBT / kWin) + w) * kCT + c) * kN + 2 * j) = h;
 #pragma unroll 4
             for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
-                const float4 pv = sP[c * kBT + t];
+                const float4 pv = sP[c * kPS + t];
                 const float4 bc = sBC[t * 8 + j];
                 float2 dA;
                 fwd_step(h, dA, pv.x, pv.y, bc.x, bc.y, al);
@@ -229,6 +234,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
     float dbias = 0.f, dDacc = 0.f;
     float* dBrow = p.dBp + cta * kN * L;
     float* dCrow = p.dCp + cta * kN * L;
+    int fw = nwin - 1;   // flat index of the current window, walking down
+    float2 hnext = *reinterpret_cast<const float2*>(ckpt + ((int64_t)fw * kCT + c) * kN + 2 * j);
     for (int blk = nblk - 1; blk >= 0; --blk) {
         const int64_t t0 = (int64_t)blk * kBT;
         __syncthreads();
@@ -256,8 +263,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 dy = gov * zv * s;
                 dzf = gov * (s * fmaf(zv, 1.f - s, 1.f));
             }
-            sP[cc * kBT + lane] = make_float4(dt, dt * uv, dy, dzf);
-            sU[cc * kBT + lane] = make_float2(uv, sp);
+            sP[cc * kPS + lane] = make_float4(dt, dt * uv, dy, dzf);
+            sU[cc * kPS + lane] = make_float2(uv, sp);
         }
         {
             const int t = tid >> 3, jj = tid & 7;
@@ -268,9 +275,10 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         }
         __syncthreads();
 
-        for (int w = kBT / kWin - 1; w >= 0; --w) {
+        for (int w = kBT / kWin - 1; w >= 0; --w, --fw) {
             const int tw = w * kWin;   // first step of the window within the block
-            const float2 he = *reinterpret_cast<const float2*>(ckpt + ((int64_t)(blk * (kBT / kWin) + w) * kCT + c) * kN + 2 * j);
+            const float2 he = hnext;   // the state entering the window
+            if (fw > 0) hnext = *reinterpret_cast<const float2*>(ckpt + ((int64_t)(fw - 1) * kCT + c) * kN + 2 * j);
             float2 hr[kWin], dAr[kWin];
             float yw;   // y of step j of the window, summed over the states
             {
@@ -278,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 float yp[kWin];
 #pragma unroll
                 for (int t = 0; t < kWin; ++t) {
-                    const float4 pv = sP[c * kBT + tw + t];
+                    const float4 pv = sP[c * kPS + tw + t];
                     const float4 bc = sBC[(tw + t) * 8 + j];
                     fwd_step(hh, dAr[t], pv.x, pv.y, bc.x, bc.y, al);
                     hr[t] = hh;
@@ -286,47 +294,49 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 }
                 yw = reduce8(yp, j);
             }
+            float4* red = sR + (S::kRedBufs == 2 ? (fw & 1) : 0) * (S::kRedBytes / 16);
             float gb[kWin], qq[kWin];
 #pragma unroll
             for (int t = kWin - 1; t >= 0; --t) {
-                const float4 pv = sP[c * kBT + tw + t];
+                const float4 pv = sP[c * kPS + tw + t];
                 const float4 bc = sBC[(tw + t) * 8 + j];
-                gs.x = fmaf(pv.z, bc.z, gs.x);   // + dy C: now dLoss/dh_t
-                gs.y = fmaf(pv.z, bc.w, gs.y);
+                gs = fma2(dup2(pv.z), make_float2(bc.z, bc.w), gs);   // + dy C: now dLoss/dh_t
                 const float2 hp = t > 0 ? hr[t - 1] : he;
-                const float2 e = make_float2(gs.x * hp.x * dAr[t].x, gs.y * hp.y * dAr[t].y);
-                dAacc.x = fmaf(e.x, pv.x, dAacc.x);
-                dAacc.y = fmaf(e.y, pv.x, dAacc.y);
+                const float2 e = mul2(mul2(gs, hp), dAr[t]);
+                dAacc = fma2(e, dup2(pv.x), dAacc);
                 gb[t] = fmaf(gs.x, bc.x, gs.y * bc.y);
                 qq[t] = fmaf(e.x, Aln.x, e.y * Aln.y);
-                sR[(c * kWin + t) * 8 + j] = make_float4(gs.x * pv.y, gs.y * pv.y, pv.z * hr[t].x, pv.z * hr[t].y);
-                gs.x *= dAr[t].x;                // carry to t-1
-                gs.y *= dAr[t].y;
-                asm volatile("" ::: "memory");   // keep the next step's loads here (register pressure)
+                const float2 db = mul2(gs, dup2(pv.y)), dc = mul2(dup2(pv.z), hr[t]);
+                red[(c * kWin + t) * 8 + j] = make_float4(db.x, db.y, dc.x, dc.y);
+                gs = mul2(gs, dAr[t]);           // carry to t-1
             }
             const float GB = reduce8(gb, j), Q = reduce8(qq, j);
             __syncwarp();
             {
                 // lane j: step tw + j of channel c
                 const int t = tw + j;
-                const float4 pv = sP[c * kBT + t];
-                const float2 uv = sU[c * kBT + t];
+                const float4 pv = sP[c * kPS + t];
+                const float2 uv = sU[c * kPS + t];
                 const float dd = fmaf(uv.x, GB, Q) * uv.y;
                 dbias += dd;
                 dDacc = fmaf(pv.z, uv.x, dDacc);
-                sP[c * kBT + t] = make_float4(fmaf(pv.x, GB, pv.z * Dc), dd, fmaf(Dc, uv.x, yw) * pv.w, 0.f);
+                sP[c * kPS + t] = make_float4(fmaf(pv.x, GB, pv.z * Dc), dd, fmaf(Dc, uv.x, yw) * pv.w, 0.f);
             }
             __syncthreads();
-            // dB, dC of these 8 steps summed over the tile's channels, in channel order
+            // dB, dC of these 8 steps summed over the tile's channels, in a fixed order
             {
-                float sum = 0.f;
+                const float* rf = reinterpret_cast<const float*>(red);
+                float s0 = 0.f, s1 = 0.f;
 #pragma unroll 8
-                for (int cc = 0; cc < kCT; ++cc) sum += sRf[cc * (kWin * 8 * 4) + tid];
+                for (int cc = 0; cc < kCT; cc += 2) {
+                    s0 += rf[cc * (kWin * 8 * 4) + tid];
+                    s1 += rf[(cc + 1) * (kWin * 8 * 4) + tid];
+                }
                 const int i = tid >> 5, jj = (tid >> 2) & 7, comp = tid & 3;
                 const int64_t t = t0 + tw + i;
-                if (t < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + t] = sum;
+                if (t < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + t] = s0 + s1;
             }
-            __syncthreads();
+            if (S::kRedBufs == 1) __syncthreads();
         }
         // the block's du, ddelta, dz rows of this warp's channels (lane = step)
         __syncwarp();
@@ -335,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int cc = warp * 4 + i;
-                const float4 o = sP[cc * kBT + lane];
+                const float4 o = sP[cc * kPS + lane];
                 const int64_t at = (row0 + cc) * L + t0 + lane;
                 static_cast<R*>(p.du)[at] = Io<T>::from(o.x);
                 static_cast<R*>(p.ddelta)[at] = Io<T>::from(o.y);

@@ -203,8 +203,10 @@ int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A
         ssm::SsdMaps maps;
         std::memset(&maps, 0, sizeof(maps));
         const uint64_t L = (uint64_t)d.seqlen;
-        const bool ok = aligned16(u) && aligned16(B) && aligned16(C) && (!z || aligned16(z)) &&
+        const bool ok = aligned16(u) && aligned16(B) && aligned16(C) && (!z || aligned16(z)) && aligned16(out) &&
                         (reinterpret_cast<uintptr_t>(delta) & 7u) == 0 &&
+                        encode_rows(&maps.out, out, 2, L, (uint64_t)(d.batch * d.dim), 64,
+                                    CU_TENSOR_MAP_SWIZZLE_128B, 64) &&
                         encode_rows(&maps.u, u, 2, L, (uint64_t)(d.batch * d.dim), 64, CU_TENSOR_MAP_SWIZZLE_128B, 64) &&
                         (!z || encode_rows(&maps.z, z, 2, L, (uint64_t)(d.batch * d.dim), 64,
                                            CU_TENSOR_MAP_SWIZZLE_128B, 64)) &&

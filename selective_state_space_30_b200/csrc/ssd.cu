@@ -16,6 +16,9 @@
 //   B' = B diag(w),  w_j = 2^(cum_end - cum_j) dt_j                   threads
 //   H  = 2^cum_end H + B'^T X                    (N x P)              tensor cores + threads
 //
+// The output tile of a chunk is written by the threads over the z tile (each thread
+// writes out(p, t) where it read z(p, t)) and leaves by a TMA store.
+//
 // Operands the tensor cores read: B, C and X straight from TMA boxes (128-byte
 // swizzle; B and C as MN-major tiles, X as K-major), M and B' as K-major tiles
 // and H as an MN-major tile written by the threads.  M, B' and H are fp32
@@ -82,14 +85,15 @@ __device__ __forceinline__ float bf16_at(const unsigned char* tile, uint32_t r, 
     return __bfloat162float(__ushort_as_bfloat16(*reinterpret_cast<const unsigned short*>(tile + tc::sw128_off(r, c))));
 }
 
-// The decay vectors of the chunk starting at t0, four steps per lane of one warp:
+// The decay vectors of one chunk from its delta bits (delta_bits: four steps per lane of one warp):
 // dt, the prefix cum (log2 units), and w = 2^(cum_end - cum) dt, the weight of each
 // step's input in the chunk's final state (at most dt, since cum only falls).
-__device__ __forceinline__ void chunk_decay(const SsdParams& p, int64_t b, int64_t h, int64_t t0, float Ah, float bias,
-                                            int lane, float* sdt, float* scum, float* sw) {
-    const unsigned short* drow =
-        reinterpret_cast<const unsigned short*>(p.delta) + (b * p.nheads + h) * p.seqlen + t0 + 4 * lane;
-    const uint2 raw = *reinterpret_cast<const uint2*>(drow);
+__device__ __forceinline__ uint2 delta_bits(const SsdParams& p, int64_t b, int64_t h, int64_t t0, int lane) {
+    return __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const unsigned short*>(p.delta) +
+                                                (b * p.nheads + h) * p.seqlen + t0 + 4 * lane));
+}
+__device__ __forceinline__ void chunk_decay(const SsdParams& p, uint2 raw, float Ah, float bias, int lane, float* sdt,
+                                            float* scum, float* sw) {
     const uint32_t w2[2] = {raw.x, raw.y};
     float dt[4], pre[4], run = 0.f;
 #pragma unroll
@@ -118,6 +122,18 @@ __device__ __forceinline__ void chunk_decay(const SsdParams& p, int64_t b, int64
     *reinterpret_cast<float4*>(scum + 4 * lane) = make_float4(cm[0], cm[1], cm[2], cm[3]);
     *reinterpret_cast<float4*>(sw + 4 * lane) = make_float4(wv[0], wv[1], wv[2], wv[3]);
 }
+
+// TMA store of a 2-D box from shared memory; bulk-group completion
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
+                 "r"(y), "r"(tc::smem_addr(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the committed stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the committed stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // 8 consecutive floats from shared memory (16-byte aligned)
 __device__ __forceinline__ void lds8f(const float* src, float (&v)[8]) {
@@ -167,6 +183,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
     const int x_row = (int)(b * Dm + d0);
     const bool gate = p.z != nullptr;
     const uint32_t tx_x = gate ? 2 * kTxX : kTxX;
+    const int nchunks = (int)(L / kQ);
 
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
@@ -178,7 +195,6 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
     tc::fence_after();
     const uint32_t tbase = *tslot;
     const uint32_t trow = tbase + ((uint32_t)(32 * quarter) << 16);
-    const int nchunks = (int)(L / kQ);
 
     // chunk 0's tiles and decay
     if (tid == 0) {
@@ -191,7 +207,12 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             if (gate) tma_2d(sZ + hb * 8192, &m.z, 64 * hb, x_row, full_x);
         }
     }
-    if (warp == 0) chunk_decay(p, b, h, 0, Ah, bias, lane, sdec, sdec + kQ, sdec + 2 * kQ);
+    // warp 0: the decay vectors of chunk 0, and the delta bits of chunk 1 one chunk ahead
+    uint2 dnext = make_uint2(0u, 0u);
+    if (warp == 0) {
+        chunk_decay(p, delta_bits(p, b, h, 0, lane), Ah, bias, lane, sdec, sdec + kQ, sdec + 2 * kQ);
+        if (nchunks > 1) dnext = delta_bits(p, b, h, kQ, lane);
+    }
 
     // the state: row n = row, channels p0 .. p0+15; skip weights of those channels
     float H[16], Dv[16];
@@ -242,7 +263,8 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         // meanwhile: the next chunk's decay, and this step's gate inputs
         if (warp == 0 && c + 1 < nchunks) {
             float* nd = sdec + ((c + 1) & 1) * kDec;
-            chunk_decay(p, b, h, t0 + kQ, Ah, bias, lane, nd, nd + kQ, nd + 2 * kQ);
+            chunk_decay(p, dnext, Ah, bias, lane, nd, nd + kQ, nd + 2 * kQ);
+            if (c + 2 < nchunks) dnext = delta_bits(p, b, h, t0 + 2 * kQ, lane);
         }
 
         const bool ok_g = mbar_wait(mb_g, ph, budget, p.status);
@@ -320,15 +342,16 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             if (with_state) tc::after_wait(cv);
             const float e = with_state ? ex2_approx(scum[row]) : 0.f;
             const unsigned char* xt = sX + (row >> 6) * 8192;
-            const unsigned char* zt = sZ + (row >> 6) * 8192;
+            unsigned char* zt = sZ + (row >> 6) * 8192;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const float x = bf16_at(xt, p0 + k, row & 63u);
                 float v = __uint_as_float(yv[k]);
                 if (with_state) v = fmaf(e, __uint_as_float(cv[k]), v);
                 v = fmaf(Dv[k], x, v);
-                if (gate) v *= silu1(bf16_at(zt, p0 + k, row & 63u));
-                p.out[(b * Dm + d0 + p0 + k) * L + t0 + row] = __float2bfloat16_rn(v);
+                unsigned short* slot = reinterpret_cast<unsigned short*>(zt + tc::sw128_off(p0 + k, row & 63u));
+                if (gate) v *= silu1(__bfloat162float(__ushort_as_bfloat16(*slot)));
+                *slot = __bfloat16_as_ushort(__float2bfloat16_rn(v));   // out(p, t) where z(p, t) was
             }
         }
         // ---- B' = B diag(w): row n = row, steps j0 .. j0+31
@@ -353,8 +376,12 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         tc::fence_before();
         __syncthreads();
 
-        // ---- S = B'^T X; then the next chunk's C and B tiles (this chunk is done with them)
+        // ---- the out tile (written over the z tile) to global; S = B'^T X; then the next
+        // chunk's C and B tiles (this chunk is done with them)
         if (tid == 0) {
+            tma_store_2d(&m.out, (int)t0, x_row, sZ);
+            tma_store_2d(&m.out, (int)t0 + 64, x_row, sZ + 8192);
+            bulk_commit();
             tc::fence_after();
             constexpr uint32_t ids = tc::idesc_bf16(128, kP, false, false);
 #pragma unroll
@@ -381,6 +408,9 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         tc::fence_after();
         // the next chunk's X and z tiles (this chunk's MMAs that read X are complete, and
         // its outputs were written before the barrier above)
+        // the out tile must be read out of shared memory before the z tile is loaded over it,
+        // or (no gate) before the next chunk's outputs are written there after the barriers below
+        if (tid == 0) bulk_wait_read();
         if (tid == 0 && c + 1 < nchunks) {
             mbar_arrive_tx(full_x, tx_x);
             for (int hb = 0; hb < 2; ++hb) {
@@ -417,6 +447,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
     // release TMEM once nothing can still write it: after a failed wait, wait (bounded) for
     // the last tensor-core batch this CTA committed
     if (failed && tid == 0 && last_bar) mbar_wait(last_bar, last_ph, budget, p.status);
+    if (tid == 0) bulk_wait_all();   // the last out tile is written before shared memory goes away
     tc::fence_before();
     __syncthreads();
     tc::fence_after();

@@ -27,10 +27,10 @@ struct SsdParams {
 };
 
 // 2-D tensor maps (time x rows), 64-step boxes with the 128-byte swizzle:
-// u and z rows (batch*dim) in boxes of 64 rows, B and C rows (batch*ngroups*dstate) in
-// boxes of 128 rows; z is unused (and may be left zero) when there is no gate.
+// u, z and out rows (batch*dim) in boxes of 64 rows, B and C rows (batch*ngroups*dstate)
+// in boxes of 128 rows; z is unused (and may be left zero) when there is no gate.
 struct SsdMaps {
-    CUtensorMap u, z, B, C;
+    CUtensorMap u, z, B, C, out;
 };
 
 // bf16 I/O, nheads < dim with dim/nheads == 64, dstate == 128, seqlen a positive multiple of 128.

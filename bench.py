@@ -422,6 +422,7 @@ def run_ours(args):
                       "frac": flops / avg_launch_s / 1e12 / tf, "peak_source": tf_src,
                       "flops_per_launch": flops, "what": "algorithmic SSD flops (G, M X, C H, B'^T X per chunk)"}
         main = dict(hbm_obj, bound="hbm") if t_hbm >= t_tc else dict(tensor_obj, bound="tensor")
+        traffic = _traffic_from_profiles(w.name, key="ssd:" + w.name, sha=_src_hash(("ssd.cu", "tcgen05.cuh")))
         roof = dict(main, traffic=traffic, roofline_frac=max(t_hbm, t_tc) / avg_launch_s,
                     hbm=hbm_obj, tensor=tensor_obj,
                     mufu_literal=dict(mufu_obj, note="B*D*L*N exps: the SSD path takes one exp per (t, head)"))

@@ -275,10 +275,15 @@ int ssm_causal_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t wi
  *     ddelta_bias   (nheads) fp32, nullable: not computed
  *     dh0           (batch, dim, dstate) fp32, nullable: not computed
  * The call allocates nothing: `workspace` (device, 256-byte aligned, at least
- * ssm_selective_scan_bwd_workspace_size bytes; about batch*dim*seqlen*4 bytes of
- * state checkpoints plus per-tile dB/dC rows) is the caller's and is scratch
- * after the call.  Two kernels on `stream`; the sums run in a fixed order, so
- * repeated calls give identical bits.  A, h0, dlast and dh0 must be 8-byte
+ * ssm_selective_scan_bwd_workspace_size bytes, which depends on the shape and on
+ * the current device's SM count; about batch*dim*seqlen*8 bytes of state
+ * checkpoints plus per-tile dB/dC rows) is the caller's and is scratch after the
+ * call; one workspace must not serve two calls at once.  Two kernels on `stream`
+ * (after two small memsets of the workspace's counters); the sums run in a fixed
+ * order, so repeated calls give identical bits.  The first kernel runs work units
+ * (32 channels x a segment of the sequence) on persistent CTAs whose bounded waits
+ * record SSM_ERR_TIMEOUT in the workspace; read it with
+ * ssm_selective_scan_bwd_device_status.  A, h0, dlast and dh0 must be 8-byte
  * aligned (else SSM_ERR_UNSUPPORTED).  SSM_ERR_INVALID_ARG for a NULL required
  * pointer (u, delta, A, B, C, dout, grads, du, ddelta, dA, dB, dC, workspace),
  * a bad shape or a workspace that is too small.
@@ -302,6 +307,10 @@ int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, const void* de
                            const float* delta_bias, int softplus, const float* h0, const void* dout,
                            const float* dlast, const ssm_grads_t* grads, void* workspace,
                            size_t workspace_bytes, ssm_stream_t stream);
+
+/* Synchronise `stream` and return the kernel-side status of the last backward call that
+ * used `workspace` (SSM_OK or SSM_ERR_TIMEOUT), clearing it. */
+int ssm_selective_scan_bwd_device_status(void* workspace, ssm_stream_t stream);
 
 /* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
 int ssm_scan_destroy(ssm_plan_t plan);

@@ -27,6 +27,7 @@ SSM_BF16 = 1
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
            "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update",
            "ssm_causal_conv1d_fwd", "ssm_selective_scan_bwd_workspace_size", "ssm_selective_scan_bwd",
+           "ssm_selective_scan_bwd_device_status",
            "ssm_scan_set_option",
            "ssm_scan_plan_schedule", "ssm_scan_destroy",
            "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
@@ -86,6 +87,7 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_bwd_workspace_size.argtypes = [dims_p, ctypes.POINTER(ctypes.c_size_t)]
     lib.ssm_selective_scan_bwd.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
                                            ctypes.POINTER(ssm_grads_t), vp, ctypes.c_size_t, vp]
+    lib.ssm_selective_scan_bwd_device_status.argtypes = [vp, vp]
     lib.ssm_scan_destroy.argtypes = [vp]
     lib.ssm_scan_device_status.argtypes = [vp, vp]
     lib.ssm_status_string.argtypes = [i32]
@@ -216,6 +218,11 @@ def ssm_selective_scan_bwd(dims: ssm_dims_t, u, delta, A, B, C, D, z, delta_bias
         1 if softplus else 0, _ptr(h0), _ptr(dout), _ptr(dlast), ctypes.byref(g), _ptr(workspace),
         int(workspace_bytes), _stream(stream))
     return _check(rc, "ssm_selective_scan_bwd") if check else rc
+
+
+def ssm_selective_scan_bwd_device_status(workspace, stream=None) -> int:
+    """Kernel-side status of the last backward call on `workspace` (syncs the stream, clears it)."""
+    return int(load_library().ssm_selective_scan_bwd_device_status(_ptr(workspace), _stream(stream)))
 
 
 def ssm_scan_destroy(plan: Optional[int]) -> int:

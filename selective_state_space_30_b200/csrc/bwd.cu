@@ -18,12 +18,17 @@
 //   da_n += g_n h_(t-1)n dt dA_tn g_n <- dA_tn g_n
 //   ddelta_t = ddt_t sigmoid(x_t),  dbias += ddelta_t,  dz_t = dout y_t silu'(z_t)
 //
-// One CTA takes 32 channels of one batch row (S6 layout, dstate 16): eight
-// warps, each four channels x 8 lanes x 2 states.  Pass 1 runs the recurrence
-// forward and stores the state at the start of every 8-step window (the
-// checkpoints).  Pass 2 walks the 32-step blocks backwards; per window it
+// A tile is 32 channels of one batch row (S6 layout, dstate 16), run by eight
+// warps, each four channels x 8 lanes x 2 states.  Its sequence is cut into
+// segments, and the work units (tile, segment) go to persistent CTAs from a
+// ticket counter: first every forward unit, segment-major, then every reverse
+// unit, last segment first.  A forward unit runs the recurrence from the state
+// its predecessor handed over and stores the state at the start of every 8-step
+// window (the checkpoints).  A reverse unit takes the state gradient from the
+// segment after it, walks its 32-step blocks backwards, and per window
 // recomputes the 8 states and decays from the checkpoint into registers, then
-// runs the window in reverse.  Sums over the states (y, sum g B, the decay term)
+// runs the window in reverse.  A unit waits (bounded) only on units with smaller
+// tickets, which running CTAs hold, so the chain always progresses.  Sums over the states (y, sum g B, the decay term)
 // are transposed shuffle reductions inside the 8 lanes of a channel; dB and dC,
 // sums over channels, go through shared memory to per-CTA partial rows, which a
 // second kernel adds in a fixed order with the per-row dA, dD and dbias
@@ -51,10 +56,19 @@ struct BwdParams {
     const float *A, *D, *bias, *h0, *dlast;
     void *du, *ddelta, *dz;
     float* dh0;
-    float *ckpt, *dBp, *dCp, *dAp, *dDp, *dbp;   // workspace
+    // workspace
+    unsigned* ticket;            // work-unit counter (zeroed before the launch)
+    int* status;                 // kernel-side ssm_status_t
+    unsigned *flag1, *flag2;     // [tile][seg]: forward / reverse segment done (zeroed before the launch)
+    float *carry1, *carry2;      // [tile][seg][kCT][kN]: state after / state gradient before a segment
+    float *ckpt, *dBp, *dCp;     // checkpoints [tile][window][kCT][kN]; dB, dC rows [tile][kN][L]
+    float *dAp, *dDp, *dbp;      // per segment and (b, d) row: [seg][row][kN], [seg][row], [seg][row]
     int64_t batch, dim, seqlen, ngroups;
-    int tiles_per_row;   // dim / kCT
+    int64_t ntiles;              // batch * dim / kCT
+    int tiles_per_row;           // dim / kCT
+    int nseg, seg_blocks;        // segments per tile, 32-step blocks per segment
     int softplus;
+    uint64_t budget_ns;          // bounded waits
 };
 
 template <typename T> struct Io;
@@ -164,211 +178,283 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = lane >> 3, j = lane & 7;
     const int c = warp * 4 + q;                    // channel within the tile
-    const int64_t cta = blockIdx.x;                // = b * tiles_per_row + tile
-    const int64_t b = cta / p.tiles_per_row;
+    __shared__ unsigned s_ticket;
     const int64_t L = p.seqlen, Dm = p.dim, G = p.ngroups;
-    const int64_t row0 = cta * kCT;                // first (b, d) row of the tile
-    const int64_t d0 = row0 - b * Dm;
-    const int64_t g = d0 / (Dm / G);
-    const int64_t d = d0 + c;
-    const T* u = static_cast<const T*>(p.u) + row0 * L;
-    const T* dl = static_cast<const T*>(p.delta) + row0 * L;
-    const T* zz = p.z ? static_cast<const T*>(p.z) + row0 * L : nullptr;
-    const T* go = static_cast<const T*>(p.dout) + row0 * L;
-    const T* Bg = static_cast<const T*>(p.B) + (b * G + g) * kN * L;
-    const T* Cg = static_cast<const T*>(p.C) + (b * G + g) * kN * L;
+    const int64_t rows = p.batch * Dm;
     const bool vec = (L % (16 / (int64_t)sizeof(T))) == 0 &&
                      ((reinterpret_cast<uintptr_t>(p.u) | reinterpret_cast<uintptr_t>(p.delta) |
                        reinterpret_cast<uintptr_t>(p.z) | reinterpret_cast<uintptr_t>(p.dout) |
                        reinterpret_cast<uintptr_t>(p.B) | reinterpret_cast<uintptr_t>(p.C)) & 15u) == 0;
     const int nblk = (int)((L + kBT - 1) / kBT);
     const int nwin = nblk * (kBT / kWin);
-    float* ckpt = p.ckpt + cta * (int64_t)nwin * kCT * kN;
+    const int64_t per_pass = p.ntiles * p.nseg;
 
-    const float2 Aln = make_float2(__ldg(p.A + d * kN + 2 * j), __ldg(p.A + d * kN + 2 * j + 1));
-    const float2 al = make_float2(Aln.x * kLog2e, Aln.y * kLog2e);
-    const float bias_c = p.bias ? __ldg(p.bias + d) : 0.f;
-    const float Dc = p.D ? __ldg(p.D + d) : 0.f;
+    for (;;) {
+        __syncthreads();   // the previous unit is done with shared memory and s_ticket
+        if (tid == 0) s_ticket = atomicAdd(p.ticket, 1u);
+        __syncthreads();
+        const int64_t k = s_ticket;
+        if (k >= 2 * per_pass) break;
+        const bool fwd = k < per_pass;
+        const int64_t kk = fwd ? k : k - per_pass;
+        const int seg = fwd ? (int)(kk / p.ntiles) : p.nseg - 1 - (int)(kk / p.ntiles);
+        const int64_t tile = kk % p.ntiles;        // = b * tiles_per_row + tile in the row
+        const int64_t b = tile / p.tiles_per_row;
+        const int64_t row0 = tile * kCT;           // first (b, d) row of the tile
+        const int64_t d0 = row0 - b * Dm;
+        const int64_t g = d0 / (Dm / G);
+        const int64_t d = d0 + c;
+        const T* u = static_cast<const T*>(p.u) + row0 * L;
+        const T* dl = static_cast<const T*>(p.delta) + row0 * L;
+        const T* zz = p.z ? static_cast<const T*>(p.z) + row0 * L : nullptr;
+        const T* go = static_cast<const T*>(p.dout) + row0 * L;
+        const T* Bg = static_cast<const T*>(p.B) + (b * G + g) * kN * L;
+        const T* Cg = static_cast<const T*>(p.C) + (b * G + g) * kN * L;
+        float* ckpt = p.ckpt + tile * (int64_t)nwin * kCT * kN;
+        const int blk0 = seg * p.seg_blocks;
+        const int blk1 = min(nblk, blk0 + p.seg_blocks);
+        const int64_t us = tile * p.nseg + seg;    // this unit's flag / carry slot
+        const float2 Aln = make_float2(__ldg(p.A + d * kN + 2 * j), __ldg(p.A + d * kN + 2 * j + 1));
+        const float2 al = make_float2(Aln.x * kLog2e, Aln.y * kLog2e);
+        const float Dc = p.D ? __ldg(p.D + d) : 0.f;
 
-    // ---------------- pass 1: the recurrence forward, checkpoints at every window start
-    float2 h = p.h0 ? *reinterpret_cast<const float2*>(p.h0 + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
-    for (int blk = 0; blk < nblk; ++blk) {
-        const int64_t t0 = (int64_t)blk * kBT;
-        __syncthreads();   // the previous block is done with the staged rows and the B tile
-        stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
-        stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
-        stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
-        __syncthreads();
-        // dt and dt*u of this warp's 4 channels, lane = step
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int cc = warp * 4 + i;
-            const float uv = staged<T>(stage, cc, lane);
-            const float xv = staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
-            float dt = p.softplus ? softplus1(xv) : xv;
-            if (t0 + lane >= L) dt = 0.f;
-            sP[cc * kPS + lane] = make_float4(dt, dt * uv, 0.f, 0.f);
+        // bounded waits (thread 0) for the units this one depends on; a wait that runs out, or
+        // a status already set by another CTA, records the failure and the unit goes on with
+        // whatever it finds (the call then reports SSM_ERR_TIMEOUT and its outputs are invalid)
+        if (tid == 0) {
+            bool ok = true;
+            const unsigned* need[2] = {nullptr, nullptr};
+            if (fwd && seg > 0) need[0] = p.flag1 + us - 1;
+            if (!fwd) {
+                need[0] = p.flag1 + us;
+                if (seg + 1 < p.nseg) need[1] = p.flag2 + us + 1;
+            }
+            for (int w = 0; w < 2; ++w) {
+                if (!need[w]) continue;
+                const uint64_t t_start = now_ns();
+                while (ld_acquire(need[w]) == 0u) {
+                    __nanosleep(128);   // leave the issue slots to the working warps of this SM
+                    if (*reinterpret_cast<volatile int*>(p.status) != SSM_OK) { ok = false; break; }
+                    if (now_ns() - t_start > p.budget_ns) {
+                        atomicCAS(p.status, SSM_OK, SSM_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok) break;
+            }
         }
-        {
-            const int t = tid >> 3, jj = tid & 7;
-            const unsigned char* sb = stage + 4 * kCT * S::kRow;
-            sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t), 0.f, 0.f);
-        }
         __syncthreads();
+
+        if (fwd) {
+            // ---------------- forward unit: the recurrence, checkpoints at every window start
+            float2 h;
+            if (seg == 0)
+                h = p.h0 ? *reinterpret_cast<const float2*>(p.h0 + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
+            else
+                h = __ldcg(reinterpret_cast<const float2*>(p.carry1 + ((us - 1) * kCT + c) * kN + 2 * j));
+            for (int blk = blk0; blk < blk1; ++blk) {
+                const int64_t t0 = (int64_t)blk * kBT;
+                __syncthreads();   // the previous block is done with the staged rows and the B tile
+                stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
+                stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
+                stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
+                __syncthreads();
+                // dt and dt*u of this warp's 4 channels, lane = step
 #pragma unroll
-        for (int w = 0; w < kBT / kWin; ++w) {
-            *reinterpret_cast<float2*>(ckpt + ((int64_t)(blk * (kBT / kWin) + w) * kCT + c) * kN + 2 * j) = h;
+                for (int i = 0; i < 4; ++i) {
+                    const int cc = warp * 4 + i;
+                    const float uv = staged<T>(stage, cc, lane);
+                    const float xv =
+                        staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
+                    float dt = p.softplus ? softplus1(xv) : xv;
+                    if (t0 + lane >= L) dt = 0.f;
+                    sP[cc * kPS + lane] = make_float4(dt, dt * uv, 0.f, 0.f);
+                }
+                {
+                    const int t = tid >> 3, jj = tid & 7;
+                    const unsigned char* sb = stage + 4 * kCT * S::kRow;
+                    sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t), 0.f, 0.f);
+                }
+                __syncthreads();
+#pragma unroll
+                for (int w = 0; w < kBT / kWin; ++w) {
+                    *reinterpret_cast<float2*>(ckpt + ((int64_t)(blk * (kBT / kWin) + w) * kCT + c) * kN + 2 * j) = h;
 #pragma unroll 4
-            for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
-                const float4 pv = sP[c * kPS + t];
-                const float4 bc = sBC[t * 8 + j];
-                float2 dA;
-                fwd_step(h, dA, pv.x, pv.y, bc.x, bc.y, al);
-            }
-        }
-    }
-
-    // ---------------- pass 2: blocks backwards, windows recomputed from their checkpoints
-    float2 gs = p.dlast ? *reinterpret_cast<const float2*>(p.dlast + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
-    float2 dAacc = make_float2(0.f, 0.f);
-    float dbias = 0.f, dDacc = 0.f;
-    float* dBrow = p.dBp + cta * kN * L;
-    float* dCrow = p.dCp + cta * kN * L;
-    int fw = nwin - 1;   // flat index of the current window, walking down
-    float2 hnext = *reinterpret_cast<const float2*>(ckpt + ((int64_t)fw * kCT + c) * kN + 2 * j);
-    for (int blk = nblk - 1; blk >= 0; --blk) {
-        const int64_t t0 = (int64_t)blk * kBT;
-        __syncthreads();
-        stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
-        stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
-        if (zz) stage_rows<T>(stage + 2 * kCT * S::kRow, zz, L, kCT, t0, L, vec, tid);
-        stage_rows<T>(stage + 3 * kCT * S::kRow, go, L, kCT, t0, L, vec, tid);
-        stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
-        stage_rows<T>(stage + (4 * kCT + kN) * S::kRow, Cg, L, kN, t0, L, vec, tid);
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int cc = warp * 4 + i;
-            const bool valid = t0 + lane < L;
-            const float uv = staged<T>(stage, cc, lane);
-            const float xv = staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
-            const float gov = staged<T>(stage + 3 * kCT * S::kRow, cc, lane);
-            float dt = p.softplus ? softplus1(xv) : xv;
-            float sp = p.softplus ? sigmoid1(xv) : 1.f;
-            if (!valid) dt = sp = 0.f;
-            float dy = gov, dzf = 0.f;
-            if (zz) {
-                const float zv = staged<T>(stage + 2 * kCT * S::kRow, cc, lane);
-                const float s = sigmoid1(zv);
-                dy = gov * zv * s;
-                dzf = gov * (s * fmaf(zv, 1.f - s, 1.f));
-            }
-            sP[cc * kPS + lane] = make_float4(dt, dt * uv, dy, dzf);
-            sU[cc * kPS + lane] = make_float2(uv, sp);
-        }
-        {
-            const int t = tid >> 3, jj = tid & 7;
-            const unsigned char* sb = stage + 4 * kCT * S::kRow;
-            const unsigned char* sc = stage + (4 * kCT + kN) * S::kRow;
-            sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t),
-                                          staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
-        }
-        __syncthreads();
-
-        for (int w = kBT / kWin - 1; w >= 0; --w, --fw) {
-            const int tw = w * kWin;   // first step of the window within the block
-            const float2 he = hnext;   // the state entering the window
-            if (fw > 0) hnext = *reinterpret_cast<const float2*>(ckpt + ((int64_t)(fw - 1) * kCT + c) * kN + 2 * j);
-            float2 hr[kWin], dAr[kWin];
-            float yw;   // y of step j of the window, summed over the states
-            {
-                float2 hh = he;
-                float yp[kWin];
-#pragma unroll
-                for (int t = 0; t < kWin; ++t) {
-                    const float4 pv = sP[c * kPS + tw + t];
-                    const float4 bc = sBC[(tw + t) * 8 + j];
-                    fwd_step(hh, dAr[t], pv.x, pv.y, bc.x, bc.y, al);
-                    hr[t] = hh;
-                    yp[t] = fmaf(bc.z, hh.x, bc.w * hh.y);
+                    for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
+                        const float4 pv = sP[c * kPS + t];
+                        const float4 bc = sBC[t * 8 + j];
+                        float2 dA;
+                        fwd_step(h, dA, pv.x, pv.y, bc.x, bc.y, al);
+                    }
                 }
-                yw = reduce8(yp, j);
             }
-            float4* red = sR + (S::kRedBufs == 2 ? (fw & 1) : 0) * (S::kRedBytes / 16);
-            float gb[kWin], qq[kWin];
-#pragma unroll
-            for (int t = kWin - 1; t >= 0; --t) {
-                const float4 pv = sP[c * kPS + tw + t];
-                const float4 bc = sBC[(tw + t) * 8 + j];
-                gs = fma2(dup2(pv.z), make_float2(bc.z, bc.w), gs);   // + dy C: now dLoss/dh_t
-                const float2 hp = t > 0 ? hr[t - 1] : he;
-                const float2 e = mul2(mul2(gs, hp), dAr[t]);
-                dAacc = fma2(e, dup2(pv.x), dAacc);
-                gb[t] = fmaf(gs.x, bc.x, gs.y * bc.y);
-                qq[t] = fmaf(e.x, Aln.x, e.y * Aln.y);
-                const float2 db = mul2(gs, dup2(pv.y)), dc = mul2(dup2(pv.z), hr[t]);
-                red[(c * kWin + t) * 8 + j] = make_float4(db.x, db.y, dc.x, dc.y);
-                gs = mul2(gs, dAr[t]);           // carry to t-1
-            }
-            const float GB = reduce8(gb, j), Q = reduce8(qq, j);
-            __syncwarp();
-            {
-                // lane j: step tw + j of channel c
-                const int t = tw + j;
-                const float4 pv = sP[c * kPS + t];
-                const float2 uv = sU[c * kPS + t];
-                const float dd = fmaf(uv.x, GB, Q) * uv.y;
-                dbias += dd;
-                dDacc = fmaf(pv.z, uv.x, dDacc);
-                sP[c * kPS + t] = make_float4(fmaf(pv.x, GB, pv.z * Dc), dd, fmaf(Dc, uv.x, yw) * pv.w, 0.f);
-            }
+            // hand the state to the next segment; the checkpoints go with it
+            *reinterpret_cast<float2*>(p.carry1 + (us * kCT + c) * kN + 2 * j) = h;
             __syncthreads();
-            // dB, dC of these 8 steps summed over the tile's channels, in a fixed order
-            {
-                const float* rf = reinterpret_cast<const float*>(red);
-                float s0 = 0.f, s1 = 0.f;
-#pragma unroll 8
-                for (int cc = 0; cc < kCT; cc += 2) {
-                    s0 += rf[cc * (kWin * 8 * 4) + tid];
-                    s1 += rf[(cc + 1) * (kWin * 8 * 4) + tid];
-                }
-                const int i = tid >> 5, jj = (tid >> 2) & 7, comp = tid & 3;
-                const int64_t t = t0 + tw + i;
-                if (t < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + t] = s0 + s1;
+            if (tid == 0) {
+                __threadfence();
+                st_release(p.flag1 + us, 1u);
             }
-            if (S::kRedBufs == 1) __syncthreads();
+            continue;
         }
-        // the block's du, ddelta, dz rows of this warp's channels (lane = step)
-        __syncwarp();
-        if (t0 + lane < L) {
-            using R = typename Io<T>::raw;
+
+        // ---------------- reverse unit: blocks backwards, windows recomputed from their checkpoints
+        float2 gs;
+        if (seg + 1 < p.nseg)
+            gs = __ldcg(reinterpret_cast<const float2*>(p.carry2 + ((us + 1) * kCT + c) * kN + 2 * j));
+        else
+            gs = p.dlast ? *reinterpret_cast<const float2*>(p.dlast + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
+        float2 dAacc = make_float2(0.f, 0.f);
+        float dbias = 0.f, dDacc = 0.f;
+        float* dBrow = p.dBp + tile * kN * L;
+        float* dCrow = p.dCp + tile * kN * L;
+        const int fw0 = blk0 * (kBT / kWin);             // first window of the segment
+        int fw = blk1 * (kBT / kWin) - 1;                // flat index of the current window, walking down
+        float2 hnext = __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)fw * kCT + c) * kN + 2 * j));
+        for (int blk = blk1 - 1; blk >= blk0; --blk) {
+            const int64_t t0 = (int64_t)blk * kBT;
+            __syncthreads();
+            stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
+            stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
+            if (zz) stage_rows<T>(stage + 2 * kCT * S::kRow, zz, L, kCT, t0, L, vec, tid);
+            stage_rows<T>(stage + 3 * kCT * S::kRow, go, L, kCT, t0, L, vec, tid);
+            stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
+            stage_rows<T>(stage + (4 * kCT + kN) * S::kRow, Cg, L, kN, t0, L, vec, tid);
+            __syncthreads();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int cc = warp * 4 + i;
-                const float4 o = sP[cc * kPS + lane];
-                const int64_t at = (row0 + cc) * L + t0 + lane;
-                static_cast<R*>(p.du)[at] = Io<T>::from(o.x);
-                static_cast<R*>(p.ddelta)[at] = Io<T>::from(o.y);
-                if (zz) static_cast<R*>(p.dz)[at] = Io<T>::from(o.z);
+                const bool valid = t0 + lane < L;
+                const float uv = staged<T>(stage, cc, lane);
+                const float xv =
+                    staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
+                const float gov = staged<T>(stage + 3 * kCT * S::kRow, cc, lane);
+                float dt = p.softplus ? softplus1(xv) : xv;
+                float sp = p.softplus ? sigmoid1(xv) : 1.f;
+                if (!valid) dt = sp = 0.f;
+                float dy = gov, dzf = 0.f;
+                if (zz) {
+                    const float zv = staged<T>(stage + 2 * kCT * S::kRow, cc, lane);
+                    const float sg = sigmoid1(zv);
+                    dy = gov * zv * sg;
+                    dzf = gov * (sg * fmaf(zv, 1.f - sg, 1.f));
+                }
+                sP[cc * kPS + lane] = make_float4(dt, dt * uv, dy, dzf);
+                sU[cc * kPS + lane] = make_float2(uv, sp);
+            }
+            {
+                const int t = tid >> 3, jj = tid & 7;
+                const unsigned char* sb = stage + 4 * kCT * S::kRow;
+                const unsigned char* sc = stage + (4 * kCT + kN) * S::kRow;
+                sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t),
+                                              staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
+            }
+            __syncthreads();
+
+            for (int w = kBT / kWin - 1; w >= 0; --w, --fw) {
+                const int tw = w * kWin;   // first step of the window within the block
+                const float2 he = hnext;   // the state entering the window
+                if (fw > fw0)
+                    hnext = __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)(fw - 1) * kCT + c) * kN + 2 * j));
+                float2 hr[kWin], dAr[kWin];
+                float yw;   // y of step j of the window, summed over the states
+                {
+                    float2 hh = he;
+                    float yp[kWin];
+#pragma unroll
+                    for (int t = 0; t < kWin; ++t) {
+                        const float4 pv = sP[c * kPS + tw + t];
+                        const float4 bc = sBC[(tw + t) * 8 + j];
+                        fwd_step(hh, dAr[t], pv.x, pv.y, bc.x, bc.y, al);
+                        hr[t] = hh;
+                        yp[t] = fmaf(bc.z, hh.x, bc.w * hh.y);
+                    }
+                    yw = reduce8(yp, j);
+                }
+                float4* red = sR + (S::kRedBufs == 2 ? (fw & 1) : 0) * (S::kRedBytes / 16);
+                float gb[kWin], qq[kWin];
+#pragma unroll
+                for (int t = kWin - 1; t >= 0; --t) {
+                    const float4 pv = sP[c * kPS + tw + t];
+                    const float4 bc = sBC[(tw + t) * 8 + j];
+                    gs = fma2(dup2(pv.z), make_float2(bc.z, bc.w), gs);   // + dy C: now dLoss/dh_t
+                    const float2 hp = t > 0 ? hr[t - 1] : he;
+                    const float2 e = mul2(mul2(gs, hp), dAr[t]);
+                    dAacc = fma2(e, dup2(pv.x), dAacc);
+                    gb[t] = fmaf(gs.x, bc.x, gs.y * bc.y);
+                    qq[t] = fmaf(e.x, Aln.x, e.y * Aln.y);
+                    const float2 db = mul2(gs, dup2(pv.y)), dc = mul2(dup2(pv.z), hr[t]);
+                    red[(c * kWin + t) * 8 + j] = make_float4(db.x, db.y, dc.x, dc.y);
+                    gs = mul2(gs, dAr[t]);           // carry to t-1
+                }
+                const float GB = reduce8(gb, j), Q = reduce8(qq, j);
+                __syncwarp();
+                {
+                    // lane j: step tw + j of channel c
+                    const int t = tw + j;
+                    const float4 pv = sP[c * kPS + t];
+                    const float2 uv = sU[c * kPS + t];
+                    const float dd = fmaf(uv.x, GB, Q) * uv.y;
+                    dbias += dd;
+                    dDacc = fmaf(pv.z, uv.x, dDacc);
+                    sP[c * kPS + t] = make_float4(fmaf(pv.x, GB, pv.z * Dc), dd, fmaf(Dc, uv.x, yw) * pv.w, 0.f);
+                }
+                __syncthreads();
+                // dB, dC of these 8 steps summed over the tile's channels, in a fixed order
+                {
+                    const float* rf = reinterpret_cast<const float*>(red);
+                    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
+                    for (int cc = 0; cc < kCT; cc += 2) {
+                        s0 += rf[cc * (kWin * 8 * 4) + tid];
+                        s1 += rf[(cc + 1) * (kWin * 8 * 4) + tid];
+                    }
+                    const int i = tid >> 5, jj = (tid >> 2) & 7, comp = tid & 3;
+                    const int64_t t = t0 + tw + i;
+                    if (t < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + t] = s0 + s1;
+                }
+                if (S::kRedBufs == 1) __syncthreads();
+            }
+            // the block's du, ddelta, dz rows of this warp's channels (lane = step)
+            __syncwarp();
+            if (t0 + lane < L) {
+                using R = typename Io<T>::raw;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int cc = warp * 4 + i;
+                    const float4 o = sP[cc * kPS + lane];
+                    const int64_t at = (row0 + cc) * L + t0 + lane;
+                    static_cast<R*>(p.du)[at] = Io<T>::from(o.x);
+                    static_cast<R*>(p.ddelta)[at] = Io<T>::from(o.y);
+                    if (zz) static_cast<R*>(p.dz)[at] = Io<T>::from(o.z);
+                }
             }
         }
-    }
 
-    // ---------------- per-row partials of the parameter gradients; dh0
-    if (p.dh0) *reinterpret_cast<float2*>(p.dh0 + (row0 + c) * kN + 2 * j) = gs;
-    *reinterpret_cast<float2*>(p.dAp + (row0 + c) * kN + 2 * j) = dAacc;
+        // hand the state gradient to the segment before; this segment's parameter partials
+        *reinterpret_cast<float2*>(p.carry2 + (us * kCT + c) * kN + 2 * j) = gs;
+        if (seg == 0 && p.dh0) *reinterpret_cast<float2*>(p.dh0 + (row0 + c) * kN + 2 * j) = gs;
+        *reinterpret_cast<float2*>(p.dAp + ((int64_t)seg * rows + row0 + c) * kN + 2 * j) = dAacc;
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-        dbias += __shfl_xor_sync(0xffffffffu, dbias, o);
-        dDacc += __shfl_xor_sync(0xffffffffu, dDacc, o);
-    }
-    if (j == 0) {
-        p.dbp[row0 + c] = dbias;
-        p.dDp[row0 + c] = dDacc;
+        for (int o = 1; o < 8; o <<= 1) {
+            dbias += __shfl_xor_sync(0xffffffffu, dbias, o);
+            dDacc += __shfl_xor_sync(0xffffffffu, dDacc, o);
+        }
+        if (j == 0) {
+            p.dbp[(int64_t)seg * rows + row0 + c] = dbias;
+            p.dDp[(int64_t)seg * rows + row0 + c] = dDacc;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            st_release(p.flag2 + us, 1u);
+        }
     }
 }
 
-// dB, dC: sum of the per-tile rows of the group; dA, dD, dbias: sum over batch rows.
+// dB, dC: sum of the per-tile rows of the group; dA, dD, dbias: sum over batch rows and
+// segments, in a fixed order.
 __global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, float* dA, float* dB, float* dC,
                                                          float* dD, float* dbias) {
     const int64_t Dm = p.dim, L = p.seqlen, G = p.ngroups;
@@ -387,9 +473,11 @@ __global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, floa
         return;
     }
     const int64_t k = i - 2 * nbc;
+    const int64_t rows = p.batch * Dm;
     if (k < Dm * kN) {
         float s = 0.f;
-        for (int64_t b = 0; b < p.batch; ++b) s += p.dAp[b * Dm * kN + k];
+        for (int64_t b = 0; b < p.batch; ++b)
+            for (int sg = 0; sg < p.nseg; ++sg) s += p.dAp[(sg * rows + b * Dm) * kN + k];
         dA[k] = s;
         return;
     }
@@ -401,30 +489,87 @@ __global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, floa
         if (!dst) return;
         const float* src = isb ? p.dbp : p.dDp;
         float s = 0.f;
-        for (int64_t b = 0; b < p.batch; ++b) s += src[b * Dm + dd];
+        for (int64_t b = 0; b < p.batch; ++b)
+            for (int sg = 0; sg < p.nseg; ++sg) s += src[sg * rows + b * Dm + dd];
         dst[dd] = s;
     }
 }
 
+// The schedule: persistent CTAs (as many as fit at once, at most one per forward unit)
+// and the cut of each tile's sequence into segments, about 8 units per CTA and pass.
+struct Sched {
+    int ctas, nseg, seg_blocks;
+};
+
+template <typename T>
+Sched make_sched(const ssm_dims_t& d, int sms, int per_sm) {
+    const int64_t ntiles = d.batch * d.dim / kCT;
+    const int64_t nblk = (d.seqlen + kBT - 1) / kBT;
+    const int64_t slots = (int64_t)sms * per_sm;
+    int64_t want = (8 * slots + ntiles - 1) / ntiles;          // segments per tile
+    int64_t sb = (nblk + want - 1) / (want > 0 ? want : 1);
+    if (sb < 4) sb = 4;                                          // at least 128 steps per unit
+    if (sb > nblk) sb = nblk > 0 ? nblk : 1;
+    Sched s;
+    s.seg_blocks = (int)sb;
+    s.nseg = (int)((nblk + sb - 1) / sb);
+    const int64_t units = ntiles * s.nseg;
+    s.ctas = (int)(units < slots ? units : slots);
+    return s;
+}
+
 struct WsLayout {
-    int64_t ckpt, dBp, dCp, dAp, dDp, dbp, total;   // byte offsets
+    int64_t ticket, flag1, flag2, zero_end;        // zeroed before every launch
+    int64_t carry1, carry2, ckpt, dBp, dCp, dAp, dDp, dbp, total;   // byte offsets
 };
 
 __host__ int64_t align256(int64_t v) { return (v + 255) & ~(int64_t)255; }
 
-WsLayout ws_layout(const ssm_dims_t& d) {
+WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
     const int64_t rows = d.batch * d.dim;
-    const int64_t ctas = rows / kCT;
+    const int64_t ntiles = rows / kCT;
     const int64_t nwin = ((d.seqlen + kBT - 1) / kBT) * (kBT / kWin);
+    const int64_t slots = ntiles * s.nseg;
     WsLayout w;
-    w.ckpt = 0;
-    w.dBp = align256(w.ckpt + ctas * nwin * kCT * kN * 4);
-    w.dCp = align256(w.dBp + ctas * kN * d.seqlen * 4);
-    w.dAp = align256(w.dCp + ctas * kN * d.seqlen * 4);
-    w.dDp = align256(w.dAp + rows * kN * 4);
-    w.dbp = align256(w.dDp + rows * 4);
-    w.total = align256(w.dbp + rows * 4);
+    w.ticket = 0;                                  // ticket (u32), status (i32)
+    w.flag1 = 256;
+    w.flag2 = align256(w.flag1 + slots * 4);
+    w.zero_end = align256(w.flag2 + slots * 4);
+    w.carry1 = w.zero_end;
+    w.carry2 = align256(w.carry1 + slots * kCT * kN * 4);
+    w.ckpt = align256(w.carry2 + slots * kCT * kN * 4);
+    w.dBp = align256(w.ckpt + ntiles * nwin * kCT * kN * 4);
+    w.dCp = align256(w.dBp + ntiles * kN * d.seqlen * 4);
+    w.dAp = align256(w.dCp + ntiles * kN * d.seqlen * 4);
+    w.dDp = align256(w.dAp + (int64_t)s.nseg * rows * kN * 4);
+    w.dbp = align256(w.dDp + (int64_t)s.nseg * rows * 4);
+    w.total = align256(w.dbp + (int64_t)s.nseg * rows * 4);
     return w;
+}
+
+// CTAs of the backward kernel that fit on one SM of the current device, and its SM count
+template <typename T>
+bool device_fit(int* sms, int* per_sm) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    if (cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<T>::TOTAL) !=
+        cudaSuccess)
+        return false;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, scan_bwd_kernel<T>, kThreads, Smem<T>::TOTAL) !=
+        cudaSuccess)
+        return false;
+    if (*per_sm < 1) *per_sm = 1;
+    return true;
+}
+
+bool plan_for(const ssm_dims_t& d, Sched* s, WsLayout* w) {
+    int sms = 0, per_sm = 0;
+    const bool ok = d.io_dtype == SSM_BF16 ? device_fit<__nv_bfloat16>(&sms, &per_sm) : device_fit<float>(&sms, &per_sm);
+    if (!ok) return false;
+    *s = d.io_dtype == SSM_BF16 ? make_sched<__nv_bfloat16>(d, sms, per_sm) : make_sched<float>(d, sms, per_sm);
+    *w = ws_layout(d, *s);
+    return true;
 }
 
 int check_dims(const ssm_dims_t* d) {
@@ -441,12 +586,8 @@ int check_dims(const ssm_dims_t* d) {
 }
 
 template <typename T>
-int launch(const BwdParams& prm, float* dA, float* dB, float* dC, float* dD, float* dbias, int64_t ctas,
-           cudaStream_t s) {
+int launch(const BwdParams& prm, float* dA, float* dB, float* dC, float* dD, float* dbias, int ctas, cudaStream_t s) {
     constexpr int smem = Smem<T>::TOTAL;
-    static const bool attr =
-        cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-    if (!attr) return SSM_ERR_CUDA;
     scan_bwd_kernel<T><<<(unsigned)ctas, kThreads, smem, s>>>(prm);
     if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
     const int64_t work = 2 * prm.batch * prm.ngroups * kN * prm.seqlen + prm.dim * kN + 2 * prm.dim;
@@ -464,8 +605,23 @@ extern "C" int ssm_selective_scan_bwd_workspace_size(const ssm_dims_t* dims, siz
     if (!bytes) return SSM_ERR_INVALID_ARG;
     const int rc = check_dims(dims);
     if (rc != SSM_OK) return rc;
-    *bytes = (size_t)ws_layout(*dims).total;
+    Sched sc;
+    WsLayout w;
+    if (!plan_for(*dims, &sc, &w)) return SSM_ERR_CUDA;
+    *bytes = (size_t)w.total;
     return SSM_OK;
+}
+
+extern "C" int ssm_selective_scan_bwd_device_status(void* workspace, ssm_stream_t stream) {
+    if (!workspace) return SSM_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int st = SSM_OK;
+    int* status = reinterpret_cast<int*>(static_cast<unsigned char*>(workspace) + 4);
+    if (cudaMemcpyAsync(&st, status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    if (st != SSM_OK && cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return SSM_ERR_CUDA;
+    return st;
 }
 
 extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, const void* delta, const float* A,
@@ -483,6 +639,7 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
         const int64_t rows = dims->batch * dims->dim, esz = dims->io_dtype == SSM_BF16 ? 2 : 4;
         const int64_t nbc = dims->batch * dims->ngroups * kN * dims->seqlen * 4;
         bool ok = cudaMemsetAsync(grads->dA, 0, dims->dim * kN * 4, s) == cudaSuccess;
+        if (workspace && workspace_bytes >= 8) ok = ok && cudaMemsetAsync(workspace, 0, 8, s) == cudaSuccess;
         if (grads->dD) ok = ok && cudaMemsetAsync(grads->dD, 0, dims->dim * 4, s) == cudaSuccess;
         if (grads->ddelta_bias) ok = ok && cudaMemsetAsync(grads->ddelta_bias, 0, dims->dim * 4, s) == cudaSuccess;
         if (nbc) ok = ok && cudaMemsetAsync(grads->dB, 0, nbc, s) == cudaSuccess &&
@@ -501,7 +658,9 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     if (!u || !delta || !A || !B || !C || !dout) return SSM_ERR_INVALID_ARG;
     if (!grads->du || !grads->ddelta || !grads->dB || !grads->dC) return SSM_ERR_INVALID_ARG;
     if (z && !grads->dz) return SSM_ERR_INVALID_ARG;
-    const WsLayout w = ws_layout(*dims);
+    Sched sc;
+    WsLayout w;
+    if (!plan_for(*dims, &sc, &w)) return SSM_ERR_CUDA;
     if (!workspace || workspace_bytes < (size_t)w.total) return SSM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) || (reinterpret_cast<uintptr_t>(A) & 7u) ||
         (h0 && (reinterpret_cast<uintptr_t>(h0) & 7u)) || (dlast && (reinterpret_cast<uintptr_t>(dlast) & 7u)) ||
@@ -512,6 +671,12 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     prm.A = A; prm.D = D; prm.bias = delta_bias; prm.h0 = h0; prm.dlast = dlast;
     prm.du = grads->du; prm.ddelta = grads->ddelta; prm.dz = grads->dz; prm.dh0 = grads->dh0;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
+    prm.ticket = reinterpret_cast<unsigned*>(ws + w.ticket);
+    prm.status = reinterpret_cast<int*>(ws + w.ticket + 4);
+    prm.flag1 = reinterpret_cast<unsigned*>(ws + w.flag1);
+    prm.flag2 = reinterpret_cast<unsigned*>(ws + w.flag2);
+    prm.carry1 = reinterpret_cast<float*>(ws + w.carry1);
+    prm.carry2 = reinterpret_cast<float*>(ws + w.carry2);
     prm.ckpt = reinterpret_cast<float*>(ws + w.ckpt);
     prm.dBp = reinterpret_cast<float*>(ws + w.dBp);
     prm.dCp = reinterpret_cast<float*>(ws + w.dCp);
@@ -520,10 +685,18 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     prm.dbp = reinterpret_cast<float*>(ws + w.dbp);
     prm.batch = dims->batch; prm.dim = dims->dim; prm.seqlen = dims->seqlen; prm.ngroups = dims->ngroups;
     prm.tiles_per_row = (int)(dims->dim / kCT);
+    prm.ntiles = dims->batch * dims->dim / kCT;
+    prm.nseg = sc.nseg;
+    prm.seg_blocks = sc.seg_blocks;
     prm.softplus = softplus ? 1 : 0;
-    const int64_t ctas = dims->batch * dims->dim / kCT;
+    prm.budget_ns = 1000000000ull;   // 1 s per wait
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the ticket, the status word and the segment flags start at zero (the status of this
+    // call is read, and cleared, by ssm_selective_scan_bwd_device_status)
+    if (cudaMemsetAsync(ws + w.ticket, 0, 8, s) != cudaSuccess ||
+        cudaMemsetAsync(ws + w.flag1, 0, (size_t)(w.zero_end - w.flag1), s) != cudaSuccess)
+        return SSM_ERR_CUDA;
     return dims->io_dtype == SSM_BF16
-               ? launch<__nv_bfloat16>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, ctas, s)
-               : launch<float>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, ctas, s);
+               ? launch<__nv_bfloat16>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, sc.ctas, s)
+               : launch<float>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, sc.ctas, s);
 }

@@ -36,9 +36,13 @@ def _recipe(kind):
 def run_bwd(dims, inp, gin, want_dh0=False, softplus=True):
     import selective_state_space_30_b200 as ssm
     dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
+    d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, io)
+    ws = torch.empty(max(ssm.ssm_selective_scan_bwd_workspace_size(d), 1), dtype=torch.uint8, device="cuda")
     g = ssm.selective_scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], to_device(gin["dout"]),
                                dev["D"], dev["z"], dev["delta_bias"], softplus, h0=to_device(gin.get("h0")),
-                               dlast=to_device(gin.get("dlast")), want_dh0=want_dh0)
+                               dlast=to_device(gin.get("dlast")), want_dh0=want_dh0, workspace=ws)
+    assert ssm.ssm_selective_scan_bwd_device_status(ws) == ssm.SSM_OK
     torch.cuda.synchronize()
     return g
 
@@ -69,7 +73,9 @@ CASES = [
     (si.Dims(2, 128, 96, 16, ngroups=2, dtype="bf16"), "c2", False, True, True),   # two groups
     (si.Dims(1, 96, 33, 16, dtype="bf16"), "plain", True, False, True),    # no z, D, bias; 33 = a block + 1
     (si.Dims(3, 32, 8, 16, dtype="bf16"), "default", False, False, True),  # shorter than a block
-    (si.Dims(2, 32, 200, 16, dtype="f32"), "default", False, False, False),  # softplus off
+    (si.Dims(2, 32, 200, 16, dtype="f32"), "default", False, False, False),  # softplus off; 2 segments
+    (si.Dims(1, 32, 1000, 16, dtype="bf16"), "c2", True, True, True),      # one tile: 8 chained segments
+    (si.Dims(2, 64, 777, 16, dtype="f32"), "c2", True, False, True),       # 7 segments, ragged, element loads
 ]
 
 

@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "scan_kernel.cuh"   // ex2_approx, rcp_approx, softplus1, kLog2e
 #include "ssm_scan.h"
@@ -548,10 +549,20 @@ WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
 }
 
 // CTAs of the backward kernel that fit on one SM of the current device, and its SM count
+// (queried once per device and dtype)
 template <typename T>
 bool device_fit(int* sms, int* per_sm) {
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static int cache[kMaxDev][2];   // {sms, per_sm}; 0 = not queried yet
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < kMaxDev && cache[dev][0] > 0) {
+        *sms = cache[dev][0];
+        *per_sm = cache[dev][1];
+        return true;
+    }
     if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
     if (cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<T>::TOTAL) !=
         cudaSuccess)
@@ -560,6 +571,10 @@ bool device_fit(int* sms, int* per_sm) {
         cudaSuccess)
         return false;
     if (*per_sm < 1) *per_sm = 1;
+    if (dev < kMaxDev) {
+        cache[dev][0] = *sms;
+        cache[dev][1] = *per_sm;
+    }
     return true;
 }
 

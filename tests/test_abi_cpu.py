@@ -106,6 +106,36 @@ def test_conv1d_host_checks(lib):
     assert f(0, 4, 16, 4, ssm.SSM_F32, None, None, None, 1, None, None) == ssm.SSM_OK
 
 
+def test_bwd_host_checks(lib):
+    """ssm_selective_scan_bwd and its workspace query reject bad shapes before touching the GPU."""
+    import selective_state_space_30_b200 as ssm
+    from selective_state_space_30_b200 import _abi
+    n = ctypes.c_size_t()
+    ws = lib.ssm_selective_scan_bwd_workspace_size
+    assert ws(ctypes.byref(ssm.make_dims(2, 32, 64, 16, 0, 1, ssm.SSM_BF16)), None) == ssm.SSM_ERR_INVALID_ARG
+    assert ws(None, ctypes.byref(n)) == ssm.SSM_ERR_INVALID_ARG
+    unsupported = [
+        ssm.make_dims(2, 64, 64, 16, 2, 1, ssm.SSM_BF16),     # per-head layout
+        ssm.make_dims(2, 32, 64, 128, 0, 1, ssm.SSM_BF16),    # dstate 128
+        ssm.make_dims(2, 48, 64, 16, 0, 1, ssm.SSM_BF16),     # 48 channels: not whole 32-channel tiles
+        ssm.make_dims(2, 64, 64, 16, 0, 4, ssm.SSM_BF16),     # 16 channels per group
+    ]
+    for d in unsupported:
+        assert ws(ctypes.byref(d), ctypes.byref(n)) == ssm.SSM_ERR_UNSUPPORTED
+    for d in (ssm.make_dims(2, 30, 64, 16, 0, 4, ssm.SSM_BF16), _abi.ssm_dims_t(2, 32, 64, 16, 32, 1, 7, 0)):
+        assert ws(ctypes.byref(d), ctypes.byref(n)) == ssm.SSM_ERR_INVALID_ARG
+    g = _abi.ssm_grads_t()
+    f = lib.ssm_selective_scan_bwd
+    d = ssm.make_dims(2, 64, 64, 16, 2, 1, ssm.SSM_BF16)
+    assert f(ctypes.byref(d), *([None] * 8), 1, None, None, None, ctypes.byref(g), None, 0, None) == \
+        ssm.SSM_ERR_UNSUPPORTED
+    d = ssm.make_dims(2, 32, 64, 16, 0, 1, ssm.SSM_BF16)
+    assert f(ctypes.byref(d), *([None] * 8), 1, None, None, None, None, None, 0, None) == ssm.SSM_ERR_INVALID_ARG
+    assert f(ctypes.byref(d), *([None] * 8), 1, None, None, None, ctypes.byref(g), None, 0, None) == \
+        ssm.SSM_ERR_INVALID_ARG                                # no dA output
+    assert lib.ssm_selective_scan_bwd_device_status(None, None) == ssm.SSM_ERR_INVALID_ARG
+
+
 def test_plan_without_a_gpu_reports_cuda_error(lib):
     import torch
     import selective_state_space_30_b200 as ssm

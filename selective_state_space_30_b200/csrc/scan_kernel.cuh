@@ -593,18 +593,18 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
                 const uint64_t tw = now_ns();
                 while (true) {
                     // 0 = ready, 1 = keep waiting, 2 = give up
-                    int verdict = 1;
+                    int outcome = 1;
                     if (lane == 0) {
-                        if (ld_acquire(p.flags + tile) >= need) verdict = 0;
-                        else if (*reinterpret_cast<volatile int*>(status) != SSM_OK) verdict = 2;
+                        if (ld_acquire(p.flags + tile) >= need) outcome = 0;
+                        else if (*reinterpret_cast<volatile int*>(status) != SSM_OK) outcome = 2;
                         else if (now_ns() - tw > budget) {
                             atomicCAS(status, SSM_OK, SSM_ERR_TIMEOUT);
-                            verdict = 2;
+                            outcome = 2;
                         }
                     }
-                    verdict = __shfl_sync(0xffffffffu, verdict, 0);
-                    if (verdict == 0) break;
-                    if (verdict == 2) { carry_ok = false; break; }
+                    outcome = __shfl_sync(0xffffffffu, outcome, 0);
+                    if (outcome == 0) break;
+                    if (outcome == 2) { carry_ok = false; break; }
                     service(false);
                     __nanosleep(200);
                 }

@@ -28,11 +28,14 @@
 // segment after it, walks its 32-step blocks backwards, and per window
 // recomputes the 8 states and decays from the checkpoint into registers, then
 // runs the window in reverse.  A unit waits (bounded) only on units with smaller
-// tickets, which running CTAs hold, so the chain always progresses.  Sums over the states (y, sum g B, the decay term)
-// are transposed shuffle reductions inside the 8 lanes of a channel; dB and dC,
-// sums over channels, go through shared memory to per-CTA partial rows, which a
-// second kernel adds in a fixed order with the per-row dA, dD and dbias
-// partials: the result does not depend on scheduling.
+// tickets, which running CTAs hold, so the chain always progresses.
+//
+// Sums over the states (y, sum g B, the decay term) are transposed shuffle
+// reductions inside the 8 lanes of a channel.  dB and dC, sums over channels, are
+// summed over a warp's four channels by shuffles at every step, then over the
+// eight warps through shared memory once per 32-step block, into per-tile partial
+// rows, which a second kernel adds in a fixed order with the per-row dA, dD and
+// dbias partials: the result does not depend on scheduling.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -94,11 +97,10 @@ struct Smem {
     static constexpr int P = STAGE + kStageRows * kRow;           // float4 [kCT][kPS]: dt, dt*u, dy, dout*silu'(z)
     static constexpr int U = P + kCT * kPS * 16;                  // float2 [kCT][kPS]: u, sigmoid(x)
     static constexpr int BC = U + kCT * kPS * 8;                  // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
-    static constexpr int RED = BC + kBT * 8 * 16;                 // float4 [bufs][kCT][kWin][8]: dB, dC terms
-    static constexpr int kRedBytes = kCT * kWin * 8 * 16;
-    // two reduction buffers (one barrier per window) where two CTAs per SM still fit
-    static constexpr int kRedBufs = RED + 2 * kRedBytes <= 112 * 1024 ? 2 : 1;
-    static constexpr int TOTAL = RED + kRedBufs * kRedBytes;
+    // per window and warp, the dB, dC terms summed over the warp's channels:
+    // float [kBT/kWin windows][8 warps][4 components][8 lanes j][kWin steps]
+    static constexpr int RED = BC + kBT * 8 * 16;
+    static constexpr int TOTAL = RED + (kBT / kWin) * 8 * 4 * 8 * kWin * 4;
 };
 
 // rows x kBT steps [t0, t0 + kBT) of `rows` rows (row r at src + r * stride) into
@@ -166,6 +168,24 @@ __device__ __forceinline__ float reduce8(const float (&v)[8], int j) {
     return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
+// The dB, dC terms of one 32-step block, held per (window, warp) in shared memory,
+// summed over the eight warps in a fixed order into the tile's rows: thread tid
+// takes four (window, component, lane j, step) entries.
+__device__ __forceinline__ void red_sum(const float* red, float* dBrow, float* dCrow, int64_t t0, int64_t L,
+                                       int tid) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int idx = tid + r * kThreads;           // 0 .. 1023
+        const int w = idx >> 8, within = idx & 255;   // window; (component, j, step)
+        float s = 0.f;
+#pragma unroll
+        for (int wp = 0; wp < 8; ++wp) s += red[(w * 8 + wp) * 256 + within];
+        const int comp = within >> 6, jj = (within >> 3) & 7, t = within & 7;
+        const int64_t ta = t0 + w * kWin + t;
+        if (ta < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + ta] = s;
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p) {
     using S = Smem<T>;
@@ -174,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
     float4* sP = reinterpret_cast<float4*>(smem + S::P);
     float2* sU = reinterpret_cast<float2*>(smem + S::U);
     float4* sBC = reinterpret_cast<float4*>(smem + S::BC);
-    float4* sR = reinterpret_cast<float4*>(smem + S::RED);
+    float* sR = reinterpret_cast<float*>(smem + S::RED);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = lane >> 3, j = lane & 7;
@@ -316,6 +336,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         for (int blk = blk1 - 1; blk >= blk0; --blk) {
             const int64_t t0 = (int64_t)blk * kBT;
             __syncthreads();
+            // the previous block's dB, dC terms (every warp has written them)
+            if (blk + 1 < blk1) red_sum(sR, dBrow, dCrow, t0 + kBT, L, tid);
             stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
             stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
             if (zz) stage_rows<T>(stage + 2 * kCT * S::kRow, zz, L, kCT, t0, L, vec, tid);
@@ -373,8 +395,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                     }
                     yw = reduce8(yp, j);
                 }
-                float4* red = sR + (S::kRedBufs == 2 ? (fw & 1) : 0) * (S::kRedBytes / 16);
-                float gb[kWin], qq[kWin];
+                float gb[kWin], qq[kWin], rw[kWin];
+                const bool q1 = q & 2, q0 = q & 1;
 #pragma unroll
                 for (int t = kWin - 1; t >= 0; --t) {
                     const float4 pv = sP[c * kPS + tw + t];
@@ -386,10 +408,19 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                     gb[t] = fmaf(gs.x, bc.x, gs.y * bc.y);
                     qq[t] = fmaf(e.x, Aln.x, e.y * Aln.y);
                     const float2 db = mul2(gs, dup2(pv.y)), dc = mul2(dup2(pv.z), hr[t]);
-                    red[(c * kWin + t) * 8 + j] = make_float4(db.x, db.y, dc.x, dc.y);
+                    // the four terms (dB_2j, dB_2j+1, dC_2j, dC_2j+1) summed over the warp's four
+                    // channels, transposed: lane (q, j) keeps component q
+                    const float a0 = (q1 ? dc.x : db.x) + __shfl_xor_sync(0xffffffffu, q1 ? db.x : dc.x, 16);
+                    const float a1 = (q1 ? dc.y : db.y) + __shfl_xor_sync(0xffffffffu, q1 ? db.y : dc.y, 16);
+                    rw[t] = (q0 ? a1 : a0) + __shfl_xor_sync(0xffffffffu, q0 ? a0 : a1, 8);
                     gs = mul2(gs, dAr[t]);           // carry to t-1
                 }
                 const float GB = reduce8(gb, j), Q = reduce8(qq, j);
+                {
+                    float4* rd = reinterpret_cast<float4*>(sR + ((w * 8 + warp) * 4 + q) * 64 + j * 8);
+                    rd[0] = make_float4(rw[0], rw[1], rw[2], rw[3]);
+                    rd[1] = make_float4(rw[4], rw[5], rw[6], rw[7]);
+                }
                 __syncwarp();
                 {
                     // lane j: step tw + j of channel c
@@ -401,21 +432,6 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                     dDacc = fmaf(pv.z, uv.x, dDacc);
                     sP[c * kPS + t] = make_float4(fmaf(pv.x, GB, pv.z * Dc), dd, fmaf(Dc, uv.x, yw) * pv.w, 0.f);
                 }
-                __syncthreads();
-                // dB, dC of these 8 steps summed over the tile's channels, in a fixed order
-                {
-                    const float* rf = reinterpret_cast<const float*>(red);
-                    float s0 = 0.f, s1 = 0.f;
-#pragma unroll 8
-                    for (int cc = 0; cc < kCT; cc += 2) {
-                        s0 += rf[cc * (kWin * 8 * 4) + tid];
-                        s1 += rf[(cc + 1) * (kWin * 8 * 4) + tid];
-                    }
-                    const int i = tid >> 5, jj = (tid >> 2) & 7, comp = tid & 3;
-                    const int64_t t = t0 + tw + i;
-                    if (t < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + t] = s0 + s1;
-                }
-                if (S::kRedBufs == 1) __syncthreads();
             }
             // the block's du, ddelta, dz rows of this warp's channels (lane = step)
             __syncwarp();
@@ -433,6 +449,9 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             }
         }
 
+        // the last block's dB, dC terms
+        __syncthreads();
+        red_sum(sR, dBrow, dCrow, (int64_t)blk0 * kBT, L, tid);
         // hand the state gradient to the segment before; this segment's parameter partials
         *reinterpret_cast<float2*>(p.carry2 + (us * kCT + c) * kN + 2 * j) = gs;
         if (seg == 0 && p.dh0) *reinterpret_cast<float2*>(p.dh0 + (row0 + c) * kN + 2 * j) = gs;

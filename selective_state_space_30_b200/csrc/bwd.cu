@@ -93,8 +93,9 @@ constexpr int kPS = kBT + 1;
 template <typename T>
 struct Smem {
     static constexpr int kRow = kBT * (int)sizeof(T) + 16;        // staged row stride (16-byte padded)
-    static constexpr int STAGE = 0;
-    static constexpr int P = STAGE + kStageRows * kRow;           // float4 [kCT][kPS]: dt, dt*u, dy, dout*silu'(z)
+    static constexpr int STAGE = 0;                               // two buffers of staged rows
+    static constexpr int kStageBytes = kStageRows * kRow;
+    static constexpr int P = STAGE + 2 * kStageBytes;             // float4 [kCT][kPS]: dt, dt*u, dy, dout*silu'(z)
     static constexpr int U = P + kCT * kPS * 16;                  // float2 [kCT][kPS]: u, sigmoid(x)
     static constexpr int BC = U + kCT * kPS * 8;                  // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
     // per window and warp, the dB, dC terms summed over the warp's channels:
@@ -104,8 +105,9 @@ struct Smem {
 };
 
 // rows x kBT steps [t0, t0 + kBT) of `rows` rows (row r at src + r * stride) into
-// shared memory, zero past L.  vec: 16-byte chunks (rows 16-byte aligned, L a
-// multiple of the chunk), else element by element.
+// shared memory, zero past L.  vec: asynchronous 16-byte copies (rows 16-byte
+// aligned, L a multiple of the chunk; complete after cp_async_wait), else element by
+// element.
 template <typename T>
 __device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int64_t stride, int rows, int64_t t0,
                                            int64_t L, bool vec, int tid) {
@@ -113,12 +115,14 @@ __device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int
     constexpr int E = 16 / (int)sizeof(T);
     constexpr int CPR = kBT / E;
     if (vec) {
+        // cp.async: zero-filled when the chunk lies past L (then the source is not read)
         for (int i = tid; i < rows * CPR; i += kThreads) {
             const int r = i / CPR, k = i % CPR;
             const int64_t t = t0 + (int64_t)k * E;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < L) v = __ldg(reinterpret_cast<const uint4*>(src + r * stride + t));
-            *reinterpret_cast<uint4*>(dst + r * Smem<T>::kRow + k * 16) = v;
+            const T* g = src + r * stride + (t < L ? t : 0);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst + r * Smem<T>::kRow + k * 16)),
+                         "l"(g), "r"(t < L ? 16 : 0)
+                         : "memory");
         }
     } else {
         const R* s = reinterpret_cast<const R*>(src);
@@ -129,6 +133,8 @@ __device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int
         }
     }
 }
+
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 template <typename T>
 __device__ __forceinline__ float staged(const unsigned char* base, int row, int k) {
@@ -190,7 +196,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p) {
     using S = Smem<T>;
     extern __shared__ __align__(16) unsigned char smem[];
-    unsigned char* stage = smem + S::STAGE;
+    unsigned char* stage_base = smem + S::STAGE;
     float4* sP = reinterpret_cast<float4*>(smem + S::P);
     float2* sU = reinterpret_cast<float2*>(smem + S::U);
     float4* sBC = reinterpret_cast<float4*>(smem + S::BC);
@@ -274,13 +280,19 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 h = p.h0 ? *reinterpret_cast<const float2*>(p.h0 + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
             else
                 h = __ldcg(reinterpret_cast<const float2*>(p.carry1 + ((us - 1) * kCT + c) * kN + 2 * j));
-            for (int blk = blk0; blk < blk1; ++blk) {
+            // the rows of the unit's first block; each block's prologue then issues the next's
+            auto issue_fwd = [&](unsigned char* sg, int64_t ts) {
+                stage_rows<T>(sg, u, L, kCT, ts, L, vec, tid);
+                stage_rows<T>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
+                stage_rows<T>(sg + 4 * kCT * S::kRow, Bg, L, kN, ts, L, vec, tid);
+            };
+            issue_fwd(stage_base, (int64_t)blk0 * kBT);
+            int cur = 0;
+            for (int blk = blk0; blk < blk1; ++blk, cur ^= 1) {
                 const int64_t t0 = (int64_t)blk * kBT;
-                __syncthreads();   // the previous block is done with the staged rows and the B tile
-                stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
-                stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
-                stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
-                __syncthreads();
+                unsigned char* stage = stage_base + cur * S::kStageBytes;
+                cp_async_wait();
+                __syncthreads();   // this block's rows are in; the previous block is done with P and BC
                 // dt and dt*u of this warp's 4 channels, lane = step
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -297,6 +309,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                     const unsigned char* sb = stage + 4 * kCT * S::kRow;
                     sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t), 0.f, 0.f);
                 }
+                // the next block's rows go into the other buffer, read last by the previous block
+                if (blk + 1 < blk1) issue_fwd(stage_base + (cur ^ 1) * S::kStageBytes, t0 + kBT);
                 __syncthreads();
 #pragma unroll
                 for (int w = 0; w < kBT / kWin; ++w) {
@@ -333,18 +347,23 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         const int fw0 = blk0 * (kBT / kWin);             // first window of the segment
         int fw = blk1 * (kBT / kWin) - 1;                // flat index of the current window, walking down
         float2 hnext = __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)fw * kCT + c) * kN + 2 * j));
-        for (int blk = blk1 - 1; blk >= blk0; --blk) {
+        auto issue_rev = [&](unsigned char* sg, int64_t ts) {
+            stage_rows<T>(sg, u, L, kCT, ts, L, vec, tid);
+            stage_rows<T>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
+            if (zz) stage_rows<T>(sg + 2 * kCT * S::kRow, zz, L, kCT, ts, L, vec, tid);
+            stage_rows<T>(sg + 3 * kCT * S::kRow, go, L, kCT, ts, L, vec, tid);
+            stage_rows<T>(sg + 4 * kCT * S::kRow, Bg, L, kN, ts, L, vec, tid);
+            stage_rows<T>(sg + (4 * kCT + kN) * S::kRow, Cg, L, kN, ts, L, vec, tid);
+        };
+        issue_rev(stage_base, (int64_t)(blk1 - 1) * kBT);
+        int cur = 0;
+        for (int blk = blk1 - 1; blk >= blk0; --blk, cur ^= 1) {
             const int64_t t0 = (int64_t)blk * kBT;
-            __syncthreads();
+            unsigned char* stage = stage_base + cur * S::kStageBytes;
+            cp_async_wait();
+            __syncthreads();   // this block's rows are in; the previous block is done with P, U, BC
             // the previous block's dB, dC terms (every warp has written them)
             if (blk + 1 < blk1) red_sum(sR, dBrow, dCrow, t0 + kBT, L, tid);
-            stage_rows<T>(stage, u, L, kCT, t0, L, vec, tid);
-            stage_rows<T>(stage + kCT * S::kRow, dl, L, kCT, t0, L, vec, tid);
-            if (zz) stage_rows<T>(stage + 2 * kCT * S::kRow, zz, L, kCT, t0, L, vec, tid);
-            stage_rows<T>(stage + 3 * kCT * S::kRow, go, L, kCT, t0, L, vec, tid);
-            stage_rows<T>(stage + 4 * kCT * S::kRow, Bg, L, kN, t0, L, vec, tid);
-            stage_rows<T>(stage + (4 * kCT + kN) * S::kRow, Cg, L, kN, t0, L, vec, tid);
-            __syncthreads();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int cc = warp * 4 + i;
@@ -373,6 +392,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t),
                                               staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
             }
+            // the next (earlier) block's rows go into the other buffer
+            if (blk > blk0) issue_rev(stage_base + (cur ^ 1) * S::kStageBytes, t0 - kBT);
             __syncthreads();
 
             for (int w = kBT / kWin - 1; w >= 0; --w, --fw) {

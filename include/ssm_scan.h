@@ -122,8 +122,12 @@ int ssm_selective_scan_fwd_h0(ssm_plan_t plan, const void* u, const void* delta,
  * tensor pointer is HOST memory (pinned memory makes the copies asynchronous).
  * The plan allocates device copies on first use (kept until ssm_scan_destroy);
  * each call copies the inputs host->device, runs the scan and copies out (and
- * last_state, if given) device->host, all on `stream`.  The host outputs are
- * complete once the stream is synchronised.
+ * last_state, if given) device->host.  With batch >= 2 the batch rows are cut
+ * into chunks (the largest divisor of batch up to 8) that are pipelined on three
+ * streams the plan owns (copies in, scans through a plan for one chunk, copies
+ * out), so the copies in both directions and the scans overlap; the call is
+ * ordered after the work already on `stream`, and later work on `stream` waits
+ * for it.  The host outputs are complete once `stream` is synchronised.
  */
 int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delta, const float* A,
                                 const void* B, const void* C, const float* D, const void* z,

@@ -59,6 +59,13 @@ struct ssm_plan_s {
     // lazily allocated device mirrors for the host-buffer entry point
     void* h_bufs[10];
     size_t h_sizes[10];
+    // the host-buffer entry point's pipeline over batch-row chunks: a plan for one chunk,
+    // streams for the copies in, the scans and the copies out, and their events
+    ssm_plan_s* sub;
+    int n_chunks;
+    cudaStream_t pipe[3];
+    cudaEvent_t ev_start, ev_end, ev_in[8], ev_run[8];
+    bool pipe_ready;
 };
 
 namespace {
@@ -293,11 +300,25 @@ const char* ssm_status_string(int status) {
     }
 }
 
+// The host-buffer pipeline's streams, events and chunk plan (built on first use).
+static void release_pipeline(ssm_plan_s* p) {
+    if (!p->pipe_ready) return;
+    for (int i = 0; i < 3; ++i) cudaStreamDestroy(p->pipe[i]);
+    cudaEventDestroy(p->ev_start);
+    cudaEventDestroy(p->ev_end);
+    for (int i = 0; i < 8; ++i) {
+        cudaEventDestroy(p->ev_in[i]);
+        cudaEventDestroy(p->ev_run[i]);
+    }
+    if (p->sub) ssm_scan_destroy(p->sub);
+    p->sub = nullptr;
+    p->pipe_ready = false;
+}
+
 int ssm_scan_plan(ssm_plan_t* out_plan, const ssm_dims_t* dims, int device) {
     if (!out_plan) return SSM_ERR_INVALID_ARG;
     *out_plan = nullptr;
     if (!dims_ok(dims)) return SSM_ERR_INVALID_ARG;
-    ssm::Variant v;
     ssm::Layout probe;
     if (!ssm::choose_layout(*dims, 1, 0, 0, &probe)) return SSM_ERR_UNSUPPORTED;
     int ndev = 0;
@@ -353,6 +374,7 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
                 return SSM_ERR_INVALID_ARG;
             if (option == SSM_OPT_SSD && value > 2) return SSM_ERR_INVALID_ARG;
             if (cudaDeviceSynchronize() != cudaSuccess) return SSM_ERR_CUDA;
+            release_pipeline(plan);   // its chunk plan follows the new options when next built
             unsigned inject = 0;
             if (cudaMemcpy(&inject, plan->ws + offsetof(ssm::WsHeader, inject), sizeof(inject),
                            cudaMemcpyDeviceToHost) != cudaSuccess)
@@ -399,6 +421,43 @@ int ssm_selective_scan_fwd(ssm_plan_t plan, const void* u, const void* delta, co
                                      last_state, stream);
 }
 
+// The same call on host buffers.  With batch >= 2 the batch rows are cut into chunks
+// (the largest divisor of batch up to 8) and pipelined on three streams the plan
+// owns: a chunk's inputs are copied in while the previous chunk is scanned and the
+// one before it is copied out, so the copies in both directions and the scans
+// overlap.  Each chunk runs through a plan for one chunk's rows.  The call starts
+// after the work already queued on `stream` and the work queued on `stream` after it
+// waits for its end.  With batch 1 everything runs in order on `stream`.
+static int build_pipeline(ssm_plan_s* p) {
+    const ssm_dims_t& d = p->dims;
+    int n = 1;
+    for (int k = 8; k >= 2; --k)
+        if (d.batch % k == 0) {
+            n = k;
+            break;
+        }
+    p->n_chunks = n;
+    if (n == 1) return SSM_OK;
+    ssm_dims_t cd = d;
+    cd.batch = d.batch / n;
+    int rc = ssm_scan_plan(&p->sub, &cd, p->device);
+    if (rc != SSM_OK) return rc;
+    p->sub->spin_limit = p->spin_limit;
+    if (p->force_ssd) {
+        rc = ssm_scan_set_option(p->sub, SSM_OPT_SSD, p->force_ssd);
+        if (rc != SSM_OK) return rc;
+    }
+    bool ok = true;
+    for (int i = 0; i < 3; ++i) ok = ok && cudaStreamCreateWithFlags(&p->pipe[i], cudaStreamNonBlocking) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&p->ev_start, cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p->ev_end, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 8; ++i)
+        ok = ok && cudaEventCreateWithFlags(&p->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&p->ev_run[i], cudaEventDisableTiming) == cudaSuccess;
+    p->pipe_ready = true;   // release_pipeline destroys what was made
+    return ok ? SSM_OK : SSM_ERR_CUDA;
+}
+
 int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delta, const float* A, const void* B,
                                 const void* C, const float* D, const void* z, const float* delta_bias, int softplus,
                                 const ssm_dims_t* dims, void* out, float* last_state, ssm_stream_t stream) {
@@ -420,29 +479,75 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
                            last_state != nullptr};
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     for (int i = 0; i < 10; ++i) {
-        if (!used[i]) continue;
-        if (plan->h_sizes[i] < bytes[i]) {
-            if (plan->h_bufs[i]) cudaFree(plan->h_bufs[i]);
-            plan->h_bufs[i] = nullptr;
-            plan->h_sizes[i] = 0;
-            if (bytes[i] && cudaMalloc(&plan->h_bufs[i], bytes[i]) != cudaSuccess) return SSM_ERR_CUDA;
-            plan->h_sizes[i] = bytes[i];
-        }
-        if (i < 8 && bytes[i] &&
-            cudaMemcpyAsync(plan->h_bufs[i], src[i], bytes[i], cudaMemcpyHostToDevice, s) != cudaSuccess)
-            return SSM_ERR_CUDA;
+        if (!used[i] || plan->h_sizes[i] >= bytes[i]) continue;
+        if (plan->h_bufs[i]) cudaFree(plan->h_bufs[i]);
+        plan->h_bufs[i] = nullptr;
+        plan->h_sizes[i] = 0;
+        if (bytes[i] && cudaMalloc(&plan->h_bufs[i], bytes[i]) != cudaSuccess) return SSM_ERR_CUDA;
+        plan->h_sizes[i] = bytes[i];
     }
-    int rc = launch_fwd(plan, plan->h_bufs[0], plan->h_bufs[1], (const float*)plan->h_bufs[2], plan->h_bufs[3],
-                        plan->h_bufs[4], D ? (const float*)plan->h_bufs[5] : nullptr, z ? plan->h_bufs[6] : nullptr,
-                        delta_bias ? (const float*)plan->h_bufs[7] : nullptr, softplus, nullptr, plan->h_bufs[8],
-                        last_state ? (float*)plan->h_bufs[9] : nullptr, s);
-    if (rc != SSM_OK) return rc;
-    if (bytes[8] && cudaMemcpyAsync(out, plan->h_bufs[8], bytes[8], cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    if (last_state && bytes[9] &&
-        cudaMemcpyAsync(last_state, plan->h_bufs[9], bytes[9], cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    return SSM_OK;
+    if (d.batch >= 2 && !plan->pipe_ready) {
+        const int rc = build_pipeline(plan);
+        if (rc != SSM_OK) {
+            release_pipeline(plan);
+            return rc;
+        }
+    }
+    if (d.batch < 2 || plan->n_chunks < 2) {
+        for (int i = 0; i < 8; ++i)
+            if (used[i] && bytes[i] &&
+                cudaMemcpyAsync(plan->h_bufs[i], src[i], bytes[i], cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return SSM_ERR_CUDA;
+        int rc = launch_fwd(plan, plan->h_bufs[0], plan->h_bufs[1], (const float*)plan->h_bufs[2], plan->h_bufs[3],
+                            plan->h_bufs[4], D ? (const float*)plan->h_bufs[5] : nullptr, z ? plan->h_bufs[6] : nullptr,
+                            delta_bias ? (const float*)plan->h_bufs[7] : nullptr, softplus, nullptr, plan->h_bufs[8],
+                            last_state ? (float*)plan->h_bufs[9] : nullptr, s);
+        if (rc != SSM_OK) return rc;
+        if (bytes[8] && cudaMemcpyAsync(out, plan->h_bufs[8], bytes[8], cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        if (last_state && bytes[9] &&
+            cudaMemcpyAsync(last_state, plan->h_bufs[9], bytes[9], cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return SSM_ERR_CUDA;
+        return SSM_OK;
+    }
+    // the pipeline: per-chunk slabs of every per-row tensor (rows of a chunk are contiguous)
+    const int n = plan->n_chunks;
+    cudaStream_t sin = plan->pipe[0], srun = plan->pipe[1], sout = plan->pipe[2];
+    bool ok = cudaEventRecord(plan->ev_start, s) == cudaSuccess;
+    for (int i = 0; i < 3; ++i) ok = ok && cudaStreamWaitEvent(plan->pipe[i], plan->ev_start, 0) == cudaSuccess;
+    // the per-channel parameters once
+    for (int i : {2, 5, 7})
+        if (ok && used[i] && bytes[i])
+            ok = cudaMemcpyAsync(plan->h_bufs[i], src[i], bytes[i], cudaMemcpyHostToDevice, sin) == cudaSuccess;
+    const bool per_row[10] = {true, true, false, true, true, false, true, false, true, true};
+    auto slab = [&](int i, int k) -> size_t { return bytes[i] / n * (size_t)k; };
+    for (int k = 0; k < n && ok; ++k) {
+        for (int i : {0, 1, 3, 4, 6}) {
+            if (!used[i] || !bytes[i] || !per_row[i]) continue;
+            ok = ok && cudaMemcpyAsync(static_cast<char*>(plan->h_bufs[i]) + slab(i, k),
+                                       static_cast<const char*>(src[i]) + slab(i, k), bytes[i] / n,
+                                       cudaMemcpyHostToDevice, sin) == cudaSuccess;
+        }
+        ok = ok && cudaEventRecord(plan->ev_in[k], sin) == cudaSuccess &&
+             cudaStreamWaitEvent(srun, plan->ev_in[k], 0) == cudaSuccess;
+        if (!ok) break;
+        auto at = [&](int i) -> void* {
+            return used[i] ? static_cast<char*>(plan->h_bufs[i]) + (per_row[i] ? slab(i, k) : 0) : nullptr;
+        };
+        const int rc = launch_fwd(plan->sub, at(0), at(1), (const float*)at(2), at(3), at(4), (const float*)at(5),
+                                  at(6), (const float*)at(7), softplus, nullptr, at(8), (float*)at(9), srun);
+        if (rc != SSM_OK) return rc;
+        ok = cudaEventRecord(plan->ev_run[k], srun) == cudaSuccess &&
+             cudaStreamWaitEvent(sout, plan->ev_run[k], 0) == cudaSuccess &&
+             cudaMemcpyAsync(static_cast<char*>(out) + slab(8, k), at(8), bytes[8] / n, cudaMemcpyDeviceToHost,
+                             sout) == cudaSuccess;
+        if (ok && last_state)
+            ok = cudaMemcpyAsync(reinterpret_cast<char*>(last_state) + slab(9, k), at(9), bytes[9] / n,
+                                 cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+    }
+    // the caller's stream resumes after the last copy out (which follows every scan)
+    ok = ok && cudaEventRecord(plan->ev_end, sout) == cudaSuccess && cudaStreamWaitEvent(s, plan->ev_end, 0) == cudaSuccess;
+    return ok ? SSM_OK : SSM_ERR_CUDA;
 }
 
 int ssm_scan_destroy(ssm_plan_t plan) {
@@ -453,6 +558,7 @@ int ssm_scan_destroy(ssm_plan_t plan) {
     if (plan->ws) cudaFree(plan->ws);
     for (int i = 0; i < 10; ++i)
         if (plan->h_bufs[i]) cudaFree(plan->h_bufs[i]);
+    release_pipeline(plan);
     plan->magic = kDead;
     delete plan;
     return SSM_OK;

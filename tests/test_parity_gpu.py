@@ -172,26 +172,42 @@ def test_misaligned_pointers_take_scalar_path():
     assert torch.equal(out, ref) and torch.equal(last, ref_last)
 
 
-def test_host_entry_point_matches_device_path():
+HOST_CASES = [
+    si.Dims(2, 64, 256, 16, dtype="bf16"),                  # two chunks of one batch row
+    si.Dims(6, 64, 200, 16, dtype="bf16"),                  # six chunks, ragged length
+    si.Dims(1, 64, 256, 16, dtype="f32"),                   # one batch row: no pipeline
+    si.Dims(4, 128, 256, 128, nheads=2, dtype="bf16"),      # four chunks through the tensor-core path
+]
+
+
+@pytest.mark.parametrize("dims", HOST_CASES, ids=lambda d: f"{d.batch}x{d.dim}x{d.seqlen}n{d.dstate}{d.dtype}")
+def test_host_entry_point_matches_oracle(dims):
+    """ssm_selective_scan_fwd_host (copies in, scan, copies out; pipelined over batch rows)
+    against the oracle, and twice in a row on the same plan."""
     import torch
     import selective_state_space_30_b200 as ssm
-    dims = si.Dims(2, 64, 256, 16, dtype="bf16")
-    inp = si.make_inputs(dims, si.Recipe(d_init="normal", delta_init="normal_half"), 6)
-    ref, ref_last = run_gpu(dims, inp)
-    d = ssm.make_dims(2, 64, 256, 16, 64, 1, ssm.SSM_BF16)
+    rec = si.Recipe(a_init="neg_uniform_1_16") if dims.head_mode else si.Recipe(d_init="normal",
+                                                                                 delta_init="normal_half")
+    inp = si.make_inputs(dims, rec, 6)
+    io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
+    d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, io)
     host = {k: np.ascontiguousarray(inp[k]) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
-    out = np.empty((2, 64, 256), dtype=np.uint16)
-    last = np.empty((2, 64, 16), dtype=np.float32)
+    odt = np.uint16 if dims.dtype == "bf16" else np.float32
+    ro, rl, rm = oracle.run_inputs(dims, inp)
     plan = ssm.ssm_scan_plan(d, 0)
     try:
-        ssm.ssm_selective_scan_fwd_host(plan, host["u"], host["delta"], host["A"], host["B"], host["C"],
-                                        host["D"], host["z"], host["delta_bias"], True, d, out, last, None)
-        torch.cuda.synchronize()
+        for _ in range(2):
+            out = np.empty((dims.batch, dims.dim, dims.seqlen), dtype=odt)
+            last = np.empty((dims.batch, dims.dim, dims.dstate), dtype=np.float32)
+            ssm.ssm_selective_scan_fwd_host(plan, host["u"], host["delta"], host["A"], host["B"], host["C"],
+                                            host["D"], host["z"], host["delta_bias"], True, d, out, last, None)
+            torch.cuda.synchronize()
+            assert ssm.ssm_scan_device_status(plan) == ssm.SSM_OK
+            got = si.to_f64(out) if dims.dtype == "bf16" else out.astype(np.float64)
+            check_out(got, ro, rm, dims.dtype)
+            check_state(last.astype(np.float64), rl)
     finally:
         ssm.ssm_scan_destroy(plan)
-    got = torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)
-    assert torch.equal(got, ref.cpu())
-    assert np.array_equal(last, ref_last.cpu().numpy())
 
 
 def test_deterministic():

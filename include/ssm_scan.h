@@ -316,6 +316,13 @@ int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, const void* de
  * used `workspace` (SSM_OK or SSM_ERR_TIMEOUT), clearing it. */
 int ssm_selective_scan_bwd_device_status(void* workspace, ssm_stream_t stream);
 
+/* Test hooks of the backward, process-wide, for tests only.  stall != 0 makes every
+ * wait of a chained work unit wait for a flag value that nothing writes, so the wait
+ * runs out, the call records SSM_ERR_TIMEOUT and its outputs are invalid;
+ * wait_budget_us > 0 replaces the default limit of a wait (about 1 s), 0 restores it.
+ * SSM_ERR_INVALID_ARG for a budget outside [0, 10 s]. */
+int ssm_selective_scan_bwd_test_hooks(int stall, int64_t wait_budget_us);
+
 /* Release the plan and its workspace.  NULL is accepted.  Synchronises the device. */
 int ssm_scan_destroy(ssm_plan_t plan);
 

@@ -23,7 +23,8 @@ from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, 
                    ssm_scan_plan_info, ssm_scan_plan_schedule, ssm_scan_set_option, ssm_selective_scan_fwd,
                    ssm_selective_scan_fwd_h0, ssm_selective_scan_fwd_host, ssm_selective_scan_fwd_noalloc,
                    ssm_selective_state_update, ssm_causal_conv1d_fwd, ssm_selective_scan_bwd,
-                   ssm_selective_scan_bwd_workspace_size, ssm_selective_scan_bwd_device_status, ssm_grads_t,
+                   ssm_selective_scan_bwd_workspace_size, ssm_selective_scan_bwd_device_status,
+                   ssm_selective_scan_bwd_test_hooks, ssm_grads_t,
                    GRAD_NAMES,
                    ssm_status_string)
 
@@ -31,7 +32,7 @@ __all__ = ["selective_scan_fwd", "selective_scan_fwd_host", "Plan", "get_plan", 
            "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0", "ssm_selective_scan_fwd_host",
            "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update", "ssm_causal_conv1d_fwd",
            "selective_scan_bwd", "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_workspace_size",
-           "ssm_selective_scan_bwd_device_status",
+           "ssm_selective_scan_bwd_device_status", "ssm_selective_scan_bwd_test_hooks",
            "ssm_scan_destroy", "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info",
            "ssm_scan_set_option", "ssm_scan_plan_schedule",
            "ssm_probe_ex2", "make_dims", "SsmError", "load_library"]

@@ -27,7 +27,7 @@ SSM_BF16 = 1
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
            "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update",
            "ssm_causal_conv1d_fwd", "ssm_selective_scan_bwd_workspace_size", "ssm_selective_scan_bwd",
-           "ssm_selective_scan_bwd_device_status",
+           "ssm_selective_scan_bwd_device_status", "ssm_selective_scan_bwd_test_hooks",
            "ssm_scan_set_option",
            "ssm_scan_plan_schedule", "ssm_scan_destroy",
            "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
@@ -88,6 +88,7 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_bwd.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
                                            ctypes.POINTER(ssm_grads_t), vp, ctypes.c_size_t, vp]
     lib.ssm_selective_scan_bwd_device_status.argtypes = [vp, vp]
+    lib.ssm_selective_scan_bwd_test_hooks.argtypes = [i32, i64]
     lib.ssm_scan_destroy.argtypes = [vp]
     lib.ssm_scan_device_status.argtypes = [vp, vp]
     lib.ssm_status_string.argtypes = [i32]
@@ -223,6 +224,12 @@ def ssm_selective_scan_bwd(dims: ssm_dims_t, u, delta, A, B, C, D, z, delta_bias
 def ssm_selective_scan_bwd_device_status(workspace, stream=None) -> int:
     """Kernel-side status of the last backward call on `workspace` (syncs the stream, clears it)."""
     return int(load_library().ssm_selective_scan_bwd_device_status(_ptr(workspace), _stream(stream)))
+
+
+def ssm_selective_scan_bwd_test_hooks(stall: bool, wait_budget_us: int = 0) -> int:
+    """Backward test hooks (see include/ssm_scan.h): make chained waits run out; shorten their limit."""
+    return _check(load_library().ssm_selective_scan_bwd_test_hooks(1 if stall else 0, int(wait_budget_us)),
+                  "ssm_selective_scan_bwd_test_hooks")
 
 
 def ssm_scan_destroy(plan: Optional[int]) -> int:

@@ -73,6 +73,7 @@ struct BwdParams {
     int nseg, seg_blocks;        // segments per tile, 32-step blocks per segment
     int softplus;
     uint64_t budget_ns;          // bounded waits
+    unsigned need;               // the flag value a wait waits for: 1, or 2 (never written) under the test hook
 };
 
 template <typename T> struct Io;
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             for (int w = 0; w < 2; ++w) {
                 if (!need[w]) continue;
                 const uint64_t t_start = now_ns();
-                while (ld_acquire(need[w]) == 0u) {
+                while (ld_acquire(need[w]) < p.need) {
                     __nanosleep(128);   // leave the issue slots to the working warps of this SM
                     if (*reinterpret_cast<volatile int*>(p.status) != SSM_OK) { ok = false; break; }
                     if (now_ns() - t_start > p.budget_ns) {
@@ -655,6 +656,18 @@ int launch(const BwdParams& prm, float* dA, float* dB, float* dC, float* dD, flo
 }  // namespace
 }  // namespace ssm
 
+// test hooks (process-wide): a stall makes every wait of a chained unit wait for a flag
+// value nobody writes, so it runs out and the call reports SSM_ERR_TIMEOUT
+static unsigned g_hook_stall = 0;
+static uint64_t g_hook_budget_ns = 0;
+
+extern "C" int ssm_selective_scan_bwd_test_hooks(int stall, int64_t wait_budget_us) {
+    if (wait_budget_us < 0 || wait_budget_us > 10000000) return SSM_ERR_INVALID_ARG;
+    g_hook_stall = stall ? 1u : 0u;
+    g_hook_budget_ns = (uint64_t)wait_budget_us * 1000ull;
+    return SSM_OK;
+}
+
 extern "C" int ssm_selective_scan_bwd_workspace_size(const ssm_dims_t* dims, size_t* bytes) {
     using namespace ssm;
     if (!bytes) return SSM_ERR_INVALID_ARG;
@@ -744,7 +757,8 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     prm.nseg = sc.nseg;
     prm.seg_blocks = sc.seg_blocks;
     prm.softplus = softplus ? 1 : 0;
-    prm.budget_ns = 1000000000ull;   // 1 s per wait
+    prm.budget_ns = g_hook_budget_ns ? g_hook_budget_ns : 1000000000ull;   // 1 s per wait
+    prm.need = g_hook_stall ? 2u : 1u;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the ticket, the status word and the segment flags start at zero (the status of this
     // call is read, and cleared, by ssm_selective_scan_bwd_device_status)

@@ -147,3 +147,28 @@ def test_bwd_full_size_mamba_130m():
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"])
     g = run_bwd(dims, inp, gin)
     check_grads(g, ref, mag, dims.dtype, what="mamba-130m ")
+
+
+def test_bwd_wait_timeout_reports_and_recovers():
+    """A chained wait that runs out (test hook: the flag it waits for is never written) ends
+    the call with SSM_ERR_TIMEOUT, without a fault; the next call on the same context and
+    workspace runs normally and matches the oracle."""
+    import selective_state_space_30_b200 as ssm
+    dims = si.Dims(1, 32, 1000, 16, dtype="bf16")          # one tile, 8 chained segments
+    inp = si.make_inputs(dims, _recipe("c2"), 47)
+    gin = si.make_grad_inputs(dims, 48)
+    d = ssm.make_dims(1, 32, 1000, 16, 32, 1, ssm.SSM_BF16)
+    ws = torch.empty(ssm.ssm_selective_scan_bwd_workspace_size(d), dtype=torch.uint8, device="cuda")
+    dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    try:
+        ssm.ssm_selective_scan_bwd_test_hooks(True, 20000)   # 20 ms per wait
+        ssm.selective_scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], to_device(gin["dout"]),
+                               dev["D"], dev["z"], dev["delta_bias"], True, workspace=ws)
+        assert ssm.ssm_selective_scan_bwd_device_status(ws) == ssm.SSM_ERR_TIMEOUT
+    finally:
+        ssm.ssm_selective_scan_bwd_test_hooks(False, 0)
+    g = ssm.selective_scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], to_device(gin["dout"]),
+                               dev["D"], dev["z"], dev["delta_bias"], True, workspace=ws)
+    assert ssm.ssm_selective_scan_bwd_device_status(ws) == ssm.SSM_OK
+    ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"])
+    check_grads(g, ref, mag, dims.dtype)

@@ -15,7 +15,7 @@
 //   dB_tn += g_n dt u_t           dC_tn += dy h_tn           (summed over channels)
 //   du_t = dt sum_n g_n B_tn + dy D
 //   ddt_t = u_t sum_n g_n B_tn + sum_n g_n h_(t-1)n a_n dA_tn
-//   da_n += g_n h_(t-1)n dt dA_tn g_n <- dA_tn g_n
+//   da_n += g_n h_(t-1)n dt dA_tn,   then g_n <- dA_tn g_n (carried to t-1)
 //   ddelta_t = ddt_t sigmoid(x_t),  dbias += ddelta_t,  dz_t = dout y_t silu'(z_t)
 //
 // A tile is 32 channels of one batch row (S6 layout, dstate 16), run by eight
@@ -28,7 +28,9 @@
 // segment after it, walks its 32-step blocks backwards, and per window
 // recomputes the 8 states and decays from the checkpoint into registers, then
 // runs the window in reverse.  A unit waits (bounded) only on units with smaller
-// tickets, which running CTAs hold, so the chain always progresses.
+// tickets, which running CTAs hold, so the chain always progresses.  Each block's
+// 32-step rows of the inputs are staged in shared memory by cp.async, double
+// buffered: a block's prologue issues the next block's rows.
 //
 // Sums over the states (y, sum g B, the decay term) are transposed shuffle
 // reductions inside the 8 lanes of a channel.  dB and dC, sums over channels, are

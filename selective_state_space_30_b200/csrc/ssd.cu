@@ -28,7 +28,9 @@
 // G (128 columns), Y (64), C H (64), S (64).
 //
 // Every wait is bounded (%globaltimer); a wait that runs out records
-// SSM_ERR_TIMEOUT and every thread leaves the chunk loop together.
+// SSM_ERR_TIMEOUT, and at the next CTA-wide vote (three per chunk) every thread
+// leaves the chunk loop together.  Threads wait for the tensor cores' results
+// themselves (tcgen05.commit -> mbarrier), without a CTA barrier.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -246,10 +248,11 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         const float* sw = sdt + 2 * kQ;
         const bool with_state = c > 0 || have_h0;
 
-        // ---- G = C B^T once the chunk's C and B tiles are in
-        const bool ok_cb = mbar_wait(full_cb, ph, budget, p.status);
-        if (__syncthreads_or(!ok_cb)) { failed = true; break; }
-        if (tid == 0) {
+        // ---- G = C B^T once the chunk's C and B tiles are in (thread 0 waits for them and
+        // issues; a wait that runs out is carried to the next CTA-wide vote)
+        bool ok = true;
+        if (tid == 0) ok = mbar_wait(full_cb, ph, budget, p.status);
+        if (tid == 0 && ok) {
             tc::fence_after();
             constexpr uint32_t id = tc::idesc_bf16(128, 128, true, true);
 #pragma unroll
@@ -267,13 +270,15 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             if (c + 2 < nchunks) dnext = delta_bits(p, b, h, t0 + 2 * kQ, lane);
         }
 
-        const bool ok_g = mbar_wait(mb_g, ph, budget, p.status);
-        if (__syncthreads_or(!ok_g)) { failed = true; break; }
+        // every thread waits for G itself
+        ok = ok && mbar_wait(mb_g, ph, budget, p.status);
         tc::fence_after();
 
         // ---- M = G o decay mask: row i = row, steps j0 .. j0+31 (a warp whose steps all lie
         // after its rows writes zeros: the causal mask)
-        if (j0 > (uint32_t)(32 * quarter + 31)) {
+        if (!ok) {
+            // a wait ran out: nothing to build, the vote below ends the loop
+        } else if (j0 > (uint32_t)(32 * quarter + 31)) {
             const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int k = 0; k < 32; k += 8)
@@ -300,8 +305,8 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         }
         tc::fence_async_smem();
         tc::fence_before();
-        const bool ok_x = mbar_wait(full_x, ph, budget, p.status);
-        if (__syncthreads_or(!ok_x)) { failed = true; break; }
+        ok = ok && mbar_wait(full_x, ph, budget, p.status);
+        if (__syncthreads_or(!ok)) { failed = true; break; }
 
         // ---- Y = M X (K-major, K = j) and C H (MN-major, K = n)
         if (tid == 0) {
@@ -328,12 +333,12 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             last_bar = mb_y;
             last_ph = ph;
         }
-        const bool ok_y = mbar_wait(mb_y, ph, budget, p.status);
-        if (__syncthreads_or(!ok_y)) { failed = true; break; }
+        // every thread waits for Y and C H itself
+        ok = mbar_wait(mb_y, ph, budget, p.status);
         tc::fence_after();
 
         // ---- outputs of step i = row, channels p0 .. p0+15
-        {
+        if (ok) {
             uint32_t yv[16], cv[16];
             tc::ld16(trow + kColY + p0, yv);
             if (with_state) tc::ld16(trow + kColCH + p0, cv);
@@ -355,7 +360,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             }
         }
         // ---- B' = B diag(w): row n = row, steps j0 .. j0+31
-        {
+        if (ok) {
             const unsigned char* bt = sB + (j0 >> 6) * 16384;
 #pragma unroll
             for (int k = 0; k < 32; k += 8) {
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         }
         tc::fence_async_smem();
         tc::fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { failed = true; break; }
 
         // ---- the out tile (written over the z tile) to global; S = B'^T X; then the next
         // chunk's C and B tiles (this chunk is done with them)
@@ -403,15 +408,15 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
                 }
             }
         }
-        const bool ok_s = mbar_wait(mb_s, ph, budget, p.status);
-        if (__syncthreads_or(!ok_s)) { failed = true; break; }
+        // every thread waits for S itself
+        ok = mbar_wait(mb_s, ph, budget, p.status);
         tc::fence_after();
         // the next chunk's X and z tiles (this chunk's MMAs that read X are complete, and
         // its outputs were written before the barrier above)
         // the out tile must be read out of shared memory before the z tile is loaded over it,
         // or (no gate) before the next chunk's outputs are written there after the barriers below
         if (tid == 0) bulk_wait_read();
-        if (tid == 0 && c + 1 < nchunks) {
+        if (tid == 0 && ok && c + 1 < nchunks) {
             mbar_arrive_tx(full_x, tx_x);
             for (int hb = 0; hb < 2; ++hb) {
                 tma_2d(sX + hb * 8192, &m.u, (int)(t0 + kQ + 64 * hb), x_row, full_x);
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         }
 
         // ---- H = 2^cum_end H + S (row n = row, channels p0 .. p0+15)
-        {
+        if (ok) {
             uint32_t sv[16];
             tc::ld16(trow + kColS + p0, sv);
             tc::wait_ld();
@@ -438,7 +443,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         }
         tc::fence_async_smem();
         tc::fence_before();
-        __syncthreads();   // H tile and the next chunk's decay are visible
+        if (__syncthreads_or(!ok)) { failed = true; break; }   // H tile and the next chunk's decay are visible
     }
     if (!failed && p.last_state) {
 #pragma unroll

@@ -13,16 +13,16 @@
 //   M  = G o [2^(cum_i - cum_j) dt_j]_{j <= i}   (causal decay mask)  threads
 //   Y  = M X + diag(2^cum) (C H)                 (Q x P)              tensor cores
 //   out = (Y + D x) silu(z)                                           threads
-//   B' = B diag(w),  w_j = 2^(cum_end - cum_j) dt_j                   threads
-//   H  = 2^cum_end H + B'^T X                    (N x P)              tensor cores + threads
+//   X' = diag(w) X,  w_j = 2^(cum_end - cum_j) dt_j                   threads
+//   H  = 2^cum_end H + B^T X'                    (N x P)              tensor cores + threads
 //
 // The output tile of a chunk is written by the threads over the z tile (each thread
 // writes out(p, t) where it read z(p, t)) and leaves by a TMA store.
 //
 // Operands the tensor cores read: B, C and X straight from TMA boxes (128-byte
-// swizzle; B and C as MN-major tiles, X as K-major), M and B' as K-major tiles
-// and H as an MN-major tile written by the threads.  M, B' and H are fp32
-// values; each goes in as a bf16 pair hi + lo (lo = the rounding residue), two
+// swizzle; B and C as MN-major tiles for G and C H, B as a K-major tile for S,
+// X K-major), M and X' as K-major tiles and H as an MN-major tile written by the
+// threads.  M, X' and H are fp32 values; each goes in as a bf16 pair hi + lo (lo = the rounding residue), two
 // MMAs per product, so the products keep about 16 significant bits: the state
 // stays within the fp32 tolerance of the recurrence.  Accumulators live in TMEM:
 // G (128 columns), Y (64), C H (64), S (64).
@@ -55,7 +55,7 @@ constexpr uint32_t kColG = 0, kColY = 128, kColCH = 192, kColS = 256;
 constexpr int OFF_C = 0;                 // C: 2 boxes (t halves) x 128 rows x 128 B
 constexpr int OFF_B = 32 * 1024;         // B: same
 constexpr int OFF_X = 64 * 1024;         // X (u rows of the head): 2 boxes x 64 rows x 128 B
-constexpr int OFF_MB = 80 * 1024;        // M, later B': hi (2 atom columns x 128 rows x 128 B), then lo
+constexpr int OFF_MB = 80 * 1024;        // M (hi: 2 atom columns x 128 rows x 128 B, then lo), later X' (hi, lo)
 constexpr int OFF_H = 144 * 1024;        // H: hi (128 rows x 128 B), then lo
 constexpr int OFF_Z = 176 * 1024;        // z (gate rows of the head): 2 boxes x 64 rows x 128 B
 constexpr int OFF_DT = 192 * 1024;       // two chunks' dt[128], cum[128], w[128] floats
@@ -359,30 +359,31 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
                 *slot = __bfloat16_as_ushort(__float2bfloat16_rn(v));   // out(p, t) where z(p, t) was
             }
         }
-        // ---- B' = B diag(w): row n = row, steps j0 .. j0+31
+        // ---- X' = diag(w) X as hi + lo in the M tile (free once Y is done): two 8-step
+        // pieces of a head-dim row per thread, laid out like the X tile (K-major, K = step)
         if (ok) {
-            const unsigned char* bt = sB + (j0 >> 6) * 16384;
 #pragma unroll
-            for (int k = 0; k < 32; k += 8) {
-                float wj[8];
-                lds8f(sw + j0 + k, wj);
-                const uint4 raw = *reinterpret_cast<const uint4*>(bt + tc::sw128_off(row, (j0 & 63u) + k));
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t e = (uint32_t)tid + (uint32_t)r * kThreadsSsd;   // 0 .. 1023
+                const uint32_t pp = e >> 4, s8 = (e & 15u) * 8u;                  // head-dim row, first step
+                const uint4 raw = *reinterpret_cast<const uint4*>(sX + (s8 >> 6) * 8192 + tc::sw128_off(pp, s8 & 63u));
                 const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                float v[8];
+                float wj[8], v[8];
+                lds8f(sw + s8, wj);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t bits = (e & 1) ? (w4[e >> 1] & 0xFFFF0000u) : (w4[e >> 1] << 16);
-                    v[e] = __uint_as_float(bits) * wj[e];
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t bits = (k & 1) ? (w4[k >> 1] & 0xFFFF0000u) : (w4[k >> 1] << 16);
+                    v[k] = __uint_as_float(bits) * wj[k];
                 }
-                store_pair8(sMhi + (j0 >> 6) * 16384, sMlo + (j0 >> 6) * 16384, row, (j0 & 63u) + k, v);
+                store_pair8(sMhi + (s8 >> 6) * 8192, sMlo + (s8 >> 6) * 8192, pp, s8 & 63u, v);
             }
         }
         tc::fence_async_smem();
         tc::fence_before();
         if (__syncthreads_or(!ok)) { failed = true; break; }
 
-        // ---- the out tile (written over the z tile) to global; S = B'^T X; then the next
-        // chunk's C and B tiles (this chunk is done with them)
+        // ---- the out tile (written over the z tile) to global; S = B^T X' (B, K-major, straight
+        // from its TMA tile); then the next chunk's C tile (B is read until S is done)
         if (tid == 0) {
             tma_store_2d(&m.out, (int)t0, x_row, sZ);
             tma_store_2d(&m.out, (int)t0 + 64, x_row, sZ + 8192);
@@ -391,21 +392,17 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             constexpr uint32_t ids = tc::idesc_bf16(128, kP, false, false);
 #pragma unroll
             for (int kk = 0; kk < kQ / 16; ++kk) {
-                const int at = (kk >> 2) * 16384 + (kk & 3) * 32;
-                const uint64_t bx = tc::desc(sX + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, tc::kSwizzle128);
-                tc::mma_bf16(tbase + kColS, tc::desc(sMhi + at, 16, 1024, tc::kSwizzle128), bx, ids, kk > 0 ? 1u : 0u);
-                tc::mma_bf16(tbase + kColS, tc::desc(sMlo + at, 16, 1024, tc::kSwizzle128), bx, ids, 1u);
+                const uint64_t ab = tc::desc(sB + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, tc::kSwizzle128);
+                const int xo = (kk >> 2) * 8192 + (kk & 3) * 32;
+                tc::mma_bf16(tbase + kColS, ab, tc::desc(sMhi + xo, 16, 1024, tc::kSwizzle128), ids, kk > 0 ? 1u : 0u);
+                tc::mma_bf16(tbase + kColS, ab, tc::desc(sMlo + xo, 16, 1024, tc::kSwizzle128), ids, 1u);
             }
             tc::commit(mb_s);
             last_bar = mb_s;
             last_ph = ph;
             if (c + 1 < nchunks) {
-                mbar_arrive_tx(full_cb, kTxCB);
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int x = (int)(t0 + kQ + 64 * hb);
-                    tma_2d(sC + hb * 16384, &m.C, x, bc_row, full_cb);
-                    tma_2d(sB + hb * 16384, &m.B, x, bc_row, full_cb);
-                }
+                mbar_arrive_tx(full_cb, kTxCB);   // C now, B once S has read it
+                for (int hb = 0; hb < 2; ++hb) tma_2d(sC + hb * 16384, &m.C, (int)(t0 + kQ + 64 * hb), bc_row, full_cb);
             }
         }
         // every thread waits for S itself
@@ -417,6 +414,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         // or (no gate) before the next chunk's outputs are written there after the barriers below
         if (tid == 0) bulk_wait_read();
         if (tid == 0 && ok && c + 1 < nchunks) {
+            for (int hb = 0; hb < 2; ++hb) tma_2d(sB + hb * 16384, &m.B, (int)(t0 + kQ + 64 * hb), bc_row, full_cb);
             mbar_arrive_tx(full_x, tx_x);
             for (int hb = 0; hb < 2; ++hb) {
                 tma_2d(sX + hb * 8192, &m.u, (int)(t0 + kQ + 64 * hb), x_row, full_x);

@@ -499,24 +499,37 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
 
 // dB, dC: sum of the per-tile rows of the group; dA, dD, dbias: sum over batch rows and
 // segments, in a fixed order.
+// vec4: four consecutive steps per thread with 16-byte loads and stores (L a multiple
+// of 4, dB and dC 16-byte aligned); every element sums its tiles in the same order.
 __global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, float* dA, float* dB, float* dC,
-                                                         float* dD, float* dbias) {
+                                                         float* dD, float* dbias, int vec4) {
     const int64_t Dm = p.dim, L = p.seqlen, G = p.ngroups;
     const int64_t nbc = p.batch * G * kN * L;
+    const int64_t vw = vec4 ? 4 : 1;
     const int64_t tpg = (Dm / G) / kCT;   // tiles per group
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < 2 * nbc) {
-        const bool isC = i >= nbc;
-        const int64_t k = isC ? i - nbc : i;
+    if (i < 2 * nbc / vw) {
+        const bool isC = i >= nbc / vw;
+        const int64_t k = (isC ? i - nbc / vw : i) * vw;
         const int64_t t = k % L, n = (k / L) % kN, bg = k / (L * kN);
         const int64_t b = bg / G, g = bg % G;
         const float* src = (isC ? p.dCp : p.dBp) + ((b * p.tiles_per_row + g * tpg) * kN + n) * L + t;
-        float s = 0.f;
-        for (int64_t m = 0; m < tpg; ++m) s += src[m * kN * L];
-        (isC ? dC : dB)[k] = s;
+        float* dst = (isC ? dC : dB) + k;
+        if (vec4) {
+            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int64_t m = 0; m < tpg; ++m) {
+                const float4 v = __ldcs(reinterpret_cast<const float4*>(src + m * kN * L));
+                s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+            }
+            *reinterpret_cast<float4*>(dst) = s;
+        } else {
+            float s = 0.f;
+            for (int64_t m = 0; m < tpg; ++m) s += src[m * kN * L];
+            *dst = s;
+        }
         return;
     }
-    const int64_t k = i - 2 * nbc;
+    const int64_t k = i - 2 * nbc / vw;
     const int64_t rows = p.batch * Dm;
     if (k < Dm * kN) {
         float s = 0.f;
@@ -648,10 +661,11 @@ int launch(const BwdParams& prm, float* dA, float* dB, float* dC, float* dD, flo
     constexpr int smem = Smem<T>::TOTAL;
     scan_bwd_kernel<T><<<(unsigned)ctas, kThreads, smem, s>>>(prm);
     if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
-    const int64_t work = 2 * prm.batch * prm.ngroups * kN * prm.seqlen + prm.dim * kN + 2 * prm.dim;
+    const int vec4 = prm.seqlen % 4 == 0 && ((reinterpret_cast<uintptr_t>(dB) | reinterpret_cast<uintptr_t>(dC)) & 15u) == 0;
+    const int64_t work = 2 * prm.batch * prm.ngroups * kN * prm.seqlen / (vec4 ? 4 : 1) + prm.dim * kN + 2 * prm.dim;
     const int64_t blocks = (work + 255) / 256;
     if (blocks > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;
-    scan_bwd_finalize<<<(unsigned)blocks, 256, 0, s>>>(prm, dA, dB, dC, dD, dbias);
+    scan_bwd_finalize<<<(unsigned)blocks, 256, 0, s>>>(prm, dA, dB, dC, dD, dbias, vec4);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

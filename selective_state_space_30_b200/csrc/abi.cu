@@ -303,15 +303,21 @@ const char* ssm_status_string(int status) {
 // The host-buffer pipeline's streams, events and chunk plan (built on first use).
 static void release_pipeline(ssm_plan_s* p) {
     if (!p->pipe_ready) return;
-    for (int i = 0; i < 3; ++i) cudaStreamDestroy(p->pipe[i]);
-    cudaEventDestroy(p->ev_start);
-    cudaEventDestroy(p->ev_end);
+    for (int i = 0; i < 3; ++i)
+        if (p->pipe[i]) cudaStreamDestroy(p->pipe[i]);
+    cudaEvent_t* evs[2] = {&p->ev_start, &p->ev_end};
+    for (cudaEvent_t* e : evs)
+        if (*e) cudaEventDestroy(*e);
     for (int i = 0; i < 8; ++i) {
-        cudaEventDestroy(p->ev_in[i]);
-        cudaEventDestroy(p->ev_run[i]);
+        if (p->ev_in[i]) cudaEventDestroy(p->ev_in[i]);
+        if (p->ev_run[i]) cudaEventDestroy(p->ev_run[i]);
     }
     if (p->sub) ssm_scan_destroy(p->sub);
     p->sub = nullptr;
+    std::memset(p->pipe, 0, sizeof(p->pipe));
+    p->ev_start = p->ev_end = nullptr;
+    std::memset(p->ev_in, 0, sizeof(p->ev_in));
+    std::memset(p->ev_run, 0, sizeof(p->ev_run));
     p->pipe_ready = false;
 }
 
@@ -442,6 +448,7 @@ static int build_pipeline(ssm_plan_s* p) {
     cd.batch = d.batch / n;
     int rc = ssm_scan_plan(&p->sub, &cd, p->device);
     if (rc != SSM_OK) return rc;
+    p->pipe_ready = true;   // from here on release_pipeline frees what was made
     p->sub->spin_limit = p->spin_limit;
     if (p->force_ssd) {
         rc = ssm_scan_set_option(p->sub, SSM_OPT_SSD, p->force_ssd);
@@ -454,7 +461,6 @@ static int build_pipeline(ssm_plan_s* p) {
     for (int i = 0; i < 8; ++i)
         ok = ok && cudaEventCreateWithFlags(&p->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
              cudaEventCreateWithFlags(&p->ev_run[i], cudaEventDisableTiming) == cudaSuccess;
-    p->pipe_ready = true;   // release_pipeline destroys what was made
     return ok ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -728,7 +728,7 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
         if (grads->ddelta_bias) ok = ok && cudaMemsetAsync(grads->ddelta_bias, 0, dims->dim * 4, s) == cudaSuccess;
         if (nbc) ok = ok && cudaMemsetAsync(grads->dB, 0, nbc, s) == cudaSuccess &&
                       cudaMemsetAsync(grads->dC, 0, nbc, s) == cudaSuccess;
-        if (rows * dims->seqlen) {
+        if (rows > 0 && dims->seqlen > 0) {
             ok = ok && cudaMemsetAsync(grads->du, 0, rows * dims->seqlen * esz, s) == cudaSuccess &&
                  cudaMemsetAsync(grads->ddelta, 0, rows * dims->seqlen * esz, s) == cudaSuccess;
             if (grads->dz) ok = ok && cudaMemsetAsync(grads->dz, 0, rows * dims->seqlen * esz, s) == cudaSuccess;

@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
     bool failed = false;
     uint64_t* last_bar = nullptr;   // thread 0: the barrier of its latest commit and that phase
     unsigned last_ph = 0;
+    int pend_cb = 0, pend_x = 0;    // thread 0: the chunk whose C, B (X, z) loads are in flight, or -1
     for (int c = 0; c < nchunks; ++c) {
         const int64_t t0 = (int64_t)c * kQ;
         const unsigned ph = (unsigned)c & 1u;
@@ -251,7 +252,10 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         // ---- G = C B^T once the chunk's C and B tiles are in (thread 0 waits for them and
         // issues; a wait that runs out is carried to the next CTA-wide vote)
         bool ok = true;
-        if (tid == 0) ok = mbar_wait(full_cb, ph, budget, p.status);
+        if (tid == 0) {
+            ok = mbar_wait(full_cb, ph, budget, p.status);
+            if (ok) pend_cb = -1;
+        }
         if (tid == 0 && ok) {
             tc::fence_after();
             constexpr uint32_t id = tc::idesc_bf16(128, 128, true, true);
@@ -306,6 +310,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         tc::fence_async_smem();
         tc::fence_before();
         ok = ok && mbar_wait(full_x, ph, budget, p.status);
+        if (tid == 0 && ok) pend_x = -1;
         if (__syncthreads_or(!ok)) { failed = true; break; }
 
         // ---- Y = M X (K-major, K = j) and C H (MN-major, K = n)
@@ -401,6 +406,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
             last_bar = mb_s;
             last_ph = ph;
             if (c + 1 < nchunks) {
+                pend_cb = c + 1;
                 mbar_arrive_tx(full_cb, kTxCB);   // C now, B once S has read it
                 for (int hb = 0; hb < 2; ++hb) tma_2d(sC + hb * 16384, &m.C, (int)(t0 + kQ + 64 * hb), bc_row, full_cb);
             }
@@ -415,6 +421,7 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
         if (tid == 0) bulk_wait_read();
         if (tid == 0 && ok && c + 1 < nchunks) {
             for (int hb = 0; hb < 2; ++hb) tma_2d(sB + hb * 16384, &m.B, (int)(t0 + kQ + 64 * hb), bc_row, full_cb);
+            pend_x = c + 1;
             mbar_arrive_tx(full_x, tx_x);
             for (int hb = 0; hb < 2; ++hb) {
                 tma_2d(sX + hb * 8192, &m.u, (int)(t0 + kQ + 64 * hb), x_row, full_x);
@@ -447,9 +454,13 @@ __global__ void __launch_bounds__(kThreadsSsd, 1) ssd_fwd_kernel(const SsdParams
 #pragma unroll
         for (int k = 0; k < 16; ++k) p.last_state[(b * Dm + d0 + p0 + k) * kN + row] = H[k];
     }
-    // release TMEM once nothing can still write it: after a failed wait, wait (bounded) for
-    // the last tensor-core batch this CTA committed
-    if (failed && tid == 0 && last_bar) mbar_wait(last_bar, last_ph, budget, p.status);
+    // release TMEM and shared memory once nothing can still write them: after a failed wait,
+    // wait (bounded) for the last tensor-core batch this CTA committed and its loads in flight
+    if (failed && tid == 0) {
+        if (last_bar) mbar_wait(last_bar, last_ph, budget, p.status);
+        if (pend_cb >= 0) mbar_wait(full_cb, (unsigned)pend_cb & 1u, budget, p.status);
+        if (pend_x >= 0) mbar_wait(full_x, (unsigned)pend_x & 1u, budget, p.status);
+    }
     if (tid == 0) bulk_wait_all();   // the last out tile is written before shared memory goes away
     tc::fence_before();
     __syncthreads();

@@ -320,7 +320,8 @@ static void bwd_rows(bjob_t* j) {
                     const double s = sigmoid_f64(z[t]);
                     const double dsilu = s * (1.0 + z[t] * (1.0 - s));
                     j->g.dz[row * L + t] = go[t] * y * dsilu;
-                    if (j->m.dz) j->m.dz[row * L + t] = fabs(go[t] * dsilu) * ym;
+                    /* silu'(z) = s + z s (1 - s) is a sum of two terms: its magnitude is s (1 + |z| (1 - s)) */
+                    if (j->m.dz) j->m.dz[row * L + t] = fabs(go[t]) * s * (1.0 + fabs(z[t]) * (1.0 - s)) * ym;
                 }
                 ADD(j->g.dD, d, dy * u[t]);
                 ADD(j->m.dD, d, fabs(dy * u[t]));

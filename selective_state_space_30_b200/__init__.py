@@ -5,6 +5,7 @@ This package binds it with ctypes (`_abi`, same names as the C entry points)
 and adds a small torch-tensor front end:
 
     out, last_state = selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus=True)
+    out, last_state = selective_scan_fn(...)   # the same, differentiable (torch autograd)
 
 PyTorch is only used for device memory and streams; the scan runs in the
 library's kernels.  There is no CPU or PyTorch fallback.
@@ -28,7 +29,7 @@ from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, 
                    GRAD_NAMES,
                    ssm_status_string)
 
-__all__ = ["selective_scan_fwd", "selective_scan_fwd_host", "Plan", "get_plan", "ssm_scan_plan",
+__all__ = ["selective_scan_fwd", "selective_scan_fwd_host", "selective_scan_fn", "Plan", "get_plan", "ssm_scan_plan",
            "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0", "ssm_selective_scan_fwd_host",
            "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update", "ssm_causal_conv1d_fwd",
            "selective_scan_bwd", "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_workspace_size",
@@ -175,3 +176,44 @@ def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None,
     ssm_selective_scan_bwd(dims, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dout, dlast, g, workspace,
                            workspace.numel() * workspace.element_size(), stream)
     return g
+
+
+_fn_cls = None
+
+
+def _selective_scan_function():
+    """The torch.autograd.Function over the forward and backward entry points (built
+    on first use, so that importing the package does not import torch)."""
+    global _fn_cls
+    if _fn_cls is not None:
+        return _fn_cls
+    import torch
+
+    class SelectiveScanFn(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, u, delta, A, B, C, D, z, delta_bias, h0, softplus):
+            out, last = selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, h0=h0)
+            ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, h0)
+            ctx.softplus = softplus
+            return out, last
+
+        @staticmethod
+        def backward(ctx, dout, dlast):
+            u, delta, A, B, C, D, z, delta_bias, h0 = ctx.saved_tensors
+            want_dh0 = h0 is not None and ctx.needs_input_grad[8]
+            g = selective_scan_bwd(u, delta, A, B, C, dout.contiguous(), D, z, delta_bias, ctx.softplus, h0=h0,
+                                   dlast=dlast.contiguous() if dlast is not None else None, want_dh0=want_dh0)
+            return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype),
+                    g["dD"] if D is not None else None, g["dz"], g["ddelta_bias"] if delta_bias is not None else None,
+                    g["dh0"], None)
+
+    _fn_cls = SelectiveScanFn
+    return _fn_cls
+
+
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True, h0=None):
+    """The forward scan as a differentiable torch operation: returns (out, last_state),
+    and the backward runs ssm_selective_scan_bwd (which covers the per-channel layout with
+    dstate 16; other shapes raise SsmError when their gradient is taken).  dB and dC are
+    formed in fp32 and returned in B's and C's dtype."""
+    return _selective_scan_function().apply(u, delta, A, B, C, D, z, delta_bias, h0, softplus)

@@ -47,7 +47,7 @@ def run_bwd(dims, inp, gin, want_dh0=False, softplus=True):
     return g
 
 
-def check_grads(g, ref, mag, dtype, what=""):
+def check_grads(g, ref, mag, dtype, what="", bf16_out=BF16_OUT):
     for k, r in ref.items():
         if r is None:
             assert g.get(k) is None, f"{what}{k}: expected no output"
@@ -56,7 +56,7 @@ def check_grads(g, ref, mag, dtype, what=""):
         assert np.all(np.isfinite(got)), f"{what}{k}: non-finite values"
         err = np.abs(got - r)
         tol = 1e-4 * mag[k]
-        if dtype == "bf16" and k in BF16_OUT:
+        if dtype == "bf16" and k in bf16_out:
             tol = tol + bf16_ulp(r)
         bad = err > tol
         if bad.any():

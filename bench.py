@@ -40,6 +40,7 @@ L2_BYTES = 126 * 1024 * 1024
 SMS = 148
 EX2_PER_CLK_PER_SM = 16          # MUFU ex2 issue rate per SM per clock (sm_80 .. sm_100 family)
 NOMINAL_SM_MHZ = 1965.0
+HBM_NOMINAL_GBS = 8000.0          # B200 HBM3e, NVIDIA's figure; the roofline's peak is the measured copy rate
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 
 
@@ -407,7 +408,8 @@ def run_ours(args):
     traffic = _traffic_from_profiles(w.name)
     hbm_obj = {"achieved": alg_bytes / avg_launch_s / 1e9, "peak": hbm_gbs, "unit": "GB/s",
                "frac": alg_bytes / avg_launch_s / 1e9 / hbm_gbs, "peak_source": peak_src,
-               "alg_bytes_per_launch": alg_bytes}
+               "alg_bytes_per_launch": alg_bytes,
+               "frac_of_nominal": alg_bytes / avg_launch_s / 1e9 / HBM_NOMINAL_GBS, "nominal_gbs": HBM_NOMINAL_GBS}
     mufu_obj = {"achieved": exps / avg_launch_s / 1e9, "peak": mufu_peak / 1e9, "unit": "Gexp/s",
                 "frac": (exps / avg_launch_s) / mufu_peak,
                 "what": "MUFU ex2: B*D*L*N exps per launch / mean launch time; peak = 148 SM x 16 ex2/clk x "

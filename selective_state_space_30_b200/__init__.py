@@ -69,8 +69,11 @@ _plans: Dict[tuple, Plan] = {}
 _plans_lock = threading.Lock()
 
 
-def get_plan(batch, dim, seqlen, dstate, nheads=0, ngroups=1, io_dtype=SSM_BF16, device=0) -> Plan:
-    key = (batch, dim, seqlen, dstate, nheads or dim, ngroups, io_dtype, device)
+def get_plan(batch, dim, seqlen, dstate, nheads=0, ngroups=1, io_dtype=SSM_BF16, device=0, stream=None) -> Plan:
+    """The cached plan of a shape on a device, one per stream: a plan's workspace
+    (ticket counter, carry flags and buffers) serves one call at a time, and the
+    calls on one stream run in order."""
+    key = (batch, dim, seqlen, dstate, nheads or dim, ngroups, io_dtype, device, _abi._stream(stream) or 0)
     with _plans_lock:
         p = _plans.get(key)
         if p is None:
@@ -113,13 +116,13 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
             if not t.is_contiguous():
                 raise ValueError(f"{name} must be contiguous")
     dev = u.device.index if u.device.index is not None else torch.cuda.current_device()
-    plan = get_plan(batch, dim, seqlen, dstate, nheads, ngroups, io, dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(u.device).cuda_stream
+    plan = get_plan(batch, dim, seqlen, dstate, nheads, ngroups, io, dev, stream)
     if out is None:
         out = torch.empty_like(u)
     if return_last_state and last_state is None:
         last_state = torch.empty((batch, dim, dstate), dtype=torch.float32, device=u.device)
-    if stream is None:
-        stream = torch.cuda.current_stream(u.device).cuda_stream
     ssm_selective_scan_fwd_h0(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, h0, out,
                               last_state if return_last_state else None, stream)
     return out, (last_state if return_last_state else None)
@@ -132,13 +135,13 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
     copies the inputs to the device, runs the scan and copies the results back."""
     import torch
     batch, dim, seqlen, dstate, nheads, ngroups, io = _shapes(u, delta, A, B)
-    plan = get_plan(batch, dim, seqlen, dstate, nheads, ngroups, io, device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device).cuda_stream
+    plan = get_plan(batch, dim, seqlen, dstate, nheads, ngroups, io, device, stream)
     if out is None:
         out = torch.empty_like(u, pin_memory=True)
     if return_last_state and last_state is None:
         last_state = torch.empty((batch, dim, dstate), dtype=torch.float32, pin_memory=True)
-    if stream is None:
-        stream = torch.cuda.current_stream(device).cuda_stream
     ssm_selective_scan_fwd_host(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, out,
                                 last_state if return_last_state else None, stream)
     return out, (last_state if return_last_state else None)

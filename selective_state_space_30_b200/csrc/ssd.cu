@@ -478,9 +478,9 @@ bool ssd_eligible(const ssm_dims_t& d) {
 int ssd_smem_bytes() { return kSmemSsd; }
 
 int ssd_launch(const SsdParams& prm, const SsdMaps& maps, int64_t grid, cudaStream_t s) {
-    static const bool attr = cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  kSmemSsd) == cudaSuccess;
-    if (!attr) return SSM_ERR_CUDA;
+    // every launch: the attribute belongs to the current device's instance of the kernel
+    if (cudaFuncSetAttribute(ssd_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemSsd) != cudaSuccess)
+        return SSM_ERR_CUDA;
     if (grid <= 0) return SSM_OK;
     ssd_fwd_kernel<<<(unsigned)grid, kThreadsSsd, kSmemSsd, s>>>(prm, maps);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;

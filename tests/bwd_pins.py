@@ -14,7 +14,8 @@ in the mutation tests) and raises AssertionError on a disagreement:
   ("Agent 229: SSM optimization patterns" page, section 2 "State Space
   Duality"): du = M^T dy + D dy with dy = dout * silu(z);
 * linearity of every gradient in (dout, dlast), and magnitudes that bound
-  the gradients.
+  the gradients;
+* dz's magnitude covering an fp32 evaluation of dz where silu'(z) cancels.
 """
 from __future__ import annotations
 
@@ -167,4 +168,32 @@ def pin_bwd_linear_in_dout(lib):
         assert np.all(m1[k] >= np.abs(g1[k]) * (1 - 1e-12) - 1e-15), f"magnitude below |grad| for {k}"
 
 
-BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_step, pin_bwd_du_transpose, pin_bwd_linear_in_dout]
+def pin_bwd_dz_magnitude_covers_fp32(lib):
+    """dz = dout y silu'(z) evaluated in fp32 (numpy float32, from the rounded fp64 y) stays within
+    1e-4 of the oracle's magnitude for dz, on a grid of z that runs through the root of
+    silu'(z) = s (1 + z (1 - s)) near z = -1.278, where the factor cancels in fp32."""
+    rng = np.random.default_rng(35)
+    L, N = 400, 4
+    c = dict(batch=1, dim=1, L=L, N=N)
+    p = _rand_problem(rng, 1, 1, L, N)
+    zg = np.concatenate([np.linspace(-1.30, -1.25, L // 2), np.linspace(-8.0, 6.0, L // 2)])
+    p["z"] = zg.reshape(1, 1, L)
+    dout = rng.standard_normal((1, 1, L))
+    grads, mags = _bwd(lib, c, p, dout)
+    # y without the gate, from the pinned forward
+    y, _, _ = _run(lib, 1, 1, L, N, dict(p, z=None))
+    s64 = 1.0 / (1.0 + np.exp(-zg))
+    # the grid reaches the cancellation: |silu'| far below the sum of its terms' magnitudes
+    assert np.min(np.abs(s64 * (1.0 + zg * (1.0 - s64))) / (s64 * (1.0 + np.abs(zg) * (1.0 - s64)))) < 1e-4
+    f = np.float32
+    z32 = zg.astype(f)
+    s32 = f(1.0) / (f(1.0) + np.exp(-z32))
+    d32 = s32 * (f(1.0) + z32 * (f(1.0) - s32))
+    dz32 = (dout[0, 0].astype(f) * y[0, 0].astype(f) * d32).astype(np.float64)
+    err = np.abs(dz32 - grads["dz"][0, 0])
+    tol = 1e-4 * mags["dz"][0, 0]
+    assert np.all(err <= tol), f"fp32 dz outside 1e-4 * mag at z = {zg[np.argmax(err - tol)]!r}"
+
+
+BWD_PINS = [pin_bwd_finite_differences, pin_bwd_single_step, pin_bwd_du_transpose, pin_bwd_linear_in_dout,
+            pin_bwd_dz_magnitude_covers_fp32]

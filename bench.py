@@ -35,7 +35,7 @@ if ROOT not in sys.path:
 
 METRIC = "selective-scan Gelem/s (B*D*L/s) fwd and % of HBM/MUFU roofline on 1 B200"
 UNIT = "Gelem/s"
-DEFAULT_WORKLOAD = "mamba-130m"
+DEFAULT_WORKLOAD = "mamba-2.8b-long"   # the largest single-GPU forward shape
 L2_BYTES = 126 * 1024 * 1024
 SMS = 148
 EX2_PER_CLK_PER_SM = 16          # MUFU ex2 issue rate per SM per clock (sm_80 .. sm_100 family)
@@ -138,7 +138,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.002):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples = []
         self.reasons = 0
         self.max_mhz = None
@@ -328,73 +328,30 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args):
+class _Nvtx:
+    """An NVTX range around a timed region (seen by Nsight tools; a no-op without them)."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        import torch
+        try:
+            torch.cuda.nvtx.range_push(self.name)
+            self.on = True
+        except Exception:  # pragma: no cover - no NVTX
+            self.on = False
+        return self
+
+    def __exit__(self, *a):
+        import torch
+        if self.on:
+            torch.cuda.nvtx.range_pop()
+
+
+def _probe_mufu(ssm, dev, sh, stream):
+    """ex2 rate of the probe kernel in this process (G ex2/s), at whatever clock the GPU runs."""
     import torch
-    import ssm_inputs as si
-    import selective_state_space_30_b200 as ssm
-
-    rank, local, world = _rank_env()
-    if world > 1:
-        torch.cuda.set_device(local)
-    init_ranks("nccl", local)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    w = si.WORKLOADS[args.workload]
-    d = w.dims
-    io = ssm.SSM_BF16 if d.dtype == "bf16" else ssm.SSM_F32
-    inp = si.make_inputs(d, w.recipe, w.seed)
-    names = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
-    alg_bytes = _alg_bytes(d)
-    # enough copies that consecutive steps never find their inputs in L2
-    copies = max(2, int(np.ceil(3 * L2_BYTES / alg_bytes)))
-    sets = []
-    for _ in range(copies):
-        t = {k: _to_dev(inp[k], dev) for k in names}
-        t["out"] = torch.empty_like(t["u"])
-        t["last"] = torch.empty(d.batch, d.dim, d.dstate, dtype=torch.float32, device=dev)
-        sets.append(t)
-    dims = ssm.make_dims(d.batch, d.dim, d.seqlen, d.dstate, d.H, d.ngroups, io)
-    plan = ssm.ssm_scan_plan(dims, local)
-    info = ssm.ssm_scan_plan_info(plan)
-    sched = ssm.ssm_scan_plan_schedule(plan)
-    stream = torch.cuda.current_stream(dev)
-    sh = stream.cuda_stream
-
-    def step(i):
-        t = sets[i % copies]
-        ssm.ssm_selective_scan_fwd(plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
-                                   t["delta_bias"], w.recipe.softplus, dims, t["out"], t["last"], sh)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    barrier()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
-        torch.cuda.synchronize(dev)
-        for i in range(args.steps):
-            starts[i].record(stream)
-            step(i)
-            ends[i].record(stream)
-        torch.cuda.synchronize(dev)
-    barrier()
-    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]), dev)
-    st = ssm.ssm_scan_device_status(plan, sh)
-    if st != ssm.SSM_OK:
-        raise RuntimeError(f"device status {ssm.ssm_status_string(st)}")
-
-    elems = d.batch * d.dim * d.seqlen
-    ms_per_step = total_ms / args.steps
-    value = job_throughput(world, elems, args.steps, total_ms)
-
-    # roofline of the scan kernel (one launch per step)
-    hbm_gbs, sm_max_mhz, peak_src = _peaks()
-    avg_launch_s = statistics.mean(launch_ms) * 1e-3
-    exps = _exps(d)
-    mufu_peak = SMS * EX2_PER_CLK_PER_SM * sm_max_mhz * 1e6        # ex2/s at the max SM clock
-    # MUFU rate measured in this process (probe kernel), at whatever clock the GPU runs
     sink = torch.empty(SMS * 8 * 256, device=dev)
     ssm.ssm_probe_ex2(sink, SMS * 8, 64, sh)
     torch.cuda.synchronize(dev)
@@ -403,9 +360,16 @@ def run_ours(args):
     ssm.ssm_probe_ex2(sink, SMS * 8, 2048, sh)
     pe1.record(stream)
     torch.cuda.synchronize(dev)
-    probe_rate = SMS * 8 * 256 * 2048 * 16 / (pe0.elapsed_time(pe1) * 1e-3)
+    return SMS * 8 * 256 * 2048 * 16 / (pe0.elapsed_time(pe1) * 1e-3)
+
+
+def _roofline(d, info, avg_launch_s, wname, probe_rate):
+    """The roofline object of one forward launch: MUFU ex2 (scan kernel) or HBM / tensor (SSD)."""
+    hbm_gbs, sm_max_mhz, peak_src = _peaks()
+    alg_bytes = _alg_bytes(d)
+    exps = _exps(d)
+    mufu_peak = SMS * EX2_PER_CLK_PER_SM * sm_max_mhz * 1e6        # ex2/s at the max SM clock
     t_roof = max(alg_bytes / (hbm_gbs * 1e9), exps / mufu_peak)
-    traffic = _traffic_from_profiles(w.name)
     hbm_obj = {"achieved": alg_bytes / avg_launch_s / 1e9, "peak": hbm_gbs, "unit": "GB/s",
                "frac": alg_bytes / avg_launch_s / 1e9 / hbm_gbs, "peak_source": peak_src,
                "alg_bytes_per_launch": alg_bytes,
@@ -424,53 +388,185 @@ def run_ours(args):
                       "frac": flops / avg_launch_s / 1e12 / tf, "peak_source": tf_src,
                       "flops_per_launch": flops, "what": "algorithmic SSD flops (G, M X, C H, B'^T X per chunk)"}
         main = dict(hbm_obj, bound="hbm") if t_hbm >= t_tc else dict(tensor_obj, bound="tensor")
-        traffic = _traffic_from_profiles(w.name, key="ssd:" + w.name, sha=_src_hash(("ssd.cu", "tcgen05.cuh")))
-        roof = dict(main, traffic=traffic, roofline_frac=max(t_hbm, t_tc) / avg_launch_s,
+        traffic = _traffic_from_profiles(wname, key="ssd:" + wname, sha=_src_hash(("ssd.cu", "tcgen05.cuh")))
+        return dict(main, traffic=traffic, roofline_frac=max(t_hbm, t_tc) / avg_launch_s,
                     hbm=hbm_obj, tensor=tensor_obj,
                     mufu_literal=dict(mufu_obj, note="B*D*L*N exps: the SSD path takes one exp per (t, head)"))
-    else:
-        roof = {"bound": "alu", "achieved": mufu_obj["achieved"], "peak": mufu_obj["peak"], "unit": "Gexp/s",
-                "frac": mufu_obj["frac"], "traffic": traffic, "what": mufu_obj["what"],
-                "roofline_frac": t_roof / avg_launch_s, "hbm": hbm_obj,
-                "mufu_probe_gexps": mufu_obj["mufu_probe_gexps"], "frac_of_probe": mufu_obj["frac_of_probe"]}
+    return {"bound": "alu", "achieved": mufu_obj["achieved"], "peak": mufu_obj["peak"], "unit": "Gexp/s",
+            "frac": mufu_obj["frac"], "traffic": _traffic_from_profiles(wname), "what": mufu_obj["what"],
+            "roofline_frac": t_roof / avg_launch_s, "hbm": hbm_obj,
+            "mufu_probe_gexps": mufu_obj["mufu_probe_gexps"], "frac_of_probe": mufu_obj["frac_of_probe"]}
 
-    # end to end through the host-buffer entry point: pinned host inputs, copies in the timed region
-    e2e = None
-    if not args.no_e2e:
-        hp = {k: _to_pinned(inp[k]) for k in names}
+
+class _ScanJob:
+    """One forward workload resident on the device: rotating input sets, a plan, and a step."""
+
+    NAMES = ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")
+
+    def __init__(self, ssm, w, dev, local):
+        import torch
+        self.ssm, self.w, self.dev = ssm, w, dev
+        d = self.d = w.dims
+        io = ssm.SSM_BF16 if d.dtype == "bf16" else ssm.SSM_F32
+        import ssm_inputs as si
+        self.inp = si.make_inputs(d, w.recipe, w.seed)
+        self.alg_bytes = _alg_bytes(d)
+        # enough copies that consecutive steps never find their inputs in L2
+        self.copies = max(2, int(np.ceil(3 * L2_BYTES / self.alg_bytes)))
+        self.sets = []
+        for _ in range(self.copies):
+            t = {k: _to_dev(self.inp[k], dev) for k in self.NAMES}
+            t["out"] = torch.empty_like(t["u"])
+            t["last"] = torch.empty(d.batch, d.dim, d.dstate, dtype=torch.float32, device=dev)
+            self.sets.append(t)
+        self.dims = ssm.make_dims(d.batch, d.dim, d.seqlen, d.dstate, d.H, d.ngroups, io)
+        self.plan = ssm.ssm_scan_plan(self.dims, local)
+        self.info = ssm.ssm_scan_plan_info(self.plan)
+        self.sched = ssm.ssm_scan_plan_schedule(self.plan)
+        self.stream = torch.cuda.current_stream(dev)
+        self.sh = self.stream.cuda_stream
+
+    def step(self, i):
+        t = self.sets[i % self.copies]
+        self.ssm.ssm_selective_scan_fwd(self.plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
+                                        t["delta_bias"], self.w.recipe.softplus, self.dims, t["out"], t["last"],
+                                        self.sh)
+
+    def timed(self, steps, warmup, local):
+        """Warm up, then time exactly `steps` launches with CUDA events on the launching stream
+        (barrier + synchronize on both sides); returns per-launch ms, the max-over-ranks total ms
+        and the clock record."""
+        import torch
+        for i in range(warmup):
+            self.step(i)
+        torch.cuda.synchronize(self.dev)
+        barrier()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        with ClockSampler(local) as clk, _Nvtx(f"timed:{self.w.name}"):
+            torch.cuda.synchronize(self.dev)
+            for i in range(steps):
+                starts[i].record(self.stream)
+                self.step(i)
+                ends[i].record(self.stream)
+            torch.cuda.synchronize(self.dev)
+        barrier()
+        launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]), self.dev)
+        st = self.ssm.ssm_scan_device_status(self.plan, self.sh)
+        if st != self.ssm.SSM_OK:
+            raise RuntimeError(f"{self.w.name}: device status {self.ssm.ssm_status_string(st)}")
+        return launch_ms, total_ms, clk.summary()
+
+    def e2e(self, steps, world):
+        """The same metric through the host-buffer entry point: pinned host inputs, copies in the timed region."""
+        import torch
+        d, ssm, names = self.d, self.ssm, self.NAMES
+        hp = {k: _to_pinned(self.inp[k]) for k in names}
         hout = torch.empty(d.batch, d.dim, d.seqlen, dtype=torch.int16 if d.dtype == "bf16" else torch.float32,
                            pin_memory=True)
         hlast = torch.empty(d.batch, d.dim, d.dstate, dtype=torch.float32, pin_memory=True)
-        e2e_steps = max(3, min(args.steps, 50))
 
         def hstep():
-            ssm.ssm_selective_scan_fwd_host(plan, hp["u"], hp["delta"], hp["A"], hp["B"], hp["C"], hp["D"],
-                                            hp["z"], hp["delta_bias"], w.recipe.softplus, dims, hout, hlast, sh)
+            ssm.ssm_selective_scan_fwd_host(self.plan, hp["u"], hp["delta"], hp["A"], hp["B"], hp["C"], hp["D"],
+                                            hp["z"], hp["delta_bias"], self.w.recipe.softplus, self.dims, hout,
+                                            hlast, self.sh)
         for _ in range(2):
             hstep()
-        torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(self.dev)
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            hstep()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ems = max_over_ranks(e0.elapsed_time(e1), dev)
+        with _Nvtx(f"e2e:{self.w.name}"):
+            e0.record(self.stream)
+            for _ in range(steps):
+                hstep()
+            e1.record(self.stream)
+            torch.cuda.synchronize(self.dev)
+        ems = max_over_ranks(e0.elapsed_time(e1), self.dev)
         h2d = sum(hp[k].numel() * hp[k].element_size() for k in names if hp[k] is not None)
         d2h = hout.numel() * hout.element_size() + hlast.numel() * hlast.element_size()
-        e2e = {"value": job_throughput(world, elems, e2e_steps, ems), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
-               "path": "ssm_selective_scan_fwd_host (pinned host buffers)"}
+        return {"value": job_throughput(world, d.batch * d.dim * d.seqlen, steps, ems), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+                "path": "ssm_selective_scan_fwd_host (pinned host buffers)"}
+
+    def close(self):
+        import torch
+        self.ssm.ssm_scan_destroy(self.plan)
+        self.sets = []
+        self.inp = None
+        torch.cuda.synchronize(self.dev)
+        torch.cuda.empty_cache()
+
+
+PER_CONFIG_MIN_MS = 40.0   # each per-config line times at least this long (more launches for small shapes)
+
+
+def _config_entry(job, launch_ms, total_ms, steps, clocks, probe_rate):
+    d = job.d
+    avg_s = statistics.mean(launch_ms) * 1e-3
+    roof = _roofline(d, job.info, avg_s, job.w.name, probe_rate)
+    elems = d.batch * d.dim * d.seqlen
+    return {"shape": {"batch": d.batch, "dim": d.dim, "seqlen": d.seqlen, "dstate": d.dstate, "nheads": d.H,
+                      "ngroups": d.ngroups, "io_dtype": d.dtype},
+            "kernel": job.info["variant"], "grid": job.info["grid"], "block": job.info["block"],
+            "schedule": job.sched, "steps": steps, "ms_per_call": total_ms / steps,
+            "gelem_s": elems * steps / (total_ms * 1e-3) / 1e9,
+            "roofline": {"bound": roof["bound"], "frac": roof["frac"], "unit": roof["unit"],
+                         "achieved": roof["achieved"], "peak": roof["peak"],
+                         "roofline_frac": roof["roofline_frac"], "hbm_frac": roof["hbm"]["frac"],
+                         "traffic": roof["traffic"], "alg_bytes_per_launch": roof["hbm"]["alg_bytes_per_launch"]},
+            "clocks": clocks}
+
+
+def run_ours(args):
+    import torch
+    import ssm_inputs as si
+    import selective_state_space_30_b200 as ssm
+
+    rank, local, world = _rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+    init_ranks("nccl", local)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = si.WORKLOADS[args.workload]
+    d = w.dims
+    stream = torch.cuda.current_stream(dev)
+    probe_rate = _probe_mufu(ssm, dev, stream.cuda_stream, stream)
+
+    # the headline: exactly K timed steps of the named workload
+    job = _ScanJob(ssm, w, dev, local)
+    launch_ms, total_ms, clocks = job.timed(args.steps, args.warmup, local)
+    elems = d.batch * d.dim * d.seqlen
+    ms_per_step = total_ms / args.steps
+    value = job_throughput(world, elems, args.steps, total_ms)
+    roof = _roofline(d, job.info, statistics.mean(launch_ms) * 1e-3, w.name, probe_rate)
+    per_config = {w.name: _config_entry(job, launch_ms, total_ms, args.steps, clocks, probe_rate)}
+    e2e = None if args.no_e2e else job.e2e(max(3, min(args.steps, 50)), world)
+    info, sched, copies, alg_bytes = job.info, job.sched, job.copies, job.alg_bytes
+    job.close()
+
+    # every other forward workload, one line each (the driver sees all five shapes)
+    if not args.no_per_config:
+        for name, wk in si.WORKLOADS.items():
+            if name == w.name:
+                continue
+            j = _ScanJob(ssm, wk, dev, local)
+            # a short probe sizes the run so that each line times at least PER_CONFIG_MIN_MS
+            pm, _, _ = j.timed(3, args.warmup, local)
+            n = max(args.steps, int(np.ceil(PER_CONFIG_MIN_MS / max(statistics.mean(pm), 1e-3))))
+            lm, tm, ck = j.timed(n, 2, local)
+            per_config[name] = _config_entry(j, lm, tm, n, ck, probe_rate)
+            j.close()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(d, w.recipe, w.seed)
 
-    ssm.ssm_scan_destroy(plan)
     finish_ranks()
     if rank != 0:
         return
+    n_launch = args.steps * info["launches_per_call"]
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32 (bf16 I/O)" if d.dtype == "bf16" else "f32",
@@ -481,7 +577,8 @@ def run_ours(args):
                        "kernel": info["variant"], "grid": info["grid"], "block": info["block"],
                        "schedule": sched},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "clocks": clk.summary(), "gpu_launches": args.steps * info["launches_per_call"]}
+            "clocks": clocks, "gpu_launches": n_launch,
+            "per_config": per_config}
     print(json.dumps(line), flush=True)
 
 
@@ -749,6 +846,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the named workload (default: also one line per other forward workload)")
     ap.add_argument("--op", default="scan", choices=["scan", "decode", "conv1d", "bwd"],
                     help="scan: the forward scan (the headline metric); decode: the single-step state update; "
                          "conv1d: the causal convolution in front of the scan; bwd: the backward scan")

@@ -159,6 +159,16 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
  *                              seqlen a multiple of 128: 0 = use it where it applies
  *                              (automatic), 1 = never (the scan kernel), 2 = required
  *                              (SSM_ERR_UNSUPPORTED for a shape it does not cover)
+ *   SSM_OPT_TIME_LANES         force the time sub-chunks per 32-step block: 1 = the
+ *                              state-parallel recurrence, 2 or 4 = sequence-parallel
+ *                              blocks (lanes split the block in time and join their
+ *                              sub-chunks by an associative scan; dstate <= 16);
+ *                              0 = automatic
+ *   SSM_OPT_TENSOR_MEMORY      the kernel that brings B and C to the lanes through
+ *                              tensor memory (bf16 I/O, dstate 16, A per channel): 0 =
+ *                              use it where it applies (automatic), 1 = never (the
+ *                              register kernel), 2 = required (SSM_ERR_UNSUPPORTED for a
+ *                              shape it does not cover)
  * Returns SSM_ERR_INVALID_ARG for an unknown option or a bad value.
  */
 typedef enum {
@@ -168,7 +178,9 @@ typedef enum {
     SSM_OPT_CONSUMER_WARPS = 4,
     SSM_OPT_WORKERS = 5,
     SSM_OPT_STATES_PER_LANE = 6,
-    SSM_OPT_SSD = 7
+    SSM_OPT_SSD = 7,
+    SSM_OPT_TIME_LANES = 8,
+    SSM_OPT_TENSOR_MEMORY = 9
 } ssm_option_t;
 int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value);
 
@@ -193,14 +205,39 @@ int ssm_scan_plan_schedule(ssm_plan_t plan, int* consumer_warps, int* seg_len, i
  *     SSM_ERR_UNSUPPORTED without launching anything.
  *   - The first call on a device looks up the array's address (once per device);
  *     make that first call before any stream capture.
- *   - All calls share the array: each clears its counters on its stream, and
- *     calls whose kernels overlap on the GPU race and must not be made.
- *   - Kernel-side conditions (a bounded wait that gave up) are not reported.
+ *   - Under CUDA's lazy module loading (the default) the array and the kernels
+ *     are placed in device memory at that first call, not when the library is
+ *     loaded: a caller that reserves all of its device memory for its own pool
+ *     should make one warm-up call first, or run with CUDA_MODULE_LOADING=EAGER.
+ *   - All calls share the array: each clears its counters, flags and status on
+ *     its stream, and calls whose kernels overlap on the GPU race and must not
+ *     be made.
+ *   - Kernel-side conditions (a bounded wait that gave up: SSM_ERR_TIMEOUT, with
+ *     out and last_state invalid) land in the array's status word; read them
+ *     with ssm_selective_scan_noalloc_device_status before the next call.
  * Calls no cudaMalloc, cudaFree or other allocating routine.
  */
 int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,
                                    const float* D, const void* z, const float* delta_bias, int softplus,
                                    const ssm_dims_t* dims, void* out, float* last_state, ssm_stream_t stream);
+
+/*
+ * The kernel-side status of the last ssm_selective_scan_fwd_noalloc call on the
+ * current device (no counterpart in the pages).  Waits for `stream`, returns the
+ * status word of the shared scratch array (SSM_OK, or SSM_ERR_TIMEOUT when a
+ * bounded wait gave up) and clears it.  Allocates nothing.  SSM_ERR_CUDA if the
+ * copy or the synchronisation fails.
+ */
+int ssm_selective_scan_noalloc_device_status(ssm_stream_t stream);
+
+/*
+ * Test hook of the allocation-free entry point (no counterpart in the pages).
+ * stall != 0 makes the chained waits of the following calls wait for a flag
+ * that nothing sets, so that they give up and report SSM_ERR_TIMEOUT;
+ * spin_limit (0 = default, else 1 .. 2^31-1; about 256 ns per unit) bounds
+ * every device-side wait of those calls.  Host-side settings of this process.
+ */
+int ssm_selective_scan_noalloc_test_hooks(int stall, int64_t spin_limit);
 
 /*
  * One step of the recurrence with the state kept in device memory: the

@@ -19,10 +19,12 @@ from . import _abi
 from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, SSM_ERR_TIMEOUT,  # noqa: F401
                    SSM_ERR_UNSUPPORTED, SSM_F32, SSM_OK, SSM_OPT_CONSUMER_WARPS, SSM_OPT_INJECT_STALL,
                    SSM_OPT_SEG_LEN, SSM_OPT_SPIN_LIMIT, SSM_OPT_SSD, SSM_OPT_STATES_PER_LANE, SSM_OPT_WORKERS,
+                   SSM_OPT_TIME_LANES, SSM_OPT_TENSOR_MEMORY,
                    SsmError, load_library, make_dims,
                    ssm_dims_t, ssm_probe_ex2, ssm_scan_destroy, ssm_scan_device_status, ssm_scan_plan,
                    ssm_scan_plan_info, ssm_scan_plan_schedule, ssm_scan_set_option, ssm_selective_scan_fwd,
                    ssm_selective_scan_fwd_h0, ssm_selective_scan_fwd_host, ssm_selective_scan_fwd_noalloc,
+                   ssm_selective_scan_noalloc_device_status, ssm_selective_scan_noalloc_test_hooks,
                    ssm_selective_state_update, ssm_causal_conv1d_fwd, ssm_selective_scan_bwd,
                    ssm_selective_scan_bwd_workspace_size, ssm_selective_scan_bwd_device_status,
                    ssm_selective_scan_bwd_test_hooks, ssm_grads_t,
@@ -31,7 +33,8 @@ from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, 
 
 __all__ = ["selective_scan_fwd", "selective_scan_fwd_host", "selective_scan_fn", "Plan", "get_plan", "ssm_scan_plan",
            "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0", "ssm_selective_scan_fwd_host",
-           "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update", "ssm_causal_conv1d_fwd",
+           "ssm_selective_scan_fwd_noalloc", "ssm_selective_scan_noalloc_device_status",
+           "ssm_selective_scan_noalloc_test_hooks", "ssm_selective_state_update", "ssm_causal_conv1d_fwd",
            "selective_scan_bwd", "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_workspace_size",
            "ssm_selective_scan_bwd_device_status", "ssm_selective_scan_bwd_test_hooks",
            "ssm_scan_destroy", "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info",

@@ -12,7 +12,8 @@ import os
 from typing import Any, Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libssmscan.so")
+# SSM_SCAN_LIBRARY names another build of the same library (the debug build, say)
+LIB_PATH = os.environ.get("SSM_SCAN_LIBRARY") or os.path.join(_HERE, "libssmscan.so")
 
 SSM_OK = 0
 SSM_ERR_INVALID_ARG = 1
@@ -25,7 +26,9 @@ SSM_BF16 = 1
 
 # every exported symbol declared in include/ssm_scan.h
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
-           "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc", "ssm_selective_state_update",
+           "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc",
+           "ssm_selective_scan_noalloc_device_status", "ssm_selective_scan_noalloc_test_hooks",
+           "ssm_selective_state_update",
            "ssm_causal_conv1d_fwd", "ssm_selective_scan_bwd_workspace_size", "ssm_selective_scan_bwd",
            "ssm_selective_scan_bwd_device_status", "ssm_selective_scan_bwd_test_hooks",
            "ssm_scan_set_option",
@@ -39,6 +42,8 @@ SSM_OPT_CONSUMER_WARPS = 4
 SSM_OPT_WORKERS = 5
 SSM_OPT_STATES_PER_LANE = 6
 SSM_OPT_SSD = 7
+SSM_OPT_TIME_LANES = 8
+SSM_OPT_TENSOR_MEMORY = 9
 
 
 class SsmError(RuntimeError):
@@ -82,6 +87,8 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_fwd_h0.argtypes = fwd_args + [vp, vp, vp, vp]
     lib.ssm_selective_scan_fwd_host.argtypes = fwd_args + [vp, vp, vp]
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, dims_p, vp, vp, vp]
+    lib.ssm_selective_scan_noalloc_device_status.argtypes = [vp]
+    lib.ssm_selective_scan_noalloc_test_hooks.argtypes = [i32, i64]
     lib.ssm_selective_state_update.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
     lib.ssm_causal_conv1d_fwd.argtypes = [i64, i64, i64, i32, i32, vp, vp, vp, i32, vp, vp]
     lib.ssm_selective_scan_bwd_workspace_size.argtypes = [dims_p, ctypes.POINTER(ctypes.c_size_t)]
@@ -181,6 +188,17 @@ def ssm_selective_scan_fwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
         1 if softplus else 0, ctypes.byref(dims), _ptr(out), _ptr(last_state), _stream(stream))
     return _check(rc, "ssm_selective_scan_fwd_noalloc") if check else rc
+
+
+def ssm_selective_scan_noalloc_device_status(stream=None) -> int:
+    """Kernel-side status of the last allocation-free call on the current device (syncs, clears it)."""
+    return int(load_library().ssm_selective_scan_noalloc_device_status(_stream(stream)))
+
+
+def ssm_selective_scan_noalloc_test_hooks(stall: bool, spin_limit: int = 0) -> int:
+    """Allocation-free entry point's test hooks (see include/ssm_scan.h)."""
+    return _check(load_library().ssm_selective_scan_noalloc_test_hooks(1 if stall else 0, int(spin_limit)),
+                  "ssm_selective_scan_noalloc_test_hooks")
 
 
 def ssm_selective_state_update(dims: ssm_dims_t, state, u, delta, A, B, C, D, z, delta_bias, softplus: bool,

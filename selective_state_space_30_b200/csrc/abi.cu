@@ -50,9 +50,10 @@ struct ssm_plan_s {
     unsigned n_units, n_ctas;
     int grid;
     const char* name;
+    ssm::FwdGeom geom;
     // options
     unsigned spin_limit;
-    int64_t force_seg_len, force_w, force_spl, force_ssd, force_workers;
+    int64_t force_seg_len, force_w, force_spl, force_ssd, force_workers, force_kt, force_tmem;
     // workspace: header | flags[n_tiles] | carry[n_tiles][CW][N]
     unsigned char* ws;
     size_t ws_bytes, flags_off, carry_off;
@@ -73,19 +74,10 @@ constexpr uint32_t kMagic = 0x53534d31u;  // "SSM1"
 constexpr uint32_t kDead = 0xdeadbeefu;
 constexpr unsigned kDefaultSpinLimit = 1u << 21;  // ~0.3-1 s of polling before a wait gives up
 
-bool dims_ok(const ssm_dims_t* d) {
-    if (!d) return false;
-    if (d->batch < 0 || d->dim <= 0 || d->seqlen < 0 || d->dstate <= 0) return false;
-    if (d->nheads <= 0 || d->ngroups <= 0) return false;
-    if (d->dim % d->nheads || d->dim % d->ngroups) return false;
-    if (d->io_dtype != SSM_F32 && d->io_dtype != SSM_BF16) return false;
-    if (d->reserved != 0) return false;
-    const int64_t lim = (int64_t)1 << 46;
-    const int64_t L = d->seqlen > 0 ? d->seqlen : 1;
-    if (d->batch > lim / d->dim || d->batch * d->dim > lim / L) return false;
-    if (d->batch * d->ngroups > lim / (d->dstate * L)) return false;
-    return true;
-}
+using ssm::aligned16;
+using ssm::dims_ok;
+using ssm::encode_rows;
+using ssm::head_mode;
 
 bool same_dims(const ssm_dims_t* a, const ssm_dims_t* b) {
     return a->batch == b->batch && a->dim == b->dim && a->seqlen == b->seqlen && a->dstate == b->dstate &&
@@ -93,7 +85,6 @@ bool same_dims(const ssm_dims_t* a, const ssm_dims_t* b) {
 }
 
 bool plan_ok(const ssm_plan_t p) { return p && p->magic == kMagic; }
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int set_device(int dev) {
     int cur = -1;
@@ -102,102 +93,45 @@ int set_device(int dev) {
     return SSM_OK;
 }
 
-bool head_mode(const ssm_dims_t& d) { return d.nheads != d.dim; }
-
-// Choose the consumer-warp count, segment length and grid; (re)allocate the workspace.
+// Choose the lane layout, segment length and grid; (re)allocate the workspace.
 int schedule(ssm_plan_s* p) {
     const ssm_dims_t& d = p->dims;
-    const int64_t Dg = d.dim / d.ngroups;
-    ssm::Layout lay;
-    if (!ssm::choose_layout(d, p->sm_count, (int)p->force_w, (int)p->force_spl, &lay)) return SSM_ERR_UNSUPPORTED;
-    const int w = lay.w;
-    const ssm::Variant& v = lay.v;
-    if (v.smem > 48 * 1024 &&
-        cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, v.fn, v.threads, v.smem) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    if (occ < 1) return SSM_ERR_UNSUPPORTED;
-    const int64_t n_tiles = ssm::layout_tiles(d, v.ch_per_tile);
-    int64_t ctas = p->sm_count;  // one persistent CTA per SM
-    if (p->force_workers > 0 && p->force_workers < ctas) ctas = p->force_workers;
-    const int64_t L = d.seqlen;
-    const int64_t seg_len = p->force_seg_len > 0 ? (p->force_seg_len + ssm::kTB - 1) / ssm::kTB * ssm::kTB
-                                                 : ssm::default_seg_len(L, n_tiles, ctas);
-    const int64_t n_seg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
-    const int64_t n_units = n_tiles * n_seg;
-    if (n_units >= (int64_t)1 << 31 || seg_len > (int64_t)1 << 30) return SSM_ERR_UNSUPPORTED;
-    if (ctas > n_units) ctas = n_units;
-    if (ctas < 1) ctas = 1;
+    ssm::FwdGeom g;
+    const int rc = ssm::fwd_geometry(d, p->sm_count, (int)p->force_w, (int)p->force_spl, (int)p->force_kt,
+                                     (int)p->force_tmem, p->force_seg_len, p->force_workers, &g);
+    if (rc != SSM_OK) return rc;
     const bool ssd_ok = ssm::ssd_eligible(d);
     if (p->force_ssd == 2 && !ssd_ok) return SSM_ERR_UNSUPPORTED;
     p->ssd = ssd_ok && p->force_ssd != 1;
-    p->w = w;
-    p->spl = lay.spl;
-    p->threads = v.threads;
-    p->ch_per_tile = v.ch_per_tile;
-    p->smem = v.smem;
-    p->tiles_per_group = (int)((Dg + v.ch_per_tile - 1) / v.ch_per_tile);
-    p->n_tiles = (int)n_tiles;
-    p->n_seg = (int)n_seg;
-    p->seg_len = (int)seg_len;
-    p->n_units = (unsigned)n_units;
-    p->n_ctas = (unsigned)ctas;
-    p->grid = (int)ctas;
-    p->name = v.name;
-    // workspace: header | flags[n_tiles] | carry[n_tiles][CT][N]
-    const size_t flags_off = 64;
-    const size_t carry_off = (flags_off + (size_t)n_tiles * 4 + 255) / 256 * 256;
-    const size_t bytes = carry_off + (size_t)n_tiles * v.ch_per_tile * d.dstate * 4;
-    if (p->ws && p->ws_bytes < bytes) {
+    p->geom = g;
+    p->w = g.lay.w;
+    p->spl = g.lay.spl;
+    p->threads = g.lay.v.threads;
+    p->ch_per_tile = g.lay.v.ch_per_tile;
+    p->smem = g.lay.v.smem;
+    p->tiles_per_group = (int)g.tiles_per_group;
+    p->n_tiles = (int)g.n_tiles;
+    p->n_seg = (int)g.n_seg;
+    p->seg_len = (int)g.seg_len;
+    p->n_units = (unsigned)g.n_units;
+    p->n_ctas = (unsigned)g.ctas;
+    p->grid = (int)g.ctas;
+    p->name = g.lay.v.name;
+    if (p->ws && p->ws_bytes < g.ws_bytes) {
         cudaFree(p->ws);
         p->ws = nullptr;
     }
     if (!p->ws) {
-        if (cudaMalloc(&p->ws, bytes) != cudaSuccess) {
+        if (cudaMalloc(&p->ws, g.ws_bytes) != cudaSuccess) {
             p->ws = nullptr;
             return SSM_ERR_CUDA;
         }
-        p->ws_bytes = bytes;
+        p->ws_bytes = g.ws_bytes;
     }
-    p->flags_off = flags_off;
-    p->carry_off = carry_off;
+    p->flags_off = g.flags_off;
+    p->carry_off = g.carry_off;
     if (cudaMemset(p->ws, 0, p->ws_bytes) != cudaSuccess) return SSM_ERR_CUDA;
     return SSM_OK;
-}
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda link).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn tensor_map_encoder() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-        tried = true;
-    }
-    return fn;
-}
-
-// A (rows x cols) row-major tensor seen as 2-D boxes of 32 steps x box_rows rows.
-bool encode_rows(CUtensorMap* m, const void* base, int esz, uint64_t cols, uint64_t rows, uint32_t box_rows,
-                 CUtensorMapSwizzle swz, uint32_t box_cols = ssm::kTB) {
-    EncodeTiledFn enc = tensor_map_encoder();
-    if (!enc || cols == 0 || rows == 0) return false;
-    const cuuint64_t gdim[2] = {cols, rows};
-    const cuuint64_t gstride[1] = {cols * (uint64_t)esz};
-    const cuuint32_t box[2] = {box_cols, box_rows};
-    const cuuint32_t es[2] = {1, 1};
-    return enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-               const_cast<void*>(base), gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A, const void* B, const void* C,
@@ -234,55 +168,9 @@ int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A
         }
         // an unaligned call takes the scan kernel below
     }
-    // Vector loads/stores need every per-lane chunk (up to 16 elements) wholly
-    // inside or outside a row and 16-byte aligned: L % 16 == 0 plus aligned bases.
-    bool vec = d.seqlen > 0 && (d.seqlen % 16 == 0) && aligned16(u) && aligned16(delta) && aligned16(B) &&
-               aligned16(C) && aligned16(out) && (!z || aligned16(z));
-    const int esz = d.io_dtype == SSM_BF16 ? 2 : 4;
-    const int64_t P = d.dim / d.nheads;
-    const int ct = plan->ch_per_tile;
-    int delta_rows = ct;
-    if (head_mode(d)) {
-        delta_rows = (int)((ct - 1) / P + 2);
-        if (delta_rows > ct) delta_rows = ct;
-    }
-    ssm::TensorMaps tm;
-    std::memset(&tm, 0, sizeof(tm));
-    if (vec) {
-        const CUtensorMapSwizzle bc_swz = esz == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-        const uint64_t L = (uint64_t)d.seqlen;
-        vec = encode_rows(&tm.u, u, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              encode_rows(&tm.delta, delta, esz, L, (uint64_t)(d.batch * d.nheads), delta_rows,
-                          CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              (!z || encode_rows(&tm.z, z, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE)) &&
-              encode_rows(&tm.B, B, esz, L, (uint64_t)(d.batch * d.ngroups * d.dstate), (uint32_t)d.dstate, bc_swz) &&
-              encode_rows(&tm.C, C, esz, L, (uint64_t)(d.batch * d.ngroups * d.dstate), (uint32_t)d.dstate, bc_swz);
-        // a shape the tensor maps cannot describe takes the element-copy path
-    }
-    ssm::Variant v;
-    if (!ssm::pick_variant(d.io_dtype, d.dstate, head_mode(d), vec, plan->w, plan->spl, &v))
-        return SSM_ERR_UNSUPPORTED;
-    ssm::FwdParams prm;
-    prm.u = u; prm.delta = delta; prm.A = A; prm.B = B; prm.C = C; prm.D = D; prm.z = z;
-    prm.bias = delta_bias; prm.h0 = h0; prm.out = out; prm.last_state = last_state;
-    prm.ws = reinterpret_cast<ssm::WsHeader*>(plan->ws);
-    prm.flags = reinterpret_cast<unsigned*>(plan->ws + plan->flags_off);
-    prm.carry = reinterpret_cast<float*>(plan->ws + plan->carry_off);
-    prm.dim = d.dim; prm.seqlen = d.seqlen; prm.nheads = d.nheads; prm.ngroups = d.ngroups;
-    prm.softplus = softplus ? 1 : 0;
-    prm.tiles_per_group = plan->tiles_per_group;
-    prm.n_tiles = plan->n_tiles;
-    prm.n_seg = plan->n_seg;
-    prm.seg_len = plan->seg_len;
-    prm.n_units = plan->n_units;
-    prm.n_ctas = plan->n_ctas;
-    prm.spin_limit = plan->spin_limit;
-    prm.delta_rows = delta_rows;
-    if (v.smem > 48 * 1024 &&
-        cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
-        return SSM_ERR_CUDA;
-    v.fn<<<plan->grid, v.threads, v.smem, stream>>>(prm, tm);
-    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    // the scan kernel (also an SSD-eligible call whose pointers the SSD path cannot take)
+    const ssm::FwdArgs a{u, delta, A, B, C, D, z, delta_bias, softplus, h0, out, last_state};
+    return ssm::fwd_launch(d, plan->geom, a, plan->ws, plan->spin_limit, stream);
 }
 }  // namespace
 
@@ -326,7 +214,7 @@ int ssm_scan_plan(ssm_plan_t* out_plan, const ssm_dims_t* dims, int device) {
     *out_plan = nullptr;
     if (!dims_ok(dims)) return SSM_ERR_INVALID_ARG;
     ssm::Layout probe;
-    if (!ssm::choose_layout(*dims, 1, 0, 0, &probe)) return SSM_ERR_UNSUPPORTED;
+    if (!ssm::choose_layout(*dims, 1, 0, 0, 0, 0, &probe)) return SSM_ERR_UNSUPPORTED;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return SSM_ERR_CUDA;
     if (set_device(device) != SSM_OK) return SSM_ERR_CUDA;
@@ -370,7 +258,9 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
         case SSM_OPT_CONSUMER_WARPS:
         case SSM_OPT_WORKERS:
         case SSM_OPT_STATES_PER_LANE:
-        case SSM_OPT_SSD: {
+        case SSM_OPT_SSD:
+        case SSM_OPT_TIME_LANES:
+        case SSM_OPT_TENSOR_MEMORY: {
             if (value < 0) return SSM_ERR_INVALID_ARG;
             if (option == SSM_OPT_CONSUMER_WARPS && value != 0 && value != 4 && value != 8 && value != 12 &&
                 value != 16)
@@ -379,6 +269,9 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
                 value != 16)
                 return SSM_ERR_INVALID_ARG;
             if (option == SSM_OPT_SSD && value > 2) return SSM_ERR_INVALID_ARG;
+            if (option == SSM_OPT_TIME_LANES && value != 0 && value != 1 && value != 2 && value != 4)
+                return SSM_ERR_INVALID_ARG;
+            if (option == SSM_OPT_TENSOR_MEMORY && value > 2) return SSM_ERR_INVALID_ARG;
             if (cudaDeviceSynchronize() != cudaSuccess) return SSM_ERR_CUDA;
             release_pipeline(plan);   // its chunk plan follows the new options when next built
             unsigned inject = 0;
@@ -389,6 +282,8 @@ int ssm_scan_set_option(ssm_plan_t plan, int option, int64_t value) {
                              : option == SSM_OPT_CONSUMER_WARPS ? &plan->force_w
                              : option == SSM_OPT_STATES_PER_LANE ? &plan->force_spl
                              : option == SSM_OPT_SSD            ? &plan->force_ssd
+                             : option == SSM_OPT_TIME_LANES     ? &plan->force_kt
+                             : option == SSM_OPT_TENSOR_MEMORY  ? &plan->force_tmem
                                                                  : &plan->force_workers;
             const int64_t old = *field;
             *field = value;

@@ -18,17 +18,24 @@
 //  * The first call on a device looks up the array's device address with
 //    cudaGetSymbolAddress (once per device, with that device current); make that
 //    first call before any stream capture.
+//  * Under CUDA's lazy module loading (the default) the array, like the kernels,
+//    is placed in device memory at that first call on each device, not when the
+//    library is loaded.  A caller that reserves all of its device memory for its
+//    own pool should make one warm-up call before reserving it, or run with
+//    CUDA_MODULE_LOADING=EAGER.
 //  * Every call shares the one array.  Each call clears the part that must start
-//    at zero (counters and flags) on its stream before its launch; calls whose
-//    kernels overlap on the GPU (two streams at once) race on the array and
-//    must not be made.
+//    at zero (counters, flags, status) on its stream before its launch; calls
+//    whose kernels overlap on the GPU (two streams at once) race on the array
+//    and must not be made.
 //  * Kernel-side conditions (a bounded wait that gave up) are recorded in the
-//    array and cleared by the next call; this entry point does not report them.
+//    array's status word.  ssm_selective_scan_noalloc_device_status reads and
+//    clears it; read it after a call and before the next one, which clears it.
 //  * Nothing here calls cudaMalloc, cudaFree or any other allocating routine.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 
@@ -76,53 +83,11 @@ int device_setup(int dev, void** addr, int* sms) {
     return SSM_OK;
 }
 
-bool dims_valid(const ssm_dims_t* d) {
-    if (!d) return false;
-    if (d->batch < 0 || d->dim <= 0 || d->seqlen < 0 || d->dstate <= 0) return false;
-    if (d->nheads <= 0 || d->ngroups <= 0) return false;
-    if (d->dim % d->nheads || d->dim % d->ngroups) return false;
-    if (d->io_dtype != SSM_F32 && d->io_dtype != SSM_BF16) return false;
-    if (d->reserved != 0) return false;
-    const int64_t lim = (int64_t)1 << 46;
-    const int64_t L = d->seqlen > 0 ? d->seqlen : 1;
-    if (d->batch > lim / d->dim || d->batch * d->dim > lim / L) return false;
-    if (d->batch * d->ngroups > lim / (d->dstate * L)) return false;
-    return true;
-}
-
-typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encoder() {
-    static std::atomic<EncodeFn> fn{nullptr};
-    EncodeFn f = fn.load(std::memory_order_acquire);
-    if (!f) {
-        void* sym = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &sym, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess) {
-            f = reinterpret_cast<EncodeFn>(sym);
-            fn.store(f, std::memory_order_release);
-        }
-    }
-    return f;
-}
-
-bool encode(CUtensorMap* m, const void* base, int esz, uint64_t cols, uint64_t rows, uint32_t box_rows,
-            CUtensorMapSwizzle swz) {
-    EncodeFn enc = encoder();
-    if (!enc || cols == 0 || rows == 0) return false;
-    const cuuint64_t gdim[2] = {cols, rows};
-    const cuuint64_t gstride[1] = {cols * (uint64_t)esz};
-    const cuuint32_t box[2] = {(cuuint32_t)ssm::kTB, box_rows};
-    const cuuint32_t es[2] = {1, 1};
-    return enc(m, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-               const_cast<void*>(base), gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Test hooks: make the chained waits of the next calls wait for a flag nobody sets,
+// and bound every wait by a spin limit (0 = the default).
+std::atomic<unsigned> g_hook_stall{0};
+std::atomic<unsigned> g_hook_spin{0};
+constexpr unsigned kDefaultSpin = 1u << 21;  // ~0.5 s of polling before a wait gives up
 
 }  // namespace
 
@@ -130,86 +95,59 @@ extern "C" int ssm_selective_scan_fwd_noalloc(const void* u, const void* delta, 
                                               const void* C, const float* D, const void* z,
                                               const float* delta_bias, int softplus, const ssm_dims_t* dims,
                                               void* out, float* last_state, ssm_stream_t stream) {
-    if (!dims_valid(dims)) return SSM_ERR_INVALID_ARG;
+    if (!ssm::dims_ok(dims)) return SSM_ERR_INVALID_ARG;
     const ssm_dims_t& d = *dims;
     if (d.batch > 0 && d.seqlen > 0 && (!u || !delta || !B || !C || !out)) return SSM_ERR_INVALID_ARG;
     if (!A) return SSM_ERR_INVALID_ARG;
-    const bool head = d.nheads != d.dim;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
+    void* scratch = nullptr;
+    int sms = 0;
+    int rc = device_setup(dev, &scratch, &sms);
+    if (rc != SSM_OK) return rc;
+    if (d.batch == 0) return SSM_OK;
+
+    // the schedule of a plan with default options (the same code as the plan path)
+    ssm::FwdGeom g;
+    rc = ssm::fwd_geometry(d, sms, 0, 0, 0, 0, 0, 0, &g);
+    if (rc != SSM_OK) return rc;
+    // the workspace must fit the static scratch
+    if (g.ws_bytes > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned char* ws = static_cast<unsigned char*>(scratch);
+    // counters, status and flags start at zero on every call (the carry region needs no clearing)
+    if (cudaMemsetAsync(ws, 0, g.carry_off, s) != cudaSuccess) return SSM_ERR_CUDA;
+    if (g_hook_stall.load() &&
+        cudaMemsetAsync(ws + offsetof(ssm::WsHeader, inject), 1, 1, s) != cudaSuccess)
+        return SSM_ERR_CUDA;
+    const unsigned spin = g_hook_spin.load() ? g_hook_spin.load() : kDefaultSpin;
+    const ssm::FwdArgs a{u, delta, A, B, C, D, z, delta_bias, softplus, nullptr, out, last_state};
+    return ssm::fwd_launch(d, g, a, ws, spin, s);
+}
+
+extern "C" int ssm_selective_scan_noalloc_device_status(ssm_stream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SSM_ERR_CUDA;
     void* scratch = nullptr;
     int sms = 0;
     const int rc = device_setup(dev, &scratch, &sms);
     if (rc != SSM_OK) return rc;
-    if (d.batch == 0) return SSM_OK;
-
-    // the schedule: the same policy as a plan (the default lane layout, one persistent CTA
-    // per SM, the default segment length)
-    const int64_t Dg = d.dim / d.ngroups;
-    ssm::Layout lay;
-    if (!ssm::choose_layout(d, sms, 0, 0, &lay)) return SSM_ERR_UNSUPPORTED;
-    const int w = lay.w;
-    const int ct = lay.v.ch_per_tile;
-    const int64_t n_tiles = ssm::layout_tiles(d, ct);
-    int64_t ctas = sms;
-    const int64_t L = d.seqlen;
-    const int64_t seg_len = ssm::default_seg_len(L, n_tiles, ctas);
-    const int64_t n_seg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
-    const int64_t n_units = n_tiles * n_seg;
-    if (n_units >= (int64_t)1 << 31) return SSM_ERR_UNSUPPORTED;
-    if (ctas > n_units) ctas = n_units;
-
-    // the workspace must fit the static scratch
-    const size_t flags_off = 64;
-    const size_t carry_off = (flags_off + (size_t)n_tiles * 4 + 255) / 256 * 256;
-    const size_t need = carry_off + (size_t)n_tiles * ct * d.dstate * 4;
-    if (need > kNoAllocScratchBytes) return SSM_ERR_UNSUPPORTED;
-
-    // vector path (tensor maps) when rows are 16-byte aligned; else guarded element copies
-    const int esz = d.io_dtype == SSM_BF16 ? 2 : 4;
-    const int64_t P = d.dim / d.nheads;
-    int delta_rows = ct;
-    if (head) {
-        delta_rows = (int)((ct - 1) / P + 2);
-        if (delta_rows > ct) delta_rows = ct;
-    }
-    bool vec = L > 0 && L % 16 == 0 && a16(u) && a16(delta) && a16(B) && a16(C) && a16(out) && (!z || a16(z));
-    ssm::TensorMaps tm;
-    std::memset(&tm, 0, sizeof(tm));
-    if (vec) {
-        const CUtensorMapSwizzle bc = esz == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-        vec = encode(&tm.u, u, esz, L, d.batch * d.dim, ct, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              encode(&tm.delta, delta, esz, L, d.batch * d.nheads, delta_rows, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-              (!z || encode(&tm.z, z, esz, L, d.batch * d.dim, ct, CU_TENSOR_MAP_SWIZZLE_NONE)) &&
-              encode(&tm.B, B, esz, L, d.batch * d.ngroups * d.dstate, (uint32_t)d.dstate, bc) &&
-              encode(&tm.C, C, esz, L, d.batch * d.ngroups * d.dstate, (uint32_t)d.dstate, bc);
-    }
-    ssm::Variant v;
-    if (!ssm::pick_variant(d.io_dtype, d.dstate, head, vec, w, lay.spl, &v)) return SSM_ERR_UNSUPPORTED;
-
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    unsigned char* ws = static_cast<unsigned char*>(scratch);
-    // counters, status and flags start at zero on every call (the carry region needs no clearing)
-    if (cudaMemsetAsync(ws, 0, carry_off, s) != cudaSuccess) return SSM_ERR_CUDA;
-    ssm::FwdParams prm;
-    prm.u = u; prm.delta = delta; prm.A = A; prm.B = B; prm.C = C; prm.D = D; prm.z = z;
-    prm.bias = delta_bias; prm.h0 = nullptr; prm.out = out; prm.last_state = last_state;
-    prm.ws = reinterpret_cast<ssm::WsHeader*>(ws);
-    prm.flags = reinterpret_cast<unsigned*>(ws + flags_off);
-    prm.carry = reinterpret_cast<float*>(ws + carry_off);
-    prm.dim = d.dim; prm.seqlen = d.seqlen; prm.nheads = d.nheads; prm.ngroups = d.ngroups;
-    prm.softplus = softplus ? 1 : 0;
-    prm.tiles_per_group = (int)((Dg + ct - 1) / ct);
-    prm.n_tiles = (int)n_tiles;
-    prm.n_seg = (int)n_seg;
-    prm.seg_len = (int)seg_len;
-    prm.n_units = (unsigned)n_units;
-    prm.n_ctas = (unsigned)ctas;
-    prm.spin_limit = 1u << 21;
-    prm.delta_rows = delta_rows;
-    if (v.smem > 48 * 1024 &&
-        cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
+    int* status = reinterpret_cast<int*>(static_cast<unsigned char*>(scratch) + offsetof(ssm::WsHeader, status));
+    int st = SSM_OK;
+    if (cudaMemcpyAsync(&st, status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
         return SSM_ERR_CUDA;
-    v.fn<<<(unsigned)ctas, v.threads, v.smem, s>>>(prm, tm);
-    return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+    if (st != SSM_OK && (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess ||
+                         cudaStreamSynchronize(s) != cudaSuccess))
+        return SSM_ERR_CUDA;
+    return st;
+}
+
+extern "C" int ssm_selective_scan_noalloc_test_hooks(int stall, int64_t spin_limit) {
+    if (spin_limit < 0 || spin_limit > 0x7fffffff) return SSM_ERR_INVALID_ARG;
+    g_hook_stall.store(stall ? 1u : 0u);
+    g_hook_spin.store((unsigned)spin_limit);
+    return SSM_OK;
 }

@@ -87,7 +87,7 @@ def to_host_f64(t) -> np.ndarray:
 
 
 OPTION_CODES = {"spin_limit": 1, "inject_stall": 2, "seg_len": 3, "warps": 4, "ctas": 5, "states_per_lane": 6,
-                "ssd": 7}
+                "ssd": 7, "time_lanes": 8, "tensor_memory": 9}
 
 
 def run_gpu(dims: si.Dims, inp: dict, h0=None, with_state=True, device="cuda", stream=None, opts=None,

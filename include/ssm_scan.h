@@ -317,11 +317,13 @@ int ssm_causal_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t wi
  *     dh0           (batch, dim, dstate) fp32, nullable: not computed
  * The call allocates nothing: `workspace` (device, 256-byte aligned, at least
  * ssm_selective_scan_bwd_workspace_size bytes, which depends on the shape and on
- * the current device's SM count; about batch*dim*seqlen*8 bytes of state
- * checkpoints plus per-tile dB/dC rows) is the caller's and is scratch after the
- * call; one workspace must not serve two calls at once.  Two kernels on `stream`
- * (after two small memsets of the workspace's counters); the sums run in a fixed
- * order, so repeated calls give identical bits.  The first kernel runs work units
+ * the current device's SM count; about batch*dim*seqlen*2 bytes of state
+ * checkpoints, one per 32 steps) is the caller's and is scratch after the call;
+ * one workspace must not serve two calls at once.  Two kernels on `stream`
+ * (after memsets of the workspace's counters and of dB and dC).  dB and dC, sums
+ * over the channels of a group, are added up by atomic adds, so their last bits
+ * may differ between calls; every other gradient is summed in a fixed order and
+ * repeats bit for bit.  The first kernel runs work units
  * (32 channels x a segment of the sequence) on persistent CTAs whose bounded waits
  * record SSM_ERR_TIMEOUT in the workspace; read it with
  * ssm_selective_scan_bwd_device_status.  A, h0, dlast and dh0 must be 8-byte

@@ -23,11 +23,12 @@
 // segments, and the work units (tile, segment) go to persistent CTAs from a
 // ticket counter: first every forward unit, segment-major, then every reverse
 // unit, last segment first.  A forward unit runs the recurrence from the state
-// its predecessor handed over and stores the state at the start of every 8-step
-// window (the checkpoints).  A reverse unit takes the state gradient from the
-// segment after it, walks its 32-step blocks backwards, and per window
-// recomputes the 8 states and decays from the checkpoint into registers, then
-// runs the window in reverse.  A unit waits (bounded) only on units with smaller
+// its predecessor handed over and stores the state at the start of every 32-step
+// block (the checkpoints).  A reverse unit takes the state gradient from the
+// segment after it and walks its blocks backwards: per block it runs the
+// recurrence forward from the block's checkpoint to get the states at the four
+// 8-step window starts (registers), then per window recomputes the 8 states and
+// decays into registers and runs the window in reverse.  A unit waits (bounded) only on units with smaller
 // tickets, which running CTAs hold, so the chain always progresses.  Each block's
 // 32-step rows of the inputs are staged in shared memory by cp.async, double
 // buffered: a block's prologue issues the next block's rows.
@@ -35,9 +36,11 @@
 // Sums over the states (y, sum g B, the decay term) are transposed shuffle
 // reductions inside the 8 lanes of a channel.  dB and dC, sums over channels, are
 // summed over a warp's four channels by shuffles at every step, then over the
-// eight warps through shared memory once per 32-step block, into per-tile partial
-// rows, which a second kernel adds in a fixed order with the per-row dA, dD and
-// dbias partials: the result does not depend on scheduling.
+// eight warps through shared memory once per 32-step block, and the tile's sums
+// are added into dB and dC by vector atomic adds (red.global.add.v4.f32) that
+// resolve in L2: no per-tile rows reach HBM, and the order of the adds between
+// tiles, so the last bits of dB and dC, may differ between calls.  A second
+// kernel adds the per-row dA, dD and dbias partials in a fixed order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -67,7 +70,9 @@ struct BwdParams {
     int* status;                 // kernel-side ssm_status_t
     unsigned *flag1, *flag2;     // [tile][seg]: forward / reverse segment done (zeroed before the launch)
     float *carry1, *carry2;      // [tile][seg][kCT][kN]: state after / state gradient before a segment
-    float *ckpt, *dBp, *dCp;     // checkpoints [tile][window][kCT][kN]; dB, dC rows [tile][kN][L]
+    float* ckpt;                 // checkpoints [tile][block][kCT][kN]
+    float *dB, *dC;              // the outputs (batch, groups, kN, L), zeroed before the launch
+    int red_vec;                 // 16-byte atomic adds into dB, dC (L % 4 == 0, aligned bases)
     float *dAp, *dDp, *dbp;      // per segment and (b, d) row: [seg][row][kN], [seg][row], [seg][row]
     int64_t batch, dim, seqlen, ngroups;
     int64_t ntiles;              // batch * dim / kCT
@@ -104,7 +109,9 @@ struct Smem {
     // per window and warp, the dB, dC terms summed over the warp's channels:
     // float [kBT/kWin windows][8 warps][4 components][8 lanes j][kWin steps]
     static constexpr int RED = BC + kBT * 8 * 16;
-    static constexpr int TOTAL = RED + (kBT / kWin) * 8 * 4 * 8 * kWin * 4;
+    // per thread, the states entering the four windows of the block being walked backwards
+    static constexpr int WST = RED + (kBT / kWin) * 8 * 4 * 8 * kWin * 4;
+    static constexpr int TOTAL = WST + (kBT / kWin) * kThreads * 8;
 };
 
 // rows x kBT steps [t0, t0 + kBT) of `rows` rows (row r at src + r * stride) into
@@ -177,21 +184,34 @@ __device__ __forceinline__ float reduce8(const float (&v)[8], int j) {
     return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
+__device__ __forceinline__ void red_add_v4(float* dst, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 // The dB, dC terms of one 32-step block, held per (window, warp) in shared memory,
-// summed over the eight warps in a fixed order into the tile's rows: thread tid
-// takes four (window, component, lane j, step) entries.
-__device__ __forceinline__ void red_sum(const float* red, float* dBrow, float* dCrow, int64_t t0, int64_t L,
+// summed over the eight warps in a fixed order and added into dB and dC (rows of the
+// tile's group, dBg / dCg) by atomic adds: thread tid takes four consecutive steps of one
+// (window, component, lane j).
+__device__ __forceinline__ void red_add(const float* red, float* dBg, float* dCg, int64_t t0, int64_t L, bool vec,
                                        int tid) {
+    const int w = tid >> 6, comp = (tid >> 4) & 3, jj = (tid >> 1) & 7, q4 = (tid & 1) * 4;
+    const int within = comp * 64 + jj * 8 + q4;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int idx = tid + r * kThreads;           // 0 .. 1023
-        const int w = idx >> 8, within = idx & 255;   // window; (component, j, step)
-        float s = 0.f;
+    for (int wp = 0; wp < 8; ++wp) {
+        const float4 v = *reinterpret_cast<const float4*>(red + (w * 8 + wp) * 256 + within);
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    const int64_t ta = t0 + w * kWin + q4;
+    float* dst = ((comp & 2) ? dCg : dBg) + (int64_t)(2 * jj + (comp & 1)) * L + ta;
+    if (vec && ta + 3 < L) {
+        red_add_v4(dst, s);
+    } else {
+        const float e[4] = {s.x, s.y, s.z, s.w};
 #pragma unroll
-        for (int wp = 0; wp < 8; ++wp) s += red[(w * 8 + wp) * 256 + within];
-        const int comp = within >> 6, jj = (within >> 3) & 7, t = within & 7;
-        const int64_t ta = t0 + w * kWin + t;
-        if (ta < L) ((comp & 2) ? dCrow : dBrow)[(int64_t)(2 * jj + (comp & 1)) * L + ta] = s;
+        for (int i = 0; i < 4; ++i)
+            if (ta + i < L) atomicAdd(dst + i, e[i]);
     }
 }
 
@@ -216,7 +236,6 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                        reinterpret_cast<uintptr_t>(p.z) | reinterpret_cast<uintptr_t>(p.dout) |
                        reinterpret_cast<uintptr_t>(p.B) | reinterpret_cast<uintptr_t>(p.C)) & 15u) == 0;
     const int nblk = (int)((L + kBT - 1) / kBT);
-    const int nwin = nblk * (kBT / kWin);
     const int64_t per_pass = p.ntiles * p.nseg;
 
     for (;;) {
@@ -240,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         const T* go = static_cast<const T*>(p.dout) + row0 * L;
         const T* Bg = static_cast<const T*>(p.B) + (b * G + g) * kN * L;
         const T* Cg = static_cast<const T*>(p.C) + (b * G + g) * kN * L;
-        float* ckpt = p.ckpt + tile * (int64_t)nwin * kCT * kN;
+        float* ckpt = p.ckpt + tile * (int64_t)nblk * kCT * kN;
         const int blk0 = seg * p.seg_blocks;
         const int blk1 = min(nblk, blk0 + p.seg_blocks);
         const int64_t us = tile * p.nseg + seg;    // this unit's flag / carry slot
@@ -277,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         __syncthreads();
 
         if (fwd) {
-            // ---------------- forward unit: the recurrence, checkpoints at every window start
+            // ---------------- forward unit: the recurrence, checkpoints at every block start
             float2 h;
             if (seg == 0)
                 h = p.h0 ? *reinterpret_cast<const float2*>(p.h0 + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
@@ -315,9 +334,9 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 // the next block's rows go into the other buffer, read last by the previous block
                 if (blk + 1 < blk1) issue_fwd(stage_base + (cur ^ 1) * S::kStageBytes, t0 + kBT);
                 __syncthreads();
+                *reinterpret_cast<float2*>(ckpt + ((int64_t)blk * kCT + c) * kN + 2 * j) = h;
 #pragma unroll
                 for (int w = 0; w < kBT / kWin; ++w) {
-                    *reinterpret_cast<float2*>(ckpt + ((int64_t)(blk * (kBT / kWin) + w) * kCT + c) * kN + 2 * j) = h;
 #pragma unroll 4
                     for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
                         const float4 pv = sP[c * kPS + t];
@@ -337,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             continue;
         }
 
-        // ---------------- reverse unit: blocks backwards, windows recomputed from their checkpoints
+        // ---------------- reverse unit: blocks backwards, windows recomputed from the block checkpoints
         float2 gs;
         if (seg + 1 < p.nseg)
             gs = __ldcg(reinterpret_cast<const float2*>(p.carry2 + ((us + 1) * kCT + c) * kN + 2 * j));
@@ -345,11 +364,11 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             gs = p.dlast ? *reinterpret_cast<const float2*>(p.dlast + (row0 + c) * kN + 2 * j) : make_float2(0.f, 0.f);
         float2 dAacc = make_float2(0.f, 0.f);
         float dbias = 0.f, dDacc = 0.f;
-        float* dBrow = p.dBp + tile * kN * L;
-        float* dCrow = p.dCp + tile * kN * L;
-        const int fw0 = blk0 * (kBT / kWin);             // first window of the segment
-        int fw = blk1 * (kBT / kWin) - 1;                // flat index of the current window, walking down
-        float2 hnext = __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)fw * kCT + c) * kN + 2 * j));
+        float* dBg = p.dB + (b * G + g) * kN * L;
+        float* dCg = p.dC + (b * G + g) * kN * L;
+        const bool rvec = p.red_vec != 0;
+        // the checkpoint of the block being walked (the next, earlier one is fetched a block ahead)
+        float2 hblk = __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)(blk1 - 1) * kCT + c) * kN + 2 * j));
         auto issue_rev = [&](unsigned char* sg, int64_t ts) {
             stage_rows<T>(sg, u, L, kCT, ts, L, vec, tid);
             stage_rows<T>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
@@ -366,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             cp_async_wait();
             __syncthreads();   // this block's rows are in; the previous block is done with P, U, BC
             // the previous block's dB, dC terms (every warp has written them)
-            if (blk + 1 < blk1) red_sum(sR, dBrow, dCrow, t0 + kBT, L, tid);
+            if (blk + 1 < blk1) red_add(sR, dBg, dCg, t0 + kBT, L, rvec, tid);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int cc = warp * 4 + i;
@@ -399,11 +418,32 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             if (blk > blk0) issue_rev(stage_base + (cur ^ 1) * S::kStageBytes, t0 - kBT);
             __syncthreads();
 
-            for (int w = kBT / kWin - 1; w >= 0; --w, --fw) {
+            const float2 hprev =
+                blk > blk0 ? __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)(blk - 1) * kCT + c) * kN + 2 * j))
+                           : make_float2(0.f, 0.f);
+            // the states entering the four windows, by the recurrence from the block checkpoint
+            // (kept in shared memory, one float2 per thread and window)
+            float2* wst = reinterpret_cast<float2*>(smem + S::WST) + tid;
+            {
+                float2 hh = hblk;
+#pragma unroll
+                for (int w = 0; w < kBT / kWin; ++w) {
+                    wst[w * kThreads] = hh;
+                    if (w + 1 < kBT / kWin) {
+#pragma unroll 4
+                        for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
+                            const float4 pv = sP[c * kPS + t];
+                            const float4 bc = sBC[t * 8 + j];
+                            float2 dA;
+                            fwd_step(hh, dA, pv.x, pv.y, bc.x, bc.y, al);
+                        }
+                    }
+                }
+            }
+            hblk = hprev;
+            for (int w = kBT / kWin - 1; w >= 0; --w) {
                 const int tw = w * kWin;   // first step of the window within the block
-                const float2 he = hnext;   // the state entering the window
-                if (fw > fw0)
-                    hnext = __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)(fw - 1) * kCT + c) * kN + 2 * j));
+                const float2 he = wst[w * kThreads];   // the state entering the window
                 float2 hr[kWin], dAr[kWin];
                 float yw;   // y of step j of the window, summed over the states
                 {
@@ -475,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
 
         // the last block's dB, dC terms
         __syncthreads();
-        red_sum(sR, dBrow, dCrow, (int64_t)blk0 * kBT, L, tid);
+        red_add(sR, dBg, dCg, (int64_t)blk0 * kBT, L, rvec, tid);
         // hand the state gradient to the segment before; this segment's parameter partials
         *reinterpret_cast<float2*>(p.carry2 + (us * kCT + c) * kN + 2 * j) = gs;
         if (seg == 0 && p.dh0) *reinterpret_cast<float2*>(p.dh0 + (row0 + c) * kN + 2 * j) = gs;
@@ -497,39 +537,11 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
     }
 }
 
-// dB, dC: sum of the per-tile rows of the group; dA, dD, dbias: sum over batch rows and
-// segments, in a fixed order.
-// vec4: four consecutive steps per thread with 16-byte loads and stores (L a multiple
-// of 4, dB and dC 16-byte aligned); every element sums its tiles in the same order.
-__global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, float* dA, float* dB, float* dC,
-                                                         float* dD, float* dbias, int vec4) {
-    const int64_t Dm = p.dim, L = p.seqlen, G = p.ngroups;
-    const int64_t nbc = p.batch * G * kN * L;
-    const int64_t vw = vec4 ? 4 : 1;
-    const int64_t tpg = (Dm / G) / kCT;   // tiles per group
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < 2 * nbc / vw) {
-        const bool isC = i >= nbc / vw;
-        const int64_t k = (isC ? i - nbc / vw : i) * vw;
-        const int64_t t = k % L, n = (k / L) % kN, bg = k / (L * kN);
-        const int64_t b = bg / G, g = bg % G;
-        const float* src = (isC ? p.dCp : p.dBp) + ((b * p.tiles_per_row + g * tpg) * kN + n) * L + t;
-        float* dst = (isC ? dC : dB) + k;
-        if (vec4) {
-            float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int64_t m = 0; m < tpg; ++m) {
-                const float4 v = __ldcs(reinterpret_cast<const float4*>(src + m * kN * L));
-                s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-            }
-            *reinterpret_cast<float4*>(dst) = s;
-        } else {
-            float s = 0.f;
-            for (int64_t m = 0; m < tpg; ++m) s += src[m * kN * L];
-            *dst = s;
-        }
-        return;
-    }
-    const int64_t k = i - 2 * nbc / vw;
+// dA, dD, dbias: sums over batch rows and segments of the per-row partials, in a fixed
+// order (dB and dC were added by the first kernel).
+__global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, float* dA, float* dD, float* dbias) {
+    const int64_t Dm = p.dim;
+    const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t rows = p.batch * Dm;
     if (k < Dm * kN) {
         float s = 0.f;
@@ -577,7 +589,7 @@ Sched make_sched(const ssm_dims_t& d, int sms, int per_sm) {
 
 struct WsLayout {
     int64_t ticket, flag1, flag2, zero_end;        // zeroed before every launch
-    int64_t carry1, carry2, ckpt, dBp, dCp, dAp, dDp, dbp, total;   // byte offsets
+    int64_t carry1, carry2, ckpt, dAp, dDp, dbp, total;   // byte offsets
 };
 
 __host__ int64_t align256(int64_t v) { return (v + 255) & ~(int64_t)255; }
@@ -585,7 +597,7 @@ __host__ int64_t align256(int64_t v) { return (v + 255) & ~(int64_t)255; }
 WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
     const int64_t rows = d.batch * d.dim;
     const int64_t ntiles = rows / kCT;
-    const int64_t nwin = ((d.seqlen + kBT - 1) / kBT) * (kBT / kWin);
+    const int64_t nblk = (d.seqlen + kBT - 1) / kBT;
     const int64_t slots = ntiles * s.nseg;
     WsLayout w;
     w.ticket = 0;                                  // ticket (u32), status (i32)
@@ -595,9 +607,7 @@ WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
     w.carry1 = w.zero_end;
     w.carry2 = align256(w.carry1 + slots * kCT * kN * 4);
     w.ckpt = align256(w.carry2 + slots * kCT * kN * 4);
-    w.dBp = align256(w.ckpt + ntiles * nwin * kCT * kN * 4);
-    w.dCp = align256(w.dBp + ntiles * kN * d.seqlen * 4);
-    w.dAp = align256(w.dCp + ntiles * kN * d.seqlen * 4);
+    w.dAp = align256(w.ckpt + ntiles * nblk * kCT * kN * 4);
     w.dDp = align256(w.dAp + (int64_t)s.nseg * rows * kN * 4);
     w.dbp = align256(w.dDp + (int64_t)s.nseg * rows * 4);
     w.total = align256(w.dbp + (int64_t)s.nseg * rows * 4);
@@ -657,15 +667,14 @@ int check_dims(const ssm_dims_t* d) {
 }
 
 template <typename T>
-int launch(const BwdParams& prm, float* dA, float* dB, float* dC, float* dD, float* dbias, int ctas, cudaStream_t s) {
+int launch(const BwdParams& prm, float* dA, float* dD, float* dbias, int ctas, cudaStream_t s) {
     constexpr int smem = Smem<T>::TOTAL;
     scan_bwd_kernel<T><<<(unsigned)ctas, kThreads, smem, s>>>(prm);
     if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
-    const int vec4 = prm.seqlen % 4 == 0 && ((reinterpret_cast<uintptr_t>(dB) | reinterpret_cast<uintptr_t>(dC)) & 15u) == 0;
-    const int64_t work = 2 * prm.batch * prm.ngroups * kN * prm.seqlen / (vec4 ? 4 : 1) + prm.dim * kN + 2 * prm.dim;
+    const int64_t work = prm.dim * kN + 2 * prm.dim;
     const int64_t blocks = (work + 255) / 256;
     if (blocks > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;
-    scan_bwd_finalize<<<(unsigned)blocks, 256, 0, s>>>(prm, dA, dB, dC, dD, dbias, vec4);
+    scan_bwd_finalize<<<(unsigned)blocks, 256, 0, s>>>(prm, dA, dD, dbias);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -762,8 +771,10 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     prm.carry1 = reinterpret_cast<float*>(ws + w.carry1);
     prm.carry2 = reinterpret_cast<float*>(ws + w.carry2);
     prm.ckpt = reinterpret_cast<float*>(ws + w.ckpt);
-    prm.dBp = reinterpret_cast<float*>(ws + w.dBp);
-    prm.dCp = reinterpret_cast<float*>(ws + w.dCp);
+    prm.dB = static_cast<float*>(grads->dB);
+    prm.dC = static_cast<float*>(grads->dC);
+    prm.red_vec = dims->seqlen % 4 == 0 &&
+                  ((reinterpret_cast<uintptr_t>(grads->dB) | reinterpret_cast<uintptr_t>(grads->dC)) & 15u) == 0;
     prm.dAp = reinterpret_cast<float*>(ws + w.dAp);
     prm.dDp = reinterpret_cast<float*>(ws + w.dDp);
     prm.dbp = reinterpret_cast<float*>(ws + w.dbp);
@@ -778,10 +789,13 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the ticket, the status word and the segment flags start at zero (the status of this
     // call is read, and cleared, by ssm_selective_scan_bwd_device_status)
+    // dB and dC are sums of atomic adds: they start at zero
+    const size_t nbc = (size_t)(dims->batch * dims->ngroups * kN * dims->seqlen) * 4;
     if (cudaMemsetAsync(ws + w.ticket, 0, 8, s) != cudaSuccess ||
-        cudaMemsetAsync(ws + w.flag1, 0, (size_t)(w.zero_end - w.flag1), s) != cudaSuccess)
+        cudaMemsetAsync(ws + w.flag1, 0, (size_t)(w.zero_end - w.flag1), s) != cudaSuccess ||
+        cudaMemsetAsync(grads->dB, 0, nbc, s) != cudaSuccess || cudaMemsetAsync(grads->dC, 0, nbc, s) != cudaSuccess)
         return SSM_ERR_CUDA;
     return dims->io_dtype == SSM_BF16
-               ? launch<__nv_bfloat16>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, sc.ctas, s)
-               : launch<float>(prm, grads->dA, grads->dB, grads->dC, grads->dD, grads->ddelta_bias, sc.ctas, s);
+               ? launch<__nv_bfloat16>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s)
+               : launch<float>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s);
 }

@@ -95,13 +95,21 @@ def test_bwd_matches_oracle(case):
 
 
 def test_bwd_is_deterministic():
+    """Every gradient but dB and dC repeats bit for bit; dB and dC are sums of atomic adds
+    over the channels of a group, so between calls they may differ only by the rounding of
+    the order of those adds (a few fp32 ulps of their terms' size)."""
     dims = si.Dims(2, 64, 130, 16, dtype="bf16")
     inp = si.make_inputs(dims, _recipe("c2"), 43)
     gin = si.make_grad_inputs(dims, 44, dlast=True)
     a = run_bwd(dims, inp, gin)
     b = run_bwd(dims, inp, gin)
     for k in a:
-        if a[k] is not None:
+        if a[k] is None:
+            continue
+        if k in ("dB", "dC"):
+            scale = float(torch.max(torch.abs(a[k]))) + 1.0
+            assert float(torch.max(torch.abs(a[k] - b[k]))) <= 1e-5 * scale, f"{k} differs beyond rounding"
+        else:
             assert torch.equal(a[k], b[k]), f"{k} differs between two identical calls"
 
 

@@ -134,8 +134,8 @@ inline int fwd_geometry(const ssm_dims_t& d, int sm_count, int force_w, int forc
     int64_t ctas = sm_count;  // one persistent CTA per SM
     if (force_workers > 0 && force_workers < ctas) ctas = force_workers;
     const int64_t L = d.seqlen;
-    const int64_t seg_len = force_seg_len > 0 ? (force_seg_len + kTB - 1) / kTB * kTB
-                                              : default_seg_len(L, n_tiles, ctas);
+    const int64_t tb = v.tb;   // segments hold whole blocks
+    const int64_t seg_len = force_seg_len > 0 ? (force_seg_len + tb - 1) / tb * tb : default_seg_len(L, n_tiles, ctas);
     const int64_t n_seg = L > 0 ? (L + seg_len - 1) / seg_len : 1;
     const int64_t n_units = n_tiles * n_seg;
     if (n_units >= (int64_t)1 << 31 || seg_len > (int64_t)1 << 30) return SSM_ERR_UNSUPPORTED;
@@ -223,17 +223,19 @@ inline int fwd_launch(const ssm_dims_t& d, const FwdGeom& g, const FwdArgs& a, u
     TensorMaps tm;
     std::memset(&tm, 0, sizeof(tm));
     if (vec) {
-        const CUtensorMapSwizzle bc_swz = esz == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+        // boxes of one block (tb steps); B and C rows of 64 bytes take the 64-byte swizzle, of 128 the 128-byte one
+        const uint32_t tb = (uint32_t)g.lay.v.tb;
+        const CUtensorMapSwizzle bc_swz = tb * esz == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
         const uint64_t L = (uint64_t)d.seqlen;
-        vec = encode_rows(&tm.u, a.u, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        vec = encode_rows(&tm.u, a.u, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE, tb) &&
               encode_rows(&tm.delta, a.delta, esz, L, (uint64_t)(d.batch * d.nheads), delta_rows,
-                          CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                          CU_TENSOR_MAP_SWIZZLE_NONE, tb) &&
               (!a.z ||
-               encode_rows(&tm.z, a.z, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE)) &&
+               encode_rows(&tm.z, a.z, esz, L, (uint64_t)(d.batch * d.dim), ct, CU_TENSOR_MAP_SWIZZLE_NONE, tb)) &&
               encode_rows(&tm.B, a.B, esz, L, (uint64_t)(d.batch * d.ngroups * d.dstate), (uint32_t)d.dstate,
-                          bc_swz) &&
+                          bc_swz, tb) &&
               encode_rows(&tm.C, a.C, esz, L, (uint64_t)(d.batch * d.ngroups * d.dstate), (uint32_t)d.dstate,
-                          bc_swz);
+                          bc_swz, tb);
         // a shape the tensor maps cannot describe takes the element-copy path
     }
     Variant v;

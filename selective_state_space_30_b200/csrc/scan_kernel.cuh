@@ -56,7 +56,9 @@
 
 namespace ssm {
 
-constexpr int kTB = 32;      // time steps per block
+constexpr int kTB = 32;      // time steps per block: the fp32 and tensor-memory kernels
+constexpr int kTB16 = 64;    // time steps per block: the register kernel with bf16 I/O
+constexpr int kSegAlign = 64;  // segment lengths are multiples of every block length
 constexpr int kStages = 3;   // shared-memory ring depth (2 where 3 do not fit)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -89,7 +91,7 @@ struct FwdParams {
     int tiles_per_group;
     int n_tiles;
     int n_seg;
-    int seg_len;       // multiple of kTB
+    int seg_len;       // a multiple of the kernel's block length
     unsigned n_units;
     unsigned n_ctas;
     unsigned spin_limit;
@@ -406,14 +408,17 @@ struct Cfg {
     static constexpr bool kHeadA = HEAD_A;
     static constexpr int kN = N;
     static constexpr int ESZ = IO<T>::kBytes;
+    // steps per block: 64 for bf16 I/O (a block's rows are 128 bytes either way, the
+    // widest hardware swizzle; the longer block halves the per-block work), 32 for fp32
+    static constexpr int TB = ESZ == 2 ? kTB16 : kTB;
     static constexpr int S = SPL;                          // states per lane
     static constexpr int TPC = N / S;                      // lanes per channel (2, 4 or 8)
     static constexpr int GW = 32 / TPC;                    // channels per consumer warp
     static constexpr int CT = W * GW;                      // channels per tile
-    static constexpr int TPT = kTB / TPC;                  // steps per lane in prologue / epilogue
+    static constexpr int TPT = TB / TPC;                   // steps per lane in prologue / epilogue
     static constexpr int WT = (ESZ == 4 || S >= 16) ? 4 : 8;  // steps per B/C register window
-    static constexpr int RB = kTB * ESZ;                   // bytes of one block row
-    static constexpr int ROW = kTB + 4;                    // per-warp float rows (padded)
+    static constexpr int RB = TB * ESZ;                    // bytes of one block row
+    static constexpr int ROW = TB + 4;                     // per-warp float rows (padded)
     static constexpr int NA = HEAD_A ? 1 : S;
     // one ring stage (1024-byte aligned): B box | C box (N rows each, hardware
     // swizzled) | u box | delta box | z box (CT rows each) | header
@@ -444,20 +449,20 @@ struct Cfg {
     static constexpr int OFF_WARP = OFF_CSLOT + 2 * CSLOT * 4;
     static constexpr int SMEM = OFF_WARP + W * WARP_F * 4;
     static constexpr int THREADS = 32 * (W + 1);
-    static_assert(S % 2 == 0 && N % S == 0 && TPC >= 2 && TPC <= 8, "lane split");
-    static_assert(TPT % 4 == 0 && TPT <= 16, "steps per lane must be 4..16");
+    // the layout compiles: lanes per channel, 4 .. 16 steps per lane, the shared-memory budget
+    static constexpr bool kFits = TPC >= 2 && TPC <= 8 && TPT % 4 == 0 && TPT <= 16 && SMEM <= 227 * 1024;
+    static_assert(S % 2 == 0 && N % S == 0, "lane split");
     static_assert(STAGE % 16 == 0 && (PSLOT * 4) % 16 == 0 && (WARP_F * 4) % 16 == 0, "16-byte aligned smem");
     static_assert(2 * kStages + 6 <= 128, "barriers fit below OFF_STAGES");
-    static_assert((N * RB) % 512 == 0, "C box keeps the swizzle phase");
-    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(RB == 64 || (N * RB) % 1024 == 0, "C box keeps the swizzle phase");
 };
 
-// Byte offset of element t of row r inside a B or C box, as the tensor-map
-// swizzle lays it out: 16-byte chunks XORed with row bits (64-byte rows: bits 1-2
-// of the row; 128-byte rows: bits 0-2).
-template <int ESZ>
+// Byte offset of element t of row r inside a B or C box of TB steps, as the
+// tensor-map swizzle lays it out: 16-byte chunks XORed with row bits (64-byte rows:
+// bits 1-2 of the row; 128-byte rows: bits 0-2).
+template <int ESZ, int TB>
 __device__ __forceinline__ int bc_off(int r, int t) {
-    constexpr int RB = kTB * ESZ;
+    constexpr int RB = TB * ESZ;
     const int byte = t * ESZ;
     const int swz = RB == 64 ? ((r >> 1) & 3) : (r & 7);
     return r * RB + ((((byte >> 4) ^ swz) & (RB / 16 - 1)) << 4) + (byte & 15);
@@ -505,7 +510,7 @@ __device__ __forceinline__ void produce(const FwdParams& p, const TensorMaps& tm
                                         const ProducerBars& br, int lane, uint64_t budget, int* status) {
     using T = typename Cf::Elem;
     constexpr bool HEAD_A = Cf::kHeadA;
-    constexpr int N = Cf::kN, CT = Cf::CT, ESZ = Cf::ESZ, RB = Cf::RB, NST = Cf::STG;
+    constexpr int N = Cf::kN, CT = Cf::CT, ESZ = Cf::ESZ, RB = Cf::RB, NST = Cf::STG, TB = Cf::TB;
     const int64_t Dm = p.dim, L = p.seqlen, H = p.nheads, G = p.ngroups;
     const int64_t Dg = Dm / G, P = Dm / H;
     unsigned fill = 0;          // blocks produced
@@ -576,7 +581,7 @@ __device__ __forceinline__ void produce(const FwdParams& p, const TensorMaps& tm
         const int64_t b = bg / G, g = bg % G, ci0 = (int64_t)ti * CT;
         const int64_t t0u = (int64_t)seg * p.seg_len;
         const int64_t t1u = t0u + p.seg_len < L ? t0u + p.seg_len : L;
-        const int nblk = L > 0 ? (int)((t1u - t0u + kTB - 1) / kTB) : 1;
+        const int nblk = L > 0 ? (int)((t1u - t0u + TB - 1) / TB) : 1;
         const bool final_seg = seg + 1 >= p.n_seg;
         const int pslot = ucount & 1;
 
@@ -663,8 +668,8 @@ __device__ __forceinline__ void produce(const FwdParams& p, const TensorMaps& tm
             const int st = fill % NST;
             unsigned char* sb = smem + Cf::OFF_STAGES + st * Cf::STAGE;
             uint64_t* full = br.fill + st;
-            const int64_t t0 = t0u + (int64_t)kb * kTB;
-            const int64_t nv = L - t0 < kTB ? (L - t0 > 0 ? L - t0 : 0) : kTB;  // valid steps in the block
+            const int64_t t0 = t0u + (int64_t)kb * TB;
+            const int64_t nv = L - t0 < TB ? (L - t0 > 0 ? L - t0 : 0) : TB;  // valid steps in the block
             int nvalid = (int)(Dg - ci0 < CT ? Dg - ci0 : CT);
             if (lane == 0) {
                 BlockHdr* hd = reinterpret_cast<BlockHdr*>(sb + Cf::OFF_HDR);
@@ -708,15 +713,15 @@ __device__ __forceinline__ void produce(const FwdParams& p, const TensorMaps& tm
                 // guarded element copies into the same layout (unaligned rows, ragged tails)
                 const T* Bb = reinterpret_cast<const T*>(p.B) + (b * G + g) * (int64_t)N * L;
                 const T* Cb = reinterpret_cast<const T*>(p.C) + (b * G + g) * (int64_t)N * L;
-                for (int e = lane; e < 2 * N * kTB; e += 32) {
-                    const int r = e / kTB, tt = e % kTB;
+                for (int e = lane; e < 2 * N * TB; e += 32) {
+                    const int r = e / TB, tt = e % TB;
                     const int w = r / N, n = r % N;
                     const T* src = (w ? Cb : Bb) + (int64_t)n * L;
-                    *reinterpret_cast<T*>(sb + Cf::OFF_BC + w * N * RB + bc_off<ESZ>(n, tt)) =
+                    *reinterpret_cast<T*>(sb + Cf::OFF_BC + w * N * RB + bc_off<ESZ, TB>(n, tt)) =
                         tt < nv ? src[t0 + tt] : T(0.f);
                 }
-                for (int e = lane; e < ntens * CT * kTB; e += 32) {
-                    const int r = e / kTB, tt = e % kTB;
+                for (int e = lane; e < ntens * CT * TB; e += 32) {
+                    const int r = e / TB, tt = e % TB;
                     const int w = r / CT, lcr = r % CT;
                     const T* src = nullptr;
                     if (w == 1) {
@@ -777,7 +782,7 @@ __global__ void __launch_bounds__(Cfg<T, N, W, HEAD_A, SPL>::THREADS, 1)
 scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
     using Cf = Cfg<T, N, W, HEAD_A, SPL>;
     constexpr int S = Cf::S, TPC = Cf::TPC, GW = Cf::GW, CT = Cf::CT, TPT = Cf::TPT, WT = Cf::WT;
-    constexpr int ROW = Cf::ROW, NA = Cf::NA, ESZ = Cf::ESZ, RB = Cf::RB;
+    constexpr int ROW = Cf::ROW, NA = Cf::NA, ESZ = Cf::ESZ, RB = Cf::RB, TB = Cf::TB;
     constexpr int NST = Cf::STG;  // ring stages
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
@@ -825,14 +830,14 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
     float* rda = wf + Cf::W_DA + cg * ROW;
     float* ry = wf + Cf::W_Y + cg * ROW;
     // this lane's states are n = s*TPC + j; byte offsets of their rows' windows in a B/C box
-    constexpr int NWIN = kTB / WT;
+    constexpr int NWIN = TB / WT;
     constexpr bool OFF_TABLE = S * NWIN <= 16;
     int boff[OFF_TABLE ? S * NWIN : S];
 #pragma unroll
     for (int s = 0; s < S; ++s) {
         if constexpr (OFF_TABLE) {
 #pragma unroll
-            for (int w = 0; w < NWIN; ++w) boff[s * NWIN + w] = bc_off<ESZ>(s * TPC + j, w * WT);
+            for (int w = 0; w < NWIN; ++w) boff[s * NWIN + w] = bc_off<ESZ, TB>(s * TPC + j, w * WT);
         } else {
             boff[s] = s * TPC + j;
         }
@@ -876,7 +881,7 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
         const int64_t drow_i = HEAD_A ? (d / P - (hd.g * Dg + hd.ci0) / P) : lc;
         const unsigned char* drow = sb + Cf::OFF_IN + (CT + drow_i) * RB + j * TPT * ESZ;
         const unsigned char* zrow = sb + Cf::OFF_IN + (2 * CT + lc) * RB + j * TPT * ESZ;
-        const bool full_blk = t0 + kTB <= hd.t1;
+        const bool full_blk = t0 + TB <= hd.t1;
         // -------- prologue: dt, dt*u (dA) of this lane's steps, two at a time
         {
             Chunk<T, TPT> cu, cd;
@@ -923,7 +928,7 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             for (int s = 0; s < S; ++s) {
                 int off;
                 if constexpr (OFF_TABLE) off = boff[s * NWIN + w];
-                else off = bc_off<ESZ>(boff[s], tw);
+                else off = bc_off<ESZ, TB>(boff[s], tw);
                 const unsigned char* rb = bcb + off;
                 const unsigned char* rc = bcb + N * RB + off;
                 if constexpr (WT * ESZ == 16) {
@@ -1066,6 +1071,7 @@ struct CfgTc {
     static constexpr int TPT = kTB / TPCS;                 // steps per lane in prologue / epilogue
     static constexpr int RB = kTB * ESZ;                   // bytes of one block row
     static constexpr int WIN = KT == 1 ? 8 : 4;            // steps per tensor-memory read
+    static constexpr int TB = kTB;                         // steps per block
     static constexpr int NSLICE = S * KT;                  // one-hot K-slices (16 columns each)
     // one ring stage (1024-byte aligned): B box | C box (16 rows of 64 bytes each, 64-byte
     // swizzle, read by the tensor cores as an MN-major operand) | u box | delta box | z box
@@ -1557,7 +1563,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
 
 // ------------------------------------------------------- segment policy
 
-// Default segment length (steps, a multiple of kTB) for a launch of `ctas`
+// Default segment length (steps, a multiple of every block length) for a launch of `ctas`
 // persistent CTAs over `n_tiles` channel tiles of a sequence of L steps.
 // Segments of one tile run one after another (each starts from the state the
 // previous one published), so a segment is the unit of load balance: about
@@ -1566,14 +1572,14 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
 // segments (64 steps) lose about a third of the throughput, and beyond eight
 // units per CTA the gain flattens, so segments stay within [256, 2048] steps.
 inline int64_t default_seg_len(int64_t L, int64_t n_tiles, int64_t ctas) {
-    if (L <= 0) return kTB;
+    if (L <= 0) return kSegAlign;
     const int64_t t = n_tiles > 0 ? n_tiles : 1;
     int64_t n_seg = (8 * ctas + t - 1) / t;
     if (n_seg < 1) n_seg = 1;
     int64_t seg = (L + n_seg - 1) / n_seg;
     if (seg > 2048) seg = 2048;
     if (seg < 256) seg = 256;
-    seg = (seg + kTB - 1) / kTB * kTB;
+    seg = (seg + kSegAlign - 1) / kSegAlign * kSegAlign;
     return seg;
 }
 
@@ -1587,18 +1593,19 @@ struct Variant {
     int threads;
     int ch_per_tile;   // CT
     int dstate;
+    int tb;            // steps per block (the tensor maps' box width)
     const char* name;
 };
 
 template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC>
 Variant make_variant(const char* name) {
     using C = Cfg<T, N, W, HEAD_A, SPL>;
-    return Variant{scan_fwd_kernel<T, N, W, HEAD_A, SPL, VEC>, C::SMEM, C::THREADS, C::CT, N, name};
+    return Variant{scan_fwd_kernel<T, N, W, HEAD_A, SPL, VEC>, C::SMEM, C::THREADS, C::CT, N, C::TB, name};
 }
 template <int W, int SPL, int KT, bool VEC>
 Variant make_variant_tc(const char* name) {
     using C = CfgTc<W, SPL, KT>;
-    return Variant{scan_fwd_tc_kernel<W, SPL, KT, VEC>, C::SMEM, C::THREADS, C::CT, 16, name};
+    return Variant{scan_fwd_tc_kernel<W, SPL, KT, VEC>, C::SMEM, C::THREADS, C::CT, 16, C::TB, name};
 }
 
 // The lane layouts compiled for a state size N: (consumer warps W, states per lane S).
@@ -1608,12 +1615,18 @@ Variant make_variant_tc(const char* name) {
 //   N >= 64: (8, N/8), (4, N/8).
 // The tensor-memory kernel (mode 1: bf16, N = 16, A per channel), with KT time sub-chunks
 // per block: (16, 2, 1), (8, 4, 1), (12, 4, 1), (16, 2, 2), (8, 2, 2).
-constexpr bool layout_exists(int N, int w, int spl) {
+constexpr bool layout_listed(int N, int w, int spl) {
     if (N <= 16)
         return (w == 16 && spl == 2) || (N == 16 && w == 12 && spl == 4) ||
                ((w == 8 || w == 4) && (spl == 2 || spl == 4));
     if (N == 32) return (w == 8 || w == 4) && spl == 4;
     return (w == 8 || w == 4) && spl == N / 8;
+}
+// a listed layout whose lane split, steps per lane and shared-memory map work out
+template <typename T, int N, int W, int SPL>
+constexpr bool layout_exists() {
+    if constexpr (layout_listed(N, W, SPL)) return Cfg<T, N, W, false, SPL>::kFits && Cfg<T, N, W, true, SPL>::kFits;
+    else return false;
 }
 constexpr bool layout_exists_tc(int w, int spl, int kt) {
     return (kt == 1 && ((w == 16 && spl == 2) || ((w == 8 || w == 12) && spl == 4))) ||
@@ -1628,7 +1641,7 @@ constexpr bool tc_fits() {
 // One function per (io dtype, N) translation unit; see fwd_*.cu.
 #define SSM_PICK_ONE(T, TN, N, W, SPL)                                                                   \
     if (mode == 0 && kt == 1 && w == W && spl == SPL) {                                                  \
-        if constexpr (layout_exists(N, W, SPL)) {                                                        \
+        if constexpr (layout_exists<T, N, W, SPL>()) {                                                   \
             if (head)                                                                                    \
                 *v = vec ? make_variant<T, N, W, true, SPL, true>("ws_" #TN "_n" #N "_w" #W "s" #SPL "t1_head_vec") \
                          : make_variant<T, N, W, true, SPL, false>("ws_" #TN "_n" #N "_w" #W "s" #SPL "t1_head");   \

@@ -536,6 +536,15 @@ def run_ours(args):
 
     # the headline: exactly K timed steps of the named workload
     job = _ScanJob(ssm, w, dev, local)
+    if args.layout:
+        # a forced kernel layout (consumer warps, states per lane, time sub-chunks, kernel: 1 = register,
+        # 2 = tensor memory), to time the kernels the plan does not pick by default
+        lw, ls, lk, lm = (int(x) for x in args.layout.split(","))
+        for opt, val in ((ssm.SSM_OPT_TENSOR_MEMORY, lm), (ssm.SSM_OPT_CONSUMER_WARPS, lw),
+                         (ssm.SSM_OPT_STATES_PER_LANE, ls), (ssm.SSM_OPT_TIME_LANES, lk)):
+            ssm.ssm_scan_set_option(job.plan, opt, val)
+        job.info = ssm.ssm_scan_plan_info(job.plan)
+        job.sched = ssm.ssm_scan_plan_schedule(job.plan)
     launch_ms, total_ms, clocks = job.timed(args.steps, args.warmup, local)
     elems = d.batch * d.dim * d.seqlen
     ms_per_step = total_ms / args.steps
@@ -846,6 +855,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layout", default="",
+                    help="force the headline's kernel layout: warps,states_per_lane,time_lanes,kernel "
+                         "(kernel 1 = register, 2 = tensor memory; 0 = automatic), e.g. 16,2,1,2")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only the named workload (default: also one line per other forward workload)")
     ap.add_argument("--op", default="scan", choices=["scan", "decode", "conv1d", "bwd"],

@@ -518,6 +518,19 @@ def _config_entry(job, launch_ms, total_ms, steps, clocks, probe_rate):
             "clocks": clocks}
 
 
+def _bench_workload(args):
+    """The named workload; with --seqlen, the same shape at a shorter sequence length (a smaller case
+    of the same kernel, for profiler captures that must stay small).  The renamed workload matches no
+    committed traffic figure."""
+    import dataclasses
+    import ssm_inputs as si
+    w = si.WORKLOADS[args.workload]
+    if not args.seqlen:
+        return w
+    return dataclasses.replace(w, name=f"{w.name}@L{args.seqlen}",
+                               dims=dataclasses.replace(w.dims, seqlen=args.seqlen))
+
+
 def run_ours(args):
     import torch
     import ssm_inputs as si
@@ -529,7 +542,7 @@ def run_ours(args):
     init_ranks("nccl", local)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = si.WORKLOADS[args.workload]
+    w = _bench_workload(args)
     d = w.dims
     stream = torch.cuda.current_stream(dev)
     probe_rate = _probe_mufu(ssm, dev, stream.cuda_stream, stream)
@@ -558,7 +571,7 @@ def run_ours(args):
     # every other forward workload, one line each (the driver sees all five shapes)
     if not args.no_per_config:
         for name, wk in si.WORKLOADS.items():
-            if name == w.name:
+            if name == args.workload:
                 continue
             j = _ScanJob(ssm, wk, dev, local)
             # a short probe sizes the run so that each line times at least PER_CONFIG_MIN_MS
@@ -779,7 +792,7 @@ def run_bwd(args):
     init_ranks("nccl", local)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    w = si.workload(args.workload)
+    w = _bench_workload(args)
     d = w.dims
     inp = si.make_inputs(d, w.recipe, w.seed)
     gin = si.make_grad_inputs(d, 1)
@@ -830,13 +843,13 @@ def run_bwd(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32 (bf16 I/O)" if d.dtype == "bf16" else "f32", "data": "synthetic (seeded splitmix64)",
-            "config": {"workload": args.workload, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen,
+            "config": {"workload": w.name, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen,
                        "dstate": d.dstate, "io_dtype": d.dtype, "parallelism": f"replicas x{world}",
                        "l2": f"inputs {in_bytes / 1e6:.0f} MB and workspace {nws / 1e6:.0f} MB (> 126 MB L2), "
                              "no flush"},
             "roofline": {"bound": "alu", "achieved": gexps, "peak": mufu_peak, "unit": "Gexp/s",
                          "frac": gexps / mufu_peak,
-                         "traffic": _traffic_from_profiles(args.workload, key="bwd:" + args.workload,
+                         "traffic": _traffic_from_profiles(w.name, key="bwd:" + w.name,
                                                            sha=_src_hash(("bwd.cu",))),
                          "peak_source": f"148 SMs x 16 ex2/clk x {sm_max_mhz:.0f} MHz ({src} sm_max_mhz)",
                          "exps_per_launch": exps,
@@ -858,6 +871,8 @@ def main():
     ap.add_argument("--layout", default="",
                     help="force the headline's kernel layout: warps,states_per_lane,time_lanes,kernel "
                          "(kernel 1 = register, 2 = tensor memory; 0 = automatic), e.g. 16,2,1,2")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="replace the workload's sequence length (a smaller case for profiler captures)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only the named workload (default: also one line per other forward workload)")
     ap.add_argument("--op", default="scan", choices=["scan", "decode", "conv1d", "bwd"],

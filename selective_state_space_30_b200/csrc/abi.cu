@@ -64,6 +64,8 @@ struct ssm_plan_s {
     // streams for the copies in, the scans and the copies out, and their events
     ssm_plan_s* sub;
     int n_chunks;
+    bool chunk_time;       // batch 1: the chunks are stretches of the sequence, chained by their states
+    float* h_state2;       // the second state buffer of a time-chunk pipeline (alternates with h_bufs[9])
     cudaStream_t pipe[3];
     cudaEvent_t ev_start, ev_end, ev_in[8], ev_run[8];
     bool pipe_ready;
@@ -202,6 +204,8 @@ static void release_pipeline(ssm_plan_s* p) {
     }
     if (p->sub) ssm_scan_destroy(p->sub);
     p->sub = nullptr;
+    if (p->h_state2) cudaFree(p->h_state2);
+    p->h_state2 = nullptr;
     std::memset(p->pipe, 0, sizeof(p->pipe));
     p->ev_start = p->ev_end = nullptr;
     std::memset(p->ev_in, 0, sizeof(p->ev_in));
@@ -322,25 +326,41 @@ int ssm_selective_scan_fwd(ssm_plan_t plan, const void* u, const void* delta, co
                                      last_state, stream);
 }
 
-// The same call on host buffers.  With batch >= 2 the batch rows are cut into chunks
-// (the largest divisor of batch up to 8) and pipelined on three streams the plan
-// owns: a chunk's inputs are copied in while the previous chunk is scanned and the
-// one before it is copied out, so the copies in both directions and the scans
-// overlap.  Each chunk runs through a plan for one chunk's rows.  The call starts
-// after the work already queued on `stream` and the work queued on `stream` after it
-// waits for its end.  With batch 1 everything runs in order on `stream`.
+// The same call on host buffers.  The problem is cut into chunks pipelined on three
+// streams the plan owns: a chunk's inputs are copied in while the previous chunk is
+// scanned and the one before it is copied out, so the copies in both directions and
+// the scans overlap.  With batch >= 2 the chunks are batch rows (the largest divisor
+// of batch up to 8).  With batch 1 they are stretches of the sequence (the most, up to
+// 8, that divide L into multiples of 64 steps of at least 1024): each chunk scans every
+// channel over its stretch, starting from the state the previous chunk ended with (the
+// initial-state entry), so every chunk runs with all of the GPU's parallelism; its
+// rows move by 2-D copies.  Each chunk runs through a plan for one chunk's shape.  The
+// call starts after the work already queued on `stream` and the work queued on
+// `stream` after it waits for its end.  A problem that splits neither way runs in
+// order on `stream`.
 static int build_pipeline(ssm_plan_s* p) {
     const ssm_dims_t& d = p->dims;
     int n = 1;
-    for (int k = 8; k >= 2; --k)
-        if (d.batch % k == 0) {
-            n = k;
-            break;
-        }
+    p->chunk_time = false;
+    if (d.batch >= 2) {
+        for (int k = 8; k >= 2; --k)
+            if (d.batch % k == 0) {
+                n = k;
+                break;
+            }
+    } else if (d.batch == 1) {
+        for (int k = 8; k >= 2; --k)
+            if (d.seqlen % k == 0 && (d.seqlen / k) % 64 == 0 && d.seqlen / k >= 1024) {
+                n = k;
+                p->chunk_time = true;
+                break;
+            }
+    }
     p->n_chunks = n;
     if (n == 1) return SSM_OK;
     ssm_dims_t cd = d;
-    cd.batch = d.batch / n;
+    if (p->chunk_time) cd.seqlen = d.seqlen / n;
+    else cd.batch = d.batch / n;
     int rc = ssm_scan_plan(&p->sub, &cd, p->device);
     if (rc != SSM_OK) return rc;
     p->pipe_ready = true;   // from here on release_pipeline frees what was made
@@ -387,14 +407,14 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
         if (bytes[i] && cudaMalloc(&plan->h_bufs[i], bytes[i]) != cudaSuccess) return SSM_ERR_CUDA;
         plan->h_sizes[i] = bytes[i];
     }
-    if (d.batch >= 2 && !plan->pipe_ready) {
+    if (d.batch >= 1 && !plan->pipe_ready && plan->n_chunks != 1) {
         const int rc = build_pipeline(plan);
         if (rc != SSM_OK) {
             release_pipeline(plan);
             return rc;
         }
     }
-    if (d.batch < 2 || plan->n_chunks < 2) {
+    if (!plan->pipe_ready || plan->n_chunks < 2) {
         for (int i = 0; i < 8; ++i)
             if (used[i] && bytes[i] &&
                 cudaMemcpyAsync(plan->h_bufs[i], src[i], bytes[i], cudaMemcpyHostToDevice, s) != cudaSuccess)
@@ -411,11 +431,59 @@ int ssm_selective_scan_fwd_host(ssm_plan_t plan, const void* u, const void* delt
             return SSM_ERR_CUDA;
         return SSM_OK;
     }
-    // the pipeline: per-chunk slabs of every per-row tensor (rows of a chunk are contiguous)
     const int n = plan->n_chunks;
     cudaStream_t sin = plan->pipe[0], srun = plan->pipe[1], sout = plan->pipe[2];
     bool ok = cudaEventRecord(plan->ev_start, s) == cudaSuccess;
     for (int i = 0; i < 3; ++i) ok = ok && cudaStreamWaitEvent(plan->pipe[i], plan->ev_start, 0) == cudaSuccess;
+    if (plan->chunk_time) {
+        // batch 1, time chunks: chunk k's rows are the (rows x Lc) block at k * rows * Lc of each device
+        // mirror, copied from (to) columns [k*Lc, (k+1)*Lc) of the host rows; the state chains the chunks
+        // through two alternating buffers
+        const size_t L = (size_t)d.seqlen, Lc = L / n;
+        const size_t rows[10] = {(size_t)d.dim, (size_t)d.nheads, 0, (size_t)(d.ngroups * d.dstate),
+                                 (size_t)(d.ngroups * d.dstate), 0, (size_t)d.dim, 0, (size_t)d.dim, 0};
+        if (!plan->h_state2 && cudaMalloc(&plan->h_state2, bytes[9] ? bytes[9] : 4) != cudaSuccess) {
+            plan->h_state2 = nullptr;
+            return SSM_ERR_CUDA;
+        }
+        if (!plan->h_bufs[9]) {
+            if (cudaMalloc(&plan->h_bufs[9], bytes[9] ? bytes[9] : 4) != cudaSuccess) return SSM_ERR_CUDA;
+            plan->h_sizes[9] = bytes[9];
+        }
+        float* state[2] = {(float*)plan->h_bufs[9], plan->h_state2};
+        for (int i : {2, 5, 7})
+            if (ok && used[i] && bytes[i])
+                ok = cudaMemcpyAsync(plan->h_bufs[i], src[i], bytes[i], cudaMemcpyHostToDevice, sin) == cudaSuccess;
+        for (int k = 0; k < n && ok; ++k) {
+            for (int i : {0, 1, 3, 4, 6}) {
+                if (!used[i] || !bytes[i]) continue;
+                ok = ok && cudaMemcpy2DAsync(static_cast<char*>(plan->h_bufs[i]) + (size_t)k * rows[i] * Lc * e, Lc * e,
+                                             static_cast<const char*>(src[i]) + (size_t)k * Lc * e, L * e, Lc * e,
+                                             rows[i], cudaMemcpyHostToDevice, sin) == cudaSuccess;
+            }
+            ok = ok && cudaEventRecord(plan->ev_in[k], sin) == cudaSuccess &&
+                 cudaStreamWaitEvent(srun, plan->ev_in[k], 0) == cudaSuccess;
+            if (!ok) break;
+            auto blk = [&](int i) -> void* {
+                return used[i] ? static_cast<char*>(plan->h_bufs[i]) + (size_t)k * rows[i] * Lc * e : nullptr;
+            };
+            const int rc = launch_fwd(plan->sub, blk(0), blk(1), (const float*)plan->h_bufs[2], blk(3), blk(4),
+                                      D ? (const float*)plan->h_bufs[5] : nullptr, blk(6),
+                                      delta_bias ? (const float*)plan->h_bufs[7] : nullptr, softplus,
+                                      k > 0 ? state[(k - 1) & 1] : nullptr, blk(8), state[k & 1], srun);
+            if (rc != SSM_OK) return rc;
+            ok = cudaEventRecord(plan->ev_run[k], srun) == cudaSuccess &&
+                 cudaStreamWaitEvent(sout, plan->ev_run[k], 0) == cudaSuccess &&
+                 cudaMemcpy2DAsync(static_cast<char*>(out) + (size_t)k * Lc * e, L * e, blk(8), Lc * e, Lc * e,
+                                   rows[8], cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+        }
+        if (ok && last_state && bytes[9])
+            ok = cudaMemcpyAsync(last_state, state[(n - 1) & 1], bytes[9], cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+        ok = ok && cudaEventRecord(plan->ev_end, sout) == cudaSuccess &&
+             cudaStreamWaitEvent(s, plan->ev_end, 0) == cudaSuccess;
+        return ok ? SSM_OK : SSM_ERR_CUDA;
+    }
+    // batch-row chunks: per-chunk slabs of every per-row tensor (rows of a chunk are contiguous)
     // the per-channel parameters once
     for (int i : {2, 5, 7})
         if (ok && used[i] && bytes[i])

@@ -210,15 +210,19 @@ def test_misaligned_pointers_take_scalar_path():
 HOST_CASES = [
     si.Dims(2, 64, 256, 16, dtype="bf16"),                  # two chunks of one batch row
     si.Dims(6, 64, 200, 16, dtype="bf16"),                  # six chunks, ragged length
-    si.Dims(1, 64, 256, 16, dtype="f32"),                   # one batch row: no pipeline
+    si.Dims(1, 64, 256, 16, dtype="f32"),                   # one batch row, too short to split: no pipeline
     si.Dims(4, 128, 256, 128, nheads=2, dtype="bf16"),      # four chunks through the tensor-core path
+    si.Dims(1, 96, 4096, 16, dtype="bf16"),                 # one batch row in four time chunks, chained states
+    si.Dims(1, 64, 6144, 16, ngroups=2, dtype="f32"),       # six time chunks, two groups
+    si.Dims(1, 128, 4096, 128, nheads=2, dtype="bf16"),     # time chunks through the tensor-core path
 ]
 
 
 @pytest.mark.parametrize("dims", HOST_CASES, ids=lambda d: f"{d.batch}x{d.dim}x{d.seqlen}n{d.dstate}{d.dtype}")
 def test_host_entry_point_matches_oracle(dims):
-    """ssm_selective_scan_fwd_host (copies in, scan, copies out; pipelined over batch rows)
-    against the oracle, and twice in a row on the same plan."""
+    """ssm_selective_scan_fwd_host (copies in, scan, copies out; pipelined over batch rows, or
+    over stretches of the sequence for one batch row) against the oracle, and twice in a row
+    on the same plan."""
     import torch
     import selective_state_space_30_b200 as ssm
     rec = si.Recipe(a_init="neg_uniform_1_16") if dims.head_mode else si.Recipe(d_init="normal",

@@ -865,7 +865,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=None,
+                    help=f"the shape (default: {DEFAULT_WORKLOAD} for the scan, a per-op default otherwise)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layout", default="",
@@ -882,22 +883,24 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.op == "decode":
-        if args.workload == DEFAULT_WORKLOAD:
+        if args.workload is None:
             args.workload = "decode-mamba-1.4b-b256"
         run_decode(args)
         return
     if args.op == "conv1d":
-        if args.workload == DEFAULT_WORKLOAD:
+        if args.workload is None:
             args.workload = "conv1d-mamba-130m"
         run_conv1d(args)
         return
     if args.op == "bwd":
-        if args.workload == DEFAULT_WORKLOAD:
+        if args.workload is None:
             args.workload = "mamba-130m"
         if args.workload not in BWD_WORKLOADS:
             raise SystemExit(f"--op bwd runs on {BWD_WORKLOADS}")
         run_bwd(args)
         return
+    if args.workload is None:
+        args.workload = DEFAULT_WORKLOAD
     if args.impl == "reference":
         run_reference(args)
     else:

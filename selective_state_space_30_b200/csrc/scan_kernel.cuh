@@ -439,7 +439,26 @@ struct Cfg {
     static constexpr int W_DU = GW * ROW;
     static constexpr int W_DA = 2 * GW * ROW;
     static constexpr int W_Y = (HEAD_A ? 3 : 2) * GW * ROW;
-    static constexpr int WARP_F = W_Y + GW * ROW;
+    // Per-lane y rows (up to 8 consumer warps, where they fit): each lane writes its
+    // partial sums of y over its S states to a row of its own, and the epilogue adds
+    // the TPC rows of a channel, so the recurrence has no cross-lane reduction.  In
+    // lane j's row, the TPT columns the epilogue of lane j reads are shifted by
+    // YSH(j) 16-byte groups, which puts the eight lanes of each shared-memory phase in
+    // different banks both when they write (same column, rows 17 groups apart) and when
+    // they read (the rows of one channel, their own columns).
+    static constexpr bool YLANE = W <= 8 && WT == 8 && TPT % 4 == 0;
+    static constexpr int YSH_MAX = TPC == 8 ? 1 : TPC - 1;
+    static constexpr int YROW = TB + 4 * YSH_MAX;
+    // Per-lane-pair y rows (16 warps, 8 lanes per channel, 64-step blocks): the
+    // recurrence does the first round of the reduction (lanes j and j^4 swap window
+    // halves) and writes the pair's sums to row j&3, the lower halves from column 0 and
+    // the upper halves from column YHALF; the epilogue adds the 4 rows.  A row is 18
+    // 16-byte groups (2 mod 8) and YHALF 9 groups (1 mod 8), so the eight lanes of a
+    // phase hit different banks on both sides.
+    static constexpr bool YPART = !YLANE && W == 16 && TPC == 8 && WT == 8 && TB == 64;
+    static constexpr int YPROW = 72, YHALF = 36;
+    static constexpr int WARP_F = W_Y + (YLANE ? 32 * YROW : YPART ? GW * 4 * YPROW : GW * ROW);
+    __device__ static constexpr int ysh(int jl) { return TPC == 8 ? jl >> 2 : jl; }
     // shared memory map (bytes)
     static constexpr int OFF_STAGES = 1024;                // barriers live below
     static constexpr int REST = 2 * PSLOT * 4 + 2 * CSLOT * 4 + W * WARP_F * 4;
@@ -828,7 +847,7 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
     float* rdt = wf + Cf::W_DT + cg * ROW;
     float* rdu = wf + Cf::W_DU + cg * ROW;
     float* rda = wf + Cf::W_DA + cg * ROW;
-    float* ry = wf + Cf::W_Y + cg * ROW;
+    float* ry = wf + Cf::W_Y + cg * (Cf::YLANE ? TPC * Cf::YROW : Cf::YPART ? 4 * Cf::YPROW : ROW);
     // this lane's states are n = s*TPC + j; byte offsets of their rows' windows in a B/C box
     constexpr int NWIN = TB / WT;
     constexpr bool OFF_TABLE = S * NWIN <= 16;
@@ -920,10 +939,15 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
         __syncwarp();
         // -------- the recurrence, one window of WT steps at a time (unrolled)
         const unsigned char* bcb = sb + Cf::OFF_BC;
-#pragma unroll
-        for (int w = 0; w < NWIN; ++w) {
+        // A window's B and C words and its dt, dt*u (dA) rows, into register set bsel.  With
+        // per-lane y rows (up to 8 consumer warps, registers to spare) the next window's set
+        // is loaded while the current one runs (up to 4 states per lane); otherwise each
+        // window loads its own.
+        constexpr bool PF = Cf::YLANE && S <= 4;
+        uint32_t bwA[PF ? 2 : 1][S][WT * ESZ / 4], cwA[PF ? 2 : 1][S][WT * ESZ / 4];
+        float dtA[PF ? 2 : 1][WT], duA[PF ? 2 : 1][WT], daA[PF ? 2 : 1][HEAD_A ? WT : 1];
+        auto load_window = [&](const int w, const int bsel) {
             const int tw = w * WT;
-            uint32_t bw[S][WT * ESZ / 4], cw_[S][WT * ESZ / 4];
 #pragma unroll
             for (int s = 0; s < S; ++s) {
                 int off;
@@ -934,27 +958,43 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
                 if constexpr (WT * ESZ == 16) {
                     const uint4 vb = *reinterpret_cast<const uint4*>(rb);
                     const uint4 vc = *reinterpret_cast<const uint4*>(rc);
-                    bw[s][0] = vb.x; bw[s][1] = vb.y; bw[s][2] = vb.z; bw[s][3] = vb.w;
-                    cw_[s][0] = vc.x; cw_[s][1] = vc.y; cw_[s][2] = vc.z; cw_[s][3] = vc.w;
+                    bwA[bsel][s][0] = vb.x; bwA[bsel][s][1] = vb.y; bwA[bsel][s][2] = vb.z; bwA[bsel][s][3] = vb.w;
+                    cwA[bsel][s][0] = vc.x; cwA[bsel][s][1] = vc.y; cwA[bsel][s][2] = vc.z; cwA[bsel][s][3] = vc.w;
                 } else {
                     const uint2 vb = *reinterpret_cast<const uint2*>(rb);
                     const uint2 vc = *reinterpret_cast<const uint2*>(rc);
-                    bw[s][0] = vb.x; bw[s][1] = vb.y;
-                    cw_[s][0] = vc.x; cw_[s][1] = vc.y;
+                    bwA[bsel][s][0] = vb.x; bwA[bsel][s][1] = vb.y;
+                    cwA[bsel][s][0] = vc.x; cwA[bsel][s][1] = vc.y;
                 }
             }
-            float dtv[WT], duv[WT], dav[HEAD_A ? WT : 1];
 #pragma unroll
             for (int q = 0; q < WT; q += 4) {
-                const float4 a = *reinterpret_cast<const float4*>(rdt + tw + q);
+                const float4 a4 = *reinterpret_cast<const float4*>(rdt + tw + q);
                 const float4 bq = *reinterpret_cast<const float4*>(rdu + tw + q);
-                dtv[q] = a.x; dtv[q + 1] = a.y; dtv[q + 2] = a.z; dtv[q + 3] = a.w;
-                duv[q] = bq.x; duv[q + 1] = bq.y; duv[q + 2] = bq.z; duv[q + 3] = bq.w;
+                dtA[bsel][q] = a4.x; dtA[bsel][q + 1] = a4.y; dtA[bsel][q + 2] = a4.z; dtA[bsel][q + 3] = a4.w;
+                duA[bsel][q] = bq.x; duA[bsel][q + 1] = bq.y; duA[bsel][q + 2] = bq.z; duA[bsel][q + 3] = bq.w;
                 if constexpr (HEAD_A) {
                     const float4 cq = *reinterpret_cast<const float4*>(rda + tw + q);
-                    dav[q] = cq.x; dav[q + 1] = cq.y; dav[q + 2] = cq.z; dav[q + 3] = cq.w;
+                    daA[bsel][q] = cq.x; daA[bsel][q + 1] = cq.y; daA[bsel][q + 2] = cq.z; daA[bsel][q + 3] = cq.w;
                 }
             }
+        };
+        if constexpr (PF) load_window(0, 0);
+#pragma unroll
+        for (int w = 0; w < NWIN; ++w) {
+            const int tw = w * WT;
+            const int bsel = PF ? (w & 1) : 0;
+            if constexpr (PF) {
+                if (w + 1 < NWIN) load_window(w + 1, (w + 1) & 1);
+            } else {
+                load_window(w, 0);
+            }
+            const auto& bw = bwA[bsel];
+            const auto& cw_ = cwA[bsel];
+            const auto& dtv = dtA[bsel];
+            const auto& duv = duA[bsel];
+            const auto& dav = daA[bsel];
+            (void)dav;
             float yw[WT];
 #pragma unroll
             for (int tt = 0; tt < WT; ++tt) {
@@ -979,11 +1019,28 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
                 }
                 yw[tt] = y2.x + y2.y;
             }
-            int off;
-            window_reduce<WT, TPC>(yw, j, off);
-            if (j % (TPC > WT ? TPC / WT : 1) == 0) {
+            if constexpr (Cf::YLANE) {
+                // this lane's partial sums to its own row (the window lies in the columns of one lane)
+                float* yl = ry + j * Cf::YROW + tw + 4 * Cf::ysh(tw / TPT);
+                *reinterpret_cast<float4*>(yl) = make_float4(yw[0], yw[1], yw[2], yw[3]);
+                *reinterpret_cast<float4*>(yl + 4) = make_float4(yw[4], yw[5], yw[6], yw[7]);
+            } else if constexpr (Cf::YPART) {
+                // the first reduction round: the lower-half lane keeps steps 0-3 of the window
+                const bool up = (j & 4) != 0;
+                float rv[4];
 #pragma unroll
-                for (int i = 0; i < (WT >= TPC ? WT / TPC : 1); ++i) ry[tw + off + i] = yw[i];
+                for (int i = 0; i < 4; ++i) rv[i] = __shfl_xor_sync(0xffffffffu, up ? yw[i] : yw[4 + i], 4);
+                const float2 s0 = add2(up ? make_float2(yw[4], yw[5]) : make_float2(yw[0], yw[1]), make_float2(rv[0], rv[1]));
+                const float2 s1 = add2(up ? make_float2(yw[6], yw[7]) : make_float2(yw[2], yw[3]), make_float2(rv[2], rv[3]));
+                *reinterpret_cast<float4*>(ry + (j & 3) * Cf::YPROW + (up ? Cf::YHALF : 0) + tw / 2) =
+                    make_float4(s0.x, s0.y, s1.x, s1.y);
+            } else {
+                int off;
+                window_reduce<WT, TPC>(yw, j, off);
+                if (j % (TPC > WT ? TPC / WT : 1) == 0) {
+#pragma unroll
+                    for (int i = 0; i < (WT >= TPC ? WT / TPC : 1); ++i) ry[tw + off + i] = yw[i];
+                }
             }
         }
         // -------- end of a unit: the state goes to the outgoing slot (or last_state)
@@ -1012,10 +1069,58 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
                 cz.w[q] = reinterpret_cast<const uint32_t*>(zrow)[q];
             }
             float o[TPT];
+            if constexpr (Cf::YLANE) {
+                // y of this lane's steps: the sum of the channel's TPC rows, added in the tree
+                // the shuffle reduction uses (rows r and r + m for m = TPC/2, ..., 1), so both
+                // readouts round alike
+                const float* yc = ry + j * TPT + 4 * Cf::ysh(j);
 #pragma unroll
-            for (int i = 0; i < TPT; i += 4) {
-                const float4 v = *reinterpret_cast<const float4*>(ry + j * TPT + i);
-                o[i] = v.x; o[i + 1] = v.y; o[i + 2] = v.z; o[i + 3] = v.w;
+                for (int i = 0; i < TPT; i += 4) {
+                    float2 lo[TPC], hi[TPC];
+#pragma unroll
+                    for (int r = 0; r < TPC; ++r) {
+                        const float4 w4 = *reinterpret_cast<const float4*>(yc + r * Cf::YROW + i);
+                        lo[r] = make_float2(w4.x, w4.y);
+                        hi[r] = make_float2(w4.z, w4.w);
+                    }
+#pragma unroll
+                    for (int m = TPC / 2; m >= 1; m >>= 1) {
+#pragma unroll
+                        for (int r = 0; r < m; ++r) {
+                            lo[r] = add2(lo[r], lo[r + m]);
+                            hi[r] = add2(hi[r], hi[r + m]);
+                        }
+                    }
+                    o[i] = lo[0].x; o[i + 1] = lo[0].y; o[i + 2] = hi[0].x; o[i + 3] = hi[0].y;
+                }
+            } else if constexpr (Cf::YPART) {
+                // this lane's steps are window j: the 4 rows' halves, added in the shuffle tree's order
+                float4 lo[4], hi[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    lo[r] = *reinterpret_cast<const float4*>(ry + r * Cf::YPROW + 4 * j);
+                    hi[r] = *reinterpret_cast<const float4*>(ry + r * Cf::YPROW + Cf::YHALF + 4 * j);
+                }
+#pragma unroll
+                for (int m = 2; m >= 1; m >>= 1) {
+#pragma unroll
+                    for (int r = 0; r < m; ++r) {
+                        const float2 a = add2(make_float2(lo[r].x, lo[r].y), make_float2(lo[r + m].x, lo[r + m].y));
+                        const float2 b = add2(make_float2(lo[r].z, lo[r].w), make_float2(lo[r + m].z, lo[r + m].w));
+                        const float2 c = add2(make_float2(hi[r].x, hi[r].y), make_float2(hi[r + m].x, hi[r + m].y));
+                        const float2 e = add2(make_float2(hi[r].z, hi[r].w), make_float2(hi[r + m].z, hi[r + m].w));
+                        lo[r] = make_float4(a.x, a.y, b.x, b.y);
+                        hi[r] = make_float4(c.x, c.y, e.x, e.y);
+                    }
+                }
+                o[0] = lo[0].x; o[1] = lo[0].y; o[2] = lo[0].z; o[3] = lo[0].w;
+                o[4] = hi[0].x; o[5] = hi[0].y; o[6] = hi[0].z; o[7] = hi[0].w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < TPT; i += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(ry + j * TPT + i);
+                    o[i] = v.x; o[i + 1] = v.y; o[i + 2] = v.z; o[i + 3] = v.w;
+                }
             }
 #pragma unroll
             for (int i = 0; i < TPT; i += 2) {

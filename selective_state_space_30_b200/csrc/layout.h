@@ -67,7 +67,11 @@ inline int64_t layout_tiles(const ssm_dims_t& d, int ct) {
 // else the one with the most tiles.  A segment of a tile runs after the
 // previous one, so tiles are the parallelism.  The kernel is latency-bound, so
 // the order prefers many consumer warps per SM sub-partition and, among those, more
-// states per lane.  The tensor-memory layouts (bf16, N = 16, A per channel: no bf16
+// states per lane.  Measured on B200 with the current readouts (bf16, N = 16):
+// 4 x 4096 channels x 4096 steps, (16, 2) 0.449 ms, (12, 4) 0.461, (8, 4) 0.470,
+// (8, 2) 0.504; 8 x 1536 x 2048, (16, 2) 0.189, (8, 4) 0.196, (8, 2) 0.202, (12, 4)
+// 0.226 (128 tiles); 1 x 5120 x 65536, (8, 2) 2.41, (4, 4) 3.64 (before the loads
+// ahead), (4, 2) 4.08, (8, 4) 4.32 (80 tiles).  The tensor-memory layouts (bf16, N = 16, A per channel: no bf16
 // unpacking and no shared-memory traffic for B and C) come last: measured on B200
 // they run no faster than the register kernel (mamba-130m 0.206 against 0.208 ms,
 // mamba-1.4b 0.489 against 0.462 ms), and their sequence-parallel blocks (kt = 2),
@@ -79,7 +83,7 @@ inline int64_t layout_tiles(const ssm_dims_t& d, int ct) {
 inline bool choose_layout(const ssm_dims_t& d, int sm_count, int force_w, int force_spl, int force_kt,
                           int force_mode, Layout* out) {
     const bool head = head_mode(d);
-    static const int order[][4] = {{12, 4, 1, 0}, {16, 2, 1, 0}, {8, 16, 1, 0}, {8, 8, 1, 0},  {8, 4, 1, 0},
+    static const int order[][4] = {{16, 2, 1, 0}, {12, 4, 1, 0}, {8, 16, 1, 0}, {8, 8, 1, 0},  {8, 4, 1, 0},
                                    {8, 2, 1, 0},  {4, 16, 1, 0}, {4, 8, 1, 0},  {4, 4, 1, 0},  {4, 2, 1, 0},
                                    {16, 2, 1, 1}, {12, 4, 1, 1}, {8, 4, 1, 1},  {16, 2, 2, 1}, {8, 2, 2, 1}};
     bool found = false;

@@ -181,9 +181,9 @@ def test_layout_option_checks():
         assert lib.ssm_scan_set_option(plan, ssm.SSM_OPT_TIME_LANES, 2) == ssm.SSM_ERR_UNSUPPORTED
     finally:
         ssm.ssm_scan_destroy(plan)
-    # 4 x 4096 channels: twelve warps with four states per lane still fill the SMs; 1 x 5120
+    # 4 x 4096 channels: sixteen warps with two states per lane fill the SMs; 1 x 5120
     # channels: eight warps with two states per lane keep a tile per SM
-    for shape, name in (((4, 4096), "ws_bf16_n16_w12s4t1_vec"), ((1, 5120), "ws_bf16_n16_w8s2t1_vec")):
+    for shape, name in (((4, 4096), "ws_bf16_n16_w16s2t1_vec"), ((1, 5120), "ws_bf16_n16_w8s2t1_vec")):
         plan = ssm.ssm_scan_plan(ssm.make_dims(shape[0], shape[1], 256, 16, shape[1], 1, ssm.SSM_BF16), 0)
         try:
             assert ssm.ssm_scan_plan_info(plan)["variant"] == name

@@ -810,24 +810,40 @@ def run_bwd(args):
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(int(x.numel() * x.element_size()) for x in list(t.values()) + [dout] if x is not None)
 
-    def step():
-        ssm.ssm_selective_scan_bwd(dims, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"],
-                                   t["delta_bias"], True, None, dout, None, g, ws, nws, stream.cuda_stream)
+    # the forward's stored states (the training path: the backward then skips its recomputation)
+    plan = ssm.ssm_scan_plan(dims, local)
+    nblk = (d.seqlen + 31) // 32
+    ck = torch.empty((d.batch, d.dim, nblk, d.dstate), **f32)
+    fout = torch.empty_like(t["u"])
+    fwd_args = (plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"], t["delta_bias"], True, dims,
+                None, fout, None)
+    ssm.ssm_selective_scan_fwd_ckpt(*fwd_args, ck, stream.cuda_stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
+    def bwd_step(states):
+        return lambda: ssm.ssm_selective_scan_bwd_ckpt(dims, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"],
+                                                       t["z"], t["delta_bias"], True, None, dout, None, states, g,
+                                                       ws, nws, stream.cuda_stream)
+
+    def timed(step, steps):
+        for _ in range(args.warmup):
             step()
-        e1.record(stream)
         torch.cuda.synchronize(dev)
-    barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    total = max_over_ranks(e0.elapsed_time(e1), dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as clk:
+            e0.record(stream)
+            for _ in range(steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier()
+        return e0.elapsed_time(e1) / steps, max_over_ranks(e0.elapsed_time(e1), dev), clk.summary()
+
+    ms, total, clocks = timed(bwd_step(ck), args.steps)
+    ms_re, total_re, _ = timed(bwd_step(None), args.steps)
+    ms_f, _, _ = timed(lambda: ssm.ssm_selective_scan_fwd_h0(*fwd_args, stream.cuda_stream), args.steps)
+    ms_fc, _, _ = timed(lambda: ssm.ssm_selective_scan_fwd_ckpt(*fwd_args, ck, stream.cuda_stream), args.steps)
+    ssm.ssm_scan_destroy(plan)
     hbm_gbs, sm_max_mhz, src = _peaks()
     finish_ranks()
     if rank != 0:
@@ -835,9 +851,19 @@ def run_bwd(args):
     elems = d.batch * d.dim * d.seqlen
     exps = _exps(d)
     mufu_peak = SMS * EX2_PER_CLK_PER_SM * sm_max_mhz * 1e6 / 1e9
-    gexps = exps / (ms * 1e-3) / 1e9
     alg = _bwd_bytes(d)
-    gbs = alg / (ms * 1e-3) / 1e9
+    ck_bytes = int(ck.numel() * 4)
+
+    def roof(ms_, traffic_key):
+        gexps = exps / (ms_ * 1e-3) / 1e9
+        gbs = alg / (ms_ * 1e-3) / 1e9
+        return {"bound": "alu", "achieved": gexps, "peak": mufu_peak, "unit": "Gexp/s", "frac": gexps / mufu_peak,
+                "traffic": _traffic_from_profiles(w.name, key=traffic_key, sha=_src_hash(("bwd.cu",))),
+                "peak_source": f"148 SMs x 16 ex2/clk x {sm_max_mhz:.0f} MHz ({src} sm_max_mhz)",
+                "exps_per_launch": exps,
+                "hbm": {"achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                        "alg_bytes_per_launch": alg, "peak_source": src}}
+
     line = {"metric": "selective-scan backward Gelem/s (B*D*L/s) on 1 B200", "op": "bwd",
             "value": job_throughput(world, elems, args.steps, total), "unit": "Gelem/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -845,17 +871,16 @@ def run_bwd(args):
             "dtype": "f32 (bf16 I/O)" if d.dtype == "bf16" else "f32", "data": "synthetic (seeded splitmix64)",
             "config": {"workload": w.name, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen,
                        "dstate": d.dstate, "io_dtype": d.dtype, "parallelism": f"replicas x{world}",
+                       "states": f"stored by the forward (ssm_selective_scan_fwd_ckpt, {ck_bytes / 1e6:.0f} MB), "
+                                 "read by ssm_selective_scan_bwd_ckpt",
                        "l2": f"inputs {in_bytes / 1e6:.0f} MB and workspace {nws / 1e6:.0f} MB (> 126 MB L2), "
                              "no flush"},
-            "roofline": {"bound": "alu", "achieved": gexps, "peak": mufu_peak, "unit": "Gexp/s",
-                         "frac": gexps / mufu_peak,
-                         "traffic": _traffic_from_profiles(w.name, key="bwd:" + w.name,
-                                                           sha=_src_hash(("bwd.cu",))),
-                         "peak_source": f"148 SMs x 16 ex2/clk x {sm_max_mhz:.0f} MHz ({src} sm_max_mhz)",
-                         "exps_per_launch": exps,
-                         "hbm": {"achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                                 "alg_bytes_per_launch": alg, "peak_source": src}},
-            "clocks": clk.summary(), "gpu_launches": 2 * args.steps}
+            "roofline": roof(ms, "bwd_ckpt:" + w.name),
+            "recompute": {"what": "ssm_selective_scan_bwd: the backward recomputes the states itself",
+                          "ms_per_step": ms_re, "value": job_throughput(world, elems, args.steps, total_re),
+                          "roofline": roof(ms_re, "bwd:" + w.name)},
+            "forward": {"ms_plain": ms_f, "ms_with_states": ms_fc, "state_bytes": ck_bytes},
+            "clocks": clocks, "gpu_launches": 2 * args.steps}
     print(json.dumps(line), flush=True)
 
 

@@ -118,6 +118,24 @@ int ssm_selective_scan_fwd_h0(ssm_plan_t plan, const void* u, const void* delta,
                               const float* h0, void* out, float* last_state, ssm_stream_t stream);
 
 /*
+ * The forward for training: ssm_selective_scan_fwd_h0 that also stores the states the
+ * backward walks from, so that ssm_selective_scan_bwd_ckpt skips its recomputation pass
+ * ("Agent 229" page, section 4 "Activation Recomputation": checkpoints at chunk
+ * boundaries, recompute inside a chunk).  ckpt (device, fp32, required, 8-byte aligned,
+ * caller-owned) receives (batch, dim, ceil(seqlen/32), dstate): element
+ * [b][d][k][n] is the state h[n] of channel (b, d) entering step 32k (k = 0 holds h0, or
+ * zero).  About batch*dim*seqlen*dstate/8 bytes.  Every other argument and output is
+ * ssm_selective_scan_fwd_h0's, bit for bit.  The register kernels store the states; a
+ * plan on the chunked (SSD) path or forced onto the tensor-memory kernel returns
+ * SSM_ERR_UNSUPPORTED.  SSM_ERR_INVALID_ARG as ssm_selective_scan_fwd, or for ckpt NULL.
+ */
+int ssm_selective_scan_fwd_ckpt(ssm_plan_t plan, const void* u, const void* delta, const float* A,
+                                const void* B, const void* C, const float* D, const void* z,
+                                const float* delta_bias, int softplus, const ssm_dims_t* dims,
+                                const float* h0, void* out, float* last_state, float* ckpt,
+                                ssm_stream_t stream);
+
+/*
  * End-to-end variant: the same arguments as ssm_selective_scan_fwd but every
  * tensor pointer is HOST memory (pinned memory makes the copies asynchronous).
  * The plan allocates device copies on first use (kept until ssm_scan_destroy);
@@ -350,6 +368,20 @@ int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, const void* de
                            const float* delta_bias, int softplus, const float* h0, const void* dout,
                            const float* dlast, const ssm_grads_t* grads, void* workspace,
                            size_t workspace_bytes, ssm_stream_t stream);
+
+/*
+ * ssm_selective_scan_bwd given the states ssm_selective_scan_fwd_ckpt stored (ckpt, the
+ * same layout; device, 8-byte aligned, read only) for the same inputs and h0: the
+ * kernel then runs no forward recomputation units and writes no checkpoints of its own,
+ * and reads ckpt instead (the workspace size is the same).  ckpt == NULL is exactly
+ * ssm_selective_scan_bwd.  The gradients are those of ssm_selective_scan_bwd (the
+ * states it would recompute are the ones the forward stored, bit for bit).
+ */
+int ssm_selective_scan_bwd_ckpt(const ssm_dims_t* dims, const void* u, const void* delta, const float* A,
+                                const void* B, const void* C, const float* D, const void* z,
+                                const float* delta_bias, int softplus, const float* h0, const void* dout,
+                                const float* dlast, const float* ckpt, const ssm_grads_t* grads,
+                                void* workspace, size_t workspace_bytes, ssm_stream_t stream);
 
 /* Synchronise `stream` and return the kernel-side status of the last backward call that
  * used `workspace` (SSM_OK or SSM_ERR_TIMEOUT), clearing it. */

@@ -23,19 +23,23 @@ from ._abi import (SSM_BF16, SSM_ERR_BOUNDS, SSM_ERR_CUDA, SSM_ERR_INVALID_ARG, 
                    SsmError, load_library, make_dims,
                    ssm_dims_t, ssm_probe_ex2, ssm_scan_destroy, ssm_scan_device_status, ssm_scan_plan,
                    ssm_scan_plan_info, ssm_scan_plan_schedule, ssm_scan_set_option, ssm_selective_scan_fwd,
-                   ssm_selective_scan_fwd_h0, ssm_selective_scan_fwd_host, ssm_selective_scan_fwd_noalloc,
+                   ssm_selective_scan_fwd_h0, ssm_selective_scan_fwd_ckpt, ssm_selective_scan_fwd_host,
+                   ssm_selective_scan_fwd_noalloc,
                    ssm_selective_scan_noalloc_device_status, ssm_selective_scan_noalloc_test_hooks,
                    ssm_selective_state_update, ssm_causal_conv1d_fwd, ssm_selective_scan_bwd,
+                   ssm_selective_scan_bwd_ckpt,
                    ssm_selective_scan_bwd_workspace_size, ssm_selective_scan_bwd_device_status,
                    ssm_selective_scan_bwd_test_hooks, ssm_grads_t,
                    GRAD_NAMES,
                    ssm_status_string)
 
 __all__ = ["selective_scan_fwd", "selective_scan_fwd_host", "selective_scan_fn", "Plan", "get_plan", "ssm_scan_plan",
-           "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0", "ssm_selective_scan_fwd_host",
+           "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0", "ssm_selective_scan_fwd_ckpt",
+           "ssm_selective_scan_fwd_host", "ckpt_shape", "bwd_covers",
            "ssm_selective_scan_fwd_noalloc", "ssm_selective_scan_noalloc_device_status",
            "ssm_selective_scan_noalloc_test_hooks", "ssm_selective_state_update", "ssm_causal_conv1d_fwd",
-           "selective_scan_bwd", "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_workspace_size",
+           "selective_scan_bwd", "ssm_selective_scan_bwd", "ssm_selective_scan_bwd_ckpt",
+           "ssm_selective_scan_bwd_workspace_size",
            "ssm_selective_scan_bwd_device_status", "ssm_selective_scan_bwd_test_hooks",
            "ssm_scan_destroy", "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info",
            "ssm_scan_set_option", "ssm_scan_plan_schedule",
@@ -101,13 +105,30 @@ def _shapes(u, delta, A, B):
     return batch, dim, seqlen, dstate, nheads, ngroups, io
 
 
+def ckpt_shape(batch: int, dim: int, seqlen: int, dstate: int) -> Tuple[int, int, int, int]:
+    """Shape of the state checkpoints ssm_selective_scan_fwd_ckpt stores (fp32): the state
+    entering every 32-step block."""
+    return (batch, dim, (seqlen + 31) // 32, dstate)
+
+
+def bwd_covers(u, delta, A, B) -> bool:
+    """Whether ssm_selective_scan_bwd covers these inputs' shape (the per-channel layout,
+    dstate 16, dim / ngroups a multiple of 32)."""
+    if u.dim() != 3 or delta.dim() != 3 or B.dim() != 4:
+        return False
+    dim, nheads, ngroups, dstate = u.shape[1], delta.shape[1], B.shape[1], B.shape[2]
+    return nheads == dim and dstate == 16 and ngroups > 0 and (dim // ngroups) % 32 == 0
+
+
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
                        h0=None, return_last_state: bool = True, out=None, last_state=None,
-                       stream=None) -> Tuple[object, Optional[object]]:
+                       stream=None, ckpt=None) -> Tuple[object, Optional[object]]:
     """Forward scan on CUDA tensors (layouts as in include/ssm_scan.h).
 
     Returns (out, last_state); last_state is None when return_last_state is False.
-    Output tensors are allocated with torch on u's device unless given.
+    Output tensors are allocated with torch on u's device unless given.  With `ckpt`
+    (fp32, ckpt_shape(...)) the call is ssm_selective_scan_fwd_ckpt, which also stores
+    the states the backward walks from.
     """
     import torch
     batch, dim, seqlen, dstate, nheads, ngroups, io = _shapes(u, delta, A, B)
@@ -126,8 +147,15 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softp
         out = torch.empty_like(u)
     if return_last_state and last_state is None:
         last_state = torch.empty((batch, dim, dstate), dtype=torch.float32, device=u.device)
-    ssm_selective_scan_fwd_h0(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, h0, out,
-                              last_state if return_last_state else None, stream)
+    if ckpt is not None:
+        if not (ckpt.is_cuda and ckpt.is_contiguous() and ckpt.dtype == torch.float32 and
+                tuple(ckpt.shape) == ckpt_shape(batch, dim, seqlen, dstate)):
+            raise ValueError("ckpt must be a contiguous fp32 CUDA tensor of ckpt_shape(batch, dim, seqlen, dstate)")
+        ssm_selective_scan_fwd_ckpt(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, h0, out,
+                                    last_state if return_last_state else None, ckpt, stream)
+    else:
+        ssm_selective_scan_fwd_h0(plan.handle, u, delta, A, B, C, D, z, delta_bias, softplus, plan.dims, h0, out,
+                                  last_state if return_last_state else None, stream)
     return out, (last_state if return_last_state else None)
 
 
@@ -151,17 +179,19 @@ def selective_scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, 
 
 
 def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None, softplus: bool = True,
-                       h0=None, dlast=None, want_dh0: bool = False, workspace=None, stream=None) -> dict:
+                       h0=None, dlast=None, want_dh0: bool = False, workspace=None, stream=None, ckpt=None) -> dict:
     """Gradients of the forward scan on CUDA tensors (see include/ssm_scan.h,
     ssm_selective_scan_bwd).  Returns a dict over GRAD_NAMES: du, ddelta, dz in
     u's dtype; dA, dB, dC, dD, ddelta_bias, dh0 fp32 (dz None without z, dh0
     only with want_dh0; dD and ddelta_bias are the gradients at D = 0 / bias = 0
     when those are not given).  The workspace is allocated with torch unless
-    given (uint8, at least ssm_selective_scan_bwd_workspace_size bytes)."""
+    given (uint8, at least ssm_selective_scan_bwd_workspace_size bytes).  `ckpt`: the
+    states selective_scan_fwd stored for the same inputs (the backward then skips
+    recomputing them), or None."""
     import torch
     batch, dim, seqlen, dstate, nheads, ngroups, io = _shapes(u, delta, A, B)
     for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("dout", dout), ("D", D),
-                    ("z", z), ("delta_bias", delta_bias), ("h0", h0), ("dlast", dlast)):
+                    ("z", z), ("delta_bias", delta_bias), ("h0", h0), ("dlast", dlast), ("ckpt", ckpt)):
         if t is not None:
             if not t.is_cuda:
                 raise ValueError(f"{name} must be a CUDA tensor")
@@ -179,8 +209,8 @@ def selective_scan_bwd(u, delta, A, B, C, dout, D=None, z=None, delta_bias=None,
          "dh0": torch.empty((batch, dim, dstate), **f32) if want_dh0 else None}
     if stream is None:
         stream = torch.cuda.current_stream(u.device).cuda_stream
-    ssm_selective_scan_bwd(dims, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dout, dlast, g, workspace,
-                           workspace.numel() * workspace.element_size(), stream)
+    ssm_selective_scan_bwd_ckpt(dims, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dout, dlast, ckpt, g,
+                                workspace, workspace.numel() * workspace.element_size(), stream)
     return g
 
 
@@ -198,17 +228,23 @@ def _selective_scan_function():
     class SelectiveScanFn(torch.autograd.Function):
         @staticmethod
         def forward(ctx, u, delta, A, B, C, D, z, delta_bias, h0, softplus):
-            out, last = selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, h0=h0)
-            ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, h0)
+            # where the backward covers the shape, the forward stores the states it walks from
+            ck = None
+            if any(ctx.needs_input_grad) and bwd_covers(u, delta, A, B) and u.numel() > 0:
+                ck = torch.empty(ckpt_shape(u.shape[0], u.shape[1], u.shape[2], B.shape[2]),
+                                 dtype=torch.float32, device=u.device)
+            out, last = selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, h0=h0, ckpt=ck)
+            ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, h0, ck)
             ctx.softplus = softplus
             return out, last
 
         @staticmethod
         def backward(ctx, dout, dlast):
-            u, delta, A, B, C, D, z, delta_bias, h0 = ctx.saved_tensors
+            u, delta, A, B, C, D, z, delta_bias, h0, ck = ctx.saved_tensors
             want_dh0 = h0 is not None and ctx.needs_input_grad[8]
             g = selective_scan_bwd(u, delta, A, B, C, dout.contiguous(), D, z, delta_bias, ctx.softplus, h0=h0,
-                                   dlast=dlast.contiguous() if dlast is not None else None, want_dh0=want_dh0)
+                                   dlast=dlast.contiguous() if dlast is not None else None, want_dh0=want_dh0,
+                                   ckpt=ck)
             return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype),
                     g["dD"] if D is not None else None, g["dz"], g["ddelta_bias"] if delta_bias is not None else None,
                     g["dh0"], None)

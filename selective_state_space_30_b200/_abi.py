@@ -26,11 +26,11 @@ SSM_BF16 = 1
 
 # every exported symbol declared in include/ssm_scan.h
 EXPORTS = ("ssm_scan_plan", "ssm_selective_scan_fwd", "ssm_selective_scan_fwd_h0",
-           "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc",
+           "ssm_selective_scan_fwd_ckpt", "ssm_selective_scan_fwd_host", "ssm_selective_scan_fwd_noalloc",
            "ssm_selective_scan_noalloc_device_status", "ssm_selective_scan_noalloc_test_hooks",
            "ssm_selective_state_update",
            "ssm_causal_conv1d_fwd", "ssm_selective_scan_bwd_workspace_size", "ssm_selective_scan_bwd",
-           "ssm_selective_scan_bwd_device_status", "ssm_selective_scan_bwd_test_hooks",
+           "ssm_selective_scan_bwd_ckpt", "ssm_selective_scan_bwd_device_status", "ssm_selective_scan_bwd_test_hooks",
            "ssm_scan_set_option",
            "ssm_scan_plan_schedule", "ssm_scan_destroy",
            "ssm_scan_device_status", "ssm_status_string", "ssm_scan_plan_info", "ssm_probe_ex2")
@@ -85,6 +85,7 @@ def load_library(path: Optional[str] = None):
     lib.ssm_scan_plan.argtypes = [ctypes.POINTER(vp), dims_p, i32]
     lib.ssm_selective_scan_fwd.argtypes = fwd_args + [vp, vp, vp]
     lib.ssm_selective_scan_fwd_h0.argtypes = fwd_args + [vp, vp, vp, vp]
+    lib.ssm_selective_scan_fwd_ckpt.argtypes = fwd_args + [vp, vp, vp, vp, vp]
     lib.ssm_selective_scan_fwd_host.argtypes = fwd_args + [vp, vp, vp]
     lib.ssm_selective_scan_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, dims_p, vp, vp, vp]
     lib.ssm_selective_scan_noalloc_device_status.argtypes = [vp]
@@ -94,6 +95,8 @@ def load_library(path: Optional[str] = None):
     lib.ssm_selective_scan_bwd_workspace_size.argtypes = [dims_p, ctypes.POINTER(ctypes.c_size_t)]
     lib.ssm_selective_scan_bwd.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
                                            ctypes.POINTER(ssm_grads_t), vp, ctypes.c_size_t, vp]
+    lib.ssm_selective_scan_bwd_ckpt.argtypes = [dims_p, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp,
+                                                ctypes.POINTER(ssm_grads_t), vp, ctypes.c_size_t, vp]
     lib.ssm_selective_scan_bwd_device_status.argtypes = [vp, vp]
     lib.ssm_selective_scan_bwd_test_hooks.argtypes = [i32, i64]
     lib.ssm_scan_destroy.argtypes = [vp]
@@ -173,6 +176,14 @@ def ssm_selective_scan_fwd_h0(plan: int, u, delta, A, B, C, D, z, delta_bias, so
     return _check(rc, "ssm_selective_scan_fwd_h0") if check else rc
 
 
+def ssm_selective_scan_fwd_ckpt(plan: int, u, delta, A, B, C, D, z, delta_bias, softplus: bool, dims: ssm_dims_t,
+                                h0, out, last_state, ckpt, stream=None, check: bool = True) -> int:
+    rc = load_library().ssm_selective_scan_fwd_ckpt(
+        plan, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if softplus else 0, ctypes.byref(dims), _ptr(h0), _ptr(out), _ptr(last_state), _ptr(ckpt), _stream(stream))
+    return _check(rc, "ssm_selective_scan_fwd_ckpt") if check else rc
+
+
 def ssm_selective_scan_fwd_host(plan: int, u, delta, A, B, C, D, z, delta_bias, softplus: bool,
                                 dims: ssm_dims_t, out, last_state, stream=None, check: bool = True) -> int:
     rc = load_library().ssm_selective_scan_fwd_host(
@@ -237,6 +248,18 @@ def ssm_selective_scan_bwd(dims: ssm_dims_t, u, delta, A, B, C, D, z, delta_bias
         1 if softplus else 0, _ptr(h0), _ptr(dout), _ptr(dlast), ctypes.byref(g), _ptr(workspace),
         int(workspace_bytes), _stream(stream))
     return _check(rc, "ssm_selective_scan_bwd") if check else rc
+
+
+def ssm_selective_scan_bwd_ckpt(dims: ssm_dims_t, u, delta, A, B, C, D, z, delta_bias, softplus: bool, h0, dout,
+                                dlast, ckpt, grads: dict, workspace, workspace_bytes: int, stream=None,
+                                check: bool = True) -> int:
+    """ssm_selective_scan_bwd given the forward's stored states (ckpt; None = recompute them)."""
+    g = ssm_grads_t(*[_ptr(grads.get(k)) for k in GRAD_NAMES])
+    rc = load_library().ssm_selective_scan_bwd_ckpt(
+        ctypes.byref(dims), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+        1 if softplus else 0, _ptr(h0), _ptr(dout), _ptr(dlast), _ptr(ckpt), ctypes.byref(g), _ptr(workspace),
+        int(workspace_bytes), _stream(stream))
+    return _check(rc, "ssm_selective_scan_bwd_ckpt") if check else rc
 
 
 def ssm_selective_scan_bwd_device_status(workspace, stream=None) -> int:

@@ -138,9 +138,10 @@ int schedule(ssm_plan_s* p) {
 
 int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A, const void* B, const void* C,
                const float* D, const void* z, const float* delta_bias, int softplus, const float* h0, void* out,
-               float* last_state, cudaStream_t stream) {
+               float* last_state, cudaStream_t stream, float* ckpt = nullptr) {
     const ssm_dims_t& d = plan->dims;
     if (d.batch == 0) return SSM_OK;
+    if (plan->ssd && ckpt) return SSM_ERR_UNSUPPORTED;   // the chunked path stores no per-block states
     if (plan->ssd) {
         // the chunked tensor-core path: 16-byte aligned TMA sources, 8-byte aligned delta rows
         ssm::SsdMaps maps;
@@ -171,7 +172,7 @@ int launch_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A
         // an unaligned call takes the scan kernel below
     }
     // the scan kernel (also an SSD-eligible call whose pointers the SSD path cannot take)
-    const ssm::FwdArgs a{u, delta, A, B, C, D, z, delta_bias, softplus, h0, out, last_state};
+    const ssm::FwdArgs a{u, delta, A, B, C, D, z, delta_bias, softplus, h0, out, last_state, ckpt};
     return ssm::fwd_launch(d, plan->geom, a, plan->ws, plan->spin_limit, stream);
 }
 }  // namespace
@@ -317,6 +318,18 @@ int ssm_selective_scan_fwd_h0(ssm_plan_t plan, const void* u, const void* delta,
     if (set_device(plan->device) != SSM_OK) return SSM_ERR_CUDA;
     return launch_fwd(plan, u, delta, A, B, C, D, z, delta_bias, softplus, h0, out, last_state,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ssm_selective_scan_fwd_ckpt(ssm_plan_t plan, const void* u, const void* delta, const float* A, const void* B,
+                                const void* C, const float* D, const void* z, const float* delta_bias,
+                                int softplus, const ssm_dims_t* dims, const float* h0, void* out, float* last_state,
+                                float* ckpt, ssm_stream_t stream) {
+    if (!plan_ok(plan) || !dims || !same_dims(dims, &plan->dims) || !ckpt) return SSM_ERR_INVALID_ARG;
+    if (plan->dims.batch > 0 && plan->dims.seqlen > 0 && (!u || !delta || !B || !C || !out)) return SSM_ERR_INVALID_ARG;
+    if (!A) return SSM_ERR_INVALID_ARG;
+    if (set_device(plan->device) != SSM_OK) return SSM_ERR_CUDA;
+    return launch_fwd(plan, u, delta, A, B, C, D, z, delta_bias, softplus, h0, out, last_state,
+                      reinterpret_cast<cudaStream_t>(stream), ckpt);
 }
 
 int ssm_selective_scan_fwd(ssm_plan_t plan, const void* u, const void* delta, const float* A, const void* B,

@@ -70,7 +70,8 @@ struct BwdParams {
     int* status;                 // kernel-side ssm_status_t
     unsigned *flag1, *flag2;     // [tile][seg]: forward / reverse segment done (zeroed before the launch)
     float *carry1, *carry2;      // [tile][seg][kCT][kN]: state after / state gradient before a segment
-    float* ckpt;                 // checkpoints [tile][block][kCT][kN]
+    float* ckpt;                 // checkpoints [b * dim + d][block][kN]: the state entering each 32-step block
+    int ext_ckpt;                // 1: ckpt holds the forward's states; no forward units run
     float *dB, *dC;              // the outputs (batch, groups, kN, L), zeroed before the launch
     int red_vec;                 // 16-byte atomic adds into dB, dC (L % 4 == 0, aligned bases)
     float *dAp, *dDp, *dbp;      // per segment and (b, d) row: [seg][row][kN], [seg][row], [seg][row]
@@ -237,15 +238,16 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                        reinterpret_cast<uintptr_t>(p.B) | reinterpret_cast<uintptr_t>(p.C)) & 15u) == 0;
     const int nblk = (int)((L + kBT - 1) / kBT);
     const int64_t per_pass = p.ntiles * p.nseg;
+    const int64_t nfwd = p.ext_ckpt ? 0 : per_pass;   // forward units come first, when they run
 
     for (;;) {
         __syncthreads();   // the previous unit is done with shared memory and s_ticket
         if (tid == 0) s_ticket = atomicAdd(p.ticket, 1u);
         __syncthreads();
         const int64_t k = s_ticket;
-        if (k >= 2 * per_pass) break;
-        const bool fwd = k < per_pass;
-        const int64_t kk = fwd ? k : k - per_pass;
+        if (k >= nfwd + per_pass) break;
+        const bool fwd = k < nfwd;
+        const int64_t kk = fwd ? k : k - nfwd;
         const int seg = fwd ? (int)(kk / p.ntiles) : p.nseg - 1 - (int)(kk / p.ntiles);
         const int64_t tile = kk % p.ntiles;        // = b * tiles_per_row + tile in the row
         const int64_t b = tile / p.tiles_per_row;
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         const T* go = static_cast<const T*>(p.dout) + row0 * L;
         const T* Bg = static_cast<const T*>(p.B) + (b * G + g) * kN * L;
         const T* Cg = static_cast<const T*>(p.C) + (b * G + g) * kN * L;
-        float* ckpt = p.ckpt + tile * (int64_t)nblk * kCT * kN;
+        float* ckpt = p.ckpt + (row0 + c) * (int64_t)nblk * kN + 2 * j;   // this thread's states, block 0
         const int blk0 = seg * p.seg_blocks;
         const int blk1 = min(nblk, blk0 + p.seg_blocks);
         const int64_t us = tile * p.nseg + seg;    // this unit's flag / carry slot
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             const unsigned* need[2] = {nullptr, nullptr};
             if (fwd && seg > 0) need[0] = p.flag1 + us - 1;
             if (!fwd) {
-                need[0] = p.flag1 + us;
+                if (!p.ext_ckpt) need[0] = p.flag1 + us;
                 if (seg + 1 < p.nseg) need[1] = p.flag2 + us + 1;
             }
             for (int w = 0; w < 2; ++w) {
@@ -334,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 // the next block's rows go into the other buffer, read last by the previous block
                 if (blk + 1 < blk1) issue_fwd(stage_base + (cur ^ 1) * S::kStageBytes, t0 + kBT);
                 __syncthreads();
-                *reinterpret_cast<float2*>(ckpt + ((int64_t)blk * kCT + c) * kN + 2 * j) = h;
+                *reinterpret_cast<float2*>(ckpt + (int64_t)blk * kN) = h;
 #pragma unroll
                 for (int w = 0; w < kBT / kWin; ++w) {
 #pragma unroll 4
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         float* dCg = p.dC + (b * G + g) * kN * L;
         const bool rvec = p.red_vec != 0;
         // the checkpoint of the block being walked (the next, earlier one is fetched a block ahead)
-        float2 hblk = __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)(blk1 - 1) * kCT + c) * kN + 2 * j));
+        float2 hblk = __ldcg(reinterpret_cast<const float2*>(ckpt + (int64_t)(blk1 - 1) * kN));
         auto issue_rev = [&](unsigned char* sg, int64_t ts) {
             stage_rows<T>(sg, u, L, kCT, ts, L, vec, tid);
             stage_rows<T>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
@@ -419,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             __syncthreads();
 
             const float2 hprev =
-                blk > blk0 ? __ldcg(reinterpret_cast<const float2*>(ckpt + ((int64_t)(blk - 1) * kCT + c) * kN + 2 * j))
+                blk > blk0 ? __ldcg(reinterpret_cast<const float2*>(ckpt + (int64_t)(blk - 1) * kN))
                            : make_float2(0.f, 0.f);
             // the states entering the four windows, by the recurrence from the block checkpoint
             // (kept in shared memory, one float2 per thread and window)
@@ -607,7 +609,7 @@ WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
     w.carry1 = w.zero_end;
     w.carry2 = align256(w.carry1 + slots * kCT * kN * 4);
     w.ckpt = align256(w.carry2 + slots * kCT * kN * 4);
-    w.dAp = align256(w.ckpt + ntiles * nblk * kCT * kN * 4);
+    w.dAp = align256(w.ckpt + ntiles * kCT * nblk * kN * 4);
     w.dDp = align256(w.dAp + (int64_t)s.nseg * rows * kN * 4);
     w.dbp = align256(w.dDp + (int64_t)s.nseg * rows * 4);
     w.total = align256(w.dbp + (int64_t)s.nseg * rows * 4);
@@ -722,6 +724,16 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
                                       const float* delta_bias, int softplus, const float* h0, const void* dout,
                                       const float* dlast, const ssm_grads_t* grads, void* workspace,
                                       size_t workspace_bytes, ssm_stream_t stream) {
+    return ssm_selective_scan_bwd_ckpt(dims, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dout, dlast, nullptr,
+                                       grads, workspace, workspace_bytes, stream);
+}
+
+extern "C" int ssm_selective_scan_bwd_ckpt(const ssm_dims_t* dims, const void* u, const void* delta, const float* A,
+                                           const void* B, const void* C, const float* D, const void* z,
+                                           const float* delta_bias, int softplus, const float* h0,
+                                           const void* dout, const float* dlast, const float* ckpt,
+                                           const ssm_grads_t* grads, void* workspace, size_t workspace_bytes,
+                                           ssm_stream_t stream) {
     using namespace ssm;
     const int rc = check_dims(dims);
     if (rc != SSM_OK) return rc;
@@ -757,7 +769,8 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     if (!workspace || workspace_bytes < (size_t)w.total) return SSM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) || (reinterpret_cast<uintptr_t>(A) & 7u) ||
         (h0 && (reinterpret_cast<uintptr_t>(h0) & 7u)) || (dlast && (reinterpret_cast<uintptr_t>(dlast) & 7u)) ||
-        (grads->dh0 && (reinterpret_cast<uintptr_t>(grads->dh0) & 7u)))
+        (grads->dh0 && (reinterpret_cast<uintptr_t>(grads->dh0) & 7u)) ||
+        (ckpt && (reinterpret_cast<uintptr_t>(ckpt) & 7u)))
         return SSM_ERR_UNSUPPORTED;
     BwdParams prm;
     prm.u = u; prm.delta = delta; prm.z = z; prm.dout = dout; prm.B = B; prm.C = C;
@@ -770,7 +783,9 @@ extern "C" int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, con
     prm.flag2 = reinterpret_cast<unsigned*>(ws + w.flag2);
     prm.carry1 = reinterpret_cast<float*>(ws + w.carry1);
     prm.carry2 = reinterpret_cast<float*>(ws + w.carry2);
-    prm.ckpt = reinterpret_cast<float*>(ws + w.ckpt);
+    // the forward's states when given (read only), else the kernel's own checkpoints in the workspace
+    prm.ckpt = ckpt ? const_cast<float*>(ckpt) : reinterpret_cast<float*>(ws + w.ckpt);
+    prm.ext_ckpt = ckpt ? 1 : 0;
     prm.dB = static_cast<float*>(grads->dB);
     prm.dC = static_cast<float*>(grads->dC);
     prm.red_vec = dims->seqlen % 4 == 0 &&

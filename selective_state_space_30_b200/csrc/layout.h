@@ -206,6 +206,7 @@ struct FwdArgs {
     const float* h0;
     void* out;
     float* last_state;
+    float* ckpt = nullptr;   // states entering every 32-step block (register kernel only)
 };
 
 // Launch the scan kernel of geometry `g` on workspace `ws` (laid out as FwdGeom says).
@@ -245,6 +246,7 @@ inline int fwd_launch(const ssm_dims_t& d, const FwdGeom& g, const FwdArgs& a, u
     Variant v;
     if (!pick_variant(d.io_dtype, d.dstate, head_mode(d), vec, g.lay.w, g.lay.spl, g.lay.kt, g.lay.mode, &v))
         return SSM_ERR_UNSUPPORTED;
+    if (a.ckpt && g.lay.mode != 0) return SSM_ERR_UNSUPPORTED;   // the tensor-memory kernel stores none
     FwdParams prm;
     prm.u = a.u; prm.delta = a.delta; prm.A = a.A; prm.B = a.B; prm.C = a.C; prm.D = a.D; prm.z = a.z;
     prm.bias = a.delta_bias; prm.h0 = a.h0; prm.out = a.out; prm.last_state = a.last_state;
@@ -261,6 +263,8 @@ inline int fwd_launch(const ssm_dims_t& d, const FwdGeom& g, const FwdArgs& a, u
     prm.n_ctas = (unsigned)g.ctas;
     prm.spin_limit = spin_limit;
     prm.delta_rows = delta_rows;
+    prm.ckpt = a.ckpt;
+    prm.ckpt_blocks = (d.seqlen + 31) / 32;
     if (v.smem > 48 * 1024 &&
         cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
         return SSM_ERR_CUDA;

@@ -96,6 +96,10 @@ struct FwdParams {
     unsigned n_ctas;
     unsigned spin_limit;
     int delta_rows;    // rows of the delta box: CT (S6 layout) or the heads a tile can touch
+    // optional (register kernel): the state entering every 32-step block, for the backward,
+    // at ckpt[((b * dim + d) * ckpt_blocks + t / 32) * N + n]; nullptr: not stored
+    float* ckpt;
+    int64_t ckpt_blocks;
 };
 
 // The five 2-D tensor maps (time x rows) the producer loads boxes through.
@@ -988,6 +992,13 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
                 if (w + 1 < NWIN) load_window(w + 1, (w + 1) & 1);
             } else {
                 load_window(w, 0);
+            }
+            // the state entering a 32-step block, for the backward (blocks start on 32-step bounds)
+            if ((tw & 31) == 0 && p.ckpt && ok && t0 + tw < hd.t1 &&
+                in_bounds(hd.b < p.batch && d < Dm && t0 + tw < L, status)) {
+                float* cp = p.ckpt + ((hd.b * Dm + d) * p.ckpt_blocks + (t0 + tw) / 32) * N;
+#pragma unroll
+                for (int s = 0; s < S; ++s) cp[s * TPC + j] = h[s];
             }
             const auto& bw = bwA[bsel];
             const auto& cw_ = cwA[bsel];

@@ -180,3 +180,124 @@ def test_bwd_wait_timeout_reports_and_recovers():
     assert ssm.ssm_selective_scan_bwd_device_status(ws) == ssm.SSM_OK
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"])
     check_grads(g, ref, mag, dims.dtype)
+
+
+# ------------------------------------------------- the forward's stored states
+
+def _prefix_states(dims, inp, h0):
+    """The oracle's state entering every 32-step block: h0 (or zero) for block 0, else the
+    last state of the oracle run over the first 32k steps."""
+    nblk = (dims.seqlen + 31) // 32
+    ref = np.zeros((dims.batch, dims.dim, nblk, dims.dstate))
+    ref[:, :, 0] = h0 if h0 is not None else 0.0
+    for k in range(1, nblk):
+        t = 32 * k
+        dk = si.Dims(dims.batch, dims.dim, t, dims.dstate, dims.nheads, dims.ngroups, dims.dtype)
+        pre = dict(inp)
+        for key in ("u", "delta", "z", "B", "C"):
+            if pre.get(key) is not None:
+                pre[key] = np.ascontiguousarray(pre[key][..., :t])
+        _, last, _ = oracle.run_inputs(dk, pre, h0=h0)
+        ref[:, :, k] = last
+    return ref
+
+
+def _fwd_ckpt(dims, inp, h0=None, opts=None):
+    """ssm_selective_scan_fwd_ckpt through the C ABI on a plan with the given options;
+    returns (out, last_state, ckpt) and the plain forward's (out, last_state)."""
+    import selective_state_space_30_b200 as ssm
+    from parity import OPTION_CODES
+    io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
+    d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, io)
+    dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    h0d = to_device(np.ascontiguousarray(h0, dtype=np.float32)) if h0 is not None else None
+    nblk = (dims.seqlen + 31) // 32
+    ck = torch.full((dims.batch, dims.dim, nblk, dims.dstate), float("nan"), device="cuda")
+    res = []
+    plan = ssm.ssm_scan_plan(d, 0)
+    try:
+        for k, v in (opts or {}).items():
+            ssm.ssm_scan_set_option(plan, OPTION_CODES[k], v)
+        for with_ckpt in (True, False):
+            out = torch.empty_like(dev["u"])
+            last = torch.empty((dims.batch, dims.dim, dims.dstate), dtype=torch.float32, device="cuda")
+            args = (plan, dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"], dev["z"],
+                    dev["delta_bias"], True, d, h0d, out, last)
+            if with_ckpt:
+                ssm.ssm_selective_scan_fwd_ckpt(*args, ck)
+            else:
+                ssm.ssm_selective_scan_fwd_h0(*args)
+            assert ssm.ssm_scan_device_status(plan) == ssm.SSM_OK
+            res.append((out, last))
+        torch.cuda.synchronize()
+    finally:
+        ssm.ssm_scan_destroy(plan)
+    return res[0], res[1], ck
+
+
+CKPT_CASES = [
+    (si.Dims(2, 64, 300, 16, dtype="bf16"), None),                                   # the plan's layout
+    (si.Dims(2, 64, 300, 16, dtype="bf16"), dict(tensor_memory=1, warps=8, states_per_lane=2)),   # per-lane rows
+    (si.Dims(1, 32, 640, 16, dtype="bf16"), dict(tensor_memory=1, warps=8, states_per_lane=2, seg_len=128)),
+    (si.Dims(2, 96, 200, 16, dtype="bf16"), dict(tensor_memory=1, warps=12, states_per_lane=4)),  # shuffles
+    (si.Dims(1, 32, 100, 16, dtype="f32"), None),                                    # 32-step blocks
+    (si.Dims(2, 64, 129, 8, dtype="bf16"), None),                                    # another dstate
+]
+
+
+@pytest.mark.parametrize("case", CKPT_CASES, ids=lambda c: f"{c[0].batch}x{c[0].dim}x{c[0].seqlen}n{c[0].dstate}"
+                                                           f"{c[0].dtype}-{'plan' if c[1] is None else c[1]['warps']}")
+def test_forward_stores_block_states(case):
+    """ssm_selective_scan_fwd_ckpt: outputs bit-equal to the plain forward, and every stored
+    state (block k: the state entering step 32k) equal, within the forward's state bound,
+    to the oracle's last state over the first 32k steps (block 0: h0)."""
+    dims, opts = case
+    inp = si.make_inputs(dims, _recipe("c2"), 51)
+    h0 = si.make_grad_inputs(dims, 52, h0=True)["h0"]
+    (out, last), (out0, last0), ck = _fwd_ckpt(dims, inp, h0, opts)
+    assert torch.equal(out, out0) and torch.equal(last, last0)
+    ref = _prefix_states(dims, inp, h0)
+    from parity import check_state
+    check_state(to_host_f64(ck), ref, what="stored states")
+
+
+def test_forward_checkpoints_refused_off_the_register_kernel():
+    import selective_state_space_30_b200 as ssm
+    dims = si.Dims(2, 64, 256, 16, dtype="bf16")
+    inp = si.make_inputs(dims, _recipe("c2"), 53)
+    with pytest.raises(ssm.SsmError):
+        _fwd_ckpt(dims, inp, None, dict(tensor_memory=2))
+
+
+@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[7], CASES[8]],
+                         ids=["2x64x100bf16", "2x64x77f32", "1x32x1000bf16", "2x64x777f32"])
+def test_bwd_with_forward_states(case):
+    """ssm_selective_scan_bwd_ckpt with the states the forward stored: every gradient but dB
+    and dC bit-equal to the backward that recomputes them (the same states, the same
+    arithmetic), dB and dC within the rounding of their atomic sums, and all within the
+    oracle's bound."""
+    import selective_state_space_30_b200 as ssm
+    dims, kind, dlast, h0, softplus = case
+    inp = si.make_inputs(dims, _recipe(kind), 41)
+    gin = si.make_grad_inputs(dims, 42, dlast=dlast, h0=h0)
+    _, _, ck = _fwd_ckpt(dims, inp, gin.get("h0"))
+    dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
+    d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, io)
+    ws = torch.empty(ssm.ssm_selective_scan_bwd_workspace_size(d), dtype=torch.uint8, device="cuda")
+    g = ssm.selective_scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], to_device(gin["dout"]),
+                               dev["D"], dev["z"], dev["delta_bias"], True, h0=to_device(gin.get("h0")),
+                               dlast=to_device(gin.get("dlast")), want_dh0=True, workspace=ws, ckpt=ck)
+    assert ssm.ssm_selective_scan_bwd_device_status(ws) == ssm.SSM_OK
+    torch.cuda.synchronize()
+    g0 = run_bwd(dims, inp, gin, want_dh0=True)
+    for k in g:
+        if g[k] is None:
+            continue
+        if k in ("dB", "dC"):
+            scale = float(torch.max(torch.abs(g0[k]))) + 1.0
+            assert float(torch.max(torch.abs(g[k] - g0[k]))) <= 1e-5 * scale, f"{k} differs beyond rounding"
+        else:
+            assert torch.equal(g[k], g0[k]), f"{k} differs from the recomputing backward"
+    ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin["dlast"], h0=gin["h0"], want_dh0=True)
+    check_grads(g, ref, mag, dims.dtype)

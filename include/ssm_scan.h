@@ -125,9 +125,10 @@ int ssm_selective_scan_fwd_h0(ssm_plan_t plan, const void* u, const void* delta,
  * caller-owned) receives (batch, dim, ceil(seqlen/32), dstate): element
  * [b][d][k][n] is the state h[n] of channel (b, d) entering step 32k (k = 0 holds h0, or
  * zero).  About batch*dim*seqlen*dstate/8 bytes.  Every other argument and output is
- * ssm_selective_scan_fwd_h0's, bit for bit.  The register kernels store the states; a
- * plan on the chunked (SSD) path or forced onto the tensor-memory kernel returns
- * SSM_ERR_UNSUPPORTED.  SSM_ERR_INVALID_ARG as ssm_selective_scan_fwd, or for ckpt NULL.
+ * ssm_selective_scan_fwd_h0's, bit for bit.  Covered: the shapes the backward covers
+ * (the S6 layout, nheads == dim, with dstate 16), on the register kernel; another shape, or
+ * a plan forced onto the tensor-memory kernel, returns SSM_ERR_UNSUPPORTED.
+ * SSM_ERR_INVALID_ARG as ssm_selective_scan_fwd, or for ckpt NULL.
  */
 int ssm_selective_scan_fwd_ckpt(ssm_plan_t plan, const void* u, const void* delta, const float* A,
                                 const void* B, const void* C, const float* D, const void* z,

@@ -243,10 +243,13 @@ inline int fwd_launch(const ssm_dims_t& d, const FwdGeom& g, const FwdArgs& a, u
                           bc_swz, tb);
         // a shape the tensor maps cannot describe takes the element-copy path
     }
+    // with stored states: the register kernel's mode-2 variant of the same layout (the
+    // tensor-memory kernel stores none)
+    if (a.ckpt && g.lay.mode != 0) return SSM_ERR_UNSUPPORTED;
     Variant v;
-    if (!pick_variant(d.io_dtype, d.dstate, head_mode(d), vec, g.lay.w, g.lay.spl, g.lay.kt, g.lay.mode, &v))
+    if (!pick_variant(d.io_dtype, d.dstate, head_mode(d), vec, g.lay.w, g.lay.spl, g.lay.kt, a.ckpt ? 2 : g.lay.mode,
+                      &v))
         return SSM_ERR_UNSUPPORTED;
-    if (a.ckpt && g.lay.mode != 0) return SSM_ERR_UNSUPPORTED;   // the tensor-memory kernel stores none
     FwdParams prm;
     prm.u = a.u; prm.delta = a.delta; prm.A = a.A; prm.B = a.B; prm.C = a.C; prm.D = a.D; prm.z = a.z;
     prm.bias = a.delta_bias; prm.h0 = a.h0; prm.out = a.out; prm.last_state = a.last_state;

@@ -189,6 +189,12 @@ __device__ __forceinline__ float2 silu2(float2 z) {
 
 __device__ __forceinline__ float silu1(float z) { return z * rcp_approx(ex2_approx(z * -kLog2e) + 1.f); }
 
+// a global store that only lanes with c set perform (a predicated store, no branch)
+__device__ __forceinline__ void st_global_if(float* p, float v, bool c) {
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q st.global.f32 [%0], %1;\n\t}" ::"l"(p), "f"(v),
+                 "r"((int)c));
+}
+
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -800,7 +806,8 @@ __device__ __forceinline__ void produce(const FwdParams& p, const TensorMaps& tm
 
 // ------------------------------------------------------------------- kernel
 
-template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC>
+// CKPT: also store the state entering every 32-step block (p.ckpt, for the backward)
+template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC, bool CKPT>
 __global__ void __launch_bounds__(Cfg<T, N, W, HEAD_A, SPL>::THREADS, 1)
 scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
     using Cf = Cfg<T, N, W, HEAD_A, SPL>;
@@ -905,6 +912,16 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
         const unsigned char* drow = sb + Cf::OFF_IN + (CT + drow_i) * RB + j * TPT * ESZ;
         const unsigned char* zrow = sb + Cf::OFF_IN + (2 * CT + lc) * RB + j * TPT * ESZ;
         const bool full_blk = t0 + TB <= hd.t1;
+        // the backward's stored states (CKPT): this lane's first state entering each 32-step
+        // part of the block, and whether that part lies in the unit
+        static_assert(TB == 32 || TB == 64, "32-step parts of a block");
+        float* ckp = nullptr;
+        bool ck0 = false, ck1 = false;
+        if constexpr (CKPT) {
+            ckp = p.ckpt + ((hd.b * Dm + d) * p.ckpt_blocks + t0 / 32) * N + j;
+            ck0 = ok && in_bounds(hd.b < p.batch && d < Dm && t0 < L, status);
+            ck1 = ck0 && t0 + 32 < hd.t1;
+        }
         // -------- prologue: dt, dt*u (dA) of this lane's steps, two at a time
         {
             Chunk<T, TPT> cu, cd;
@@ -993,12 +1010,12 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             } else {
                 load_window(w, 0);
             }
-            // the state entering a 32-step block, for the backward (blocks start on 32-step bounds)
-            if ((tw & 31) == 0 && p.ckpt && ok && t0 + tw < hd.t1 &&
-                in_bounds(hd.b < p.batch && d < Dm && t0 + tw < L, status)) {
-                float* cp = p.ckpt + ((hd.b * Dm + d) * p.ckpt_blocks + (t0 + tw) / 32) * N;
+            // the state entering a 32-step block, for the backward (blocks start on 32-step
+            // bounds).  Predicated stores, not a branch: the unrolled windows stay one stretch
+            // of straight-line code for the scheduler.
+            if (CKPT && (tw & 31) == 0) {
 #pragma unroll
-                for (int s = 0; s < S; ++s) cp[s * TPC + j] = h[s];
+                for (int s = 0; s < S; ++s) st_global_if(ckp + (tw / 32) * N + s * TPC, h[s], tw == 0 ? ck0 : ck1);
             }
             const auto& bw = bwA[bsel];
             const auto& cw_ = cwA[bsel];
@@ -1713,10 +1730,10 @@ struct Variant {
     const char* name;
 };
 
-template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC>
+template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC, bool CKPT = false>
 Variant make_variant(const char* name) {
     using C = Cfg<T, N, W, HEAD_A, SPL>;
-    return Variant{scan_fwd_kernel<T, N, W, HEAD_A, SPL, VEC>, C::SMEM, C::THREADS, C::CT, N, C::TB, name};
+    return Variant{scan_fwd_kernel<T, N, W, HEAD_A, SPL, VEC, CKPT>, C::SMEM, C::THREADS, C::CT, N, C::TB, name};
 }
 template <int W, int SPL, int KT, bool VEC>
 Variant make_variant_tc(const char* name) {
@@ -1729,6 +1746,8 @@ Variant make_variant_tc(const char* name) {
 //   N <= 16: (16, 2), (8, 4), (8, 2), (4, 4), (4, 2), and (12, 4) for N = 16;
 //   N = 32: (8, 4), (4, 4);
 //   N >= 64: (8, N/8), (4, N/8).
+// Mode 2 is the register kernel that also stores the states for the backward (N = 16, A
+// per channel).
 // The tensor-memory kernel (mode 1: bf16, N = 16, A per channel), with KT time sub-chunks
 // per block: (16, 2, 1), (8, 4, 1), (12, 4, 1), (16, 2, 2), (8, 2, 2).
 constexpr bool layout_listed(int N, int w, int spl) {
@@ -1756,8 +1775,17 @@ constexpr bool tc_fits() {
 
 // One function per (io dtype, N) translation unit; see fwd_*.cu.
 #define SSM_PICK_ONE(T, TN, N, W, SPL)                                                                   \
-    if (mode == 0 && kt == 1 && w == W && spl == SPL) {                                                  \
+    if ((mode == 0 || mode == 2) && kt == 1 && w == W && spl == SPL) {                                   \
         if constexpr (layout_exists<T, N, W, SPL>()) {                                                   \
+            if (mode == 2) {                                                                             \
+                if constexpr (N == 16) {                                                                 \
+                    if (head) return false;                                                              \
+                    *v = vec ? make_variant<T, N, W, false, SPL, true, true>("ws_" #TN "_n" #N "_w" #W "s" #SPL "t1_ckpt_vec") \
+                             : make_variant<T, N, W, false, SPL, false, true>("ws_" #TN "_n" #N "_w" #W "s" #SPL "t1_ckpt"); \
+                    return true;                                                                         \
+                }                                                                                        \
+                return false;                                                                            \
+            }                                                                                            \
             if (head)                                                                                    \
                 *v = vec ? make_variant<T, N, W, true, SPL, true>("ws_" #TN "_n" #N "_w" #W "s" #SPL "t1_head_vec") \
                          : make_variant<T, N, W, true, SPL, false>("ws_" #TN "_n" #N "_w" #W "s" #SPL "t1_head");   \

@@ -241,7 +241,7 @@ CKPT_CASES = [
     (si.Dims(1, 32, 640, 16, dtype="bf16"), dict(tensor_memory=1, warps=8, states_per_lane=2, seg_len=128)),
     (si.Dims(2, 96, 200, 16, dtype="bf16"), dict(tensor_memory=1, warps=12, states_per_lane=4)),  # shuffles
     (si.Dims(1, 32, 100, 16, dtype="f32"), None),                                    # 32-step blocks
-    (si.Dims(2, 64, 129, 8, dtype="bf16"), None),                                    # another dstate
+    (si.Dims(2, 64, 777, 16, dtype="f32"), dict(tensor_memory=1, warps=16, states_per_lane=2, seg_len=128)),
 ]
 
 
@@ -261,12 +261,18 @@ def test_forward_stores_block_states(case):
     check_state(to_host_f64(ck), ref, what="stored states")
 
 
-def test_forward_checkpoints_refused_off_the_register_kernel():
+@pytest.mark.parametrize("dims,opts", [(si.Dims(2, 64, 256, 16, dtype="bf16"), dict(tensor_memory=2)),
+                                       (si.Dims(2, 64, 129, 8, dtype="bf16"), None),
+                                       (si.Dims(2, 64, 128, 16, nheads=4, dtype="bf16"), None)],
+                         ids=["tensor-memory", "dstate8", "per-head"])
+def test_forward_checkpoints_refused_outside_the_backward(dims, opts):
+    """The states are stored where the backward can use them: the register kernel, the S6
+    layout, dstate 16; elsewhere the call is refused (SSM_ERR_UNSUPPORTED)."""
     import selective_state_space_30_b200 as ssm
-    dims = si.Dims(2, 64, 256, 16, dtype="bf16")
-    inp = si.make_inputs(dims, _recipe("c2"), 53)
+    recipe = si.Recipe(a_init="neg_uniform_1_16") if dims.head_mode else _recipe("c2")
+    inp = si.make_inputs(dims, recipe, 53)
     with pytest.raises(ssm.SsmError):
-        _fwd_ckpt(dims, inp, None, dict(tensor_memory=2))
+        _fwd_ckpt(dims, inp, None, opts)
 
 
 @pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[7], CASES[8]],

@@ -47,6 +47,31 @@ def main():
         ro, rl, rm = oracle.run_inputs(dims, inp)
         check_out(to_host_f64(out), ro, rm, dt, what=f"debug build {dims} {opts}")
         check_state(to_host_f64(last), rl, what=f"debug build last_state {dims} {opts}")
+    # the forward variant that also stores the backward's states (S6 layout, N = 16)
+    import torch
+    from parity import OPTION_CODES, to_device
+    for b, dm, L, dt, opts in [(2, 80, 300, "bf16", {}), (3, 40, 257, "f32", {}), (1, 17, 5, "bf16", {}),
+                               (2, 64, 333, "bf16", dict(tensor_memory=1, warps=8, states_per_lane=2, seg_len=128))]:
+        dims = si.Dims(b, dm, L, 16, dtype=dt)
+        inp = si.make_inputs(dims, si.Recipe(d_init="normal", delta_init="normal_half"), 5 + L)
+        out0, last0 = run_gpu(dims, inp, opts=opts)
+        io = ssm.SSM_BF16 if dt == "bf16" else ssm.SSM_F32
+        d = ssm.make_dims(b, dm, L, 16, dm, 1, io)
+        dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+        out = torch.empty_like(dev["u"])
+        last = torch.empty((b, dm, 16), dtype=torch.float32, device="cuda")
+        ck = torch.empty((b, dm, (L + 31) // 32, 16), dtype=torch.float32, device="cuda")
+        plan = ssm.ssm_scan_plan(d, 0)
+        try:
+            for k, v in opts.items():
+                ssm.ssm_scan_set_option(plan, OPTION_CODES[k], v)
+            ssm.ssm_selective_scan_fwd_ckpt(plan, dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev["D"],
+                                            dev["z"], dev["delta_bias"], True, d, None, out, last, ck)
+            assert ssm.ssm_scan_device_status(plan) == ssm.SSM_OK, f"stored-state forward {dims} {opts}"
+            torch.cuda.synchronize()
+        finally:
+            ssm.ssm_scan_destroy(plan)
+        assert torch.equal(out, out0) and torch.equal(last, last0), f"stored-state forward differs {dims} {opts}"
     print("debug build: all shapes SSM_OK and at parity")
 
 

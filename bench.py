@@ -768,7 +768,7 @@ def run_conv1d(args):
 
 # ------------------------------------------------------------------ backward scan
 
-BWD_WORKLOADS = ("mamba-130m", "mamba-1.4b", "mamba-2.8b-long")
+BWD_WORKLOADS = ("mamba-130m", "mamba-1.4b", "mamba-2.8b-long", "mamba2-n128")
 
 
 def _bwd_bytes(d):
@@ -776,8 +776,10 @@ def _bwd_bytes(d):
     du, ddelta, dz written in the I/O dtype, dB, dC fp32, dA, dD, dbias fp32."""
     e = 2 if d.dtype == "bf16" else 4
     elems = d.batch * d.dim * d.seqlen
+    helems = d.batch * d.H * d.seqlen          # delta and ddelta rows: per channel, or per head
     bc = d.batch * d.ngroups * d.dstate * d.seqlen
-    return 7 * elems * e + 2 * bc * e + 2 * bc * 4 + 2 * (d.dim * d.dstate + 2 * d.dim) * 4
+    nA = d.H if d.head_mode else d.dim * d.dstate
+    return 5 * elems * e + 2 * helems * e + 2 * bc * e + 2 * bc * 4 + 2 * (nA + d.dim + d.H) * 4
 
 
 def run_bwd(args):
@@ -810,14 +812,17 @@ def run_bwd(args):
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum(int(x.numel() * x.element_size()) for x in list(t.values()) + [dout] if x is not None)
 
-    # the forward's stored states (the training path: the backward then skips its recomputation)
+    # the forward's stored states (the training path: the backward then skips its recomputation),
+    # where the tiled backward takes the shape; the generic backward always recomputes
+    stored = ssm.bwd_covers(t["u"], t["delta"], t["A"], t["B"])
     plan = ssm.ssm_scan_plan(dims, local)
     nblk = (d.seqlen + 31) // 32
-    ck = torch.empty((d.batch, d.dim, nblk, d.dstate), **f32)
+    ck = torch.empty((d.batch, d.dim, nblk, d.dstate), **f32) if stored else None
     fout = torch.empty_like(t["u"])
     fwd_args = (plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"], t["delta_bias"], True, dims,
                 None, fout, None)
-    ssm.ssm_selective_scan_fwd_ckpt(*fwd_args, ck, stream.cuda_stream)
+    if stored:
+        ssm.ssm_selective_scan_fwd_ckpt(*fwd_args, ck, stream.cuda_stream)
 
     def bwd_step(states):
         return lambda: ssm.ssm_selective_scan_bwd_ckpt(dims, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"],
@@ -839,10 +844,13 @@ def run_bwd(args):
         barrier()
         return e0.elapsed_time(e1) / steps, max_over_ranks(e0.elapsed_time(e1), dev), clk.summary()
 
-    ms, total, clocks = timed(bwd_step(ck), args.steps)
-    ms_re, total_re, _ = timed(bwd_step(None), args.steps)
+    ms_re, total_re, clocks_re = timed(bwd_step(None), args.steps)
+    if stored:
+        ms, total, clocks = timed(bwd_step(ck), args.steps)
+        ms_fc, _, _ = timed(lambda: ssm.ssm_selective_scan_fwd_ckpt(*fwd_args, ck, stream.cuda_stream), args.steps)
+    else:
+        ms, total, clocks, ms_fc = ms_re, total_re, clocks_re, None
     ms_f, _, _ = timed(lambda: ssm.ssm_selective_scan_fwd_h0(*fwd_args, stream.cuda_stream), args.steps)
-    ms_fc, _, _ = timed(lambda: ssm.ssm_selective_scan_fwd_ckpt(*fwd_args, ck, stream.cuda_stream), args.steps)
     ssm.ssm_scan_destroy(plan)
     hbm_gbs, sm_max_mhz, src = _peaks()
     finish_ranks()
@@ -852,7 +860,7 @@ def run_bwd(args):
     exps = _exps(d)
     mufu_peak = SMS * EX2_PER_CLK_PER_SM * sm_max_mhz * 1e6 / 1e9
     alg = _bwd_bytes(d)
-    ck_bytes = int(ck.numel() * 4)
+    ck_bytes = int(ck.numel() * 4) if stored else 0
 
     def roof(ms_, traffic_key):
         gexps = exps / (ms_ * 1e-3) / 1e9
@@ -871,16 +879,17 @@ def run_bwd(args):
             "dtype": "f32 (bf16 I/O)" if d.dtype == "bf16" else "f32", "data": "synthetic (seeded splitmix64)",
             "config": {"workload": w.name, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen,
                        "dstate": d.dstate, "io_dtype": d.dtype, "parallelism": f"replicas x{world}",
-                       "states": f"stored by the forward (ssm_selective_scan_fwd_ckpt, {ck_bytes / 1e6:.0f} MB), "
-                                 "read by ssm_selective_scan_bwd_ckpt",
+                       "states": (f"stored by the forward (ssm_selective_scan_fwd_ckpt, {ck_bytes / 1e6:.0f} MB), "
+                                  "read by ssm_selective_scan_bwd_ckpt") if stored else
+                                 "recomputed (the generic backward: per-head layout or dstate other than 16)",
                        "l2": f"inputs {in_bytes / 1e6:.0f} MB and workspace {nws / 1e6:.0f} MB (> 126 MB L2), "
                              "no flush"},
-            "roofline": roof(ms, "bwd_ckpt:" + w.name),
+            "roofline": roof(ms, ("bwd_ckpt:" if stored else "bwd:") + w.name),
             "recompute": {"what": "ssm_selective_scan_bwd: the backward recomputes the states itself",
                           "ms_per_step": ms_re, "value": job_throughput(world, elems, args.steps, total_re),
                           "roofline": roof(ms_re, "bwd:" + w.name)},
             "forward": {"ms_plain": ms_f, "ms_with_states": ms_fc, "state_bytes": ck_bytes},
-            "clocks": clocks, "gpu_launches": 2 * args.steps}
+            "clocks": clocks, "gpu_launches": (2 if stored else 4) * args.steps}
     print(json.dumps(line), flush=True)
 
 

@@ -322,8 +322,14 @@ int ssm_causal_conv1d_fwd(int64_t batch, int64_t dim, int64_t seqlen, int32_t wi
  *     ddelta_bias += ddelta,  dD += dy * u,  dz = dout * y * silu'(z)
  *     dh0 = g after step 0
  *
- * Covered: the S6 layout (nheads == dim), dstate 16, dim/ngroups a multiple of
- * 32; other shapes return SSM_ERR_UNSUPPORTED.  Inputs and layouts are the
+ * Covered: every layout with dstate in {8, 16, 32, 64, 128}; other dstates return
+ * SSM_ERR_UNSUPPORTED.  The S6 layout (nheads == dim) with dstate 16 and dim/ngroups a
+ * multiple of 32 runs on the tiled kernel described below.  Every other covered shape
+ * (the per-head layout, where A, delta and delta_bias are per head and ddelta, dA and
+ * ddelta_bias are summed over each head's channels; the other dstates) runs on a generic
+ * kernel: one CTA per group of channels for the whole sequence (no inter-CTA waits),
+ * states recomputed from workspace checkpoints every 256 steps; correct, not tuned, and
+ * its ddelta for the per-head layout is a sum of atomic adds as well.  Inputs and layouts are the
  * forward's (h0 nullable: zero); dout is (batch, dim, seqlen) in the io dtype,
  * dlast (batch, dim, dstate) fp32.  Outputs (ssm_grads_t, device memory owned
  * by the caller, every one overwritten):

@@ -255,7 +255,7 @@ def _selective_scan_function():
 
 def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True, h0=None):
     """The forward scan as a differentiable torch operation: returns (out, last_state),
-    and the backward runs ssm_selective_scan_bwd (which covers the per-channel layout with
-    dstate 16; other shapes raise SsmError when their gradient is taken).  dB and dC are
-    formed in fp32 and returned in B's and C's dtype."""
+    and the backward runs ssm_selective_scan_bwd (dstate 8 to 128, both layouts; on the
+    shapes its tiled kernel takes, the forward also stores the states the backward walks
+    back from).  dB and dC are formed in fp32 and returned in B's and C's dtype."""
     return _selective_scan_function().apply(u, delta, A, B, C, D, z, delta_bias, h0, softplus)

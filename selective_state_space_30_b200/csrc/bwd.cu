@@ -47,6 +47,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "bwd_generic.h"
 #include "scan_kernel.cuh"   // ex2_approx, rcp_approx, softplus1, kLog2e
 #include "ssm_scan.h"
 
@@ -699,6 +700,10 @@ extern "C" int ssm_selective_scan_bwd_workspace_size(const ssm_dims_t* dims, siz
     using namespace ssm;
     if (!bytes) return SSM_ERR_INVALID_ARG;
     const int rc = check_dims(dims);
+    if (rc == SSM_ERR_UNSUPPORTED && bwd_generic_supported(*dims) == SSM_OK) {
+        *bytes = (size_t)bwd_generic_workspace_bytes(*dims);
+        return SSM_OK;
+    }
     if (rc != SSM_OK) return rc;
     Sched sc;
     WsLayout w;
@@ -736,33 +741,45 @@ extern "C" int ssm_selective_scan_bwd_ckpt(const ssm_dims_t* dims, const void* u
                                            ssm_stream_t stream) {
     using namespace ssm;
     const int rc = check_dims(dims);
-    if (rc != SSM_OK) return rc;
+    // the shapes the tiled kernel does not take (per-head layout, dstate other than 16, tiles
+    // that do not divide a group) run on the generic backward
+    const bool generic = rc == SSM_ERR_UNSUPPORTED && bwd_generic_supported(*dims) == SSM_OK;
+    if (rc != SSM_OK && !generic) return rc;
     if (!grads || !grads->dA) return SSM_ERR_INVALID_ARG;
+    if (generic && ckpt) return SSM_ERR_INVALID_ARG;   // the forward stores states only for the tiled kernel's shapes
     if (dims->batch == 0 || dims->seqlen == 0) {
         // no steps (the per-step tensors are empty and may be NULL): every gradient is zero, dh0 = dlast
         cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        const int64_t N = dims->dstate;
         const int64_t rows = dims->batch * dims->dim, esz = dims->io_dtype == SSM_BF16 ? 2 : 4;
-        const int64_t nbc = dims->batch * dims->ngroups * kN * dims->seqlen * 4;
-        bool ok = cudaMemsetAsync(grads->dA, 0, dims->dim * kN * 4, s) == cudaSuccess;
+        const int64_t nbc = dims->batch * dims->ngroups * N * dims->seqlen * 4;
+        const int64_t nA = dims->nheads != dims->dim ? dims->nheads : dims->dim * N;
+        bool ok = cudaMemsetAsync(grads->dA, 0, nA * 4, s) == cudaSuccess;
         if (workspace && workspace_bytes >= 8) ok = ok && cudaMemsetAsync(workspace, 0, 8, s) == cudaSuccess;
         if (grads->dD) ok = ok && cudaMemsetAsync(grads->dD, 0, dims->dim * 4, s) == cudaSuccess;
-        if (grads->ddelta_bias) ok = ok && cudaMemsetAsync(grads->ddelta_bias, 0, dims->dim * 4, s) == cudaSuccess;
+        if (grads->ddelta_bias) ok = ok && cudaMemsetAsync(grads->ddelta_bias, 0, dims->nheads * 4, s) == cudaSuccess;
         if (nbc) ok = ok && cudaMemsetAsync(grads->dB, 0, nbc, s) == cudaSuccess &&
                       cudaMemsetAsync(grads->dC, 0, nbc, s) == cudaSuccess;
         if (rows > 0 && dims->seqlen > 0) {
             ok = ok && cudaMemsetAsync(grads->du, 0, rows * dims->seqlen * esz, s) == cudaSuccess &&
-                 cudaMemsetAsync(grads->ddelta, 0, rows * dims->seqlen * esz, s) == cudaSuccess;
+                 cudaMemsetAsync(grads->ddelta, 0, dims->batch * dims->nheads * dims->seqlen * esz, s) == cudaSuccess;
             if (grads->dz) ok = ok && cudaMemsetAsync(grads->dz, 0, rows * dims->seqlen * esz, s) == cudaSuccess;
         }
         if (grads->dh0 && rows) {
-            ok = ok && (dlast ? cudaMemcpyAsync(grads->dh0, dlast, rows * kN * 4, cudaMemcpyDeviceToDevice, s)
-                              : cudaMemsetAsync(grads->dh0, 0, rows * kN * 4, s)) == cudaSuccess;
+            ok = ok && (dlast ? cudaMemcpyAsync(grads->dh0, dlast, rows * N * 4, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(grads->dh0, 0, rows * N * 4, s)) == cudaSuccess;
         }
         return ok ? SSM_OK : SSM_ERR_CUDA;
     }
     if (!u || !delta || !A || !B || !C || !dout) return SSM_ERR_INVALID_ARG;
     if (!grads->du || !grads->ddelta || !grads->dB || !grads->dC) return SSM_ERR_INVALID_ARG;
     if (z && !grads->dz) return SSM_ERR_INVALID_ARG;
+    if (generic) {
+        if (!workspace || workspace_bytes < (size_t)bwd_generic_workspace_bytes(*dims)) return SSM_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u) return SSM_ERR_UNSUPPORTED;
+        return bwd_generic_launch(*dims, u, delta, A, B, C, D, z, delta_bias, softplus, h0, dout, dlast, *grads,
+                                  static_cast<unsigned char*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+    }
     Sched sc;
     WsLayout w;
     if (!plan_for(*dims, &sc, &w)) return SSM_ERR_CUDA;

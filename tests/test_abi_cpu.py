@@ -114,21 +114,31 @@ def test_bwd_host_checks(lib):
     ws = lib.ssm_selective_scan_bwd_workspace_size
     assert ws(ctypes.byref(ssm.make_dims(2, 32, 64, 16, 0, 1, ssm.SSM_BF16)), None) == ssm.SSM_ERR_INVALID_ARG
     assert ws(None, ctypes.byref(n)) == ssm.SSM_ERR_INVALID_ARG
-    unsupported = [
+    generic = [
         ssm.make_dims(2, 64, 64, 16, 2, 1, ssm.SSM_BF16),     # per-head layout
         ssm.make_dims(2, 32, 64, 128, 0, 1, ssm.SSM_BF16),    # dstate 128
         ssm.make_dims(2, 48, 64, 16, 0, 1, ssm.SSM_BF16),     # 48 channels: not whole 32-channel tiles
         ssm.make_dims(2, 64, 64, 16, 0, 4, ssm.SSM_BF16),     # 16 channels per group
+        ssm.make_dims(2, 32, 600, 8, 0, 1, ssm.SSM_F32),      # dstate 8, three 256-step segments
     ]
-    for d in unsupported:
-        assert ws(ctypes.byref(d), ctypes.byref(n)) == ssm.SSM_ERR_UNSUPPORTED
+    for d in generic:   # the generic backward: header, ddelta sums, per-row partials, a state per segment
+        assert ws(ctypes.byref(d), ctypes.byref(n)) == ssm.SSM_OK
+        nseg = (d.seqlen + 255) // 256
+        need = 256 + d.batch * d.nheads * d.seqlen * 4 + d.batch * d.dim * d.dstate * 4 + d.batch * d.dim * 4 + \
+            d.batch * d.dim * nseg * d.dstate * 4
+        assert need <= n.value <= need + 4 * 256
+    for d in (ssm.make_dims(2, 32, 64, 24, 0, 1, ssm.SSM_BF16), ssm.make_dims(2, 32, 64, 256, 0, 1, ssm.SSM_BF16)):
+        assert ws(ctypes.byref(d), ctypes.byref(n)) == ssm.SSM_ERR_UNSUPPORTED    # dstate 24, 256
     for d in (ssm.make_dims(2, 30, 64, 16, 0, 4, ssm.SSM_BF16), _abi.ssm_dims_t(2, 32, 64, 16, 32, 1, 7, 0)):
         assert ws(ctypes.byref(d), ctypes.byref(n)) == ssm.SSM_ERR_INVALID_ARG
     g = _abi.ssm_grads_t()
     f = lib.ssm_selective_scan_bwd
-    d = ssm.make_dims(2, 64, 64, 16, 2, 1, ssm.SSM_BF16)
+    d = ssm.make_dims(2, 32, 64, 24, 0, 1, ssm.SSM_BF16)
     assert f(ctypes.byref(d), *([None] * 8), 1, None, None, None, ctypes.byref(g), None, 0, None) == \
         ssm.SSM_ERR_UNSUPPORTED
+    d = ssm.make_dims(2, 64, 64, 16, 2, 1, ssm.SSM_BF16)      # per-head: generic, but no dA output
+    assert f(ctypes.byref(d), *([None] * 8), 1, None, None, None, ctypes.byref(g), None, 0, None) == \
+        ssm.SSM_ERR_INVALID_ARG
     d = ssm.make_dims(2, 32, 64, 16, 0, 1, ssm.SSM_BF16)
     assert f(ctypes.byref(d), *([None] * 8), 1, None, None, None, None, None, 0, None) == ssm.SSM_ERR_INVALID_ARG
     assert f(ctypes.byref(d), *([None] * 8), 1, None, None, None, ctypes.byref(g), None, 0, None) == \

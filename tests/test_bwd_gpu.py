@@ -136,9 +136,11 @@ def test_bwd_argument_checks():
                                           check=False)
     ok = ssm.make_dims(1, 32, 16, 16, 0, 1, ssm.SSM_BF16)
     assert ssm.ssm_selective_scan_bwd_workspace_size(ok) <= ws.numel()
-    assert call(ssm.make_dims(1, 32, 16, 128, 0, 1, ssm.SSM_BF16)) == ssm.SSM_ERR_UNSUPPORTED    # dstate 128
-    assert call(ssm.make_dims(1, 64, 16, 16, 2, 1, ssm.SSM_BF16)) == ssm.SSM_ERR_UNSUPPORTED     # per-head layout
-    assert call(ssm.make_dims(1, 48, 16, 16, 0, 1, ssm.SSM_BF16)) == ssm.SSM_ERR_UNSUPPORTED     # dim not x32
+    # shapes outside the tiled kernel run on the generic backward
+    assert call(ssm.make_dims(1, 32, 16, 128, 0, 1, ssm.SSM_BF16)) == ssm.SSM_OK                 # dstate 128
+    assert call(ssm.make_dims(1, 64, 16, 16, 2, 1, ssm.SSM_BF16)) == ssm.SSM_OK                  # per-head layout
+    assert call(ssm.make_dims(1, 48, 16, 16, 0, 1, ssm.SSM_BF16)) == ssm.SSM_OK                  # dim not x32
+    assert call(ssm.make_dims(1, 32, 16, 24, 0, 1, ssm.SSM_BF16)) == ssm.SSM_ERR_UNSUPPORTED     # dstate 24
     assert call(ok, z=x) == ssm.SSM_ERR_INVALID_ARG                                              # z without dz
     assert call(ok, nbytes=16) == ssm.SSM_ERR_INVALID_ARG                                        # workspace too small
     assert call(ok, g=dict(grads, dB=None)) == ssm.SSM_ERR_INVALID_ARG                           # missing output
@@ -307,3 +309,64 @@ def test_bwd_with_forward_states(case):
             assert torch.equal(g[k], g0[k]), f"{k} differs from the recomputing backward"
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin["dlast"], h0=gin["h0"], want_dh0=True)
     check_grads(g, ref, mag, dims.dtype)
+
+
+# ------------------------------------------ the generic backward (other layouts)
+
+GENERIC_CASES = [
+    # (dims, recipe kind, dlast, h0, softplus): shapes the tiled kernel does not take
+    (si.Dims(2, 64, 100, 16, nheads=4, dtype="bf16"), "head", True, True, True),     # per-head, dstate 16
+    (si.Dims(1, 128, 300, 128, nheads=2, dtype="bf16"), "head", True, True, True),   # the Mamba-2 shape, small
+    (si.Dims(2, 64, 160, 64, nheads=8, ngroups=2, dtype="f32"), "head", False, False, True),   # heads and groups
+    (si.Dims(2, 24, 77, 8, dtype="f32"), "c2", True, True, True),                    # dstate 8
+    (si.Dims(2, 40, 260, 32, ngroups=2, dtype="bf16"), "c2", False, True, True),     # dstate 32, two groups
+    (si.Dims(1, 16, 513, 64, dtype="f32"), "c2", True, False, True),                 # two segments and a step
+    (si.Dims(2, 48, 90, 16, dtype="bf16"), "c2", True, True, True),                  # 48 channels: no 32-channel tile
+    (si.Dims(1, 32, 70, 128, nheads=4, dtype="f32"), "plainhead", False, False, False),   # no z, D, bias; no softplus
+]
+
+
+def _generic_recipe(kind):
+    if kind == "head":
+        return si.Recipe(a_init="neg_uniform_1_16", d_init="normal", delta_init="normal_half")
+    if kind == "plainhead":
+        return si.Recipe(a_init="neg_uniform_1_16", has_D=False, has_z=False, has_bias=False,
+                         delta_init="normal_half")
+    if kind == "c2":
+        return si.Recipe(a_init="neg_uniform_1_16", d_init="normal", delta_init="normal_half")
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("case", GENERIC_CASES,
+                         ids=lambda c: f"{c[0].batch}x{c[0].dim}x{c[0].seqlen}n{c[0].dstate}h{c[0].H}g{c[0].ngroups}"
+                                       f"{c[0].dtype}-{c[1]}")
+def test_generic_bwd_matches_oracle(case):
+    """The per-head layout and dstate 8 to 128 run on the generic backward: every gradient
+    against the oracle's, within the same bound as the tiled kernel."""
+    dims, kind, dlast, h0, softplus = case
+    inp = si.make_inputs(dims, _generic_recipe(kind), 61)
+    if not softplus:
+        inp["delta"] = (np.abs(si.make_inputs(dims, _generic_recipe("head"), 61)["delta"]) *
+                        np.float32(0.05)).astype(np.float32)
+        if dims.dtype == "bf16":
+            raise AssertionError("the no-softplus case is fp32")
+    inp["softplus"] = softplus
+    gin = si.make_grad_inputs(dims, 62, dlast=dlast, h0=h0)
+    ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin["dlast"], h0=gin["h0"], want_dh0=True)
+    g = run_bwd(dims, inp, gin, want_dh0=True, softplus=softplus)
+    check_grads(g, ref, mag, dims.dtype, what=f"{dims} ")
+
+
+def test_generic_bwd_refuses_stored_states_and_odd_dstate():
+    """The forward stores no states for these shapes, so a ckpt pointer is an argument
+    error; a dstate outside {8, 16, 32, 64, 128} is unsupported."""
+    import selective_state_space_30_b200 as ssm
+    x = torch.zeros(1 << 16, device="cuda")
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    grads = {k: x for k in ("du", "ddelta", "dA", "dB", "dC")}
+    head = ssm.make_dims(1, 64, 16, 16, 4, 1, ssm.SSM_BF16)
+    assert ssm.ssm_selective_scan_bwd_ckpt(head, x, x, x, x, x, None, None, None, True, None, x, None, x, grads,
+                                           ws, ws.numel(), check=False) == ssm.SSM_ERR_INVALID_ARG
+    odd = ssm.make_dims(1, 32, 16, 12, 0, 1, ssm.SSM_BF16)
+    assert ssm.ssm_selective_scan_bwd(odd, x, x, x, x, x, None, None, None, True, None, x, None, grads, ws,
+                                      ws.numel(), check=False) == ssm.SSM_ERR_UNSUPPORTED

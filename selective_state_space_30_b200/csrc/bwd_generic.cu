@@ -9,7 +9,8 @@
 // the channels of head h, dA[h] over its channels and states.
 //
 // One CTA owns `cpb` channels of one batch row (inside one group) for the whole
-// sequence, one thread per (channel, state): nothing waits on another CTA.
+// sequence, one thread per (channel, state), up to 256 threads (512 from dstate 64
+// on): nothing waits on another CTA.
 //   1. A forward pass stores the state at the start of every segment (256 steps)
 //      in the workspace.
 //   2. Segments are then taken last to first.  A forward pass over the segment
@@ -36,7 +37,7 @@ namespace {
 constexpr int gK = 32;                 // steps per block
 constexpr int gSegB = 8;               // blocks per segment
 constexpr int gSeg = gK * gSegB;       // steps per segment (a workspace checkpoint each)
-constexpr int gMaxThreads = 256;
+constexpr int gMaxThreads = 512;
 
 struct GParams {
     const void *u, *delta, *z, *dout, *B, *C;
@@ -52,6 +53,7 @@ struct GParams {
     int nseg;           // segments of gSeg steps
     int softplus;
     int head;           // 1: one scalar A per head
+    int red_vec;        // dB, dC rows take 16-byte atomic adds (L % 4 == 0, 16-byte aligned)
 };
 
 template <typename T> struct GIo;
@@ -69,6 +71,11 @@ template <> struct GIo<__nv_bfloat16> {
 };
 
 __device__ __forceinline__ float gsigmoid(float x) { return rcp_approx(1.f + ex2_approx(x * -kLog2e)); }
+
+__device__ __forceinline__ void gred4(float* dst, const float (&v)[4]) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3])
+                 : "memory");
+}
 
 // Shared memory (floats) for T = cpb * N threads; rows of T + 1 floats so that a
 // thread walking one row of states and its neighbours walking the next rows meet
@@ -224,12 +231,13 @@ __global__ void __launch_bounds__(gMaxThreads) scan_bwd_generic_kernel(const GPa
                 const int cc = pr / gK, k = pr % gK;
                 const int64_t t = t0 + k;
                 const float dt = at(PC_DT, cc, k);
+                const float dAh = ex2_approx(dt * a2);   // one A per head: the decay of every state
                 float y = 0.f, gB = 0.f, q = 0.f;
                 for (int nn = tl; nn < N; nn += TS) {
                     const int idx = cc * N + nn;
                     const float gv = sG[k * TP + idx];
                     const float Ann = p.head ? An : __ldg(p.A + (d0 + cc) * N + nn);
-                    const float dA = ex2_approx(dt * (Ann * kLog2e));
+                    const float dA = p.head ? dAh : ex2_approx(dt * (Ann * kLog2e));
                     y = fmaf(sC[nn * KP + k], sH[(k + 1) * TP + idx], y);
                     gB = fmaf(gv, sB[nn * KP + k], gB);
                     q = fmaf(gv * sH[k * TP + idx], Ann * dA, q);
@@ -254,19 +262,32 @@ __global__ void __launch_bounds__(gMaxThreads) scan_bwd_generic_kernel(const GPa
                 }
             }
             // pass B: per (state, step), dB = sum over channels of g dt u, dC = of dy h_t
-            for (int i = tid; i < N * gK; i += NT) {
-                const int nn = i / gK, k = i % gK;
-                const int64_t t = t0 + k;
-                if (t >= L) continue;
-                float sb = 0.f, sc = 0.f;
+            // (four consecutive steps per thread: one 16-byte atomic add each for dB and dC)
+            for (int i = tid; i < N * (gK / 4); i += NT) {
+                const int nn = i / (gK / 4), k4 = (i % (gK / 4)) * 4;
+                if (t0 + k4 >= L) continue;
+                float sb[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int cc = 0; cc < cpb; ++cc) {
                     const int idx = cc * N + nn;
-                    sb = fmaf(sG[k * TP + idx], at(PC_DU, cc, k), sb);
-                    sc = fmaf(at(PC_DY, cc, k), sH[(k + 1) * TP + idx], sc);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int k = k4 + e;
+                        sb[e] = fmaf(sG[k * TP + idx], at(PC_DU, cc, k), sb[e]);
+                        sc[e] = fmaf(at(PC_DY, cc, k), sH[(k + 1) * TP + idx], sc[e]);
+                    }
                 }
-                const int64_t off = ((b * G + g) * N + nn) * L + t;
-                atomicAdd(p.dB + off, sb);
-                atomicAdd(p.dC + off, sc);
+                const int64_t off = ((b * G + g) * N + nn) * L + t0 + k4;
+                if (p.red_vec && t0 + k4 + 3 < L) {
+                    gred4(p.dB + off, sb);
+                    gred4(p.dC + off, sc);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (t0 + k4 + e < L) {
+                            atomicAdd(p.dB + off + e, sb[e]);
+                            atomicAdd(p.dC + off + e, sc[e]);
+                        }
+                }
             }
         }
     }
@@ -346,10 +367,11 @@ struct GLayout {
     int64_t dd, dA, dD, ck, total;   // byte offsets after the 256-byte header
 };
 
-// channels per CTA: the largest power of two up to 256 / N that divides dim / ngroups
+// channels per CTA: the largest power of two up to 256 / N (512 / N from N = 64 on) that divides
+// dim / ngroups
 int gcpb(const ssm_dims_t& d) {
     const int64_t per_group = d.dim / d.ngroups;
-    int c = 256 / (int)d.dstate;
+    int c = (d.dstate >= 64 ? 512 : 256) / (int)d.dstate;
     while (c > 1 && per_group % c) c >>= 1;
     return c;
 }
@@ -420,6 +442,7 @@ int bwd_generic_launch(const ssm_dims_t& d, const void* u, const void* delta, co
     prm.nseg = (int)((d.seqlen + gSeg - 1) / gSeg);
     prm.softplus = softplus ? 1 : 0;
     prm.head = d.nheads != d.dim ? 1 : 0;
+    prm.red_vec = d.seqlen % 4 == 0 && ((reinterpret_cast<uintptr_t>(gr.dB) | reinterpret_cast<uintptr_t>(gr.dC)) & 15u) == 0;
     const int64_t N = d.dstate;
     const size_t nbc = (size_t)(d.batch * d.ngroups * N * d.seqlen) * 4;
     // the header (status: nothing here waits, so it stays SSM_OK), the ddelta sums, dB and dC start at zero

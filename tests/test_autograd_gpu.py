@@ -61,3 +61,26 @@ def test_autograd_without_optional_inputs():
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"])
     got = {GRAD_OF[k]: leaves[k].grad for k in leaves}
     check_grads(got, {k: ref[k] for k in got}, mag, "f32", what="autograd, no options ")
+
+
+@pytest.mark.parametrize("dims", [si.Dims(2, 64, 130, 16, nheads=4, dtype="bf16"),
+                                  si.Dims(1, 128, 200, 128, nheads=2, dtype="bf16")],
+                         ids=["per-head-n16", "per-head-n128"])
+def test_autograd_per_head_layout(dims):
+    """The per-head (Mamba-2) layout through selective_scan_fn: the forward (the scan
+    kernel, or the chunked tensor-core path for dstate 128) and the generic backward;
+    every leaf's gradient against the oracle's, A and delta_bias per head."""
+    import selective_state_space_30_b200 as ssm
+    inp = si.make_inputs(dims, si.Recipe(a_init="neg_uniform_1_16", d_init="normal", delta_init="normal_half"), 55)
+    inp["softplus"] = True
+    gin = si.make_grad_inputs(dims, 56, dlast=True)
+    leaves = {k: to_device(inp[k]).requires_grad_() for k in INPUTS}
+    out, last = ssm.selective_scan_fn(*(leaves[k] for k in INPUTS), softplus=True)
+    torch.autograd.backward([out, last], [to_device(gin["dout"]), to_device(gin["dlast"])])
+    torch.cuda.synchronize()
+    ref_out, ref_last, mag_out = oracle.run_inputs(dims, inp)
+    check_out(to_host_f64(out.detach()), ref_out, mag_out, dims.dtype)
+    ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin["dlast"])
+    got = {GRAD_OF[k]: leaves[k].grad for k in INPUTS}
+    check_grads(got, {k: ref[k] for k in got}, mag, dims.dtype, what="autograd, per head ",
+                bf16_out=BF16_OUT + ("dB", "dC"))

@@ -37,7 +37,6 @@ namespace {
 constexpr int gK = 32;                 // steps per block
 constexpr int gSegB = 8;               // blocks per segment
 constexpr int gSeg = gK * gSegB;       // steps per segment (a workspace checkpoint each)
-constexpr int gMaxThreads = 512;
 
 struct GParams {
     const void *u, *delta, *z, *dout, *B, *C;
@@ -96,8 +95,10 @@ struct GSmem {
 };
 enum { PC_DT = 0, PC_DU, PC_U, PC_X, PC_DY, PC_DOUT, PC_Z };
 
-template <typename T, int N>
-__global__ void __launch_bounds__(gMaxThreads) scan_bwd_generic_kernel(const GParams p) {
+// PREF: the CTA holds at least 4 channels (at most 8 B and C values per thread and block),
+// so a block's inputs fit in registers and are loaded one block ahead
+template <typename T, int N, bool PREF>
+__global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(const GParams p) {
     extern __shared__ float gsm[];
     const GSmem S(N, p.cpb);
     const int NT = S.T, TP = S.TP;
@@ -125,44 +126,108 @@ __global__ void __launch_bounds__(gMaxThreads) scan_bwd_generic_kernel(const GPa
     const float a2 = An * kLog2e;
     const int nblk = (int)((L + gK - 1) / gK);
 
-    // block blk into shared memory: per (channel, step) dt and dt*u (full: also u, the
-    // softplus argument x, dy = dout silu(z), dout, z), and the B (full: and C) rows
-    auto stage = [&](int blk, bool full) {
+    // Block blk in two halves: load() reads its inputs into registers (issued a block
+    // ahead, so the loads are in flight while the current block runs), store() writes
+    // them to shared memory with the per-(channel, step) values: dt and dt*u (full: also
+    // u, the softplus argument x, dy = dout silu(z), dout, z), and the B (full: C) rows.
+    constexpr int PPT = gK / N > 0 ? gK / N : 1;   // (channel, step) pairs per thread, at most
+    constexpr int BPT = PREF ? 8 : 1;               // B (C) values per thread, at most
+    float ru[PPT], rx[PPT], rdo[PPT], rz[PPT], rb[BPT], rc[BPT];
+    auto load = [&](int blk, bool full) {
+        if constexpr (!PREF) return;   // fewer than 4 channels: store() loads for itself
         const int64_t t0 = (int64_t)blk * gK;
-        for (int i = tid; i < cpb * gK; i += NT) {
-            const int cc = i / gK, k = i % gK;
-            const int64_t t = t0 + k, dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
-            float dt = 0.f, du = 0.f, uv = 0.f, x = 0.f, dy = 0.f, dov = 0.f, zv = 0.f;
-            if (t < L) {
-                uv = GIo<T>::ld(p.u, rr * L + t);
-                x = GIo<T>::ld(p.delta, (b * H + hh) * L + t) + (p.bias ? __ldg(p.bias + hh) : 0.f);
-                dt = p.softplus ? softplus1(x) : x;
-                du = dt * uv;
-                if (full) {
-                    dov = GIo<T>::ld(p.dout, rr * L + t);
-                    if (p.z) {
-                        zv = GIo<T>::ld(p.z, rr * L + t);
-                        dy = dov * (zv * gsigmoid(zv));
-                    } else {
-                        dy = dov;
+#pragma unroll
+        for (int e = 0; e < PPT; ++e) {
+            const int i = tid + e * NT;
+            ru[e] = rx[e] = rdo[e] = rz[e] = 0.f;
+            if (i < cpb * gK) {
+                const int cc = i / gK, k = i % gK;
+                const int64_t t = t0 + k, dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
+                if (t < L) {
+                    ru[e] = GIo<T>::ld(p.u, rr * L + t);
+                    rx[e] = GIo<T>::ld(p.delta, (b * H + hh) * L + t) + (p.bias ? __ldg(p.bias + hh) : 0.f);
+                    if (full) {
+                        rdo[e] = GIo<T>::ld(p.dout, rr * L + t);
+                        if (p.z) rz[e] = GIo<T>::ld(p.z, rr * L + t);
                     }
                 }
             }
-            at(PC_DT, cc, k) = dt;
-            at(PC_DU, cc, k) = du;
-            if (full) {
-                at(PC_U, cc, k) = uv;
-                at(PC_X, cc, k) = x;
-                at(PC_DY, cc, k) = dy;
-                at(PC_DOUT, cc, k) = dov;
-                at(PC_Z, cc, k) = zv;
+        }
+#pragma unroll
+        for (int e = 0; e < BPT; ++e) {
+            const int i = tid + e * NT;
+            rb[e] = rc[e] = 0.f;
+            if (i < N * gK) {
+                const int nn = i / gK, k = i % gK;
+                const int64_t t = t0 + k, off = ((b * G + g) * N + nn) * L + t;
+                if (t < L) {
+                    rb[e] = GIo<T>::ld(p.B, off);
+                    if (full) rc[e] = GIo<T>::ld(p.C, off);
+                }
             }
         }
-        for (int i = tid; i < N * gK; i += NT) {
-            const int nn = i / gK, k = i % gK;
-            const int64_t t = t0 + k, off = ((b * G + g) * N + nn) * L + t;
-            sB[nn * KP + k] = t < L ? GIo<T>::ld(p.B, off) : 0.f;
-            if (full) sC[nn * KP + k] = t < L ? GIo<T>::ld(p.C, off) : 0.f;
+    };
+    auto store = [&](int blk, bool full) {
+        const int64_t t0 = (int64_t)blk * gK;
+        if constexpr (!PREF) {
+            // no registers to spare: load and store in one go
+            for (int i = tid; i < cpb * gK; i += NT) {
+                const int cc = i / gK, k = i % gK;
+                const int64_t t = t0 + k, dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
+                float dt = 0.f, uv = 0.f, x = 0.f, dov = 0.f, zv = 0.f;
+                if (t < L) {
+                    uv = GIo<T>::ld(p.u, rr * L + t);
+                    x = GIo<T>::ld(p.delta, (b * H + hh) * L + t) + (p.bias ? __ldg(p.bias + hh) : 0.f);
+                    dt = p.softplus ? softplus1(x) : x;
+                    if (full) {
+                        dov = GIo<T>::ld(p.dout, rr * L + t);
+                        if (p.z) zv = GIo<T>::ld(p.z, rr * L + t);
+                    }
+                }
+                at(PC_DT, cc, k) = dt;
+                at(PC_DU, cc, k) = dt * uv;
+                if (full) {
+                    at(PC_U, cc, k) = uv;
+                    at(PC_X, cc, k) = x;
+                    at(PC_DY, cc, k) = p.z ? dov * (zv * gsigmoid(zv)) : dov;
+                    at(PC_DOUT, cc, k) = dov;
+                    at(PC_Z, cc, k) = zv;
+                }
+            }
+            for (int i = tid; i < N * gK; i += NT) {
+                const int nn = i / gK, k = i % gK;
+                const int64_t t = t0 + k, off = ((b * G + g) * N + nn) * L + t;
+                sB[nn * KP + k] = t < L ? GIo<T>::ld(p.B, off) : 0.f;
+                if (full) sC[nn * KP + k] = t < L ? GIo<T>::ld(p.C, off) : 0.f;
+            }
+            return;
+        }
+#pragma unroll
+        for (int e = 0; e < PPT; ++e) {
+            const int i = tid + e * NT;
+            if (i < cpb * gK) {
+                const int cc = i / gK, k = i % gK;
+                const bool valid = t0 + k < L;   // past L: no step (dt = 0)
+                const float dt = valid ? (p.softplus ? softplus1(rx[e]) : rx[e]) : 0.f;
+                at(PC_DT, cc, k) = dt;
+                at(PC_DU, cc, k) = dt * ru[e];
+                if (full) {
+                    at(PC_U, cc, k) = ru[e];
+                    at(PC_X, cc, k) = rx[e];
+                    at(PC_DY, cc, k) = p.z ? rdo[e] * (rz[e] * gsigmoid(rz[e])) : rdo[e];
+                    at(PC_DOUT, cc, k) = rdo[e];
+                    at(PC_Z, cc, k) = rz[e];
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < BPT; ++e) {
+            const int i = tid + e * NT;
+            if (i < N * gK) {
+                const int nn = i / gK, k = i % gK;
+                sB[nn * KP + k] = rb[e];
+                if (full) sC[nn * KP + k] = rc[e];
+            }
         }
     };
     // the recurrence over the staged block from state h (steps past L have dt = 0: no
@@ -179,11 +244,13 @@ __global__ void __launch_bounds__(gMaxThreads) scan_bwd_generic_kernel(const GPa
 
     // ---- 1. forward: the state entering every segment, into the workspace
     float h = p.h0 ? __ldg(p.h0 + row * N + n) : 0.f;
+    if (nblk > 0) load(0, false);
     for (int blk = 0; blk < nblk; ++blk) {
         if (blk % gSegB == 0) p.ckpt[(row * p.nseg + blk / gSegB) * N + n] = h;
         __syncthreads();   // the previous block is done with the staged arrays
-        stage(blk, false);
+        store(blk, false);
         __syncthreads();
+        if (blk + 1 < nblk) load(blk + 1, false);
         h = run_block(h, false);
     }
 
@@ -196,18 +263,22 @@ __global__ void __launch_bounds__(gMaxThreads) scan_bwd_generic_kernel(const GPa
     for (int seg = p.nseg - 1; seg >= 0; --seg) {
         const int b0 = seg * gSegB, b1 = min(nblk, b0 + gSegB);
         float hs = p.ckpt[(row * p.nseg + seg) * N + n];
+        load(b0, false);
         for (int blk = b0; blk < b1; ++blk) {
             sBlk[(blk - b0) * NT + tid] = hs;
             __syncthreads();
-            stage(blk, false);
+            store(blk, false);
             __syncthreads();
+            if (blk + 1 < b1) load(blk + 1, false);
+            else load(b1 - 1, true);   // the first block of the walk
             hs = run_block(hs, false);
         }
         for (int blk = b1 - 1; blk >= b0; --blk) {
             const int64_t t0 = (int64_t)blk * gK;
             __syncthreads();
-            stage(blk, true);
+            store(blk, true);
             __syncthreads();
+            if (blk > b0) load(blk - 1, true);
             run_block(sBlk[(blk - b0) * NT + tid], true);
             // the state gradient back through the block: g += dy C is dLoss/dh_t
             for (int k = gK - 1; k >= 0; --k) {
@@ -387,17 +458,20 @@ GLayout glayout(const ssm_dims_t& d) {
     return w;
 }
 
-template <typename T, int N>
-int glaunch(const GParams& prm, unsigned grid, cudaStream_t s) {
+template <typename T, int N, bool PREF>
+int glaunch_one(const GParams& prm, unsigned grid, cudaStream_t s) {
     const GSmem S(N, prm.cpb);
     const size_t smem = (size_t)S.total * 4;
     if (smem > 227 * 1024) return SSM_ERR_UNSUPPORTED;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(scan_bwd_generic_kernel<T, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(scan_bwd_generic_kernel<T, N, PREF>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return SSM_ERR_CUDA;
-    scan_bwd_generic_kernel<T, N><<<grid, (unsigned)S.T, smem, s>>>(prm);
+    scan_bwd_generic_kernel<T, N, PREF><<<grid, (unsigned)S.T, smem, s>>>(prm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+template <typename T, int N>
+int glaunch(const GParams& prm, unsigned grid, cudaStream_t s) {
+    return prm.cpb >= 4 ? glaunch_one<T, N, true>(prm, grid, s) : glaunch_one<T, N, false>(prm, grid, s);
 }
 
 template <typename T>

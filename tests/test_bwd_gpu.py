@@ -323,6 +323,8 @@ GENERIC_CASES = [
     (si.Dims(1, 16, 513, 64, dtype="f32"), "c2", True, False, True),                 # two segments and a step
     (si.Dims(2, 48, 90, 16, dtype="bf16"), "c2", True, True, True),                  # 48 channels: no 32-channel tile
     (si.Dims(1, 32, 70, 128, nheads=4, dtype="f32"), "plainhead", False, False, False),   # no z, D, bias; no softplus
+    (si.Dims(1, 6, 70, 32, dtype="f32"), "c2", True, True, True),                     # 2 channels per CTA
+    (si.Dims(2, 2, 50, 128, nheads=1, dtype="bf16"), "head", True, False, True),      # one head of 2 channels
 ]
 
 

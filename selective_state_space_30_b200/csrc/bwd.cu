@@ -57,9 +57,14 @@ namespace {
 constexpr int kN = 16;         // states per channel
 constexpr int kBT = 32;        // steps per staged block
 constexpr int kWin = 8;        // steps per recomputed window (= one 8-lane reduction)
-constexpr int kCT = 32;        // channels per CTA
-constexpr int kThreads = 256;  // 8 warps x 4 channels x 8 lanes
-constexpr int kStageRows = 4 * kCT + 2 * kN;   // u, delta, z, dout rows; B, C rows
+// A CTA of NW warps (8, or 4 where 32-channel tiles would leave CTA slots idle), each
+// warp 4 channels x 8 lanes x 2 states.
+template <int NW>
+struct Bw {
+    static constexpr int CT = 4 * NW;                   // channels per CTA (a tile)
+    static constexpr int THREADS = 32 * NW;
+    static constexpr int STAGE_ROWS = 4 * CT + 2 * kN;  // u, delta, z, dout rows; B, C rows
+};
 
 struct BwdParams {
     const void *u, *delta, *z, *dout, *B, *C;
@@ -70,15 +75,15 @@ struct BwdParams {
     unsigned* ticket;            // work-unit counter (zeroed before the launch)
     int* status;                 // kernel-side ssm_status_t
     unsigned *flag1, *flag2;     // [tile][seg]: forward / reverse segment done (zeroed before the launch)
-    float *carry1, *carry2;      // [tile][seg][kCT][kN]: state after / state gradient before a segment
+    float *carry1, *carry2;      // [tile][seg][CT][kN]: state after / state gradient before a segment
     float* ckpt;                 // checkpoints [b * dim + d][block][kN]: the state entering each 32-step block
     int ext_ckpt;                // 1: ckpt holds the forward's states; no forward units run
     float *dB, *dC;              // the outputs (batch, groups, kN, L), zeroed before the launch
     int red_vec;                 // 16-byte atomic adds into dB, dC (L % 4 == 0, aligned bases)
     float *dAp, *dDp, *dbp;      // per segment and (b, d) row: [seg][row][kN], [seg][row], [seg][row]
     int64_t batch, dim, seqlen, ngroups;
-    int64_t ntiles;              // batch * dim / kCT
-    int tiles_per_row;           // dim / kCT
+    int64_t ntiles;              // batch * dim / CT (channels per tile)
+    int tiles_per_row;           // dim / CT
     int nseg, seg_blocks;        // segments per tile, 32-step blocks per segment
     int softplus;
     uint64_t budget_ns;          // bounded waits
@@ -100,29 +105,31 @@ template <> struct Io<__nv_bfloat16> {
 // shared memory (bytes).  The per-step rows P and U have kPS = kBT + 1 entries per
 // channel, so the four channels a warp reads at one step sit in different banks.
 constexpr int kPS = kBT + 1;
-template <typename T>
+template <typename T, int NW>
 struct Smem {
+    static constexpr int CT = Bw<NW>::CT;
     static constexpr int kRow = kBT * (int)sizeof(T) + 16;        // staged row stride (16-byte padded)
     static constexpr int STAGE = 0;                               // two buffers of staged rows
-    static constexpr int kStageBytes = kStageRows * kRow;
-    static constexpr int P = STAGE + 2 * kStageBytes;             // float4 [kCT][kPS]: dt, dt*u, dy, dout*silu'(z)
-    static constexpr int U = P + kCT * kPS * 16;                  // float2 [kCT][kPS]: u, sigmoid(x)
-    static constexpr int BC = U + kCT * kPS * 8;                  // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
+    static constexpr int kStageBytes = Bw<NW>::STAGE_ROWS * kRow;
+    static constexpr int P = STAGE + 2 * kStageBytes;             // float4 [CT][kPS]: dt, dt*u, dy, dout*silu'(z)
+    static constexpr int U = P + CT * kPS * 16;                   // float2 [CT][kPS]: u, sigmoid(x)
+    static constexpr int BC = U + CT * kPS * 8;                   // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
     // per window and warp, the dB, dC terms summed over the warp's channels:
-    // float [kBT/kWin windows][8 warps][4 components][8 lanes j][kWin steps]
+    // float [kBT/kWin windows][NW warps][4 components][8 lanes j][kWin steps]
     static constexpr int RED = BC + kBT * 8 * 16;
     // per thread, the states entering the four windows of the block being walked backwards
-    static constexpr int WST = RED + (kBT / kWin) * 8 * 4 * 8 * kWin * 4;
-    static constexpr int TOTAL = WST + (kBT / kWin) * kThreads * 8;
+    static constexpr int WST = RED + (kBT / kWin) * NW * 4 * 8 * kWin * 4;
+    static constexpr int TOTAL = WST + (kBT / kWin) * Bw<NW>::THREADS * 8;
 };
 
 // rows x kBT steps [t0, t0 + kBT) of `rows` rows (row r at src + r * stride) into
 // shared memory, zero past L.  vec: asynchronous 16-byte copies (rows 16-byte
 // aligned, L a multiple of the chunk; complete after cp_async_wait), else element by
 // element.
-template <typename T>
+template <typename T, int NW>
 __device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int64_t stride, int rows, int64_t t0,
                                            int64_t L, bool vec, int tid) {
+    constexpr int kThreads = Bw<NW>::THREADS;
     using R = typename Io<T>::raw;
     constexpr int E = 16 / (int)sizeof(T);
     constexpr int CPR = kBT / E;
@@ -132,7 +139,7 @@ __device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int
             const int r = i / CPR, k = i % CPR;
             const int64_t t = t0 + (int64_t)k * E;
             const T* g = src + r * stride + (t < L ? t : 0);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst + r * Smem<T>::kRow + k * 16)),
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst + r * Smem<T, NW>::kRow + k * 16)),
                          "l"(g), "r"(t < L ? 16 : 0)
                          : "memory");
         }
@@ -141,7 +148,7 @@ __device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int
         for (int i = tid; i < rows * kBT; i += kThreads) {
             const int r = i / kBT, k = i % kBT;
             const int64_t t = t0 + k;
-            reinterpret_cast<R*>(dst + r * Smem<T>::kRow)[k] = t < L ? s[r * stride + t] : (R)0;
+            reinterpret_cast<R*>(dst + r * Smem<T, NW>::kRow)[k] = t < L ? s[r * stride + t] : (R)0;
         }
     }
 }
@@ -150,7 +157,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_al
 
 template <typename T>
 __device__ __forceinline__ float staged(const unsigned char* base, int row, int k) {
-    return Io<T>::f(reinterpret_cast<const typename Io<T>::raw*>(base + row * Smem<T>::kRow)[k]);
+    return Io<T>::f(reinterpret_cast<const typename Io<T>::raw*>(base + row * Smem<T, 8>::kRow)[k]);
 }
 
 __device__ __forceinline__ float sigmoid1(float x) { return rcp_approx(1.f + ex2_approx(x * -kLog2e)); }
@@ -192,34 +199,39 @@ __device__ __forceinline__ void red_add_v4(float* dst, float4 v) {
 }
 
 // The dB, dC terms of one 32-step block, held per (window, warp) in shared memory,
-// summed over the eight warps in a fixed order and added into dB and dC (rows of the
-// tile's group, dBg / dCg) by atomic adds: thread tid takes four consecutive steps of one
-// (window, component, lane j).
+// summed over the NW warps in a fixed order and added into dB and dC (rows of the
+// tile's group, dBg / dCg) by atomic adds: each of the 256 items is four consecutive
+// steps of one (window, component, lane j).
+template <int NW>
 __device__ __forceinline__ void red_add(const float* red, float* dBg, float* dCg, int64_t t0, int64_t L, bool vec,
                                        int tid) {
-    const int w = tid >> 6, comp = (tid >> 4) & 3, jj = (tid >> 1) & 7, q4 = (tid & 1) * 4;
-    const int within = comp * 64 + jj * 8 + q4;
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int wp = 0; wp < 8; ++wp) {
-        const float4 v = *reinterpret_cast<const float4*>(red + (w * 8 + wp) * 256 + within);
-        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-    }
-    const int64_t ta = t0 + w * kWin + q4;
-    float* dst = ((comp & 2) ? dCg : dBg) + (int64_t)(2 * jj + (comp & 1)) * L + ta;
-    if (vec && ta + 3 < L) {
-        red_add_v4(dst, s);
-    } else {
-        const float e[4] = {s.x, s.y, s.z, s.w};
+    for (int it = tid; it < 256; it += Bw<NW>::THREADS) {
+        const int w = it >> 6, comp = (it >> 4) & 3, jj = (it >> 1) & 7, q4 = (it & 1) * 4;
+        const int within = comp * 64 + jj * 8 + q4;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (ta + i < L) atomicAdd(dst + i, e[i]);
+        for (int wp = 0; wp < NW; ++wp) {
+            const float4 v = *reinterpret_cast<const float4*>(red + (w * NW + wp) * 256 + within);
+            s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        }
+        const int64_t ta = t0 + w * kWin + q4;
+        float* dst = ((comp & 2) ? dCg : dBg) + (int64_t)(2 * jj + (comp & 1)) * L + ta;
+        if (vec && ta + 3 < L) {
+            red_add_v4(dst, s);
+        } else {
+            const float e[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (ta + i < L) atomicAdd(dst + i, e[i]);
+        }
     }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p) {
-    using S = Smem<T>;
+template <typename T, int NW>
+__global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdParams p) {
+    using S = Smem<T, NW>;
+    constexpr int kCT = Bw<NW>::CT, kThreads = Bw<NW>::THREADS;
     extern __shared__ __align__(16) unsigned char smem[];
     unsigned char* stage_base = smem + S::STAGE;
     float4* sP = reinterpret_cast<float4*>(smem + S::P);
@@ -307,9 +319,9 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 h = __ldcg(reinterpret_cast<const float2*>(p.carry1 + ((us - 1) * kCT + c) * kN + 2 * j));
             // the rows of the unit's first block; each block's prologue then issues the next's
             auto issue_fwd = [&](unsigned char* sg, int64_t ts) {
-                stage_rows<T>(sg, u, L, kCT, ts, L, vec, tid);
-                stage_rows<T>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
-                stage_rows<T>(sg + 4 * kCT * S::kRow, Bg, L, kN, ts, L, vec, tid);
+                stage_rows<T, NW>(sg, u, L, kCT, ts, L, vec, tid);
+                stage_rows<T, NW>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
+                stage_rows<T, NW>(sg + 4 * kCT * S::kRow, Bg, L, kN, ts, L, vec, tid);
             };
             issue_fwd(stage_base, (int64_t)blk0 * kBT);
             int cur = 0;
@@ -329,8 +341,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                     if (t0 + lane >= L) dt = 0.f;
                     sP[cc * kPS + lane] = make_float4(dt, dt * uv, 0.f, 0.f);
                 }
-                {
-                    const int t = tid >> 3, jj = tid & 7;
+                for (int it = tid; it < kBT * 8; it += kThreads) {
+                    const int t = it >> 3, jj = it & 7;
                     const unsigned char* sb = stage + 4 * kCT * S::kRow;
                     sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t), 0.f, 0.f);
                 }
@@ -373,12 +385,12 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
         // the checkpoint of the block being walked (the next, earlier one is fetched a block ahead)
         float2 hblk = __ldcg(reinterpret_cast<const float2*>(ckpt + (int64_t)(blk1 - 1) * kN));
         auto issue_rev = [&](unsigned char* sg, int64_t ts) {
-            stage_rows<T>(sg, u, L, kCT, ts, L, vec, tid);
-            stage_rows<T>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
-            if (zz) stage_rows<T>(sg + 2 * kCT * S::kRow, zz, L, kCT, ts, L, vec, tid);
-            stage_rows<T>(sg + 3 * kCT * S::kRow, go, L, kCT, ts, L, vec, tid);
-            stage_rows<T>(sg + 4 * kCT * S::kRow, Bg, L, kN, ts, L, vec, tid);
-            stage_rows<T>(sg + (4 * kCT + kN) * S::kRow, Cg, L, kN, ts, L, vec, tid);
+            stage_rows<T, NW>(sg, u, L, kCT, ts, L, vec, tid);
+            stage_rows<T, NW>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
+            if (zz) stage_rows<T, NW>(sg + 2 * kCT * S::kRow, zz, L, kCT, ts, L, vec, tid);
+            stage_rows<T, NW>(sg + 3 * kCT * S::kRow, go, L, kCT, ts, L, vec, tid);
+            stage_rows<T, NW>(sg + 4 * kCT * S::kRow, Bg, L, kN, ts, L, vec, tid);
+            stage_rows<T, NW>(sg + (4 * kCT + kN) * S::kRow, Cg, L, kN, ts, L, vec, tid);
         };
         issue_rev(stage_base, (int64_t)(blk1 - 1) * kBT);
         int cur = 0;
@@ -388,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
             cp_async_wait();
             __syncthreads();   // this block's rows are in; the previous block is done with P, U, BC
             // the previous block's dB, dC terms (every warp has written them)
-            if (blk + 1 < blk1) red_add(sR, dBg, dCg, t0 + kBT, L, rvec, tid);
+            if (blk + 1 < blk1) red_add<NW>(sR, dBg, dCg, t0 + kBT, L, rvec, tid);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int cc = warp * 4 + i;
@@ -410,8 +422,8 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 sP[cc * kPS + lane] = make_float4(dt, dt * uv, dy, dzf);
                 sU[cc * kPS + lane] = make_float2(uv, sp);
             }
-            {
-                const int t = tid >> 3, jj = tid & 7;
+            for (int it = tid; it < kBT * 8; it += kThreads) {
+                const int t = it >> 3, jj = it & 7;
                 const unsigned char* sb = stage + 4 * kCT * S::kRow;
                 const unsigned char* sc = stage + (4 * kCT + kN) * S::kRow;
                 sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t),
@@ -484,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
                 }
                 const float GB = reduce8(gb, j), Q = reduce8(qq, j);
                 {
-                    float4* rd = reinterpret_cast<float4*>(sR + ((w * 8 + warp) * 4 + q) * 64 + j * 8);
+                    float4* rd = reinterpret_cast<float4*>(sR + ((w * NW + warp) * 4 + q) * 64 + j * 8);
                     rd[0] = make_float4(rw[0], rw[1], rw[2], rw[3]);
                     rd[1] = make_float4(rw[4], rw[5], rw[6], rw[7]);
                 }
@@ -518,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 2) scan_bwd_kernel(const BwdParams p
 
         // the last block's dB, dC terms
         __syncthreads();
-        red_add(sR, dBg, dCg, (int64_t)blk0 * kBT, L, rvec, tid);
+        red_add<NW>(sR, dBg, dCg, (int64_t)blk0 * kBT, L, rvec, tid);
         // hand the state gradient to the segment before; this segment's parameter partials
         *reinterpret_cast<float2*>(p.carry2 + (us * kCT + c) * kN + 2 * j) = gs;
         if (seg == 0 && p.dh0) *reinterpret_cast<float2*>(p.dh0 + (row0 + c) * kN + 2 * j) = gs;
@@ -571,11 +583,12 @@ __global__ void __launch_bounds__(256) scan_bwd_finalize(const BwdParams p, floa
 // and the cut of each tile's sequence into segments, about 8 units per CTA and pass.
 struct Sched {
     int ctas, nseg, seg_blocks;
+    int nw, ct;   // warps per CTA and channels per tile
 };
 
-template <typename T>
-Sched make_sched(const ssm_dims_t& d, int sms, int per_sm) {
-    const int64_t ntiles = d.batch * d.dim / kCT;
+Sched make_sched(const ssm_dims_t& d, int sms, int per_sm, int nw) {
+    const int ct = 4 * nw;
+    const int64_t ntiles = d.batch * d.dim / ct;
     const int64_t nblk = (d.seqlen + kBT - 1) / kBT;
     const int64_t slots = (int64_t)sms * per_sm;
     int64_t want = (8 * slots + ntiles - 1) / ntiles;          // segments per tile
@@ -583,6 +596,8 @@ Sched make_sched(const ssm_dims_t& d, int sms, int per_sm) {
     if (sb < 4) sb = 4;                                          // at least 128 steps per unit
     if (sb > nblk) sb = nblk > 0 ? nblk : 1;
     Sched s;
+    s.nw = nw;
+    s.ct = ct;
     s.seg_blocks = (int)sb;
     s.nseg = (int)((nblk + sb - 1) / sb);
     const int64_t units = ntiles * s.nseg;
@@ -599,7 +614,8 @@ __host__ int64_t align256(int64_t v) { return (v + 255) & ~(int64_t)255; }
 
 WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
     const int64_t rows = d.batch * d.dim;
-    const int64_t ntiles = rows / kCT;
+    const int64_t ct = s.ct;
+    const int64_t ntiles = rows / ct;
     const int64_t nblk = (d.seqlen + kBT - 1) / kBT;
     const int64_t slots = ntiles * s.nseg;
     WsLayout w;
@@ -608,9 +624,9 @@ WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
     w.flag2 = align256(w.flag1 + slots * 4);
     w.zero_end = align256(w.flag2 + slots * 4);
     w.carry1 = w.zero_end;
-    w.carry2 = align256(w.carry1 + slots * kCT * kN * 4);
-    w.ckpt = align256(w.carry2 + slots * kCT * kN * 4);
-    w.dAp = align256(w.ckpt + ntiles * kCT * nblk * kN * 4);
+    w.carry2 = align256(w.carry1 + slots * ct * kN * 4);
+    w.ckpt = align256(w.carry2 + slots * ct * kN * 4);
+    w.dAp = align256(w.ckpt + ntiles * ct * nblk * kN * 4);
     w.dDp = align256(w.dAp + (int64_t)s.nseg * rows * kN * 4);
     w.dbp = align256(w.dDp + (int64_t)s.nseg * rows * 4);
     w.total = align256(w.dbp + (int64_t)s.nseg * rows * 4);
@@ -619,7 +635,7 @@ WsLayout ws_layout(const ssm_dims_t& d, const Sched& s) {
 
 // CTAs of the backward kernel that fit on one SM of the current device, and its SM count
 // (queried once per device and dtype)
-template <typename T>
+template <typename T, int NW>
 bool device_fit(int* sms, int* per_sm) {
     constexpr int kMaxDev = 64;
     static std::mutex mu;
@@ -633,11 +649,11 @@ bool device_fit(int* sms, int* per_sm) {
         return true;
     }
     if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-    if (cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<T>::TOTAL) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(scan_bwd_kernel<T, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<T, NW>::TOTAL) != cudaSuccess)
         return false;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, scan_bwd_kernel<T>, kThreads, Smem<T>::TOTAL) !=
-        cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, scan_bwd_kernel<T, NW>, Bw<NW>::THREADS,
+                                                      Smem<T, NW>::TOTAL) != cudaSuccess)
         return false;
     if (*per_sm < 1) *per_sm = 1;
     if (dev < kMaxDev) {
@@ -647,11 +663,20 @@ bool device_fit(int* sms, int* per_sm) {
     return true;
 }
 
+// The CTA size: 8 warps (32-channel tiles), or 4 warps (16-channel tiles) when the
+// 32-channel tiles are fewer than the CTAs that fit at once: each tile's chain of units
+// runs in order, so the tiles bound the CTAs at work (one batch row of 5120 channels: 160
+// tiles against 296 slots).
 bool plan_for(const ssm_dims_t& d, Sched* s, WsLayout* w) {
+    const bool bf = d.io_dtype == SSM_BF16;
     int sms = 0, per_sm = 0;
-    const bool ok = d.io_dtype == SSM_BF16 ? device_fit<__nv_bfloat16>(&sms, &per_sm) : device_fit<float>(&sms, &per_sm);
-    if (!ok) return false;
-    *s = d.io_dtype == SSM_BF16 ? make_sched<__nv_bfloat16>(d, sms, per_sm) : make_sched<float>(d, sms, per_sm);
+    if (!(bf ? device_fit<__nv_bfloat16, 8>(&sms, &per_sm) : device_fit<float, 8>(&sms, &per_sm))) return false;
+    int nw = 8;
+    if (d.batch * d.dim / 32 < (int64_t)sms * per_sm) {
+        nw = 4;
+        if (!(bf ? device_fit<__nv_bfloat16, 4>(&sms, &per_sm) : device_fit<float, 4>(&sms, &per_sm))) return false;
+    }
+    *s = make_sched(d, sms, per_sm, nw);
     *w = ws_layout(d, *s);
     return true;
 }
@@ -664,15 +689,15 @@ int check_dims(const ssm_dims_t* d) {
     if (d->batch > ((int64_t)1 << 40) / d->dim || (d->seqlen > 0 && d->batch * d->dim > ((int64_t)1 << 40) / d->seqlen))
         return SSM_ERR_INVALID_ARG;
     // what the kernel covers: the S6 layout, dstate 16, whole 32-channel tiles inside a group
-    if (d->nheads != d->dim || d->dstate != kN || (d->dim / d->ngroups) % kCT != 0) return SSM_ERR_UNSUPPORTED;
-    if (d->batch * d->dim / kCT > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;
+    if (d->nheads != d->dim || d->dstate != kN || (d->dim / d->ngroups) % 32 != 0) return SSM_ERR_UNSUPPORTED;
+    if (d->batch * d->dim / 16 > 0x7FFFFFFF) return SSM_ERR_UNSUPPORTED;
     return SSM_OK;
 }
 
-template <typename T>
+template <typename T, int NW>
 int launch(const BwdParams& prm, float* dA, float* dD, float* dbias, int ctas, cudaStream_t s) {
-    constexpr int smem = Smem<T>::TOTAL;
-    scan_bwd_kernel<T><<<(unsigned)ctas, kThreads, smem, s>>>(prm);
+    constexpr int smem = Smem<T, NW>::TOTAL;
+    scan_bwd_kernel<T, NW><<<(unsigned)ctas, Bw<NW>::THREADS, smem, s>>>(prm);
     if (cudaGetLastError() != cudaSuccess) return SSM_ERR_CUDA;
     const int64_t work = prm.dim * kN + 2 * prm.dim;
     const int64_t blocks = (work + 255) / 256;
@@ -811,8 +836,8 @@ extern "C" int ssm_selective_scan_bwd_ckpt(const ssm_dims_t* dims, const void* u
     prm.dDp = reinterpret_cast<float*>(ws + w.dDp);
     prm.dbp = reinterpret_cast<float*>(ws + w.dbp);
     prm.batch = dims->batch; prm.dim = dims->dim; prm.seqlen = dims->seqlen; prm.ngroups = dims->ngroups;
-    prm.tiles_per_row = (int)(dims->dim / kCT);
-    prm.ntiles = dims->batch * dims->dim / kCT;
+    prm.tiles_per_row = (int)(dims->dim / sc.ct);
+    prm.ntiles = dims->batch * dims->dim / sc.ct;
     prm.nseg = sc.nseg;
     prm.seg_blocks = sc.seg_blocks;
     prm.softplus = softplus ? 1 : 0;
@@ -827,7 +852,9 @@ extern "C" int ssm_selective_scan_bwd_ckpt(const ssm_dims_t* dims, const void* u
         cudaMemsetAsync(ws + w.flag1, 0, (size_t)(w.zero_end - w.flag1), s) != cudaSuccess ||
         cudaMemsetAsync(grads->dB, 0, nbc, s) != cudaSuccess || cudaMemsetAsync(grads->dC, 0, nbc, s) != cudaSuccess)
         return SSM_ERR_CUDA;
-    return dims->io_dtype == SSM_BF16
-               ? launch<__nv_bfloat16>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s)
-               : launch<float>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s);
+    if (dims->io_dtype == SSM_BF16)
+        return sc.nw == 8 ? launch<__nv_bfloat16, 8>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s)
+                          : launch<__nv_bfloat16, 4>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s);
+    return sc.nw == 8 ? launch<float, 8>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s)
+                      : launch<float, 4>(prm, grads->dA, grads->dD, grads->ddelta_bias, sc.ctas, s);
 }

@@ -111,12 +111,16 @@ struct Smem {
     static constexpr int kRow = kBT * (int)sizeof(T) + 16;        // staged row stride (16-byte padded)
     static constexpr int STAGE = 0;                               // two buffers of staged rows
     static constexpr int kStageBytes = Bw<NW>::STAGE_ROWS * kRow;
-    static constexpr int P = STAGE + 2 * kStageBytes;             // float4 [CT][kPS]: dt, dt*u, dy, dout*silu'(z)
-    static constexpr int U = P + CT * kPS * 16;                   // float2 [CT][kPS]: u, sigmoid(x)
-    static constexpr int BC = U + CT * kPS * 8;                   // float4 [kBT][8]: B_2j, B_2j+1, C_2j, C_2j+1
+    // Per-step values in 8-byte pairs: a lane reads only the pairs a pass needs (the
+    // shared-memory pipe moves a lane's bytes, broadcast or not).
+    static constexpr int PA = STAGE + 2 * kStageBytes;            // float2 [CT][kPS]: dt, dt*u
+    static constexpr int PB = PA + CT * kPS * 8;                  // float2 [CT][kPS]: dy, dout*silu'(z)
+    static constexpr int U = PB + CT * kPS * 8;                   // float2 [CT][kPS]: u, sigmoid(x)
+    static constexpr int BS = U + CT * kPS * 8;                   // float2 [kBT][8]: B_2j, B_2j+1
+    static constexpr int CS = BS + kBT * 8 * 8;                   // float2 [kBT][8]: C_2j, C_2j+1
     // per window and warp, the dB, dC terms summed over the warp's channels:
     // float [kBT/kWin windows][NW warps][4 components][8 lanes j][kWin steps]
-    static constexpr int RED = BC + kBT * 8 * 16;
+    static constexpr int RED = CS + kBT * 8 * 8;
     // per thread, the states entering the four windows of the block being walked backwards
     static constexpr int WST = RED + (kBT / kWin) * NW * 4 * 8 * kWin * 4;
     static constexpr int TOTAL = WST + (kBT / kWin) * Bw<NW>::THREADS * 8;
@@ -234,9 +238,11 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
     constexpr int kCT = Bw<NW>::CT, kThreads = Bw<NW>::THREADS;
     extern __shared__ __align__(16) unsigned char smem[];
     unsigned char* stage_base = smem + S::STAGE;
-    float4* sP = reinterpret_cast<float4*>(smem + S::P);
+    float2* sPa = reinterpret_cast<float2*>(smem + S::PA);
+    float2* sPb = reinterpret_cast<float2*>(smem + S::PB);
     float2* sU = reinterpret_cast<float2*>(smem + S::U);
-    float4* sBC = reinterpret_cast<float4*>(smem + S::BC);
+    float2* sB = reinterpret_cast<float2*>(smem + S::BS);
+    float2* sC = reinterpret_cast<float2*>(smem + S::CS);
     float* sR = reinterpret_cast<float*>(smem + S::RED);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -339,12 +345,12 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                         staged<T>(stage + kCT * S::kRow, cc, lane) + (p.bias ? __ldg(p.bias + d0 + cc) : 0.f);
                     float dt = p.softplus ? softplus1(xv) : xv;
                     if (t0 + lane >= L) dt = 0.f;
-                    sP[cc * kPS + lane] = make_float4(dt, dt * uv, 0.f, 0.f);
+                    sPa[cc * kPS + lane] = make_float2(dt, dt * uv);
                 }
                 for (int it = tid; it < kBT * 8; it += kThreads) {
                     const int t = it >> 3, jj = it & 7;
                     const unsigned char* sb = stage + 4 * kCT * S::kRow;
-                    sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t), 0.f, 0.f);
+                    sB[t * 8 + jj] = make_float2(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t));
                 }
                 // the next block's rows go into the other buffer, read last by the previous block
                 if (blk + 1 < blk1) issue_fwd(stage_base + (cur ^ 1) * S::kStageBytes, t0 + kBT);
@@ -354,10 +360,10 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                 for (int w = 0; w < kBT / kWin; ++w) {
 #pragma unroll 4
                     for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
-                        const float4 pv = sP[c * kPS + t];
-                        const float4 bc = sBC[t * 8 + j];
+                        const float2 pv = sPa[c * kPS + t];
+                        const float2 bb = sB[t * 8 + j];
                         float2 dA;
-                        fwd_step(h, dA, pv.x, pv.y, bc.x, bc.y, al);
+                        fwd_step(h, dA, pv.x, pv.y, bb.x, bb.y, al);
                     }
                 }
             }
@@ -419,15 +425,16 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                     dy = gov * zv * sg;
                     dzf = gov * (sg * fmaf(zv, 1.f - sg, 1.f));
                 }
-                sP[cc * kPS + lane] = make_float4(dt, dt * uv, dy, dzf);
+                sPa[cc * kPS + lane] = make_float2(dt, dt * uv);
+                sPb[cc * kPS + lane] = make_float2(dy, dzf);
                 sU[cc * kPS + lane] = make_float2(uv, sp);
             }
             for (int it = tid; it < kBT * 8; it += kThreads) {
                 const int t = it >> 3, jj = it & 7;
                 const unsigned char* sb = stage + 4 * kCT * S::kRow;
                 const unsigned char* sc = stage + (4 * kCT + kN) * S::kRow;
-                sBC[t * 8 + jj] = make_float4(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t),
-                                              staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
+                sB[t * 8 + jj] = make_float2(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t));
+                sC[t * 8 + jj] = make_float2(staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
             }
             // the next (earlier) block's rows go into the other buffer
             if (blk > blk0) issue_rev(stage_base + (cur ^ 1) * S::kStageBytes, t0 - kBT);
@@ -447,10 +454,10 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                     if (w + 1 < kBT / kWin) {
 #pragma unroll 4
                         for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
-                            const float4 pv = sP[c * kPS + t];
-                            const float4 bc = sBC[t * 8 + j];
+                            const float2 pv = sPa[c * kPS + t];
+                            const float2 bb = sB[t * 8 + j];
                             float2 dA;
-                            fwd_step(hh, dA, pv.x, pv.y, bc.x, bc.y, al);
+                            fwd_step(hh, dA, pv.x, pv.y, bb.x, bb.y, al);
                         }
                     }
                 }
@@ -466,11 +473,12 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                     float yp[kWin];
 #pragma unroll
                     for (int t = 0; t < kWin; ++t) {
-                        const float4 pv = sP[c * kPS + tw + t];
-                        const float4 bc = sBC[(tw + t) * 8 + j];
-                        fwd_step(hh, dAr[t], pv.x, pv.y, bc.x, bc.y, al);
+                        const float2 pv = sPa[c * kPS + tw + t];
+                        const float2 bb = sB[(tw + t) * 8 + j];
+                        const float2 cc = sC[(tw + t) * 8 + j];
+                        fwd_step(hh, dAr[t], pv.x, pv.y, bb.x, bb.y, al);
                         hr[t] = hh;
-                        yp[t] = fmaf(bc.z, hh.x, bc.w * hh.y);
+                        yp[t] = fmaf(cc.x, hh.x, cc.y * hh.y);
                     }
                     yw = reduce8(yp, j);
                 }
@@ -478,15 +486,17 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                 const bool q1 = q & 2, q0 = q & 1;
 #pragma unroll
                 for (int t = kWin - 1; t >= 0; --t) {
-                    const float4 pv = sP[c * kPS + tw + t];
-                    const float4 bc = sBC[(tw + t) * 8 + j];
-                    gs = fma2(dup2(pv.z), make_float2(bc.z, bc.w), gs);   // + dy C: now dLoss/dh_t
+                    const float2 pv = sPa[c * kPS + tw + t];   // dt, dt*u
+                    const float dy = sPb[c * kPS + tw + t].x;
+                    const float2 bb = sB[(tw + t) * 8 + j];
+                    const float2 cc = sC[(tw + t) * 8 + j];
+                    gs = fma2(dup2(dy), cc, gs);   // + dy C: now dLoss/dh_t
                     const float2 hp = t > 0 ? hr[t - 1] : he;
                     const float2 e = mul2(mul2(gs, hp), dAr[t]);
                     dAacc = fma2(e, dup2(pv.x), dAacc);
-                    gb[t] = fmaf(gs.x, bc.x, gs.y * bc.y);
+                    gb[t] = fmaf(gs.x, bb.x, gs.y * bb.y);
                     qq[t] = fmaf(e.x, Aln.x, e.y * Aln.y);
-                    const float2 db = mul2(gs, dup2(pv.y)), dc = mul2(dup2(pv.z), hr[t]);
+                    const float2 db = mul2(gs, dup2(pv.y)), dc = mul2(dup2(dy), hr[t]);
                     // the four terms (dB_2j, dB_2j+1, dC_2j, dC_2j+1) summed over the warp's four
                     // channels, transposed: lane (q, j) keeps component q
                     const float a0 = (q1 ? dc.x : db.x) + __shfl_xor_sync(0xffffffffu, q1 ? db.x : dc.x, 16);
@@ -504,12 +514,14 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                 {
                     // lane j: step tw + j of channel c
                     const int t = tw + j;
-                    const float4 pv = sP[c * kPS + t];
+                    const float dt = sPa[c * kPS + t].x;
+                    const float2 pb = sPb[c * kPS + t];   // dy, dout*silu'(z)
                     const float2 uv = sU[c * kPS + t];
                     const float dd = fmaf(uv.x, GB, Q) * uv.y;
                     dbias += dd;
-                    dDacc = fmaf(pv.z, uv.x, dDacc);
-                    sP[c * kPS + t] = make_float4(fmaf(pv.x, GB, pv.z * Dc), dd, fmaf(Dc, uv.x, yw) * pv.w, 0.f);
+                    dDacc = fmaf(pb.x, uv.x, dDacc);
+                    sPa[c * kPS + t] = make_float2(fmaf(dt, GB, pb.x * Dc), dd);
+                    sPb[c * kPS + t].x = fmaf(Dc, uv.x, yw) * pb.y;
                 }
             }
             // the block's du, ddelta, dz rows of this warp's channels (lane = step)
@@ -519,11 +531,11 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int cc = warp * 4 + i;
-                    const float4 o = sP[cc * kPS + lane];
+                    const float2 o = sPa[cc * kPS + lane];
                     const int64_t at = (row0 + cc) * L + t0 + lane;
                     static_cast<R*>(p.du)[at] = Io<T>::from(o.x);
                     static_cast<R*>(p.ddelta)[at] = Io<T>::from(o.y);
-                    if (zz) static_cast<R*>(p.dz)[at] = Io<T>::from(o.z);
+                    if (zz) static_cast<R*>(p.dz)[at] = Io<T>::from(sPb[cc * kPS + lane].x);
                 }
             }
         }

@@ -816,8 +816,8 @@ def run_bwd(args):
     # where the tiled backward takes the shape; the generic backward always recomputes
     stored = ssm.bwd_covers(t["u"], t["delta"], t["A"], t["B"])
     plan = ssm.ssm_scan_plan(dims, local)
-    nblk = (d.seqlen + 31) // 32
-    ck = torch.empty((d.batch, d.dim, nblk, d.dstate), **f32) if stored else None
+    nwin = (d.seqlen + 7) // 8
+    ck = torch.empty((d.batch, d.dim, nwin, d.dstate), **f32) if stored else None
     fout = torch.empty_like(t["u"])
     fwd_args = (plan, t["u"], t["delta"], t["A"], t["B"], t["C"], t["D"], t["z"], t["delta_bias"], True, dims,
                 None, fout, None)

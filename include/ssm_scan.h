@@ -122,9 +122,10 @@ int ssm_selective_scan_fwd_h0(ssm_plan_t plan, const void* u, const void* delta,
  * backward walks from, so that ssm_selective_scan_bwd_ckpt skips its recomputation pass
  * ("Agent 229" page, section 4 "Activation Recomputation": checkpoints at chunk
  * boundaries, recompute inside a chunk).  ckpt (device, fp32, required, 8-byte aligned,
- * caller-owned) receives (batch, dim, ceil(seqlen/32), dstate): element
- * [b][d][k][n] is the state h[n] of channel (b, d) entering step 32k (k = 0 holds h0, or
- * zero).  About batch*dim*seqlen*dstate/8 bytes.  Every other argument and output is
+ * caller-owned) receives (batch, dim, ceil(seqlen/8), dstate): element
+ * [b][d][k][n] is the state h[n] of channel (b, d) entering step 8k (k = 0 holds h0, or
+ * zero): the start of every 8-step window the backward recomputes, so that it rebuilds
+ * none.  About batch*dim*seqlen*dstate/2 bytes.  Every other argument and output is
  * ssm_selective_scan_fwd_h0's, bit for bit.  Covered: the shapes the backward covers
  * (the S6 layout, nheads == dim, with dstate 16), on the register kernel; another shape, or
  * a plan forced onto the tensor-memory kernel, returns SSM_ERR_UNSUPPORTED.
@@ -378,9 +379,10 @@ int ssm_selective_scan_bwd(const ssm_dims_t* dims, const void* u, const void* de
 
 /*
  * ssm_selective_scan_bwd given the states ssm_selective_scan_fwd_ckpt stored (ckpt, the
- * same layout; device, 8-byte aligned, read only) for the same inputs and h0: the
- * kernel then runs no forward recomputation units and writes no checkpoints of its own,
- * and reads ckpt instead (the workspace size is the same).  ckpt == NULL is exactly
+ * same layout; device, 8-byte aligned (16-byte aligned: copied in 16-byte pieces), read
+ * only) for the same inputs and h0: the kernel then runs no forward recomputation units,
+ * writes no checkpoints of its own and rebuilds no window starts: it reads them from ckpt
+ * (the workspace size is the same).  ckpt == NULL is exactly
  * ssm_selective_scan_bwd.  The gradients are those of ssm_selective_scan_bwd (the
  * states it would recompute are the ones the forward stored, bit for bit).
  */

@@ -107,8 +107,8 @@ def _shapes(u, delta, A, B):
 
 def ckpt_shape(batch: int, dim: int, seqlen: int, dstate: int) -> Tuple[int, int, int, int]:
     """Shape of the state checkpoints ssm_selective_scan_fwd_ckpt stores (fp32): the state
-    entering every 32-step block."""
-    return (batch, dim, (seqlen + 31) // 32, dstate)
+    entering every 8-step window."""
+    return (batch, dim, (seqlen + 7) // 8, dstate)
 
 
 def bwd_covers(u, delta, A, B) -> bool:

@@ -27,8 +27,10 @@
 // block (the checkpoints).  A reverse unit takes the state gradient from the
 // segment after it and walks its blocks backwards: per block it runs the
 // recurrence forward from the block's checkpoint to get the states at the four
-// 8-step window starts (registers), then per window recomputes the 8 states and
-// decays into registers and runs the window in reverse.  A unit waits (bounded) only on units with smaller
+// 8-step window starts (shared memory), then per window recomputes the 8 states and
+// decays into registers and runs the window in reverse.  Given the forward's stored
+// states (one per 8-step window, ssm_selective_scan_bwd_ckpt), no forward unit runs and
+// the window starts are copied in with the block's rows instead of rebuilt.  A unit waits (bounded) only on units with smaller
 // tickets, which running CTAs hold, so the chain always progresses.  Each block's
 // 32-step rows of the inputs are staged in shared memory by cp.async, double
 // buffered: a block's prologue issues the next block's rows.
@@ -76,8 +78,11 @@ struct BwdParams {
     int* status;                 // kernel-side ssm_status_t
     unsigned *flag1, *flag2;     // [tile][seg]: forward / reverse segment done (zeroed before the launch)
     float *carry1, *carry2;      // [tile][seg][CT][kN]: state after / state gradient before a segment
-    float* ckpt;                 // checkpoints [b * dim + d][block][kN]: the state entering each 32-step block
-    int ext_ckpt;                // 1: ckpt holds the forward's states; no forward units run
+    // the kernel's checkpoints [b * dim + d][block][kN] (the state entering each 32-step block),
+    // or with ext_ckpt the forward's stored states [b * dim + d][window][kN] (the state entering
+    // each 8-step window); then no forward units run
+    float* ckpt;
+    int ext_ckpt;
     float *dB, *dC;              // the outputs (batch, groups, kN, L), zeroed before the launch
     int red_vec;                 // 16-byte atomic adds into dB, dC (L % 4 == 0, aligned bases)
     float *dAp, *dDp, *dbp;      // per segment and (b, d) row: [seg][row][kN], [seg][row], [seg][row]
@@ -110,7 +115,12 @@ struct Smem {
     static constexpr int CT = Bw<NW>::CT;
     static constexpr int kRow = kBT * (int)sizeof(T) + 16;        // staged row stride (16-byte padded)
     static constexpr int STAGE = 0;                               // two buffers of staged rows
-    static constexpr int kStageBytes = Bw<NW>::STAGE_ROWS * kRow;
+    // in each stage buffer after the rows: the states entering the block's four windows,
+    // float [CT][kWinStride] (a channel's 4 x kN, padded so that two channels' reads of one
+    // window meet different banks)
+    static constexpr int kWinStride = (kBT / kWin) * kN + 16;
+    static constexpr int WINS = Bw<NW>::STAGE_ROWS * kRow;
+    static constexpr int kStageBytes = WINS + CT * kWinStride * 4;
     // Per-step values in 8-byte pairs: a lane reads only the pairs a pass needs (the
     // shared-memory pipe moves a lane's bytes, broadcast or not).
     static constexpr int PA = STAGE + 2 * kStageBytes;            // float2 [CT][kPS]: dt, dt*u
@@ -121,9 +131,7 @@ struct Smem {
     // per window and warp, the dB, dC terms summed over the warp's channels:
     // float [kBT/kWin windows][NW warps][4 components][8 lanes j][kWin steps]
     static constexpr int RED = CS + kBT * 8 * 8;
-    // per thread, the states entering the four windows of the block being walked backwards
-    static constexpr int WST = RED + (kBT / kWin) * NW * 4 * 8 * kWin * 4;
-    static constexpr int TOTAL = WST + (kBT / kWin) * Bw<NW>::THREADS * 8;
+    static constexpr int TOTAL = RED + (kBT / kWin) * NW * 4 * 8 * kWin * 4;
 };
 
 // rows x kBT steps [t0, t0 + kBT) of `rows` rows (row r at src + r * stride) into
@@ -158,6 +166,30 @@ __device__ __forceinline__ void stage_rows(unsigned char* dst, const T* src, int
 }
 
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// The forward's stored states entering windows [win0, win0 + 4) of the tile's CT channels
+// (channel cc's row at ck + cc * nwin * kN) into the block's window area, zero past nwin.
+// vec: 16-byte asynchronous copies (ck 16-byte aligned), else element by element.
+template <typename T, int NW>
+__device__ __forceinline__ void stage_wins(float* dst, const float* ck, int64_t nwin, int64_t win0, bool vec,
+                                           int tid) {
+    constexpr int kCT = Bw<NW>::CT, kThreads = Bw<NW>::THREADS;
+    constexpr int CPC = (kBT / kWin) * kN / 4;   // 16-byte chunks per channel
+    for (int i = tid; i < kCT * CPC; i += kThreads) {
+        const int cc = i / CPC, k = i % CPC;
+        const int64_t win = win0 + k / (kN / 4);
+        const bool in = win < nwin;
+        const float* g = ck + ((int64_t)cc * nwin + (in ? win : 0)) * kN + (k % (kN / 4)) * 4;
+        float* sm = dst + cc * Smem<T, NW>::kWinStride + k * 4;
+        if (vec) {
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(sm)), "l"(g), "r"(in ? 16 : 0)
+                         : "memory");
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sm[e] = in ? g[e] : 0.f;
+        }
+    }
+}
 
 template <typename T>
 __device__ __forceinline__ float staged(const unsigned char* base, int row, int k) {
@@ -388,9 +420,16 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
         float* dBg = p.dB + (b * G + g) * kN * L;
         float* dCg = p.dC + (b * G + g) * kN * L;
         const bool rvec = p.red_vec != 0;
-        // the checkpoint of the block being walked (the next, earlier one is fetched a block ahead)
-        float2 hblk = __ldcg(reinterpret_cast<const float2*>(ckpt + (int64_t)(blk1 - 1) * kN));
+        // the checkpoint of the block being walked (the next, earlier one is fetched a block
+        // ahead); with the forward's states, the window starts come with the block's rows
+        const bool ext = p.ext_ckpt != 0;
+        float2 hblk = ext ? make_float2(0.f, 0.f)
+                          : __ldcg(reinterpret_cast<const float2*>(ckpt + (int64_t)(blk1 - 1) * kN));
+        const int64_t nwin = (L + kWin - 1) / kWin;
+        const float* cktile = p.ckpt + row0 * nwin * kN;
+        const bool ckvec = (reinterpret_cast<uintptr_t>(p.ckpt) & 15u) == 0;
         auto issue_rev = [&](unsigned char* sg, int64_t ts) {
+            if (ext) stage_wins<T, NW>(reinterpret_cast<float*>(sg + S::WINS), cktile, nwin, ts / kWin, ckvec, tid);
             stage_rows<T, NW>(sg, u, L, kCT, ts, L, vec, tid);
             stage_rows<T, NW>(sg + kCT * S::kRow, dl, L, kCT, ts, L, vec, tid);
             if (zz) stage_rows<T, NW>(sg + 2 * kCT * S::kRow, zz, L, kCT, ts, L, vec, tid);
@@ -440,17 +479,17 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
             if (blk > blk0) issue_rev(stage_base + (cur ^ 1) * S::kStageBytes, t0 - kBT);
             __syncthreads();
 
-            const float2 hprev =
-                blk > blk0 ? __ldcg(reinterpret_cast<const float2*>(ckpt + (int64_t)(blk - 1) * kN))
-                           : make_float2(0.f, 0.f);
-            // the states entering the four windows, by the recurrence from the block checkpoint
-            // (kept in shared memory, one float2 per thread and window)
-            float2* wst = reinterpret_cast<float2*>(smem + S::WST) + tid;
-            {
+            // the states entering the four windows: staged with the rows (the forward's), or by
+            // the recurrence from the block checkpoint
+            float* wins = reinterpret_cast<float*>(stage + S::WINS) + c * S::kWinStride + 2 * j;
+            if (!ext) {
+                const float2 hprev =
+                    blk > blk0 ? __ldcg(reinterpret_cast<const float2*>(ckpt + (int64_t)(blk - 1) * kN))
+                               : make_float2(0.f, 0.f);
                 float2 hh = hblk;
 #pragma unroll
                 for (int w = 0; w < kBT / kWin; ++w) {
-                    wst[w * kThreads] = hh;
+                    *reinterpret_cast<float2*>(wins + w * kN) = hh;
                     if (w + 1 < kBT / kWin) {
 #pragma unroll 4
                         for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
@@ -461,11 +500,11 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                         }
                     }
                 }
+                hblk = hprev;
             }
-            hblk = hprev;
             for (int w = kBT / kWin - 1; w >= 0; --w) {
                 const int tw = w * kWin;   // first step of the window within the block
-                const float2 he = wst[w * kThreads];   // the state entering the window
+                const float2 he = *reinterpret_cast<const float2*>(wins + w * kN);   // the state entering the window
                 float2 hr[kWin], dAr[kWin];
                 float yw;   // y of step j of the window, summed over the states
                 {

@@ -206,7 +206,7 @@ struct FwdArgs {
     const float* h0;
     void* out;
     float* last_state;
-    float* ckpt = nullptr;   // states entering every 32-step block (register kernel only)
+    float* ckpt = nullptr;   // states entering every 8-step window (register kernel only)
 };
 
 // Launch the scan kernel of geometry `g` on workspace `ws` (laid out as FwdGeom says).
@@ -267,7 +267,7 @@ inline int fwd_launch(const ssm_dims_t& d, const FwdGeom& g, const FwdArgs& a, u
     prm.spin_limit = spin_limit;
     prm.delta_rows = delta_rows;
     prm.ckpt = a.ckpt;
-    prm.ckpt_blocks = (d.seqlen + 31) / 32;
+    prm.ckpt_wins = (d.seqlen + 7) / 8;
     if (v.smem > 48 * 1024 &&
         cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem) != cudaSuccess)
         return SSM_ERR_CUDA;

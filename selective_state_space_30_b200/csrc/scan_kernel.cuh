@@ -96,10 +96,10 @@ struct FwdParams {
     unsigned n_ctas;
     unsigned spin_limit;
     int delta_rows;    // rows of the delta box: CT (S6 layout) or the heads a tile can touch
-    // optional (register kernel): the state entering every 32-step block, for the backward,
-    // at ckpt[((b * dim + d) * ckpt_blocks + t / 32) * N + n]; nullptr: not stored
+    // optional (register kernel): the state entering every 8-step window, for the backward,
+    // at ckpt[((b * dim + d) * ckpt_wins + t / 8) * N + n]; nullptr: not stored
     float* ckpt;
-    int64_t ckpt_blocks;
+    int64_t ckpt_wins;
 };
 
 // The five 2-D tensor maps (time x rows) the producer loads boxes through.
@@ -806,7 +806,7 @@ __device__ __forceinline__ void produce(const FwdParams& p, const TensorMaps& tm
 
 // ------------------------------------------------------------------- kernel
 
-// CKPT: also store the state entering every 32-step block (p.ckpt, for the backward)
+// CKPT: also store the state entering every 8-step window (p.ckpt, for the backward)
 template <typename T, int N, int W, bool HEAD_A, int SPL, bool VEC, bool CKPT>
 __global__ void __launch_bounds__(Cfg<T, N, W, HEAD_A, SPL>::THREADS, 1)
 scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
@@ -912,15 +912,14 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
         const unsigned char* drow = sb + Cf::OFF_IN + (CT + drow_i) * RB + j * TPT * ESZ;
         const unsigned char* zrow = sb + Cf::OFF_IN + (2 * CT + lc) * RB + j * TPT * ESZ;
         const bool full_blk = t0 + TB <= hd.t1;
-        // the backward's stored states (CKPT): this lane's first state entering each 32-step
-        // part of the block, and whether that part lies in the unit
-        static_assert(TB == 32 || TB == 64, "32-step parts of a block");
+        // the backward's stored states (CKPT): this lane's first state entering each 8-step
+        // window of the block, and whether the lane's row is in bounds
+        static_assert(Cf::WT == 4 || Cf::WT == 8, "windows on 8-step bounds");
         float* ckp = nullptr;
-        bool ck0 = false, ck1 = false;
+        bool ck0 = false;
         if constexpr (CKPT) {
-            ckp = p.ckpt + ((hd.b * Dm + d) * p.ckpt_blocks + t0 / 32) * N + j;
+            ckp = p.ckpt + ((hd.b * Dm + d) * p.ckpt_wins + t0 / 8) * N + j;
             ck0 = ok && in_bounds(hd.b < p.batch && d < Dm && t0 < L, status);
-            ck1 = ck0 && t0 + 32 < hd.t1;
         }
         // -------- prologue: dt, dt*u (dA) of this lane's steps, two at a time
         {
@@ -1010,12 +1009,13 @@ scan_fwd_kernel(const FwdParams p, const __grid_constant__ TensorMaps tm) {
             } else {
                 load_window(w, 0);
             }
-            // the state entering a 32-step block, for the backward (blocks start on 32-step
+            // the state entering an 8-step window, for the backward (blocks start on 8-step
             // bounds).  Predicated stores, not a branch: the unrolled windows stay one stretch
             // of straight-line code for the scheduler.
-            if (CKPT && (tw & 31) == 0) {
+            if (CKPT && (tw & 7) == 0) {
+                const bool ckw = tw == 0 ? ck0 : ck0 && t0 + tw < hd.t1;
 #pragma unroll
-                for (int s = 0; s < S; ++s) st_global_if(ckp + (tw / 32) * N + s * TPC, h[s], tw == 0 ? ck0 : ck1);
+                for (int s = 0; s < S; ++s) st_global_if(ckp + (tw / 8) * N + s * TPC, h[s], ckw);
             }
             const auto& bw = bwA[bsel];
             const auto& cw_ = cwA[bsel];

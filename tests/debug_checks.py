@@ -60,7 +60,7 @@ def main():
         dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
         out = torch.empty_like(dev["u"])
         last = torch.empty((b, dm, 16), dtype=torch.float32, device="cuda")
-        ck = torch.empty((b, dm, (L + 31) // 32, 16), dtype=torch.float32, device="cuda")
+        ck = torch.empty((b, dm, (L + 7) // 8, 16), dtype=torch.float32, device="cuda")
         plan = ssm.ssm_scan_plan(d, 0)
         try:
             for k, v in opts.items():

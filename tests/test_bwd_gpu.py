@@ -187,13 +187,13 @@ def test_bwd_wait_timeout_reports_and_recovers():
 # ------------------------------------------------- the forward's stored states
 
 def _prefix_states(dims, inp, h0):
-    """The oracle's state entering every 32-step block: h0 (or zero) for block 0, else the
-    last state of the oracle run over the first 32k steps."""
-    nblk = (dims.seqlen + 31) // 32
-    ref = np.zeros((dims.batch, dims.dim, nblk, dims.dstate))
+    """The oracle's state entering every 8-step window: h0 (or zero) for window 0, else the
+    last state of the oracle run over the first 8k steps."""
+    nwin = (dims.seqlen + 7) // 8
+    ref = np.zeros((dims.batch, dims.dim, nwin, dims.dstate))
     ref[:, :, 0] = h0 if h0 is not None else 0.0
-    for k in range(1, nblk):
-        t = 32 * k
+    for k in range(1, nwin):
+        t = 8 * k
         dk = si.Dims(dims.batch, dims.dim, t, dims.dstate, dims.nheads, dims.ngroups, dims.dtype)
         pre = dict(inp)
         for key in ("u", "delta", "z", "B", "C"):
@@ -213,8 +213,8 @@ def _fwd_ckpt(dims, inp, h0=None, opts=None):
     d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, io)
     dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
     h0d = to_device(np.ascontiguousarray(h0, dtype=np.float32)) if h0 is not None else None
-    nblk = (dims.seqlen + 31) // 32
-    ck = torch.full((dims.batch, dims.dim, nblk, dims.dstate), float("nan"), device="cuda")
+    nwin = (dims.seqlen + 7) // 8
+    ck = torch.full((dims.batch, dims.dim, nwin, dims.dstate), float("nan"), device="cuda")
     res = []
     plan = ssm.ssm_scan_plan(d, 0)
     try:
@@ -249,10 +249,10 @@ CKPT_CASES = [
 
 @pytest.mark.parametrize("case", CKPT_CASES, ids=lambda c: f"{c[0].batch}x{c[0].dim}x{c[0].seqlen}n{c[0].dstate}"
                                                            f"{c[0].dtype}-{'plan' if c[1] is None else c[1]['warps']}")
-def test_forward_stores_block_states(case):
+def test_forward_stores_window_states(case):
     """ssm_selective_scan_fwd_ckpt: outputs bit-equal to the plain forward, and every stored
-    state (block k: the state entering step 32k) equal, within the forward's state bound,
-    to the oracle's last state over the first 32k steps (block 0: h0)."""
+    state (window k: the state entering step 8k) equal, within the forward's state bound,
+    to the oracle's last state over the first 8k steps (window 0: h0)."""
     dims, opts = case
     inp = si.make_inputs(dims, _recipe("c2"), 51)
     h0 = si.make_grad_inputs(dims, 52, h0=True)["h0"]
@@ -309,6 +309,40 @@ def test_bwd_with_forward_states(case):
             assert torch.equal(g[k], g0[k]), f"{k} differs from the recomputing backward"
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin["dlast"], h0=gin["h0"], want_dh0=True)
     check_grads(g, ref, mag, dims.dtype)
+
+
+def test_bwd_with_forward_states_8_byte_aligned():
+    """Stored states at an address that is 8- but not 16-byte aligned take the element copies
+    instead of the 16-byte ones: the same gradients (dB and dC within their rounding)."""
+    import selective_state_space_30_b200 as ssm
+    dims, kind, dlast, h0, softplus = CASES[0]
+    inp = si.make_inputs(dims, _recipe(kind), 43)
+    gin = si.make_grad_inputs(dims, 44, dlast=dlast, h0=h0)
+    _, _, ck = _fwd_ckpt(dims, inp, gin.get("h0"))
+    buf = torch.empty(ck.numel() + 2, dtype=torch.float32, device="cuda")
+    ck8 = buf[2:].view(ck.shape)
+    ck8.copy_(ck)
+    assert ck8.data_ptr() % 16 == 8
+    dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    io = ssm.SSM_BF16 if dims.dtype == "bf16" else ssm.SSM_F32
+    d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, io)
+    ws = torch.empty(ssm.ssm_selective_scan_bwd_workspace_size(d), dtype=torch.uint8, device="cuda")
+    res = []
+    for c in (ck, ck8):
+        res.append(ssm.selective_scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"],
+                                          to_device(gin["dout"]), dev["D"], dev["z"], dev["delta_bias"], True,
+                                          h0=to_device(gin.get("h0")), dlast=to_device(gin.get("dlast")),
+                                          want_dh0=True, workspace=ws, ckpt=c))
+        assert ssm.ssm_selective_scan_bwd_device_status(ws) == ssm.SSM_OK
+    torch.cuda.synchronize()
+    for k in res[0]:
+        if res[0][k] is None:
+            continue
+        if k in ("dB", "dC"):
+            scale = float(torch.max(torch.abs(res[0][k]))) + 1.0
+            assert float(torch.max(torch.abs(res[1][k] - res[0][k]))) <= 1e-5 * scale, k
+        else:
+            assert torch.equal(res[0][k], res[1][k]), k
 
 
 # ------------------------------------------ the generic backward (other layouts)

@@ -862,15 +862,18 @@ def run_bwd(args):
     alg = _bwd_bytes(d)
     ck_bytes = int(ck.numel() * 4) if stored else 0
 
-    def roof(ms_, traffic_key):
+    def roof(ms_, traffic_key, state_bytes=0):
+        # algorithmic bytes: the call's inputs read and outputs written (the stored states are
+        # an input of the stored-state call)
+        a = alg + state_bytes
         gexps = exps / (ms_ * 1e-3) / 1e9
-        gbs = alg / (ms_ * 1e-3) / 1e9
+        gbs = a / (ms_ * 1e-3) / 1e9
         return {"bound": "alu", "achieved": gexps, "peak": mufu_peak, "unit": "Gexp/s", "frac": gexps / mufu_peak,
                 "traffic": _traffic_from_profiles(w.name, key=traffic_key, sha=_src_hash(("bwd.cu",))),
                 "peak_source": f"148 SMs x 16 ex2/clk x {sm_max_mhz:.0f} MHz ({src} sm_max_mhz)",
                 "exps_per_launch": exps,
                 "hbm": {"achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                        "alg_bytes_per_launch": alg, "peak_source": src}}
+                        "alg_bytes_per_launch": a, "state_bytes_read": state_bytes, "peak_source": src}}
 
     line = {"metric": "selective-scan backward Gelem/s (B*D*L/s) on 1 B200", "op": "bwd",
             "value": job_throughput(world, elems, args.steps, total), "unit": "Gelem/s",
@@ -879,12 +882,12 @@ def run_bwd(args):
             "dtype": "f32 (bf16 I/O)" if d.dtype == "bf16" else "f32", "data": "synthetic (seeded splitmix64)",
             "config": {"workload": w.name, "batch": d.batch, "dim": d.dim, "seqlen": d.seqlen,
                        "dstate": d.dstate, "io_dtype": d.dtype, "parallelism": f"replicas x{world}",
-                       "states": (f"stored by the forward (ssm_selective_scan_fwd_ckpt, {ck_bytes / 1e6:.0f} MB), "
-                                  "read by ssm_selective_scan_bwd_ckpt") if stored else
+                       "states": (f"stored by the forward every 8 steps (ssm_selective_scan_fwd_ckpt, "
+                                  f"{ck_bytes / 1e6:.0f} MB), read by ssm_selective_scan_bwd_ckpt") if stored else
                                  "recomputed (the generic backward: per-head layout or dstate other than 16)",
                        "l2": f"inputs {in_bytes / 1e6:.0f} MB and workspace {nws / 1e6:.0f} MB (> 126 MB L2), "
                              "no flush"},
-            "roofline": roof(ms, ("bwd_ckpt:" if stored else "bwd:") + w.name),
+            "roofline": roof(ms, ("bwd_ckpt:" if stored else "bwd:") + w.name, ck_bytes),
             "recompute": {"what": "ssm_selective_scan_bwd: the backward recomputes the states itself",
                           "ms_per_step": ms_re, "value": job_throughput(world, elems, args.steps, total_re),
                           "roofline": roof(ms_re, "bwd:" + w.name)},

@@ -227,10 +227,10 @@ def _selective_scan_function():
 
     class SelectiveScanFn(torch.autograd.Function):
         @staticmethod
-        def forward(ctx, u, delta, A, B, C, D, z, delta_bias, h0, softplus):
+        def forward(ctx, u, delta, A, B, C, D, z, delta_bias, h0, softplus, store_states):
             # where the backward covers the shape, the forward stores the states it walks from
             ck = None
-            if any(ctx.needs_input_grad) and bwd_covers(u, delta, A, B) and u.numel() > 0:
+            if store_states and any(ctx.needs_input_grad) and bwd_covers(u, delta, A, B) and u.numel() > 0:
                 ck = torch.empty(ckpt_shape(u.shape[0], u.shape[1], u.shape[2], B.shape[2]),
                                  dtype=torch.float32, device=u.device)
             out, last = selective_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus, h0=h0, ckpt=ck)
@@ -247,15 +247,17 @@ def _selective_scan_function():
                                    ckpt=ck)
             return (g["du"], g["ddelta"], g["dA"], g["dB"].to(B.dtype), g["dC"].to(C.dtype),
                     g["dD"] if D is not None else None, g["dz"], g["ddelta_bias"] if delta_bias is not None else None,
-                    g["dh0"], None)
+                    g["dh0"], None, None)
 
     _fn_cls = SelectiveScanFn
     return _fn_cls
 
 
-def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True, h0=None):
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True, h0=None,
+                      store_states: bool = True):
     """The forward scan as a differentiable torch operation: returns (out, last_state),
-    and the backward runs ssm_selective_scan_bwd (dstate 8 to 128, both layouts; on the
+    and the backward runs ssm_selective_scan_bwd (dstate 8 to 128, both layouts).  On the
     shapes its tiled kernel takes, the forward also stores the states the backward walks
-    back from).  dB and dC are formed in fp32 and returned in B's and C's dtype."""
-    return _selective_scan_function().apply(u, delta, A, B, C, D, z, delta_bias, h0, softplus)
+    back from (ckpt_shape: B*D*L*N/2 bytes) unless store_states is False; the backward then
+    recomputes them.  dB and dC are formed in fp32 and returned in B's and C's dtype."""
+    return _selective_scan_function().apply(u, delta, A, B, C, D, z, delta_bias, h0, softplus, store_states)

@@ -93,3 +93,29 @@ def test_unused_last_state_and_unwanted_h0(oracle_backed):
     for k, name in (("u", "du"), ("B", "dB"), ("D", "dD"), ("delta_bias", "ddelta_bias")):
         np.testing.assert_allclose(_np(p[k].grad), g[name], rtol=1e-12, atol=1e-14)
     assert p["h0"].grad is None
+
+
+@pytest.mark.parametrize("store_states", [True, False])
+def test_states_stored_only_when_asked(monkeypatch, store_states):
+    """On a shape the tiled backward covers (S6 layout, dstate 16, 32 channels), the forward
+    is handed a state buffer of ckpt_shape and the backward the same buffer; with
+    store_states False neither gets one (the backward recomputes the states)."""
+    seen = {}
+
+    def fwd(*a, ckpt=None, **kw):
+        seen["fwd"] = ckpt
+        return _fake_fwd(*a, **kw)
+
+    def bwd(*a, ckpt=None, **kw):
+        seen["bwd"] = ckpt
+        return _fake_bwd(*a, **kw)
+
+    monkeypatch.setattr(ssm, "selective_scan_fwd", fwd)
+    monkeypatch.setattr(ssm, "selective_scan_bwd", bwd)
+    p = _problem(np.random.default_rng(9), 1, 32, 6, 16)
+    out, last = ssm.selective_scan_fn(*(p[k] for k in ORDER[:8]), True, p["h0"], store_states=store_states)
+    (out.sum() + last.sum()).backward()
+    if store_states:
+        assert tuple(seen["fwd"].shape) == ssm.ckpt_shape(1, 32, 6, 16) and seen["bwd"] is seen["fwd"]
+    else:
+        assert seen["fwd"] is None and seen["bwd"] is None

@@ -21,8 +21,9 @@ GRAD_OF = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "
            "delta_bias": "ddelta_bias"}
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_autograd_matches_oracle(dtype):
+@pytest.mark.parametrize("dtype,store_states", [("bf16", True), ("f32", True), ("bf16", False)])
+def test_autograd_matches_oracle(dtype, store_states):
+    """store_states False: the forward stores nothing and the backward recomputes the states."""
     import selective_state_space_30_b200 as ssm
     dims = si.Dims(2, 64, 100, 16, dtype=dtype)
     inp = si.make_inputs(dims, _recipe("c2"), 51)
@@ -30,7 +31,7 @@ def test_autograd_matches_oracle(dtype):
     gin = si.make_grad_inputs(dims, 52, dlast=True, h0=True)
     leaves = {k: to_device(inp[k]).requires_grad_() for k in INPUTS}
     h0 = to_device(gin["h0"]).requires_grad_()
-    out, last = ssm.selective_scan_fn(*(leaves[k] for k in INPUTS), softplus=True, h0=h0)
+    out, last = ssm.selective_scan_fn(*(leaves[k] for k in INPUTS), softplus=True, h0=h0, store_states=store_states)
     torch.autograd.backward([out, last], [to_device(gin["dout"]), to_device(gin["dlast"])])
     torch.cuda.synchronize()
 

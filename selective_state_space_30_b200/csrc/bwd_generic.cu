@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "bwd_generic.h"
 #include "scan_kernel.cuh"   // ex2_approx, rcp_approx, softplus1, kLog2e
@@ -57,10 +58,14 @@ struct GParams {
 
 template <typename T> struct GIo;
 template <> struct GIo<float> {
+    using raw = float;
+    __device__ static float f(raw v) { return v; }
     __device__ static float ld(const void* p, int64_t i) { return static_cast<const float*>(p)[i]; }
     __device__ static void st(void* p, int64_t i, float v) { static_cast<float*>(p)[i] = v; }
 };
 template <> struct GIo<__nv_bfloat16> {
+    using raw = unsigned short;
+    __device__ static float f(raw v) { return __uint_as_float((uint32_t)v << 16); }
     __device__ static float ld(const void* p, int64_t i) {
         return __uint_as_float((uint32_t) static_cast<const unsigned short*>(p)[i] << 16);
     }
@@ -76,33 +81,42 @@ __device__ __forceinline__ void gred4(float* dst, const float (&v)[4]) {
                  : "memory");
 }
 
-// Shared memory (floats) for T = cpb * N threads; rows of T + 1 floats so that a
-// thread walking one row of states and its neighbours walking the next rows meet
-// different banks.
+// Shared memory (floats) for T = cpb * N threads.  The state and state-gradient rows
+// (sH, sG) are T + 1 floats long, so that a thread walking one row and its neighbours
+// walking the next meet different banks.  B and C are kept per step, [step][N + 1]: a
+// thread reads its own state's column and a team a step's row, both without bank
+// conflicts.  The per-(channel, step) arrays are [channel][KP] with KP a multiple of 4:
+// a thread reads four steps of its channel in one 16-byte load.
+constexpr int KP = gK + 4;
+enum { PC_DT = 0, PC_DU, PC_U, PC_X, PC_DY, PC_DOUT, PC_Z, PC_DA, PC_W, kPC };
+// PC_DA, PC_W (one A per head): the step's decay dA = exp(dt A) and dt dA, formed once per
+// (channel, step) for all of its states
 struct GSmem {
-    int T, TP, N, cpb;
-    int H, G, BLK, Bs, Cs, PC;   // offsets: sH, sG, sBlk, sB, sC, per-(channel, step) arrays
+    int T, TP, N, NB, cpb, NCH;
+    int H, G, BLK, Bs, Cs, PART, PC;   // offsets: sH, sG, sBlk, sB, sC, chunk sums, per-(channel, step) arrays
     int total;
-    __host__ __device__ GSmem(int n, int c) : T(c * n), TP(c * n + 1), N(n), cpb(c) {
+    __host__ __device__ GSmem(int n, int c)
+        : T(c * n), TP(c * n + 1), N(n), NB(n + 1), cpb(c), NCH((n + 31) / 32) {
         H = 0;                              // [gK + 1][TP]: the state entering the block, then after each step
         G = H + (gK + 1) * TP;              // [gK][TP]: dLoss/dh_t of each step
         BLK = G + gK * TP;                  // [gSegB][T]: the state entering each block of the segment
-        Bs = BLK + gSegB * T;               // [N][gK + 1]: B of the block
-        Cs = Bs + N * (gK + 1);             // [N][gK + 1]: C of the block
-        PC = Cs + N * (gK + 1);             // 7 arrays [cpb][gK + 1]: dt, dt*u, u, x, dy, dout, z
-        total = PC + 7 * cpb * (gK + 1);
+        Bs = BLK + gSegB * T;               // [gK][NB]: B of the block
+        Cs = Bs + gK * NB;                  // [gK][NB]: C of the block
+        PART = Cs + gK * NB;                // [cpb * NCH chunks][3][gK]: a chunk's parts of y, sum g B, the decay term
+        PC = (PART + cpb * NCH * 3 * gK + 3) / 4 * 4;   // kPC arrays [cpb][KP], 16-byte aligned
+        total = PC + kPC * cpb * KP;
     }
 };
-enum { PC_DT = 0, PC_DU, PC_U, PC_X, PC_DY, PC_DOUT, PC_Z };
 
 // PREF: the CTA holds at least 4 channels (at most 8 B and C values per thread and block),
-// so a block's inputs fit in registers and are loaded one block ahead
-template <typename T, int N, bool PREF>
+// so a block's inputs fit in registers and are loaded one block ahead.  HEAD: one scalar A
+// per head (the decay of a step is the same for every state of a channel).
+template <typename T, int N, bool PREF, bool HEAD>
 __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(const GParams p) {
-    extern __shared__ float gsm[];
+    extern __shared__ __align__(16) float gsm[];
     const GSmem S(N, p.cpb);
     const int NT = S.T, TP = S.TP;
-    constexpr int KP = gK + 1;
+    constexpr int NB = N + 1;
     const int tid = threadIdx.x;
     const int c = tid / N, n = tid % N;
     const int64_t L = p.seqlen, Dm = p.dim, H = p.nheads, G = p.ngroups;
@@ -117,22 +131,44 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     float* sBlk = gsm + S.BLK;
     float* sB = gsm + S.Bs;
     float* sC = gsm + S.Cs;
+    float* sPart = gsm + S.PART;
     float* pc = gsm + S.PC;
     const int cpb = p.cpb;
     auto at = [&](int arr, int cc, int k) -> float& { return pc[(arr * cpb + cc) * KP + k]; };
+    auto at4 = [&](int arr, int cc, int k) -> float4 {
+        return *reinterpret_cast<const float4*>(pc + (arr * cpb + cc) * KP + k);
+    };
+    // every channel of the CTA in one head: the head's ddelta terms are summed here first
+    const bool one_head = HEAD && d0 / P == (d0 + cpb - 1) / P;
 
     // A of this thread's (channel, state), natural units and log2 units
-    const float An = p.head ? __ldg(p.A + d / P) : __ldg(p.A + d * N + n);
+    const float An = HEAD ? __ldg(p.A + d / P) : __ldg(p.A + d * N + n);
     const float a2 = An * kLog2e;
     const int nblk = (int)((L + gK - 1) / gK);
 
     // Block blk in two halves: load() reads its inputs into registers (issued a block
     // ahead, so the loads are in flight while the current block runs), store() writes
     // them to shared memory with the per-(channel, step) values: dt and dt*u (full: also
-    // u, the softplus argument x, dy = dout silu(z), dout, z), and the B (full: C) rows.
+    // u, the softplus argument x, dy = dout silu(z), dout, z; one A per head: dA, dt dA),
+    // and the B (full: C) rows.
     constexpr int PPT = gK / N > 0 ? gK / N : 1;   // (channel, step) pairs per thread, at most
-    constexpr int BPT = PREF ? 8 : 1;               // B (C) values per thread, at most
-    float ru[PPT], rx[PPT], rdo[PPT], rz[PPT], rb[BPT], rc[BPT];
+    // B and C rows in 16-byte pieces of EPC steps: CPR pieces per row and block, at most VPT
+    // per thread (PREF: at least 4 channels, so at least 4 N threads)
+    constexpr int EPC = 16 / (int)sizeof(T), CPR = gK / EPC;
+    constexpr int VPT = PREF ? (CPR / 4 > 0 ? CPR / 4 : 1) : 1;
+    const bool vecbc = ((reinterpret_cast<uintptr_t>(p.B) | reinterpret_cast<uintptr_t>(p.C)) & 15u) == 0 &&
+                       L % EPC == 0;
+    float ru[PPT], rx[PPT], rdo[PPT], rz[PPT];
+    uint4 rb[VPT], rc[VPT];
+    // EPC elements of row `src` from step t, zero past L (16-byte load when vecbc and whole)
+    auto piece = [&](const void* src, int64_t off, int64_t t) -> uint4 {
+        if (vecbc && t + EPC <= L) return __ldg(reinterpret_cast<const uint4*>(static_cast<const T*>(src) + off));
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        typename GIo<T>::raw* e = reinterpret_cast<typename GIo<T>::raw*>(&v);
+        for (int j = 0; j < EPC; ++j)
+            if (t + j < L) e[j] = reinterpret_cast<const typename GIo<T>::raw*>(src)[off + j];
+        return v;
+    };
     auto load = [&](int blk, bool full) {
         if constexpr (!PREF) return;   // fewer than 4 channels: store() loads for itself
         const int64_t t0 = (int64_t)blk * gK;
@@ -154,17 +190,32 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             }
         }
 #pragma unroll
-        for (int e = 0; e < BPT; ++e) {
+        for (int e = 0; e < VPT; ++e) {
             const int i = tid + e * NT;
-            rb[e] = rc[e] = 0.f;
-            if (i < N * gK) {
-                const int nn = i / gK, k = i % gK;
-                const int64_t t = t0 + k, off = ((b * G + g) * N + nn) * L + t;
-                if (t < L) {
-                    rb[e] = GIo<T>::ld(p.B, off);
-                    if (full) rc[e] = GIo<T>::ld(p.C, off);
-                }
+            if (i < N * CPR) {
+                const int nn = i / CPR, q = i % CPR;
+                const int64_t t = t0 + q * EPC, off = ((b * G + g) * N + nn) * L + t;
+                rb[e] = piece(p.B, off, t);
+                if (full) rc[e] = piece(p.C, off, t);
             }
+        }
+    };
+    // the per-(channel, step) values of one pair from its inputs (past L: dt = 0, so dA = 1)
+    auto put = [&](int cc, int k, bool valid, float uv, float x, float dov, float zv, bool full) {
+        const float dt = valid ? (p.softplus ? softplus1(x) : x) : 0.f;
+        at(PC_DT, cc, k) = dt;
+        at(PC_DU, cc, k) = dt * uv;
+        if (HEAD) {
+            const float dA = ex2_approx(dt * (__ldg(p.A + (d0 + cc) / P) * kLog2e));
+            at(PC_DA, cc, k) = dA;
+            at(PC_W, cc, k) = dt * dA;
+        }
+        if (full) {
+            at(PC_U, cc, k) = uv;
+            at(PC_X, cc, k) = x;
+            at(PC_DY, cc, k) = p.z ? dov * (zv * gsigmoid(zv)) : dov;
+            at(PC_DOUT, cc, k) = dov;
+            at(PC_Z, cc, k) = zv;
         }
     };
     auto store = [&](int blk, bool full) {
@@ -174,31 +225,22 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             for (int i = tid; i < cpb * gK; i += NT) {
                 const int cc = i / gK, k = i % gK;
                 const int64_t t = t0 + k, dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
-                float dt = 0.f, uv = 0.f, x = 0.f, dov = 0.f, zv = 0.f;
+                float uv = 0.f, x = 0.f, dov = 0.f, zv = 0.f;
                 if (t < L) {
                     uv = GIo<T>::ld(p.u, rr * L + t);
                     x = GIo<T>::ld(p.delta, (b * H + hh) * L + t) + (p.bias ? __ldg(p.bias + hh) : 0.f);
-                    dt = p.softplus ? softplus1(x) : x;
                     if (full) {
                         dov = GIo<T>::ld(p.dout, rr * L + t);
                         if (p.z) zv = GIo<T>::ld(p.z, rr * L + t);
                     }
                 }
-                at(PC_DT, cc, k) = dt;
-                at(PC_DU, cc, k) = dt * uv;
-                if (full) {
-                    at(PC_U, cc, k) = uv;
-                    at(PC_X, cc, k) = x;
-                    at(PC_DY, cc, k) = p.z ? dov * (zv * gsigmoid(zv)) : dov;
-                    at(PC_DOUT, cc, k) = dov;
-                    at(PC_Z, cc, k) = zv;
-                }
+                put(cc, k, t < L, uv, x, dov, zv, full);
             }
             for (int i = tid; i < N * gK; i += NT) {
                 const int nn = i / gK, k = i % gK;
                 const int64_t t = t0 + k, off = ((b * G + g) * N + nn) * L + t;
-                sB[nn * KP + k] = t < L ? GIo<T>::ld(p.B, off) : 0.f;
-                if (full) sC[nn * KP + k] = t < L ? GIo<T>::ld(p.C, off) : 0.f;
+                sB[k * NB + nn] = t < L ? GIo<T>::ld(p.B, off) : 0.f;
+                if (full) sC[k * NB + nn] = t < L ? GIo<T>::ld(p.C, off) : 0.f;
             }
             return;
         }
@@ -207,37 +249,41 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             const int i = tid + e * NT;
             if (i < cpb * gK) {
                 const int cc = i / gK, k = i % gK;
-                const bool valid = t0 + k < L;   // past L: no step (dt = 0)
-                const float dt = valid ? (p.softplus ? softplus1(rx[e]) : rx[e]) : 0.f;
-                at(PC_DT, cc, k) = dt;
-                at(PC_DU, cc, k) = dt * ru[e];
-                if (full) {
-                    at(PC_U, cc, k) = ru[e];
-                    at(PC_X, cc, k) = rx[e];
-                    at(PC_DY, cc, k) = p.z ? rdo[e] * (rz[e] * gsigmoid(rz[e])) : rdo[e];
-                    at(PC_DOUT, cc, k) = rdo[e];
-                    at(PC_Z, cc, k) = rz[e];
-                }
+                put(cc, k, t0 + k < L, ru[e], rx[e], rdo[e], rz[e], full);
             }
         }
 #pragma unroll
-        for (int e = 0; e < BPT; ++e) {
+        for (int e = 0; e < VPT; ++e) {
             const int i = tid + e * NT;
-            if (i < N * gK) {
-                const int nn = i / gK, k = i % gK;
-                sB[nn * KP + k] = rb[e];
-                if (full) sC[nn * KP + k] = rc[e];
+            if (i < N * CPR) {
+                const int nn = i / CPR, k0 = (i % CPR) * EPC;
+                const typename GIo<T>::raw* vb = reinterpret_cast<const typename GIo<T>::raw*>(&rb[e]);
+                const typename GIo<T>::raw* vc = reinterpret_cast<const typename GIo<T>::raw*>(&rc[e]);
+#pragma unroll
+                for (int j = 0; j < EPC; ++j) {
+                    sB[(k0 + j) * NB + nn] = GIo<T>::f(vb[j]);
+                    if (full) sC[(k0 + j) * NB + nn] = GIo<T>::f(vc[j]);
+                }
             }
         }
     };
     // the recurrence over the staged block from state h (steps past L have dt = 0: no
     // change); keep: every state into sH (row 0 the entering state, row k + 1 after step k)
-    auto run_block = [&](float h, bool keep) -> float {
+    auto run_block = [&](float h, auto keep_c) -> float {
+        constexpr bool keep = decltype(keep_c)::value;   // a compile-time choice: no branch per step
         if (keep) sH[tid] = h;
-        for (int k = 0; k < gK; ++k) {
-            const float dA = ex2_approx(at(PC_DT, c, k) * a2);
-            h = fmaf(dA, h, at(PC_DU, c, k) * sB[n * KP + k]);
-            if (keep) sH[(k + 1) * TP + tid] = h;
+#pragma unroll 1
+        for (int k0 = 0; k0 < gK; k0 += 4) {
+            const float4 du4 = at4(PC_DU, c, k0);
+            const float4 x4 = HEAD ? at4(PC_DA, c, k0) : at4(PC_DT, c, k0);
+            const float duv[4] = {du4.x, du4.y, du4.z, du4.w}, xv[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = k0 + e;
+                const float dA = HEAD ? xv[e] : ex2_approx(xv[e] * a2);
+                h = fmaf(dA, h, duv[e] * sB[k * NB + n]);
+                if (keep) sH[(k + 1) * TP + tid] = h;
+            }
         }
         return h;
     };
@@ -251,15 +297,15 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
         store(blk, false);
         __syncthreads();
         if (blk + 1 < nblk) load(blk + 1, false);
-        h = run_block(h, false);
+        h = run_block(h, std::false_type{});
     }
 
     // ---- 2. segments last to first
     float gst = p.dlast ? __ldg(p.dlast + row * N + n) : 0.f;   // dLoss/dh after the last step
     float da = 0.f, dDacc = 0.f;
-    // pass A: one team of TS consecutive threads per (channel, step) sums over the states
-    constexpr int TS = N > gK ? N / gK : 1;
-    const int team = tid / TS, tl = tid % TS, nteams = NT / TS;
+    // pass A: a warp per chunk of up to 32 states of one channel, a lane per step
+    constexpr int NCH = (N + 31) / 32, NC = N < 32 ? N : 32;
+    const int warp = tid / 32, lane = tid % 32, nwarps = NT / 32 > 0 ? NT / 32 : 1;
     for (int seg = p.nseg - 1; seg >= 0; --seg) {
         const int b0 = seg * gSegB, b1 = min(nblk, b0 + gSegB);
         float hs = p.ckpt[(row * p.nseg + seg) * N + n];
@@ -271,7 +317,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             __syncthreads();
             if (blk + 1 < b1) load(blk + 1, false);
             else load(b1 - 1, true);   // the first block of the walk
-            hs = run_block(hs, false);
+            hs = run_block(hs, std::false_type{});
         }
         for (int blk = b1 - 1; blk >= b0; --blk) {
             const int64_t t0 = (int64_t)blk * gK;
@@ -279,72 +325,147 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             store(blk, true);
             __syncthreads();
             if (blk > b0) load(blk - 1, true);
-            run_block(sBlk[(blk - b0) * NT + tid], true);
+            run_block(sBlk[(blk - b0) * NT + tid], std::true_type{});
+            const int kend = (int)(L - t0 < gK ? L - t0 : gK);   // steps of the block inside L
             // the state gradient back through the block: g += dy C is dLoss/dh_t
-            for (int k = gK - 1; k >= 0; --k) {
-                if (t0 + k < L) {
-                    gst = fmaf(at(PC_DY, c, k), sC[n * KP + k], gst);
-                    sG[k * TP + tid] = gst;
-                    const float dt = at(PC_DT, c, k);
-                    const float dA = ex2_approx(dt * a2);
-                    da = fmaf(gst * sH[k * TP + tid], dt * dA, da);
-                    gst *= dA;
-                } else {
-                    sG[k * TP + tid] = 0.f;
+#pragma unroll 1
+            for (int k0 = gK - 4; k0 >= 0; k0 -= 4) {
+                const float4 dy4 = at4(PC_DY, c, k0);
+                const float4 x4 = HEAD ? at4(PC_DA, c, k0) : at4(PC_DT, c, k0);
+                const float4 w4 = HEAD ? at4(PC_W, c, k0) : x4;
+                const float dyv[4] = {dy4.x, dy4.y, dy4.z, dy4.w}, xv[4] = {x4.x, x4.y, x4.z, x4.w};
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int e = 3; e >= 0; --e) {
+                    const int k = k0 + e;
+                    if (k < kend) {
+                        gst = fmaf(dyv[e], sC[k * NB + n], gst);
+                        sG[k * TP + tid] = gst;
+                        float dA, w;
+                        if (HEAD) {
+                            dA = xv[e];
+                            w = wv[e];
+                        } else {
+                            dA = ex2_approx(xv[e] * a2);
+                            w = xv[e] * dA;
+                        }
+                        da = fmaf(gst * sH[k * TP + tid], w, da);
+                        gst *= dA;
+                    } else {
+                        sG[k * TP + tid] = 0.f;
+                    }
                 }
             }
             if (n == 0)
                 for (int k = 0; k < gK; ++k)
-                    if (t0 + k < L) dDacc = fmaf(at(PC_DY, c, k), at(PC_U, c, k), dDacc);
+                    if (k < kend) dDacc = fmaf(at(PC_DY, c, k), at(PC_U, c, k), dDacc);
             __syncthreads();   // sH and sG complete
-            // pass A: per (channel, step), y = sum C h, gB = sum g B, q = sum g h_(t-1) A dA
-            for (int pr = team; pr < cpb * gK; pr += nteams) {
-                const int cc = pr / gK, k = pr % gK;
-                const int64_t t = t0 + k;
-                const float dt = at(PC_DT, cc, k);
-                const float dAh = ex2_approx(dt * a2);   // one A per head: the decay of every state
-                float y = 0.f, gB = 0.f, q = 0.f;
-                for (int nn = tl; nn < N; nn += TS) {
-                    const int idx = cc * N + nn;
-                    const float gv = sG[k * TP + idx];
-                    const float Ann = p.head ? An : __ldg(p.A + (d0 + cc) * N + nn);
-                    const float dA = p.head ? dAh : ex2_approx(dt * (Ann * kLog2e));
-                    y = fmaf(sC[nn * KP + k], sH[(k + 1) * TP + idx], y);
-                    gB = fmaf(gv, sB[nn * KP + k], gB);
-                    q = fmaf(gv * sH[k * TP + idx], Ann * dA, q);
-                }
-#pragma unroll
-                for (int o = 1; o < TS; o <<= 1) {
-                    y += __shfl_xor_sync(0xffffffffu, y, o);
-                    gB += __shfl_xor_sync(0xffffffffu, gB, o);
-                    q += __shfl_xor_sync(0xffffffffu, q, o);
-                }
-                if (tl == 0 && t < L) {
-                    const int64_t dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
-                    const float uv = at(PC_U, cc, k), dy = at(PC_DY, cc, k);
-                    const float Dv = p.D ? __ldg(p.D + dd) : 0.f;
-                    GIo<T>::st(p.du, rr * L + t, fmaf(dt, gB, dy * Dv));
-                    const float ddt = fmaf(uv, gB, q);
-                    atomicAdd(p.dd_acc + (b * H + hh) * L + t, p.softplus ? ddt * gsigmoid(at(PC_X, cc, k)) : ddt);
-                    if (p.z) {
-                        const float zv = at(PC_Z, cc, k), sg = gsigmoid(zv);
-                        GIo<T>::st(p.dz, rr * L + t, at(PC_DOUT, cc, k) * fmaf(Dv, uv, y) * (sg * fmaf(zv, 1.f - sg, 1.f)));
+            // pass A, first half: per chunk and step (lane), the chunk's parts of y = sum C h,
+            // gB = sum g B and q = sum g h_(t-1) (A dA) into sPart.  No shuffles: the lanes walk
+            // rows of odd length, so they meet different banks.
+            if (NT >= 32) {
+                for (int ch = warp; ch < cpb * NCH; ch += nwarps) {
+                    const int cc = ch / NCH, n0 = (ch % NCH) * NC, k = lane;
+                    const float* grow = sG + k * TP + cc * N + n0;
+                    const float* hrow = sH + (k + 1) * TP + cc * N + n0;
+                    const float* prow = sH + k * TP + cc * N + n0;
+                    const float* brow = sB + k * NB + n0;
+                    const float* crow = sC + k * NB + n0;
+                    const float dt = at(PC_DT, cc, k);
+                    float y = 0.f, gB = 0.f, q = 0.f;
+#pragma unroll 8
+                    for (int i = 0; i < NC; ++i) {
+                        const float gv = grow[i];
+                        y = fmaf(crow[i], hrow[i], y);
+                        gB = fmaf(gv, brow[i], gB);
+                        if (HEAD) {
+                            q = fmaf(gv, prow[i], q);
+                        } else {
+                            const float Ann = __ldg(p.A + (d0 + cc) * N + n0 + i);
+                            q = fmaf(gv * prow[i], Ann * ex2_approx(dt * (Ann * kLog2e)), q);
+                        }
                     }
+                    float* pp = sPart + ch * 3 * gK + k;
+                    pp[0] = y;
+                    pp[gK] = gB;
+                    pp[2 * gK] = q;
+                }
+            } else {
+                // fewer than 32 threads (one channel of dstate 8 or 16): a thread per step
+                for (int it = tid; it < cpb * NCH * gK; it += NT) {
+                    const int ch = it / gK, k = it % gK, cc = ch / NCH, n0 = (ch % NCH) * NC;
+                    const float dt = at(PC_DT, cc, k);
+                    float y = 0.f, gB = 0.f, q = 0.f;
+                    for (int i = 0; i < NC; ++i) {
+                        const float gv = sG[k * TP + cc * N + n0 + i], hp = sH[k * TP + cc * N + n0 + i];
+                        y = fmaf(sC[k * NB + n0 + i], sH[(k + 1) * TP + cc * N + n0 + i], y);
+                        gB = fmaf(gv, sB[k * NB + n0 + i], gB);
+                        if (HEAD) {
+                            q = fmaf(gv, hp, q);
+                        } else {
+                            const float Ann = __ldg(p.A + (d0 + cc) * N + n0 + i);
+                            q = fmaf(gv * hp, Ann * ex2_approx(dt * (Ann * kLog2e)), q);
+                        }
+                    }
+                    float* pp = sPart + ch * 3 * gK + k;
+                    pp[0] = y;
+                    pp[gK] = gB;
+                    pp[2 * gK] = q;
+                }
+            }
+            __syncthreads();
+            // second half: per (channel, step), the chunks' parts added in order, then the outputs
+            for (int it = tid; it < cpb * gK; it += NT) {
+                const int cc = it / gK, k = it % gK;
+                const int64_t t = t0 + k;
+                if (t >= L) continue;
+                float y = 0.f, gB = 0.f, q = 0.f;
+#pragma unroll
+                for (int j = 0; j < NCH; ++j) {
+                    const float* pp = sPart + (cc * NCH + j) * 3 * gK + k;
+                    y += pp[0];
+                    gB += pp[gK];
+                    q += pp[2 * gK];
+                }
+                const float dt = at(PC_DT, cc, k);
+                const int64_t dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
+                if (HEAD) q *= __ldg(p.A + hh) * at(PC_DA, cc, k);   // one decay for every state
+                const float uv = at(PC_U, cc, k), dy = at(PC_DY, cc, k);
+                const float Dv = p.D ? __ldg(p.D + dd) : 0.f;
+                GIo<T>::st(p.du, rr * L + t, fmaf(dt, gB, dy * Dv));
+                const float ddt = fmaf(uv, gB, q);
+                const float ddl = p.softplus ? ddt * gsigmoid(at(PC_X, cc, k)) : ddt;
+                if (one_head) at(PC_X, cc, k) = ddl;   // summed over the CTA's channels below
+                else atomicAdd(p.dd_acc + (b * H + hh) * L + t, ddl);
+                if (p.z) {
+                    const float zv = at(PC_Z, cc, k), sg = gsigmoid(zv);
+                    GIo<T>::st(p.dz, rr * L + t, at(PC_DOUT, cc, k) * fmaf(Dv, uv, y) * (sg * fmaf(zv, 1.f - sg, 1.f)));
+                }
+            }
+            if (one_head) {
+                __syncthreads();   // every channel's ddelta terms of the block are in
+                if (tid < gK && t0 + tid < L) {
+                    float s = 0.f;
+                    for (int cc = 0; cc < cpb; ++cc) s += at(PC_X, cc, tid);
+                    atomicAdd(p.dd_acc + (b * H + d0 / P) * L + t0 + tid, s);
                 }
             }
             // pass B: per (state, step), dB = sum over channels of g dt u, dC = of dy h_t
-            // (four consecutive steps per thread: one 16-byte atomic add each for dB and dC)
+            // (four consecutive steps per thread: one 16-byte atomic add each for dB and dC;
+            // consecutive threads take consecutive states)
             for (int i = tid; i < N * (gK / 4); i += NT) {
-                const int nn = i / (gK / 4), k4 = (i % (gK / 4)) * 4;
+                const int nn = i % N, k4 = (i / N) * 4;
                 if (t0 + k4 >= L) continue;
                 float sb[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int cc = 0; cc < cpb; ++cc) {
                     const int idx = cc * N + nn;
+                    const float4 du4 = at4(PC_DU, cc, k4), dy4 = at4(PC_DY, cc, k4);
+                    const float duv[4] = {du4.x, du4.y, du4.z, du4.w}, dyv[4] = {dy4.x, dy4.y, dy4.z, dy4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int k = k4 + e;
-                        sb[e] = fmaf(sG[k * TP + idx], at(PC_DU, cc, k), sb[e]);
-                        sc[e] = fmaf(at(PC_DY, cc, k), sH[(k + 1) * TP + idx], sc[e]);
+                        sb[e] = fmaf(sG[k * TP + idx], duv[e], sb[e]);
+                        sc[e] = fmaf(dyv[e], sH[(k + 1) * TP + idx], sc[e]);
                     }
                 }
                 const int64_t off = ((b * G + g) * N + nn) * L + t0 + k4;
@@ -458,20 +579,22 @@ GLayout glayout(const ssm_dims_t& d) {
     return w;
 }
 
-template <typename T, int N, bool PREF>
+template <typename T, int N, bool PREF, bool HEAD>
 int glaunch_one(const GParams& prm, unsigned grid, cudaStream_t s) {
     const GSmem S(N, prm.cpb);
     const size_t smem = (size_t)S.total * 4;
     if (smem > 227 * 1024) return SSM_ERR_UNSUPPORTED;
-    if (smem > 48 * 1024 && cudaFuncSetAttribute(scan_bwd_generic_kernel<T, N, PREF>,
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(scan_bwd_generic_kernel<T, N, PREF, HEAD>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return SSM_ERR_CUDA;
-    scan_bwd_generic_kernel<T, N, PREF><<<grid, (unsigned)S.T, smem, s>>>(prm);
+    scan_bwd_generic_kernel<T, N, PREF, HEAD><<<grid, (unsigned)S.T, smem, s>>>(prm);
     return cudaGetLastError() == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 template <typename T, int N>
 int glaunch(const GParams& prm, unsigned grid, cudaStream_t s) {
-    return prm.cpb >= 4 ? glaunch_one<T, N, true>(prm, grid, s) : glaunch_one<T, N, false>(prm, grid, s);
+    if (prm.head)
+        return prm.cpb >= 4 ? glaunch_one<T, N, true, true>(prm, grid, s) : glaunch_one<T, N, false, true>(prm, grid, s);
+    return prm.cpb >= 4 ? glaunch_one<T, N, true, false>(prm, grid, s) : glaunch_one<T, N, false, false>(prm, grid, s);
 }
 
 template <typename T>

@@ -359,6 +359,8 @@ GENERIC_CASES = [
     (si.Dims(1, 32, 70, 128, nheads=4, dtype="f32"), "plainhead", False, False, False),   # no z, D, bias; no softplus
     (si.Dims(1, 6, 70, 32, dtype="f32"), "c2", True, True, True),                     # 2 channels per CTA
     (si.Dims(2, 2, 50, 128, nheads=1, dtype="bf16"), "head", True, False, True),      # one head of 2 channels
+    (si.Dims(1, 128, 256, 128, nheads=2, dtype="bf16"), "head", True, True, True),   # 16-byte B and C loads
+    (si.Dims(2, 64, 96, 32, dtype="bf16"), "c2", True, False, True),                 # the same, dstate 32
 ]
 
 

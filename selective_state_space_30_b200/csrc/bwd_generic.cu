@@ -93,7 +93,7 @@ enum { PC_DT = 0, PC_DU, PC_U, PC_X, PC_DY, PC_DOUT, PC_Z, PC_DA, PC_W, kPC };
 // (channel, step) for all of its states
 struct GSmem {
     int T, TP, N, NB, cpb, NCH;
-    int H, G, BLK, Bs, Cs, PART, PC;   // offsets: sH, sG, sBlk, sB, sC, chunk sums, per-(channel, step) arrays
+    int H, G, BLK, Bs, Cs, PART, PC, DD, KC;   // offsets: sH, sG, sBlk, sB, sC, chunk sums, per-(channel, step) arrays
     int total;
     __host__ __device__ GSmem(int n, int c)
         : T(c * n), TP(c * n + 1), N(n), NB(n + 1), cpb(c), NCH((n + 31) / 32) {
@@ -104,7 +104,9 @@ struct GSmem {
         Cs = Bs + gK * NB;                  // [gK][NB]: C of the block
         PART = Cs + gK * NB;                // [cpb * NCH chunks][3][gK]: a chunk's parts of y, sum g B, the decay term
         PC = (PART + cpb * NCH * 3 * gK + 3) / 4 * 4;   // kPC arrays [cpb][KP], 16-byte aligned
-        total = PC + kPC * cpb * KP;
+        DD = PC + kPC * cpb * KP;           // [cpb][gK]: a block's ddelta terms (channels of one head)
+        KC = DD + cpb * gK;                 // [cpb][4]: per channel A of its head, D, delta_bias of its row
+        total = KC + 4 * cpb;
     }
 };
 
@@ -133,6 +135,8 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     float* sC = gsm + S.Cs;
     float* sPart = gsm + S.PART;
     float* pc = gsm + S.PC;
+    float* sDD = gsm + S.DD;
+    float* sKc = gsm + S.KC;
     const int cpb = p.cpb;
     auto at = [&](int arr, int cc, int k) -> float& { return pc[(arr * cpb + cc) * KP + k]; };
     auto at4 = [&](int arr, int cc, int k) -> float4 {
@@ -143,6 +147,13 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
 
     // A of this thread's (channel, state), natural units and log2 units
     const float An = HEAD ? __ldg(p.A + d / P) : __ldg(p.A + d * N + n);
+    // per-channel constants, read once (the first block's staging follows a barrier)
+    for (int cc = tid; cc < cpb; cc += NT) {
+        const int64_t dd = d0 + cc, hh = dd / P;
+        sKc[cc * 4 + 0] = HEAD ? __ldg(p.A + hh) : 0.f;
+        sKc[cc * 4 + 1] = p.D ? __ldg(p.D + dd) : 0.f;
+        sKc[cc * 4 + 2] = p.bias ? __ldg(p.bias + hh) : 0.f;
+    }
     const float a2 = An * kLog2e;
     const int nblk = (int)((L + gK - 1) / gK);
 
@@ -181,7 +192,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
                 const int64_t t = t0 + k, dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
                 if (t < L) {
                     ru[e] = GIo<T>::ld(p.u, rr * L + t);
-                    rx[e] = GIo<T>::ld(p.delta, (b * H + hh) * L + t) + (p.bias ? __ldg(p.bias + hh) : 0.f);
+                    rx[e] = GIo<T>::ld(p.delta, (b * H + hh) * L + t);   // delta_bias added at staging
                     if (full) {
                         rdo[e] = GIo<T>::ld(p.dout, rr * L + t);
                         if (p.z) rz[e] = GIo<T>::ld(p.z, rr * L + t);
@@ -201,12 +212,13 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
         }
     };
     // the per-(channel, step) values of one pair from its inputs (past L: dt = 0, so dA = 1)
-    auto put = [&](int cc, int k, bool valid, float uv, float x, float dov, float zv, bool full) {
+    auto put = [&](int cc, int k, bool valid, float uv, float xd, float dov, float zv, bool full) {
+        const float x = xd + sKc[cc * 4 + 2];   // + delta_bias
         const float dt = valid ? (p.softplus ? softplus1(x) : x) : 0.f;
         at(PC_DT, cc, k) = dt;
         at(PC_DU, cc, k) = dt * uv;
         if (HEAD) {
-            const float dA = ex2_approx(dt * (__ldg(p.A + (d0 + cc) / P) * kLog2e));
+            const float dA = ex2_approx(dt * (sKc[cc * 4 + 0] * kLog2e));
             at(PC_DA, cc, k) = dA;
             at(PC_W, cc, k) = dt * dA;
         }
@@ -228,7 +240,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
                 float uv = 0.f, x = 0.f, dov = 0.f, zv = 0.f;
                 if (t < L) {
                     uv = GIo<T>::ld(p.u, rr * L + t);
-                    x = GIo<T>::ld(p.delta, (b * H + hh) * L + t) + (p.bias ? __ldg(p.bias + hh) : 0.f);
+                    x = GIo<T>::ld(p.delta, (b * H + hh) * L + t);
                     if (full) {
                         dov = GIo<T>::ld(p.dout, rr * L + t);
                         if (p.z) zv = GIo<T>::ld(p.z, rr * L + t);
@@ -306,6 +318,19 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     // pass A: a warp per chunk of up to 32 states of one channel, a lane per step
     constexpr int NCH = (N + 31) / 32, NC = N < 32 ? N : 32;
     const int warp = tid / 32, lane = tid % 32, nwarps = NT / 32 > 0 ? NT / 32 : 1;
+    // channels of one head: a block's ddelta terms wait in sDD, and the threads of the first
+    // gK steps add them up and into dd_acc after the next barrier (one atomic add per step)
+    int64_t dd_t0 = -1;
+    auto flush_dd = [&]() {
+        if (one_head && dd_t0 >= 0) {
+            if (tid < gK && dd_t0 + tid < L) {
+                float s = 0.f;
+                for (int cc = 0; cc < cpb; ++cc) s += sDD[cc * gK + tid];
+                atomicAdd(p.dd_acc + (b * H + d0 / P) * L + dd_t0 + tid, s);
+            }
+            dd_t0 = -1;
+        }
+    };
     for (int seg = p.nseg - 1; seg >= 0; --seg) {
         const int b0 = seg * gSegB, b1 = min(nblk, b0 + gSegB);
         float hs = p.ckpt[(row * p.nseg + seg) * N + n];
@@ -322,6 +347,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
         for (int blk = b1 - 1; blk >= b0; --blk) {
             const int64_t t0 = (int64_t)blk * gK;
             __syncthreads();
+            flush_dd();   // the previous block's (its terms are in after the barrier)
             store(blk, true);
             __syncthreads();
             if (blk > b0) load(blk - 1, true);
@@ -429,27 +455,20 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
                 }
                 const float dt = at(PC_DT, cc, k);
                 const int64_t dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
-                if (HEAD) q *= __ldg(p.A + hh) * at(PC_DA, cc, k);   // one decay for every state
+                if (HEAD) q *= sKc[cc * 4 + 0] * at(PC_DA, cc, k);   // one decay for every state
                 const float uv = at(PC_U, cc, k), dy = at(PC_DY, cc, k);
-                const float Dv = p.D ? __ldg(p.D + dd) : 0.f;
+                const float Dv = sKc[cc * 4 + 1];
                 GIo<T>::st(p.du, rr * L + t, fmaf(dt, gB, dy * Dv));
                 const float ddt = fmaf(uv, gB, q);
                 const float ddl = p.softplus ? ddt * gsigmoid(at(PC_X, cc, k)) : ddt;
-                if (one_head) at(PC_X, cc, k) = ddl;   // summed over the CTA's channels below
+                if (one_head) sDD[cc * gK + k] = ddl;   // summed over the CTA's channels after the next barrier
                 else atomicAdd(p.dd_acc + (b * H + hh) * L + t, ddl);
                 if (p.z) {
                     const float zv = at(PC_Z, cc, k), sg = gsigmoid(zv);
                     GIo<T>::st(p.dz, rr * L + t, at(PC_DOUT, cc, k) * fmaf(Dv, uv, y) * (sg * fmaf(zv, 1.f - sg, 1.f)));
                 }
             }
-            if (one_head) {
-                __syncthreads();   // every channel's ddelta terms of the block are in
-                if (tid < gK && t0 + tid < L) {
-                    float s = 0.f;
-                    for (int cc = 0; cc < cpb; ++cc) s += at(PC_X, cc, tid);
-                    atomicAdd(p.dd_acc + (b * H + d0 / P) * L + t0 + tid, s);
-                }
-            }
+            dd_t0 = t0;
             // pass B: per (state, step), dB = sum over channels of g dt u, dC = of dy h_t
             // (four consecutive steps per thread: one 16-byte atomic add each for dB and dC;
             // consecutive threads take consecutive states)
@@ -483,6 +502,8 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             }
         }
     }
+    __syncthreads();
+    flush_dd();
     if (p.dh0) p.dh0[row * N + n] = gst;
     p.dA_part[row * N + n] = da;
     if (n == 0) p.dD_part[row] = dDacc;

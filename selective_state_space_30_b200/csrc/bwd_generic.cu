@@ -318,15 +318,15 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     // pass A: a warp per chunk of up to 32 states of one channel, a lane per step
     constexpr int NCH = (N + 31) / 32, NC = N < 32 ? N : 32;
     const int warp = tid / 32, lane = tid % 32, nwarps = NT / 32 > 0 ? NT / 32 : 1;
-    // channels of one head: a block's ddelta terms wait in sDD, and the threads of the first
-    // gK steps add them up and into dd_acc after the next barrier (one atomic add per step)
+    // channels of one head: a block's ddelta terms wait in sDD, and after the next barrier a
+    // thread per step adds them up and into dd_acc (one atomic add per step)
     int64_t dd_t0 = -1;
     auto flush_dd = [&]() {
         if (one_head && dd_t0 >= 0) {
-            if (tid < gK && dd_t0 + tid < L) {
+            for (int k = tid; k < gK && dd_t0 + k < L; k += NT) {   // fewer threads than steps: a loop
                 float s = 0.f;
-                for (int cc = 0; cc < cpb; ++cc) s += sDD[cc * gK + tid];
-                atomicAdd(p.dd_acc + (b * H + d0 / P) * L + dd_t0 + tid, s);
+                for (int cc = 0; cc < cpb; ++cc) s += sDD[cc * gK + k];
+                atomicAdd(p.dd_acc + (b * H + d0 / P) * L + dd_t0 + k, s);
             }
             dd_t0 = -1;
         }

@@ -361,6 +361,8 @@ GENERIC_CASES = [
     (si.Dims(2, 2, 50, 128, nheads=1, dtype="bf16"), "head", True, False, True),      # one head of 2 channels
     (si.Dims(1, 128, 256, 128, nheads=2, dtype="bf16"), "head", True, True, True),   # 16-byte B and C loads
     (si.Dims(2, 64, 96, 32, dtype="bf16"), "c2", True, False, True),                 # the same, dstate 32
+    (si.Dims(1, 2, 70, 8, nheads=1, dtype="f32"), "head", True, True, True),         # 16 threads: fewer than the steps
+    (si.Dims(2, 3, 45, 8, dtype="f32"), "c2", False, True, True),                    # 8 threads per CTA
 ]
 
 

@@ -149,7 +149,9 @@ def test_bwd_argument_checks():
 
 def test_bwd_full_size_mamba_130m():
     """The bench workload (mamba-130m: 8 x 1536 x 2048, N = 16, bf16), every gradient against
-    the full fp64 oracle backward."""
+    the full fp64 oracle backward: the recomputing call, and the call with the states the
+    forward stored (both in the bench's launch configuration: 8-warp CTAs)."""
+    import selective_state_space_30_b200 as ssm
     w = si.workload("mamba-130m")
     dims = w.dims
     inp = si.make_inputs(dims, w.recipe, w.seed)
@@ -157,6 +159,16 @@ def test_bwd_full_size_mamba_130m():
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"])
     g = run_bwd(dims, inp, gin)
     check_grads(g, ref, mag, dims.dtype, what="mamba-130m ")
+    del g
+    _, _, ck = _fwd_ckpt(dims, inp)
+    dev = {k: to_device(inp.get(k)) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    d = ssm.make_dims(dims.batch, dims.dim, dims.seqlen, dims.dstate, dims.H, dims.ngroups, ssm.SSM_BF16)
+    ws = torch.empty(ssm.ssm_selective_scan_bwd_workspace_size(d), dtype=torch.uint8, device="cuda")
+    g = ssm.selective_scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], to_device(gin["dout"]),
+                               dev["D"], dev["z"], dev["delta_bias"], True, workspace=ws, ckpt=ck)
+    assert ssm.ssm_selective_scan_bwd_device_status(ws) == ssm.SSM_OK
+    torch.cuda.synchronize()
+    check_grads(g, ref, mag, dims.dtype, what="mamba-130m, stored states ")
 
 
 def test_bwd_wait_timeout_reports_and_recovers():
@@ -277,8 +289,10 @@ def test_forward_checkpoints_refused_outside_the_backward(dims, opts):
         _fwd_ckpt(dims, inp, None, opts)
 
 
-@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[7], CASES[8]],
-                         ids=["2x64x100bf16", "2x64x77f32", "1x32x1000bf16", "2x64x777f32"])
+@pytest.mark.parametrize("case", [CASES[0], CASES[2], CASES[4], CASES[5], CASES[7], CASES[8],
+                                  (si.Dims(2, 32, 5, 16, dtype="bf16"), "c2", True, True, True)],
+                         ids=["2x64x100bf16", "2x64x77f32", "1x96x33bf16", "3x32x8bf16", "1x32x1000bf16",
+                              "2x64x777f32", "2x32x5bf16"])
 def test_bwd_with_forward_states(case):
     """ssm_selective_scan_bwd_ckpt with the states the forward stored: every gradient but dB
     and dC bit-equal to the backward that recomputes them (the same states, the same

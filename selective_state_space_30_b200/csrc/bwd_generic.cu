@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     auto run_block = [&](float h, auto keep_c) -> float {
         constexpr bool keep = decltype(keep_c)::value;   // a compile-time choice: no branch per step
         if (keep) sH[tid] = h;
-#pragma unroll 1
+#pragma unroll 2
         for (int k0 = 0; k0 < gK; k0 += 4) {
             const float4 du4 = at4(PC_DU, c, k0);
             const float4 x4 = HEAD ? at4(PC_DA, c, k0) : at4(PC_DT, c, k0);
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             run_block(sBlk[(blk - b0) * NT + tid], std::true_type{});
             const int kend = (int)(L - t0 < gK ? L - t0 : gK);   // steps of the block inside L
             // the state gradient back through the block: g += dy C is dLoss/dh_t
-#pragma unroll 1
+#pragma unroll 2
             for (int k0 = gK - 4; k0 >= 0; k0 -= 4) {
                 const float4 dy4 = at4(PC_DY, c, k0);
                 const float4 x4 = HEAD ? at4(PC_DA, c, k0) : at4(PC_DT, c, k0);

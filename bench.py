@@ -300,6 +300,82 @@ def cpu_oracle_sample(d, recipe, seed, target_s=12.0):
             "sample": f"{what} x L={d.seqlen} (N={d.dstate}), fp64, {dt:.1f} s"}
 
 
+def _grow_timed(run, target_s, kmax=1 << 16):
+    """run(k) -> (seconds, units): grow k (up to kmax, the whole workload) until one run takes
+    about target_s (at least a third of it); returns (seconds, units, k)."""
+    k = 1
+    while True:
+        dt, units = run(k)
+        if dt >= target_s / 3 or k >= kmax:
+            return dt, units, k
+        k = min(kmax, int(k * min(64.0, max(2.0, target_s / max(dt, 1e-3)))))
+
+
+def cpu_oracle_bwd_sample(d, recipe, seed, target_s=8.0):
+    """Time the fp64 oracle backward (as it stands) on a bounded sample: batch row 1 and a
+    growing number of channels (whole heads in the per-head layout) of the workload's shape."""
+    import oracle
+    import ssm_inputs as si
+    cores = _cores()
+    P = d.dim // d.H if d.head_mode else 1
+    maxk = d.dim // P
+
+    def run(k):
+        k = min(k, maxk)
+        sub = si.Dims(1, k * P, d.seqlen, d.dstate, nheads=k if d.head_mode else 0, ngroups=1, dtype=d.dtype)
+        inp = si.make_inputs(sub, recipe, seed)
+        dout = si.make_grad_inputs(sub, seed + 1)["dout"]
+        t0 = time.perf_counter()
+        oracle.run_inputs_bwd(sub, inp, dout, nthreads=cores)
+        return time.perf_counter() - t0, k * P * d.seqlen
+
+    dt, units, k = _grow_timed(run, target_s, maxk)
+    return {"value": units / dt / 1e9, "unit": "Gelem/s", "cores": cores, "kind": "oracle",
+            "sample": f"{units // d.seqlen} channels x L={d.seqlen} (N={d.dstate}, batch row 1), fp64 backward, "
+                      f"{dt:.1f} s"}
+
+
+def cpu_oracle_decode_sample(dims, recipe, target_s=5.0):
+    """Time the fp64 oracle on decode steps (a scan of one step from a state) of a growing
+    number of batch rows of the decode shape."""
+    import oracle
+    import ssm_inputs as si
+    cores = _cores()
+
+    def run(k):
+        k = min(k, dims.batch)
+        sub = si.Dims(k, dims.dim, 1, dims.dstate, nheads=dims.nheads, ngroups=dims.ngroups, dtype=dims.dtype)
+        inp = si.make_inputs(sub, recipe, 0)
+        h0 = np.random.default_rng(1).standard_normal((k, dims.dim, dims.dstate))
+        t0 = time.perf_counter()
+        oracle.run_inputs(sub, inp, h0=h0, nthreads=cores)
+        return time.perf_counter() - t0, k * dims.dim
+
+    dt, units, k = _grow_timed(run, target_s, dims.batch)
+    return {"value": units / dt / 1e9, "unit": "Gelem/s", "cores": cores, "kind": "oracle",
+            "sample": f"{k} batch rows x {dims.dim} channels, one step (N={dims.dstate}), fp64, {dt:.1f} s"}
+
+
+def cpu_oracle_conv1d_sample(sh, target_s=5.0):
+    """Time the fp64 oracle convolution on a growing number of channels of one batch row."""
+    import oracle
+    cores = _cores()
+    rng = np.random.default_rng(0)
+
+    def run(k):
+        k = min(k, sh["batch"] * sh["dim"])
+        x = rng.standard_normal((1, k, sh["seqlen"]))
+        w = rng.standard_normal((k, sh["width"]))
+        b = rng.standard_normal(k)
+        t0 = time.perf_counter()
+        oracle.causal_conv1d(x, w, b, True)
+        return time.perf_counter() - t0, k * sh["seqlen"]
+
+    dt, units, k = _grow_timed(run, target_s, sh["batch"] * sh["dim"])
+    return {"value": units / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": f"{k} channels x L={sh['seqlen']} (width {sh['width']}), fp64, one thread, {dt:.1f} s"}
+
+
 # ------------------------------------------------------------------ arms
 
 def run_reference(args):
@@ -678,7 +754,9 @@ def run_decode(args):
     if rank != 0:
         return
     gbs = alg / (ms * 1e-3) / 1e9
-    line = {"metric": "selective-state-update (decode step) GB/s on 1 B200", "op": "decode",
+    cpu = None if (world > 1 or args.no_cpu_baseline) else cpu_oracle_decode_sample(dims, rec)
+    line = {"metric": "selective-state-update (decode step) Gelem/s (batch rows x channels per second) on 1 B200",
+            "op": "decode",
             "value": world * dims.batch * dims.dim * args.steps / (total * 1e-3) / 1e9, "unit": "Gelem/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -686,8 +764,10 @@ def run_decode(args):
             "config": dict(sh, workload=args.workload,
                            l2=f"{copies} rotating state/input sets of {alg / 1e6:.0f} MB, no flush"),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                         "traffic": None, "peak_source": src, "alg_bytes_per_launch": alg},
-            "clocks": clk.summary(), "gpu_launches": args.steps}
+                         "traffic": _traffic_from_profiles(args.workload, key="decode:" + args.workload,
+                                                           sha=_src_hash(("decode.cu",))),
+                         "peak_source": src, "alg_bytes_per_launch": alg},
+            "cpu_baseline": cpu, "clocks": clk.summary(), "gpu_launches": args.steps}
     print(json.dumps(line), flush=True)
 
 
@@ -753,6 +833,7 @@ def run_conv1d(args):
     if rank != 0:
         return
     gbs = alg / (ms * 1e-3) / 1e9
+    cpu = None if (world > 1 or args.no_cpu_baseline) else cpu_oracle_conv1d_sample(sh)
     line = {"metric": "causal conv1d (d_conv taps + SiLU) Gelem/s on 1 B200", "op": "conv1d",
             "value": job_throughput(world, elems, args.steps, total), "unit": "Gelem/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -761,8 +842,10 @@ def run_conv1d(args):
             "config": dict(sh, workload=args.workload,
                            l2=f"{copies} rotating input sets of {alg / 1e6:.0f} MB, no flush"),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                         "traffic": None, "peak_source": src, "alg_bytes_per_launch": alg},
-            "clocks": clk.summary(), "gpu_launches": args.steps}
+                         "traffic": _traffic_from_profiles(args.workload, key="conv1d:" + args.workload,
+                                                           sha=_src_hash(("conv1d.cu",))),
+                         "peak_source": src, "alg_bytes_per_launch": alg},
+            "cpu_baseline": cpu, "clocks": clk.summary(), "gpu_launches": args.steps}
     print(json.dumps(line), flush=True)
 
 
@@ -853,6 +936,7 @@ def run_bwd(args):
     ms_f, _, _ = timed(lambda: ssm.ssm_selective_scan_fwd_h0(*fwd_args, stream.cuda_stream), args.steps)
     ssm.ssm_scan_destroy(plan)
     hbm_gbs, sm_max_mhz, src = _peaks()
+    cpu = None if (world > 1 or args.no_cpu_baseline) else cpu_oracle_bwd_sample(d, w.recipe, w.seed)
     finish_ranks()
     if rank != 0:
         return
@@ -892,7 +976,7 @@ def run_bwd(args):
                           "ms_per_step": ms_re, "value": job_throughput(world, elems, args.steps, total_re),
                           "roofline": roof(ms_re, "bwd:" + w.name)},
             "forward": {"ms_plain": ms_f, "ms_with_states": ms_fc, "state_bytes": ck_bytes},
-            "clocks": clocks, "gpu_launches": (2 if stored else 4) * args.steps}
+            "cpu_baseline": cpu, "clocks": clocks, "gpu_launches": (2 if stored else 4) * args.steps}
     print(json.dumps(line), flush=True)
 
 

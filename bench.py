@@ -660,6 +660,10 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(d, w.recipe, w.seed)
+        # the oracle beside every other shape too, on a shorter sample each
+        for name, e in per_config.items():
+            wk = si.WORKLOADS[name]
+            e["cpu_baseline"] = cpu_oracle_sample(wk.dims, wk.recipe, wk.seed, target_s=3.0)
 
     finish_ranks()
     if rank != 0:

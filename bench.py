@@ -957,7 +957,8 @@ def run_bwd(args):
         gexps = exps / (ms_ * 1e-3) / 1e9
         gbs = a / (ms_ * 1e-3) / 1e9
         return {"bound": "alu", "achieved": gexps, "peak": mufu_peak, "unit": "Gexp/s", "frac": gexps / mufu_peak,
-                "traffic": _traffic_from_profiles(w.name, key=traffic_key, sha=_src_hash(("bwd.cu",))),
+                "traffic": _traffic_from_profiles(w.name, key=traffic_key,
+                                                  sha=_src_hash(("bwd.cu",) if stored else ("bwd_generic.cu",))),
                 "peak_source": f"148 SMs x 16 ex2/clk x {sm_max_mhz:.0f} MHz ({src} sm_max_mhz)",
                 "exps_per_launch": exps,
                 "hbm": {"achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,

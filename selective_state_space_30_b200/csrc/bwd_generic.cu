@@ -96,7 +96,7 @@ struct GSmem {
     int H, G, BLK, Bs, Cs, PART, PC, DD, KC;   // offsets: sH, sG, sBlk, sB, sC, chunk sums, per-(channel, step) arrays
     int total;
     __host__ __device__ GSmem(int n, int c)
-        : T(c * n), TP(c * n + 1), N(n), NB(n + 1), cpb(c), NCH((n + 31) / 32) {
+        : T(c * n), TP(c * n + 4), N(n), NB(n + 4), cpb(c), NCH((n + 31) / 32) {
         H = 0;                              // [gK + 1][TP]: the state entering the block, then after each step
         G = H + (gK + 1) * TP;              // [gK][TP]: dLoss/dh_t of each step
         BLK = G + gK * TP;                  // [gSegB][T]: the state entering each block of the segment
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     extern __shared__ __align__(16) float gsm[];
     const GSmem S(N, p.cpb);
     const int NT = S.T, TP = S.TP;
-    constexpr int NB = N + 1;
+    constexpr int NB = N + 4;
     const int tid = threadIdx.x;
     const int c = tid / N, n = tid % N;
     const int64_t L = p.seqlen, Dm = p.dim, H = p.nheads, G = p.ngroups;
@@ -142,6 +142,11 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     auto at4 = [&](int arr, int cc, int k) -> float4 {
         return *reinterpret_cast<const float4*>(pc + (arr * cpb + cc) * KP + k);
     };
+    // one A per head with at least 32 states: dA's terms are w_t sum_n g h_(t-1) per (channel,
+    // step), the decay sum pass A forms anyway; the (channel, step) threads of pass A add them
+    // (one item each: cpb * gK <= cpb * N threads)
+    constexpr bool DA_SUM = HEAD && N >= 32;
+    float da_item = 0.f;
     // every channel of the CTA in one head: the head's ddelta terms are summed here first
     const bool one_head = HEAD && d0 / P == (d0 + cpb - 1) / P;
 
@@ -375,7 +380,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
                             dA = ex2_approx(xv[e] * a2);
                             w = xv[e] * dA;
                         }
-                        da = fmaf(gst * sH[k * TP + tid], w, da);
+                        if (!DA_SUM) da = fmaf(gst * sH[k * TP + tid], w, da);
                         gst *= dA;
                     } else {
                         sG[k * TP + tid] = 0.f;
@@ -387,8 +392,9 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
                     if (k < kend) dDacc = fmaf(at(PC_DY, c, k), at(PC_U, c, k), dDacc);
             __syncthreads();   // sH and sG complete
             // pass A, first half: per chunk and step (lane), the chunk's parts of y = sum C h,
-            // gB = sum g B and q = sum g h_(t-1) (A dA) into sPart.  No shuffles: the lanes walk
-            // rows of odd length, so they meet different banks.
+            // gB = sum g B and q = sum g h_(t-1) (A dA) into sPart.  No shuffles: each lane reads
+            // its step's rows four states at a time, and rows 4 mod 32 floats apart put the eight
+            // lanes of a 16-byte phase in different banks.
             if (NT >= 32) {
                 for (int ch = warp; ch < cpb * NCH; ch += nwarps) {
                     const int cc = ch / NCH, n0 = (ch % NCH) * NC, k = lane;
@@ -399,16 +405,26 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
                     const float* crow = sC + k * NB + n0;
                     const float dt = at(PC_DT, cc, k);
                     float y = 0.f, gB = 0.f, q = 0.f;
-#pragma unroll 8
-                    for (int i = 0; i < NC; ++i) {
-                        const float gv = grow[i];
-                        y = fmaf(crow[i], hrow[i], y);
-                        gB = fmaf(gv, brow[i], gB);
-                        if (HEAD) {
-                            q = fmaf(gv, prow[i], q);
-                        } else {
-                            const float Ann = __ldg(p.A + (d0 + cc) * N + n0 + i);
-                            q = fmaf(gv * prow[i], Ann * ex2_approx(dt * (Ann * kLog2e)), q);
+#pragma unroll 2
+                    for (int i0 = 0; i0 < NC; i0 += 4) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(grow + i0);
+                        const float4 h4 = *reinterpret_cast<const float4*>(hrow + i0);
+                        const float4 p4 = *reinterpret_cast<const float4*>(prow + i0);
+                        const float4 b4 = *reinterpret_cast<const float4*>(brow + i0);
+                        const float4 c4 = *reinterpret_cast<const float4*>(crow + i0);
+                        const float gv[4] = {g4.x, g4.y, g4.z, g4.w}, hv[4] = {h4.x, h4.y, h4.z, h4.w};
+                        const float pv[4] = {p4.x, p4.y, p4.z, p4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                        const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            y = fmaf(cv[e], hv[e], y);
+                            gB = fmaf(gv[e], bv[e], gB);
+                            if (HEAD) {
+                                q = fmaf(gv[e], pv[e], q);
+                            } else {
+                                const float Ann = __ldg(p.A + (d0 + cc) * N + n0 + i0 + e);
+                                q = fmaf(gv[e] * pv[e], Ann * ex2_approx(dt * (Ann * kLog2e)), q);
+                            }
                         }
                     }
                     float* pp = sPart + ch * 3 * gK + k;
@@ -455,6 +471,7 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
                 }
                 const float dt = at(PC_DT, cc, k);
                 const int64_t dd = d0 + cc, hh = dd / P, rr = b * Dm + dd;
+                if (DA_SUM) da_item = fmaf(q, at(PC_W, cc, k), da_item);   // sum_n g h_(t-1) times dt dA
                 if (HEAD) q *= sKc[cc * 4 + 0] * at(PC_DA, cc, k);   // one decay for every state
                 const float uv = at(PC_U, cc, k), dy = at(PC_DY, cc, k);
                 const float Dv = sKc[cc * 4 + 1];
@@ -505,7 +522,16 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     __syncthreads();
     flush_dd();
     if (p.dh0) p.dh0[row * N + n] = gst;
-    p.dA_part[row * N + n] = da;
+    if constexpr (DA_SUM) {
+        // channel cc's total from the gK pass-A threads of warp cc (their items are (cc, step))
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) da_item += __shfl_xor_sync(0xffffffffu, da_item, o);
+        p.dA_part[row * N + n] = 0.f;
+        __syncthreads();
+        if (tid < cpb * gK && lane == 0) p.dA_part[(b * Dm + d0 + tid / gK) * N] = da_item;
+    } else {
+        p.dA_part[row * N + n] = da;
+    }
     if (n == 0) p.dD_part[row] = dDacc;
 }
 

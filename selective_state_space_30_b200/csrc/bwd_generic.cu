@@ -146,6 +146,9 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
     // step), the decay sum pass A forms anyway; the (channel, step) threads of pass A add them
     // (one item each: cpb * gK <= cpb * N threads)
     constexpr bool DA_SUM = HEAD && N >= 32;
+    // pass B's first thread: past the threads of pass A's second half when half the CTA or
+    // more is left for it, so that the two phases overlap instead of queueing on one thread
+    const int pb0 = NT >= 2 * cpb * gK ? cpb * gK : 0;
     float da_item = 0.f;
     // every channel of the CTA in one head: the head's ddelta terms are summed here first
     const bool one_head = HEAD && d0 / P == (d0 + cpb - 1) / P;
@@ -489,7 +492,8 @@ __global__ void __launch_bounds__(N >= 64 ? 512 : 256) scan_bwd_generic_kernel(c
             // pass B: per (state, step), dB = sum over channels of g dt u, dC = of dy h_t
             // (four consecutive steps per thread: one 16-byte atomic add each for dB and dC;
             // consecutive threads take consecutive states)
-            for (int i = tid; i < N * (gK / 4); i += NT) {
+            // (where there are threads to spare, not on those that ran pass A's second half)
+            for (int i = tid - pb0; i >= 0 && i < N * (gK / 4); i += NT - pb0) {
                 const int nn = i % N, k4 = (i / N) * 4;
                 if (t0 + k4 >= L) continue;
                 float sb[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};

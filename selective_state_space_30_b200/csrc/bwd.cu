@@ -196,6 +196,22 @@ __device__ __forceinline__ float staged(const unsigned char* base, int row, int 
     return Io<T>::f(reinterpret_cast<const typename Io<T>::raw*>(base + row * Smem<T, 8>::kRow)[k]);
 }
 
+// a (B_2j, B_2j+1) or (C_2j, C_2j+1) pair in shared memory: two bf16 in one word for bf16
+// I/O (half the shared-memory bytes; unpacked on use), a float2 for fp32
+template <typename T> struct BCPair;
+template <> struct BCPair<float> {
+    using W = float2;
+    __device__ static W pack(float a, float b) { return make_float2(a, b); }
+    __device__ static float2 get(W w) { return w; }
+};
+template <> struct BCPair<__nv_bfloat16> {
+    using W = uint32_t;
+    __device__ static W pack(float a, float b) {
+        return (__float_as_uint(b) & 0xFFFF0000u) | (__float_as_uint(a) >> 16);   // exact: a, b are bf16 values
+    }
+    __device__ static float2 get(W w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
+};
+
 __device__ __forceinline__ float sigmoid1(float x) { return rcp_approx(1.f + ex2_approx(x * -kLog2e)); }
 
 // One step of the recurrence on the lane's two states, as f32x2 pairs (the same
@@ -273,8 +289,9 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
     float2* sPa = reinterpret_cast<float2*>(smem + S::PA);
     float2* sPb = reinterpret_cast<float2*>(smem + S::PB);
     float2* sU = reinterpret_cast<float2*>(smem + S::U);
-    float2* sB = reinterpret_cast<float2*>(smem + S::BS);
-    float2* sC = reinterpret_cast<float2*>(smem + S::CS);
+    using BW = BCPair<T>;
+    typename BW::W* sB = reinterpret_cast<typename BW::W*>(smem + S::BS);
+    typename BW::W* sC = reinterpret_cast<typename BW::W*>(smem + S::CS);
     float* sR = reinterpret_cast<float*>(smem + S::RED);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -382,7 +399,7 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                 for (int it = tid; it < kBT * 8; it += kThreads) {
                     const int t = it >> 3, jj = it & 7;
                     const unsigned char* sb = stage + 4 * kCT * S::kRow;
-                    sB[t * 8 + jj] = make_float2(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t));
+                    sB[t * 8 + jj] = BW::pack(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t));
                 }
                 // the next block's rows go into the other buffer, read last by the previous block
                 if (blk + 1 < blk1) issue_fwd(stage_base + (cur ^ 1) * S::kStageBytes, t0 + kBT);
@@ -393,7 +410,7 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
 #pragma unroll 4
                     for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
                         const float2 pv = sPa[c * kPS + t];
-                        const float2 bb = sB[t * 8 + j];
+                        const float2 bb = BW::get(sB[t * 8 + j]);
                         float2 dA;
                         fwd_step(h, dA, pv.x, pv.y, bb.x, bb.y, al);
                     }
@@ -472,8 +489,8 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                 const int t = it >> 3, jj = it & 7;
                 const unsigned char* sb = stage + 4 * kCT * S::kRow;
                 const unsigned char* sc = stage + (4 * kCT + kN) * S::kRow;
-                sB[t * 8 + jj] = make_float2(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t));
-                sC[t * 8 + jj] = make_float2(staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
+                sB[t * 8 + jj] = BW::pack(staged<T>(sb, 2 * jj, t), staged<T>(sb, 2 * jj + 1, t));
+                sC[t * 8 + jj] = BW::pack(staged<T>(sc, 2 * jj, t), staged<T>(sc, 2 * jj + 1, t));
             }
             // the next (earlier) block's rows go into the other buffer
             if (blk > blk0) issue_rev(stage_base + (cur ^ 1) * S::kStageBytes, t0 - kBT);
@@ -494,7 +511,7 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
 #pragma unroll 4
                         for (int t = w * kWin; t < (w + 1) * kWin; ++t) {
                             const float2 pv = sPa[c * kPS + t];
-                            const float2 bb = sB[t * 8 + j];
+                            const float2 bb = BW::get(sB[t * 8 + j]);
                             float2 dA;
                             fwd_step(hh, dA, pv.x, pv.y, bb.x, bb.y, al);
                         }
@@ -513,8 +530,8 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
 #pragma unroll
                     for (int t = 0; t < kWin; ++t) {
                         const float2 pv = sPa[c * kPS + tw + t];
-                        const float2 bb = sB[(tw + t) * 8 + j];
-                        const float2 cc = sC[(tw + t) * 8 + j];
+                        const float2 bb = BW::get(sB[(tw + t) * 8 + j]);
+                        const float2 cc = BW::get(sC[(tw + t) * 8 + j]);
                         fwd_step(hh, dAr[t], pv.x, pv.y, bb.x, bb.y, al);
                         hr[t] = hh;
                         yp[t] = fmaf(cc.x, hh.x, cc.y * hh.y);
@@ -527,8 +544,8 @@ __global__ void __launch_bounds__(32 * NW, 16 / NW) scan_bwd_kernel(const BwdPar
                 for (int t = kWin - 1; t >= 0; --t) {
                     const float2 pv = sPa[c * kPS + tw + t];   // dt, dt*u
                     const float dy = sPb[c * kPS + tw + t].x;
-                    const float2 bb = sB[(tw + t) * 8 + j];
-                    const float2 cc = sC[(tw + t) * 8 + j];
+                    const float2 bb = BW::get(sB[(tw + t) * 8 + j]);
+                    const float2 cc = BW::get(sC[(tw + t) * 8 + j]);
                     gs = fma2(dup2(dy), cc, gs);   // + dy C: now dLoss/dh_t
                     const float2 hp = t > 0 ? hr[t - 1] : he;
                     const float2 e = mul2(mul2(gs, hp), dAr[t]);

@@ -11,7 +11,7 @@ import torch
 import oracle
 import ssm_inputs as si
 from parity import check_out, check_state, run_gpu, to_device, to_host_f64
-from test_bwd_gpu import check_grads
+from test_bwd_gpu import check_grads, grad_scale
 
 pytestmark = pytest.mark.gpu
 
@@ -70,7 +70,7 @@ def test_fuzz_backward(seed):
     torch.cuda.synchronize()
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin.get("dlast"), h0=gin.get("h0"),
                                      want_dh0=with_h0)
-    check_grads(g, ref, mag, dims.dtype, what=f"{dims} ")
+    check_grads(g, ref, mag, dims.dtype, what=f"{dims} ", gscale=grad_scale(inp, gin, dims.seqlen))
 
 
 @pytest.mark.parametrize("seed", range(24))
@@ -105,3 +105,11 @@ def test_fuzz_backward_with_stored_states(seed):
     ref, mag = oracle.run_inputs_bwd(dims, inp, gin["dout"], dlast=gin.get("dlast"), h0=gin.get("h0"),
                                      want_dh0=with_h0)
     check_grads(g, ref, mag, dims.dtype, what=f"{dims}, stored states ")
+
+
+@pytest.mark.parametrize("seed", [78, 138, 324, 360, 401])
+def test_fuzz_backward_deep_decay(seed):
+    """Seeds of the backward draw (dstate 64 or 128, A down to -128) whose decays fall
+    below fp32's smallest normal number: the kernel's dh0 is zero where the fp64 oracle's
+    is about 1e-38, within the tolerance's floor of 2^-126 times the state gradient bound."""
+    test_fuzz_backward(seed)
